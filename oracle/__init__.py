@@ -1,0 +1,99 @@
+"""fp64 CPU oracle for the chunk-KDA forward -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, ``__graft_entry__.smoke()`` and bench.py's cpu_baseline /
+``--impl reference`` legs may import this package.  The product path
+(``chunked_gated_delta_12_b200`` and its CUDA library) never does, and shares
+no code with it: the only thing both sides read is the seeded input generator,
+which holds no KDA arithmetic.
+
+``kda_fwd`` is the plain token-by-token recurrence in ``kda_oracle.c`` (C,
+fp64, pthreads over independent (document, head) chains).  ``chunked.py`` is a
+second, independent formulation (chunked UT/WY algebra in numpy fp64) used
+only to cross-check the recurrence.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.c with gcc into oracle/libkda_oracle.so (no GPU needed)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f = lib.kda_oracle_fwd
+        f.restype = ctypes.c_int
+        f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                              ctypes.c_double, ctypes.c_int, ctypes.c_void_p,
+                                              ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _f32(x) -> np.ndarray:
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def kda_fwd(q, k, v, g, beta, cu_seqlens, scale: float | None = None, eps: float = 1e-6,
+            erase: bool = True, chains=None, n_threads: int | None = None,
+            return_state: bool = False):
+    """Token-recurrence KDA forward in fp64.
+
+    q, k, g: [T, H, K] (any float dtype; widened exactly to fp32 then fp64 inside)
+    v: [T, H, V]; beta: [T, H]; cu_seqlens: [n_docs + 1] int.
+    chains: optional list of chain ids (doc * H + head) to compute; other rows of
+    the result are NaN.  Returns o [T, H, V] fp64 (and the final states
+    [n_chains, K, V] if ``return_state``).
+    """
+    q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
+    beta = _f32(beta)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    T, H, K = q.shape
+    V = v.shape[2]
+    assert k.shape == (T, H, K) and g.shape == (T, H, K) and v.shape[:2] == (T, H)
+    assert beta.shape == (T, H)
+    n_docs = len(cu) - 1
+    if scale is None:
+        scale = 1.0 / np.sqrt(K)
+    ch = None if chains is None else np.ascontiguousarray(chains, dtype=np.int32)
+    n_chains = n_docs * H if ch is None else len(ch)
+    out = np.full((T, H, V), np.nan, dtype=np.float64)
+    fs = np.zeros((n_chains, K, V), dtype=np.float64) if return_state else None
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    rc = _load().kda_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu),
+                                n_docs, T, H, K, V, float(scale), float(eps), int(bool(erase)),
+                                _ptr(ch), n_chains, _ptr(out), _ptr(fs), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (cu_seqlens or sizes malformed)")
+    return (out, fs) if return_state else out
+
+
+def chain_rows(cu_seqlens, H: int, chain: int) -> tuple[int, int, int]:
+    """(first token, end token, head) of chain id doc * H + head."""
+    doc, h = divmod(int(chain), H)
+    return int(cu_seqlens[doc]), int(cu_seqlens[doc + 1]), h
