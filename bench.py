@@ -1,0 +1,310 @@
+"""Chunk-KDA forward benchmark (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+
+A step is one chunk-KDA forward over the whole workload (default: the dense
+4 x 8192 batch, H = 32, K = V = 128, bf16 q/k/v, fp32 g and beta), inputs
+already resident in HBM.  Under torchrun every rank runs its own replica of
+the workload (documents and heads are independent; no collective on the data
+path), so per-GPU work is fixed and the line reports weak scaling.
+
+`--impl reference` times the fp64 CPU oracle on this host's cores instead
+(rank 0 only), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk-KDA fwd Mtokens/s at H=32,K=V=128 bf16; TFLOP/s and % of roofline"
+UNIT = "Mtokens/s"
+BYTES_PER_TOKEN_HEAD = 1540          # q,k,v bf16 768 + g fp32 512 + beta 4 + o bf16 256
+FLOPS_PER_TOKEN_HEAD = 180224        # 6 d^2 + 10 C d, d = 128, C = 64 (dense chunk tiles)
+FLOPS_PER_TOKEN_HEAD_TRI = 139264    # same, skipping the zero triangles
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j.get("bf16_tflops", 1590.0)), "measured"
+    return FALLBACK_HBM_GBS, 1590.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunked_gated_delta_12_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel sources still match."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    rec = j.get("per_launch_bytes", {}).get(workload_name)
+    return None if rec is None else float(rec)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev = dev_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._th = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                r = subprocess.run(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                   timeout=5)
+                parts = [x.strip() for x in r.stdout.strip().split(",")]
+                if len(parts) == 7:
+                    self.samples.append(parts)
+            except Exception:
+                pass
+            self._stop.wait(0.05)
+
+    def __enter__(self):
+        self._th = threading.Thread(target=self._run, daemon=True)
+        self._th.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._th.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def oracle_sample_rate(w, d, tokens: int, n_threads: int):
+    """Time the fp64 oracle on the first `tokens` tokens of document 0 (all heads)."""
+    import oracle
+    from chunked_gated_delta_12_b200.inputs import bf16_bits_to_f32
+    tokens = min(tokens, int(d["cu_seqlens"][1]))
+    sl = slice(0, tokens)
+    f = lambda key: bf16_bits_to_f32(d[key][sl]).reshape(d[key][sl].shape)
+    q, k, v = f("q"), f("k"), f("v")
+    g, b = np.ascontiguousarray(d["g"][sl]), np.ascontiguousarray(d["beta"][sl])
+    t0 = time.perf_counter()
+    oracle.kda_fwd(q, k, v, g, b, [0, tokens], n_threads=n_threads)
+    dt = time.perf_counter() - t0
+    return tokens / dt / 1e6, dt, tokens
+
+
+def run_reference(args, w, d):
+    """fp64 oracle on the host cores: each step a bounded sample of the workload."""
+    cores = os.cpu_count() or 1
+    # calibrate: seconds per token (all heads) at this core count
+    _, dt, n = oracle_sample_rate(w, d, 64, cores)
+    per_tok = dt / n
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    tokens = int(max(64, min(4096, budget / per_tok)))
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, d, tokens, cores)
+    times = []
+    for _ in range(args.steps):
+        _, dt, n = oracle_sample_rate(w, d, tokens, cores)
+        times.append(dt)
+    total = sum(times)
+    value = args.steps * n / total / 1e6
+    sample = (f"first {n} tokens of document 0 of {w.name}, all {w.H} heads "
+              f"({w.H} independent chains, fp64 token recurrence)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(w.describe(), sample_tokens=n),
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": cores,
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    from chunked_gated_delta_12_b200.inputs import generate, workload
+    w = workload(args.workload)
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        d = generate(w)
+        run_reference(args, w, d)
+        return
+
+    import torch
+    import chunked_gated_delta_12_b200 as kda
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = generate(w)
+    host = {}
+    for key in ("q", "k", "v"):
+        host[key] = torch.from_numpy(d[key].view(np.int16)).view(torch.bfloat16).pin_memory()
+    host["g"] = torch.from_numpy(d["g"]).pin_memory()
+    host["beta"] = torch.from_numpy(d["beta"]).pin_memory()
+    host["cu_seqlens"] = torch.from_numpy(d["cu_seqlens"]).pin_memory()
+    dv = {key: t.to(dev) for key, t in host.items()}
+    out = torch.empty_like(dv["q"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_chunk_fwd(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"], dv["cu_seqlens"], out=out,
+                          stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    kda.device_status(stream)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    # timed region: K steps, events on the launching stream (one kernel launch per step)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    smi_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(smi_index) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    kda.device_status(stream)
+    per_launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    elapsed_ms = ev[0].elapsed_time(ev[-1])
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs -> device, forward, result -> host
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for key in host:
+            dv[key].copy_(host[key], non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    tokens_all = w.T * world
+    ms_step = elapsed_ms / args.steps
+    value = tokens_all / (ms_step * 1e-3) / 1e6
+    hbm_peak, tc_peak, peak_kind = peaks()
+    launch_ms = float(np.mean(per_launch_ms))
+    alg_bytes = w.T * w.H * BYTES_PER_TOKEN_HEAD
+    achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
+    tflops = w.T * w.H * FLOPS_PER_TOKEN_HEAD / (launch_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(w.describe(), l2="inputs 1.6 GB per step > 126 MB L2; no flush",
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name),
+                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
+                     "launch_ms": launch_ms},
+        "tflops": {"dense_tile": tflops, "triangle_exact": tflops * FLOPS_PER_TOKEN_HEAD_TRI / FLOPS_PER_TOKEN_HEAD,
+                   "frac_of_bf16_peak": tflops / tc_peak},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "e2e": {"value": tokens_all / (e2e_ms * 1e-3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        rate, dt, n = oracle_sample_rate(w, d, 1024, cores)
+        if dt < 5.0:   # grow the sample towards ~10 s of CPU work
+            rate, dt, n = oracle_sample_rate(w, d, int(min(w.lengths[0], 1024 * 10.0 / max(dt, 1e-3))), cores)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"first {n} tokens of document 0, all {w.H} heads, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,8 @@
+"""chunked_gated_delta_12_b200: chunk-KDA forward for B200 (sm_100a).
+
+The compute lives in libkda.so (CUDA, C ABI in include/kda.h); this package
+only marshals torch tensors into that ABI.
+"""
+from ._lib import KdaError, device_status, kda_chunk_fwd, lib
+
+__all__ = ["kda_chunk_fwd", "device_status", "KdaError", "lib"]

@@ -1,0 +1,95 @@
+"""ctypes binding of libkda (include/kda.h): argument marshalling only.
+
+Every step of the forward runs in the CUDA library; nothing here computes.
+If libkda.so is missing or the device is not sm_100, calls raise -- there is
+no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkda.so")
+
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED_DEVICE", 3: "KDA_ERR_CUDA",
+          4: "KDA_ERR_NO_MEMORY", 5: "KDA_ERR_TIMEOUT", 6: "KDA_ERR_BAD_SEQLENS"}
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libkda.so not built ({LIB_PATH}); run "
+                              "`python -m chunked_gated_delta_12_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.kda_chunk_fwd.restype = i32
+        L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp]
+        L.kda_last_error.restype = ctypes.c_char_p
+        L.kda_last_error.argtypes = []
+        L.kda_device_status.restype = i32
+        L.kda_device_status.argtypes = [vp]
+        L.kda_abi_version.restype = i32
+        L.kda_abi_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise KdaError(rc, lib().kda_last_error().decode())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, cu_seqlens: torch.Tensor, out: torch.Tensor | None = None,
+                  stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Chunked KDA forward through libkda's kda_chunk_fwd.
+
+    q, k, v: [T, H, 128] bf16 (a leading batch dim of 1 is accepted); g: [T, H, 128] fp32;
+    beta: [T, H] fp32; cu_seqlens: [n_docs + 1] int32, all on the same CUDA device.
+    Returns out [T, H, 128] bf16 (allocated by torch if not given).
+    """
+    if q.dim() == 4:
+        q, k, v, g = (x.squeeze(0) for x in (q, k, v, g))
+        beta = beta.squeeze(0)
+    T, H, D = q.shape
+    for name, t, dt, shape in (("q", q, torch.bfloat16, (T, H, D)), ("k", k, torch.bfloat16, (T, H, D)),
+                               ("v", v, torch.bfloat16, (T, H, D)), ("g", g, torch.float32, (T, H, D)),
+                               ("beta", beta, torch.float32, (T, H))):
+        if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or not t.is_cuda:
+            raise KdaError(1, f"{name} must be a contiguous CUDA {dt} tensor of shape {shape} "
+                              f"(got {t.dtype} {tuple(t.shape)})")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise KdaError(1, "cu_seqlens must be a 1-d int32 CUDA tensor")
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                             cu_seqlens.numel() - 1, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))
+    _check(rc)
+    return out
+
+
+def device_status(stream: torch.cuda.Stream | None = None) -> None:
+    """Synchronise the stream and raise if a kernel flagged bad cu_seqlens or a timeout."""
+    _check(lib().kda_device_status(ctypes.c_void_p(_stream_handle(stream))))

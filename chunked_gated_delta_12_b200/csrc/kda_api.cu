@@ -1,0 +1,137 @@
+// kda_api.cu -- the extern "C" boundary of libkda (declared in include/kda.h).
+//
+// Argument marshalling and validation only: every step of the forward runs in
+// the CUDA kernels.  Checks follow the "first violated condition" convention
+// of fused_kda_unsupported_reason on the kda_fused page of
+// nemo_automodel.components.models.kimi_k3: the first failing check is
+// reported and nothing is launched; there is no fallback.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "../../include/kda.h"
+#include "kda_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+kda_status fail(kda_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+// One status word per device; its device address is looked up once per device.
+__device__ int g_kda_status_word;
+
+constexpr int kMaxDevices = 64;
+int *g_status_ptr[kMaxDevices] = {nullptr};
+std::mutex g_status_mu;
+
+kda_status status_ptr(int dev, int **out) {
+    if (dev < 0 || dev >= kMaxDevices) return fail(KDA_ERR_UNSUPPORTED_DEVICE, "device id %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_kda_status_word);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    *out = g_status_ptr[dev];
+    return KDA_OK;
+}
+
+kda_status check_device(int *dev_out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+        return fail(KDA_ERR_UNSUPPORTED_DEVICE,
+                    "device %d is sm_%d%d; libkda is built for sm_100a (B200) only", dev, major, minor);
+    *dev_out = dev;
+    return KDA_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_last_error(void) { return g_err; }
+
+int kda_abi_version(void) { return 1; }
+
+kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                         const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                         uint16_t *out, void *stream) {
+    g_err[0] = '\0';
+    if (n_docs < 1) return fail(KDA_ERR_INVALID_ARG, "n_docs must be >= 1 (got %d)", n_docs);
+    if (H < 1) return fail(KDA_ERR_INVALID_ARG, "H must be >= 1 (got %d)", H);
+    if (T < 0) return fail(KDA_ERR_INVALID_ARG, "T must be >= 0 (got %lld)", (long long)T);
+    if (T > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "T must fit int32 (cu_seqlens is int32)");
+    if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if (T == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !out) return fail(KDA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) || !aligned(out, 16))
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, g and out must be 16-byte aligned");
+    if (!aligned(beta, 4) || !aligned(cu_seqlens, 4))
+        return fail(KDA_ERR_INVALID_ARG, "beta and cu_seqlens must be 4-byte aligned");
+    const size_t nel = (size_t)T * (size_t)H * KDA_HEAD_DIM;
+    const size_t ob = nel * 2;
+    if (overlaps(out, ob, q, ob) || overlaps(out, ob, k, ob) || overlaps(out, ob, v, ob) ||
+        overlaps(out, ob, g, nel * 4) || overlaps(out, ob, beta, (size_t)T * H * 4))
+        return fail(KDA_ERR_INVALID_ARG, "out must not alias an input");
+    int dev = -1;
+    kda_status s = check_device(&dev);
+    if (s != KDA_OK) return s;
+    int *status = nullptr;
+    s = status_ptr(dev, &status);
+    if (s != KDA_OK) return s;
+    // one CTA per (document, head, value slice): split the value columns in two
+    // when there are too few chains to cover the 148 SMs
+    const int64_t chains = (int64_t)n_docs * H;
+    const int v_slice = chains >= 112 ? 128 : 64;
+    if (chains * (KDA_HEAD_DIM / v_slice) > (int64_t)INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large for one launch");
+    cudaError_t e = kda::launch_fwd_mma(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status, v_slice,
+                                        static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+    return KDA_OK;
+}
+
+kda_status kda_device_status(void *stream) {
+    g_err[0] = '\0';
+    int dev = -1;
+    kda_status s = check_device(&dev);
+    if (s != KDA_OK) return s;
+    int *status = nullptr;
+    s = status_ptr(dev, &status);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int h = 0;
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(status, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "device status read: %s", cudaGetErrorString(e));
+    if (h == kda::kStatusBadSeqlens) return fail(KDA_ERR_BAD_SEQLENS, "cu_seqlens malformed (seen on device)");
+    if (h == kda::kStatusTimeout) return fail(KDA_ERR_TIMEOUT, "a device-side wait timed out");
+    return KDA_OK;
+}
+
+}  // extern "C"

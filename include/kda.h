@@ -1,0 +1,97 @@
+/*
+ * kda.h -- C ABI of libkda, the B200 (sm_100a) chunk-KDA forward.
+ *
+ * Kimi Delta Attention (KDA) is the gated delta rule with a per-key-channel
+ * decay.  Per document and head, with the 128 x 128 fp32 state S starting at 0:
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = scale * S_t^T q_t,          scale = 1/sqrt(128)
+ *
+ * with q_t and k_t l2-normalised inside the op (q / sqrt(|q|^2 + 1e-6)).
+ *
+ * Scope follows the fused-kernel contract of the kda_fused page of
+ * nemo_automodel.components.models.kimi_k3 (module description and
+ * fused_chunk_kda): head dims K = V = 128, packed layout (batch 1, int32
+ * cu_seqlens; a dense batch of B equal-length sequences is passed as B packed
+ * documents with cu_seqlens = [0, L, 2L, ..., BL]), q/k l2-normalised inside
+ * the kernel, a bounded log gate, no initial or final state, no context
+ * parallelism, chunk mode only.  Like fused_kda_unsupported_reason on that
+ * page, every call that falls outside this scope is rejected with the first
+ * violated condition (kda_last_error); there is no fallback path of any kind.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,        /* bad pointer, size or alignment (see kda_last_error) */
+    KDA_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not sm_100 (B200-class)          */
+    KDA_ERR_CUDA = 3,               /* a CUDA runtime call or launch failed               */
+    KDA_ERR_NO_MEMORY = 4,          /* reserved: libkda allocates no device memory        */
+    KDA_ERR_TIMEOUT = 5,            /* a device-side bounded wait gave up                 */
+    KDA_ERR_BAD_SEQLENS = 6         /* cu_seqlens content found malformed on the device   */
+} kda_status;
+
+/* Head dimension the kernels are specialised to (K = V). */
+#define KDA_HEAD_DIM 128
+
+/*
+ * kda_chunk_fwd -- chunked KDA forward, o = KDA(q, k, v, g, beta) per document.
+ *
+ * Operation: the recurrence in the header comment, evaluated chunk-wise
+ * (64-token chunks starting at each document start) in the exact UT/WY
+ * algebra; output equal to the token recurrence up to rounding.  This is
+ * fused_chunk_kda(q, k, v, g, beta, cu_seqlens) of the kda_fused page, whose
+ * return convention is (o, None): no final state.
+ *
+ * Arguments (all arrays DEVICE memory, C-contiguous, 16-byte aligned):
+ *   q, k, v    [T, H, 128] bf16 (uint16 bit patterns), token-major, then head, then channel
+ *   g          [T, H, 128] fp32 per-key-channel log decay; precondition -5 <= g <= 0
+ *              (the bounded gate; values outside are not checked and may lose accuracy)
+ *   beta       [T, H] fp32 write strength, expected in [0, 1]
+ *   cu_seqlens [n_docs + 1] int32, cu[0] = 0, non-decreasing, cu[n_docs] = T;
+ *              zero-length documents are allowed and produce nothing
+ *   n_docs     >= 1
+ *   T          total tokens (>= 0); T = 0 returns KDA_OK without launching
+ *   H          heads (>= 1); q, k and v share H (no grouped heads)
+ *   out        [T, H, 128] bf16 (uint16), written for every token in [0, T); must not
+ *              alias any input
+ *   stream     cudaStream_t (NULL = legacy default stream); the call is asynchronous
+ *
+ * Ownership: the caller owns every buffer; libkda keeps no pointer after the
+ * enqueued work and allocates no device memory.
+ *
+ * Errors: argument and device checks return KDA_ERR_INVALID_ARG /
+ * KDA_ERR_UNSUPPORTED_DEVICE with a message in kda_last_error() and launch
+ * nothing.  A malformed cu_seqlens table cannot be seen from the host without
+ * a sync; the kernel detects it, skips the affected documents and records
+ * KDA_ERR_BAD_SEQLENS, which kda_device_status() reports.
+ */
+kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const float *g, const float *beta, const int32_t *cu_seqlens,
+                         int n_docs, int64_t T, int H, uint16_t *out, void *stream);
+
+/* Thread-local description of the first violated condition of the last failing call. */
+const char *kda_last_error(void);
+
+/*
+ * kda_device_status -- synchronise `stream`, then return and clear the
+ * device-side status word of the current device (KDA_OK, KDA_ERR_BAD_SEQLENS or
+ * KDA_ERR_TIMEOUT), or KDA_ERR_CUDA if the synchronisation itself failed.
+ */
+kda_status kda_device_status(void *stream);
+
+/* ABI version of this header (bumped on any signature change). */
+int kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

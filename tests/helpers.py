@@ -1,0 +1,56 @@
+"""Shared test helpers: workload -> device tensors, oracle comparison."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from chunked_gated_delta_12_b200.inputs import bf16_bits_to_f32
+
+RTOL_L2 = 1e-2      # relative L2 error bound on bf16 outputs
+ATOL_MAX = 5e-2     # max absolute error bound on bf16 outputs
+
+
+def to_device(d: dict):
+    import torch
+    dev = torch.device("cuda")
+    t = {}
+    for key in ("q", "k", "v"):
+        t[key] = torch.from_numpy(np.ascontiguousarray(d[key]).view(np.int16)).view(torch.bfloat16).to(dev)
+    t["g"] = torch.from_numpy(np.ascontiguousarray(d["g"])).to(dev)
+    t["beta"] = torch.from_numpy(np.ascontiguousarray(d["beta"])).to(dev)
+    t["cu_seqlens"] = torch.from_numpy(np.ascontiguousarray(d["cu_seqlens"], dtype=np.int32)).to(dev)
+    return t
+
+
+def out_to_f64(o) -> np.ndarray:
+    import torch
+    bits = o.view(torch.int16).cpu().numpy().view(np.uint16)
+    return bf16_bits_to_f32(bits).reshape(bits.shape).astype(np.float64)
+
+
+def oracle_out(d: dict, chains=None, **kw) -> np.ndarray:
+    f = lambda key: bf16_bits_to_f32(d[key]).reshape(d[key].shape)
+    return oracle.kda_fwd(f("q"), f("k"), f("v"), d["g"], d["beta"], d["cu_seqlens"], chains=chains, **kw)
+
+
+def chain_slices(cu, H, chains):
+    for ch in chains:
+        doc, h = divmod(int(ch), H)
+        yield int(cu[doc]), int(cu[doc + 1]), h
+
+
+def compare(got: np.ndarray, ref: np.ndarray, cu, H, chains=None) -> tuple[float, float]:
+    """rel-L2 and max-abs error over the rows of `chains` (all chains if None)."""
+    if chains is None:
+        chains = range((len(cu) - 1) * H)
+    num = den = 0.0
+    mx = 0.0
+    for s, e, h in chain_slices(cu, H, chains):
+        if e == s:
+            continue
+        a, b = got[s:e, h], ref[s:e, h]
+        assert np.isfinite(a).all(), "non-finite output"
+        num += float(((a - b) ** 2).sum())
+        den += float((b ** 2).sum())
+        mx = max(mx, float(np.abs(a - b).max()))
+    return (num ** 0.5) / max(den ** 0.5, 1e-300), mx

@@ -1,0 +1,70 @@
+"""libkda loads, exports every entry point include/kda.h declares, and rejects
+bad arguments on the host before touching a device.  CPU only."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunked_gated_delta_12_b200 import _lib
+from chunked_gated_delta_12_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "kda_chunk_fwd" in names and "kda_last_error" in names
+    for n in names:
+        assert hasattr(L, n), f"libkda.so does not export {n}"
+
+
+def test_abi_version(L):
+    assert L.kda_abi_version() == 1
+
+
+FAKE = 0x10000000  # never dereferenced: every case below fails a host-side check first
+
+
+def call(L, q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, n_docs=1, T=64, H=1, out=FAKE + (1 << 30)):
+    vp = ctypes.c_void_p
+    return L.kda_chunk_fwd(vp(q), vp(k), vp(v), vp(g), vp(beta), vp(cu), n_docs, T, H, vp(out), None)
+
+
+def test_rejects_bad_sizes(L):
+    assert call(L, n_docs=0) == 1 and b"n_docs" in L.kda_last_error()
+    assert call(L, H=0) == 1 and b"H must" in L.kda_last_error()
+    assert call(L, T=-1) == 1
+    assert call(L, cu=0) == 1 and b"cu_seqlens" in L.kda_last_error()
+
+
+def test_empty_is_noop(L):
+    assert call(L, T=0) == 0
+
+
+def test_rejects_null_misaligned_and_aliasing(L):
+    assert call(L, q=0) == 1 and b"NULL" in L.kda_last_error()
+    assert call(L, k=FAKE + 8) == 1 and b"aligned" in L.kda_last_error()
+    assert call(L, beta=FAKE + 2) == 1
+    assert call(L, out=FAKE) == 1 and b"alias" in L.kda_last_error()
+
+
+def test_no_device_is_an_error_not_a_fallback(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc = call(L)
+    assert rc in (2, 3), rc            # UNSUPPORTED_DEVICE or CUDA error, never OK
+    assert L.kda_last_error()
