@@ -180,11 +180,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="DOCSxLEN:H -- a custom dense workload with the same distributions "
+                         "(e.g. 4x2048:32 for a profiling case larger than L2)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
-    from chunked_gated_delta_12_b200.inputs import generate, workload
-    w = workload(args.workload)
+    from chunked_gated_delta_12_b200.inputs import custom_workload, generate, workload
+    if args.shape:
+        docs_len, heads = args.shape.split(":")
+        n_docs, doc_len = (int(x) for x in docs_len.split("x"))
+        w = custom_workload(f"dense_{n_docs}x{doc_len}_H{heads}", [doc_len] * n_docs, int(heads), seed=20262)
+    else:
+        w = workload(args.workload)
 
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
@@ -252,14 +261,14 @@ def main():
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.e2e_steps):
+    for _ in range(0 if args.no_e2e else args.e2e_steps):
         for key in host:
             dv[key].copy_(host[key], non_blocking=True)
         step()
         host_out.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps) if not args.no_e2e else float("nan")
     if world > 1:
         import torch.distributed as dist
         t = torch.tensor([e2e_ms], device=dev)
