@@ -108,8 +108,11 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
     const int v_slice = chains >= 112 ? 128 : 64;
     if (chains * (KDA_HEAD_DIM / v_slice) > (int64_t)INT32_MAX)
         return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large for one launch");
-    cudaError_t e = kda::launch_fwd_tc(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status, v_slice,
-                                        static_cast<cudaStream_t>(stream));
+    cudaError_t e = v_slice == 128
+                        ? kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status,
+                                               static_cast<cudaStream_t>(stream))
+                        : kda::launch_fwd_tc(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status, v_slice,
+                                             static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return KDA_OK;
 }

@@ -133,10 +133,12 @@ __device__ __forceinline__ void mbar_init(uint32_t saddr, uint32_t count) {
 }
 __device__ __forceinline__ bool mbar_try(uint32_t saddr, uint32_t parity) {
     uint32_t ok;
+    // the suspend-time hint (ns) lets the hardware park the thread until the phase
+    // completes instead of spinning through the issue slots
     asm volatile(
-        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\nselp.b32 %0, 1, 0, P;\n}\n"
+        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\nselp.b32 %0, 1, 0, P;\n}\n"
         : "=r"(ok)
-        : "r"(saddr), "r"(parity)
+        : "r"(saddr), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
