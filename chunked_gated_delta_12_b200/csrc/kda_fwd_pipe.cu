@@ -3,12 +3,12 @@
 //
 // Two chunks are in flight per CTA.  In step s all 16 warps first prepare chunk
 // s; then warps 0-11 finish chunk s's intra-chunk work while warps 12-15 run
-// chunk s-1's state update on the tensor cores.  The state is kept transposed,
-// S^T[v][c] in fp32 in tensor memory (lane = value column v), so that both the
-// bf16 copy of the state and the corrected values U~ are tcgen05 A operands
-// read straight from TMEM -- no shared-memory round trip on the state chain.
+// chunk s-1's state update on the tensor cores and the row norms of chunk s+1.
+// The state is kept transposed, S^T[v][c] in fp32 in tensor memory (lane =
+// value column v), so that both the bf16 copy of the state and the corrected
+// values U~ are tcgen05 A operands read straight from TMEM.
 //
-// Per chunk (rows r, i; Gamma = in-chunk cumsum of g; scale-free notation):
+// Per chunk (rows r, i; Gamma = in-chunk cumsum of g):
 //   A_kk[r,i] = beta_r k^_r.(k^_i e^{Gamma_r - Gamma_i}) (i < r),  A_qk (i <= r)
 //   T' = (I + A_kk)^-1 diag(beta)
 //   W  = T' K^e^Gamma,  U = T' V,  Q' = Q^e^Gamma - A_qk W,  U' = A_qk U
@@ -19,11 +19,17 @@
 //          D    = V^T [T'; A_qk T']^T                              -> [U^T | U'^T]
 //   state  D   += S^T_bf16 (TMEM) B2                               -> [U~^T | O^T]
 //          S^T += U~^T_bf16 (TMEM) Kd                               (after S^T <- S^T Diag(e^{Gamma_last}))
-// The gate exponent is split at 16-row sub-block boundaries exactly as in the
-// non-pipelined kernel (kda_fwd_tc.cu).  Every tensor-core wait is
-// time-limited and reports KDA_ERR_TIMEOUT.
+// q, k, g and v tiles arrive by TMA (2-D tensor maps over [T, H*128], no
+// multicast); rows past the document end are masked with selects (and v rows
+// zeroed) because a tile may reach into the next document.  The gate exponent
+// is split at 16-row sub-block boundaries exactly as in kda_fwd_tc.cu.  Every
+// wait is time-limited and reports KDA_ERR_TIMEOUT.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
+
+#include <mutex>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -33,7 +39,6 @@ namespace kda {
 namespace pipe_path {
 
 constexpr int kThreads = 512;
-constexpr int kIntraThreads = 384;            // warps 0-11
 constexpr int kStateTid0 = 384;               // first thread of warps 12-15
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSF = 0;                   // S^T fp32          [128 lanes v][128 cols c]
@@ -47,10 +52,10 @@ constexpr int kBlkPitch = 20;
 constexpr int kBlkFloats = 16 * kBlkPitch;
 
 struct Smem {
-    static constexpr int Q = 0;            // raw q [64][128] bf16 (pitch 256) -> q^E1 [c][r] SW128
-    static constexpr int K = 16384;        // raw k                             -> k^E1 [c][r] SW128
-    static constexpr int G = 32768;        // raw g [64][128] fp32 (pitch 512)
-    static constexpr int V = 65536;        // raw v, MN-major SW128 (64 K-rows, two 64-wide atoms)
+    static constexpr int Q = 0;            // raw q: two TMA boxes [64 rows][64 ch] (128 B rows) -> q^E1 [c][r] SW128
+    static constexpr int K = 16384;        // raw k                                                -> k^E1 [c][r] SW128
+    static constexpr int G = 32768;        // raw g: four TMA boxes [64 rows][32 ch] fp32
+    static constexpr int V = 65536;        // raw v: two TMA boxes, 128B-swizzled = MN-major SW128 atoms
     static constexpr int KR = 81920;       // k^E2 [c][r] SW128 -> A1 = [T'; A_qk T'] (K-major, 128 rows)
     static constexpr int KGT = 98304;      // (k^ e^Gamma)^T, K-major [c][r]
     static constexpr int KDT = 114688;     // two buffers: (k^ e^{Gamma_last-Gamma})^T, K-major [c][r]
@@ -66,29 +71,27 @@ struct Smem {
     static constexpr int PS = TOT + 2048;            // fp32 [10][128]
     static constexpr int DC = PS + 5120;             // fp32 [2][128]
     static constexpr int XT = DC + 1024;             // fp32 [6][16][8]
-    static constexpr int MBAR = XT + 3072;           // u64 [4]
-    static constexpr int TBASE = MBAR + 32;
+    static constexpr int MBAR = XT + 3072;           // u64 [8]
+    static constexpr int TBASE = MBAR + 64;
     static constexpr int ABORT = TBASE + 16;
     static constexpr int BYTES = ABORT + 16;
     static constexpr int ALLOC = BYTES + 1024;
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
 
+enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV };
+
 __device__ __forceinline__ void bar_intra() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void bar_state() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
+// tf32 warp MMA on fp32 bit patterns (the tensor core ignores the low mantissa bits)
+__device__ __forceinline__ void mma_tf32(float (&d)[4], float a0, float a1, float a2, float a3, float b0, float b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        : "r"(__float_as_uint(a0)), "r"(__float_as_uint(a1)), "r"(__float_as_uint(a2)), "r"(__float_as_uint(a3)),
+          "r"(__float_as_uint(b0)), "r"(__float_as_uint(b1)));
 }
 // tcgen05.mma with A in TMEM
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -118,24 +121,8 @@ __device__ __forceinline__ uint4 pack8(const float *x, float s) {
 __device__ __forceinline__ int pair_R(int p) { return p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0; }
 __device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
 
-__device__ __forceinline__ void load_qk(uint8_t *sm, const uint16_t *q, const uint16_t *k, int64_t tok0, int L,
-                                        int H, int h, int t0, int nthr) {
-    for (int idx = t0; idx < 64 * 16; idx += nthr) {
-        const int row = idx >> 4, ch = idx & 15;
-        const bool ok = row < L;
-        const int64_t off = ok ? ((tok0 + row) * H + h) * kHeadDim + ch * 8 : 0;
-        cp_async16(smem_u32(sm + Smem::Q + row * 256 + ch * 16), q + off, ok ? 16 : 0);
-        cp_async16(smem_u32(sm + Smem::K + row * 256 + ch * 16), k + off, ok ? 16 : 0);
-    }
-}
-__device__ __forceinline__ void load_gb(uint8_t *sm, const float *g, const float *beta, int64_t tok0, int L, int H,
-                                        int h, int buf) {
-    for (int idx = threadIdx.x; idx < 64 * 32; idx += kThreads) {
-        const int row = idx >> 5, ch = idx & 31;
-        const bool ok = row < L;
-        const int64_t off = ok ? ((tok0 + row) * H + h) * kHeadDim + ch * 4 : 0;
-        cp_async16(smem_u32(sm + Smem::G + row * 512 + ch * 16), g + off, ok ? 16 : 0);
-    }
+// beta rows [tok0, tok0 + L) of head h (threads 0-63; rows >= L zero-filled)
+__device__ __forceinline__ void load_beta(uint8_t *sm, const float *beta, int64_t tok0, int L, int H, int h, int buf) {
     if (threadIdx.x < 64) {
         const int row = threadIdx.x;
         const bool ok = row < L;
@@ -146,21 +133,15 @@ __device__ __forceinline__ void load_gb(uint8_t *sm, const float *g, const float
                      : "memory");
     }
 }
-__device__ __forceinline__ void load_v(uint8_t *sm, const uint16_t *v, int64_t tok0, int L, int H, int h, int t0,
-                                       int nthr) {
-    for (int idx = t0; idx < 64 * 16; idx += nthr) {
-        const int row = idx >> 4, ch = idx & 15;
-        const bool ok = row < L;
-        const int64_t off = ok ? ((tok0 + row) * H + h) * kHeadDim + ch * 8 : 0;
-        cp_async16(smem_u32(sm + Smem::V) + tc::mnmaj_chunk(ch, row, 64), v + off, ok ? 16 : 0);
-    }
-}
+
+struct Maps {
+    CUtensorMap q, k, g, v;
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
-    kda_fwd_pipe_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
-                        const uint16_t *__restrict__ v, const float *__restrict__ g,
-                        const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int n_docs,
-                        int64_t T, int H, uint16_t *__restrict__ out, int *__restrict__ status) {
+    kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
+                        const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
+                        uint16_t *__restrict__ out, int *__restrict__ status) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
@@ -179,6 +160,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (doc_end == doc_start) return;
     const int nchunks = (int)((doc_end - doc_start + 63) / 64);
+    auto chunk_len = [&](int i) -> int {
+        const int64_t rem = doc_end - (doc_start + 64 * (int64_t)i);
+        return rem <= 0 ? 0 : (rem < 64 ? (int)rem : 64);
+    };
 
     float *f_rq = reinterpret_cast<float *>(sm + S::RQ);
     float *f_rk = reinterpret_cast<float *>(sm + S::RK);
@@ -187,32 +172,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *f_akk = reinterpret_cast<float *>(sm + S::AKK);
     float *f_tm = reinterpret_cast<float *>(sm + S::TM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::ABORT);
-    const uint32_t mbar_wq = smem_u32(sm + S::MBAR), mbar_u = mbar_wq + 8, mbar_2 = mbar_wq + 16,
-                   mbar_4 = mbar_wq + 24;
+    const uint32_t mb = smem_u32(sm + S::MBAR);
+    auto mbar = [&](int i) -> uint32_t { return mb + 8u * (uint32_t)i; };
     const uint32_t sbase = smem_u32(sm);
+    const int xq = h * kHeadDim;          // TMA x coordinate of this head's channel 0
+
+    auto issue_qk = [&](int i) {          // q, k tiles of chunk i (one thread)
+        const int y = (int)(doc_start + 64 * (int64_t)i);
+        tc::mbar_expect_tx(mbar(kMbQK), 32768u);
+        tc::tma_load_2d(sbase + S::Q, &maps.q, xq, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::Q + 8192, &maps.q, xq + 64, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::K, &maps.k, xq, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::K + 8192, &maps.k, xq + 64, y, mbar(kMbQK));
+    };
+    auto issue_g = [&](int i) {
+        const int y = (int)(doc_start + 64 * (int64_t)i);
+        tc::mbar_expect_tx(mbar(kMbG), 32768u);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tc::tma_load_2d(sbase + S::G + 8192 * b, &maps.g, xq + 32 * b, y, mbar(kMbG));
+    };
+    auto issue_v = [&](int i) {
+        const int y = (int)(doc_start + 64 * (int64_t)i);
+        tc::mbar_expect_tx(mbar(kMbV), 16384u);
+        tc::tma_load_2d(sbase + S::V, &maps.v, xq, y, mbar(kMbV));
+        tc::tma_load_2d(sbase + S::V + 8192, &maps.v, xq + 64, y, mbar(kMbV));
+    };
+    // 1/|q_r| and 1/|k_r| for rows r0..r0+15 of the raw tiles (rows >= Li count as zero).
+    // Each lane sums its 4 channels for all 32 (tensor, row) pairs, then a transposed
+    // butterfly (31 shuffles) leaves lane l with the total of pair l.
+    auto norms16 = [&](int r0, int Li) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = r0 + i;
+            const uint32_t off = (lane >> 4) * 8192 + r * 128 + (lane & 15) * 8;
+            uint2 qa = *reinterpret_cast<const uint2 *>(sm + S::Q + off);
+            uint2 ka = *reinterpret_cast<const uint2 *>(sm + S::K + off);
+            if (r >= Li) qa = ka = make_uint2(0u, 0u);
+            const float2 q01 = unpack_bf16(qa.x), q23 = unpack_bf16(qa.y);
+            const float2 k01 = unpack_bf16(ka.x), k23 = unpack_bf16(ka.y);
+            v[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
+            v[16 + i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+        }
+#pragma unroll
+        for (int lv = 0; lv < 5; ++lv) {
+            const int o = 16 >> lv, half = 16 >> lv;
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int j = 0; j < half; ++j) {
+                const float send = up ? v[j] : v[j + half];
+                const float keep = up ? v[j + half] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        float *dst = lane < 16 ? f_rq : f_rk;
+        dst[r0 + (lane & 15)] = rsqrtf(v[0] + 1e-6f);
+    };
 
     // ---- setup ----
     if (warp == 0) tc::alloc(smem_u32(sm + S::TBASE), kTmemCols);
     if (tid == 0) {
-        tc::mbar_init(mbar_wq, 1);
-        tc::mbar_init(mbar_u, 1);
-        tc::mbar_init(mbar_2, 1);
-        tc::mbar_init(mbar_4, 1);
+        for (int i = 0; i < 7; ++i) tc::mbar_init(mbar(i), 1);
         *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    {
-        const int L0 = (int)(doc_end - doc_start < 64 ? doc_end - doc_start : 64);
-        load_qk(sm, q, k, doc_start, L0, H, h, tid, kThreads);
-        load_gb(sm, g, beta, doc_start, L0, H, h, 0);
-        cp_async_commit();
+    __syncthreads();
+    if (tid == 0) {
+        issue_qk(0);
+        issue_g(0);
     }
+    load_beta(sm, beta, doc_start, chunk_len(0), H, h, 0);
+    cp_async_commit();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + S::TBASE);
     const int lq = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * lq) << 16);
-    if (warp >= 12) {   // S^T = 0
+    if (warp >= 12) {
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.f;
@@ -220,95 +257,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c0 = 0; c0 < 128; c0 += 32) tc::st32(lane_base + kSF + c0, z);
         tc::wait_st();
     }
+    // norms of chunk 0
+    if (!tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit)) *abort_flag = 1;
+    if (warp < 4) norms16(warp * 16, chunk_len(0));
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
 
-    bool aborted = false;
+    bool aborted = *abort_flag != 0;
     const float out_scale = rsqrtf((float)kHeadDim);
 
-    for (int s = 0; s <= nchunks; ++s) {
+    for (int s = 0; s <= nchunks && !aborted; ++s) {
         const bool have_intra = s < nchunks;        // chunk s: prep + intra
         const bool have_state = s >= 1;             // chunk s-1: state update + output
-        const int64_t tok0 = doc_start + 64 * (int64_t)s;
-        const int L = have_intra ? (int)(doc_end - tok0 < 64 ? doc_end - tok0 : 64) : 0;
-        const int64_t ntok0 = tok0 + 64;
-        const int nL = (int)(doc_end - ntok0 < 64 ? doc_end - ntok0 : 64);    // <= 0: no chunk s+1
+        const bool have_next = s + 1 < nchunks;     // chunk s+1 exists
+        const int L = chunk_len(s);
+        const int nL = chunk_len(s + 1);
         const int buf = s & 1;
+        const uint32_t par = (uint32_t)(s & 1);
 
-        // ---- top: raw(s) landed; the previous step's U product is done (V, KR free) ----
+        // ---- top: beta(s) landed; the previous step's U product is done (V, KR free) ----
         cp_async_wait_all();
         if (have_state) {
-            if (!tc::mbar_wait(mbar_u, (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
+            if (!tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
         }
         tc::fence_before();
         __syncthreads();
         tc::fence_after();
         if (*abort_flag) { aborted = true; break; }
-        // v(s) for this step's U product (intra warps; waited on before that product)
-        if (tid < kIntraThreads) {
-            if (have_intra) load_v(sm, v, tok0, L, H, h, tid, kIntraThreads);
-            cp_async_commit();
+        if (tid == 0 && have_intra) {
+            tc::fence_proxy_async();
+            issue_v(s);
         }
 
         float ql[16], kl[16], kr[16];
-        float lg0 = 0.f;
+        float lg0 = 0.f, lg15 = 0.f;
         const int pc = tid & 127, pR = tid >> 7;
         if (have_intra) {
-            // ---- norms: warp w handles rows 4w..4w+3 ----
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = warp * 4 + i;
-                const uint2 qa = *reinterpret_cast<const uint2 *>(sm + S::Q + r * 256 + lane * 8);
-                const uint2 ka = *reinterpret_cast<const uint2 *>(sm + S::K + r * 256 + lane * 8);
-                const float2 q01 = unpack_bf16(qa.x), q23 = unpack_bf16(qa.y);
-                const float2 k01 = unpack_bf16(ka.x), k23 = unpack_bf16(ka.y);
-                float sq = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
-                float sk = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
-                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                }
-                if (lane == 0) {
-                    f_rq[r] = rsqrtf(sq + 1e-6f);
-                    f_rk[r] = rsqrtf(sk + 1e-6f);
-                }
-            }
-        }
-        __syncthreads();
-        float lg15 = 0.f;
-        if (have_intra) {
             // ---- prep pass 1: thread = (channel c, row block R) ----
+            bool ok = tc::mbar_wait(mbar(kMbQK), par, kWaitLimit);
+            ok = tc::mbar_wait(mbar(kMbG), par, kWaitLimit) && ok;
+            if (!ok) *abort_flag = 1;
             float lg[16];
             float acc = 0.f;
+            const uint8_t *gcol = sm + S::G + (pc >> 5) * 8192 + (pc & 31) * 4;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                acc += *reinterpret_cast<const float *>(sm + S::G + (16 * pR + j) * 512 + pc * 4);
+                const int r = 16 * pR + j;
+                const float gv = *reinterpret_cast<const float *>(gcol + r * 128);
+                acc += r < L ? gv * kLog2e : 0.f;         // log2-scaled gate cumsum
                 lg[j] = acc;
             }
             lg0 = lg[0];
             lg15 = lg[15];
             f_tot[pR * 128 + pc] = lg15;
+            const uint8_t *qcol = sm + S::Q + (pc >> 6) * 8192 + (pc & 63) * 2;
+            const uint8_t *kcol = sm + S::K + (pc >> 6) * 8192 + (pc & 63) * 2;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int r = 16 * pR + j;
-                const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + S::Q + r * 256 + pc * 2));
-                const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + S::K + r * 256 + pc * 2));
-                const float qh = qv * f_rq[r], kh = kv * f_rk[r];
-                const float e1 = fast_exp2((lg[j] - lg0) * kLog2e);
-                const float e2 = fast_exp2((lg15 - lg[j]) * kLog2e);
-                ql[j] = qh * e1;
-                kl[j] = kh * e1;
-                kr[j] = kh * e2;
+            for (int j4 = 0; j4 < 16; j4 += 4) {
+                const float4 rq4 = *reinterpret_cast<const float4 *>(f_rq + 16 * pR + j4);
+                const float4 rk4 = *reinterpret_cast<const float4 *>(f_rk + 16 * pR + j4);
+                const float rqv[4] = {rq4.x, rq4.y, rq4.z, rq4.w};
+                const float rkv[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = j4 + jj, r = 16 * pR + j;
+                    float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qcol + r * 128));
+                    float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kcol + r * 128));
+                    qv = r < L ? qv : 0.f;
+                    kv = r < L ? kv : 0.f;
+                    const float e1 = fast_exp2(lg[j] - lg0);
+                    const float e2 = fast_exp2(lg15 - lg[j]);
+                    const float qh = qv * rqv[jj], kh = kv * rkv[jj];
+                    ql[j] = qh * e1;
+                    kl[j] = kh * e1;
+                    kr[j] = kh * e2;
+                }
             }
         }
         __syncthreads();   // raw q, k, g read; block sums published
-        // raw g is dead: the next chunk's g and beta
-        if (nL > 0) load_gb(sm, g, beta, ntok0, nL, H, h, buf ^ 1);
+        // raw g, beta(s+1) buffer are free: the next chunk's g and beta
+        if (tid == 0 && have_next) {
+            tc::fence_proxy_async();
+            issue_g(s + 1);
+        }
+        if (have_next) load_beta(sm, beta, doc_start + 64 * (int64_t)(s + 1), nL, H, h, buf ^ 1);
         cp_async_commit();
         if (have_intra) {
-            // ---- prep pass 2 ----
+            // ---- prep pass 2 (log2-scaled Gamma) ----
             float offs[5];
             offs[0] = 0.f;
 #pragma unroll
@@ -316,12 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float gm = offs[pR] + lg0;
             const float ge = offs[pR + 1];
             const float gl = offs[4];
-            const float P = fast_exp2(gm * kLog2e);
-            const float Dk = fast_exp2((gl - ge) * kLog2e);
+            const float P = fast_exp2(gm);
+            const float Dk = fast_exp2(gl - ge);
 #pragma unroll
             for (int I = 0; I < 4; ++I)
-                if (I <= pR) f_ps[pair_of(pR, I) * 128 + pc] = fast_exp2((gm - offs[I + 1]) * kLog2e);
-            if (pR == 0) reinterpret_cast<float *>(sm + S::DC)[buf * 128 + pc] = fast_exp2(gl * kLog2e);
+                if (I <= pR) f_ps[pair_of(pR, I) * 128 + pc] = fast_exp2(gm - offs[I + 1]);
+            if (pR == 0) reinterpret_cast<float *>(sm + S::DC)[buf * 128 + pc] = fast_exp2(gl);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int j0 = half * 8;
@@ -415,37 +451,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                             make_uint4(0, 0, 0, 0);
                     }
                 }
-            }
-            bar_intra();
-            // q^E1 / k^E1 consumed: the next chunk's raw q, k
-            if (nL > 0) load_qk(sm, q, k, ntok0, nL, H, h, tid, kIntraThreads);
-            cp_async_commit();
-            if (have_intra) {
-                const float *f_beta = reinterpret_cast<const float *>(sm + S::BETA + buf * 256);
-                // ---- T = (I + A_kk)^-1: diagonal blocks, one column per lane ----
-                if (warp < 4 && lane < 16) {
-                    const int R = warp, col = lane;
-                    const float *blk = f_akk + pair_of(R, R) * kBlkFloats;
-                    float x[16];
+                bar_intra();
+                // q^E1 / k^E1 consumed: the next chunk's raw q, k
+                if (tid == 0 && have_next) {
+                    tc::fence_proxy_async();
+                    issue_qk(s + 1);
+                }
+                // ---- T = (I + A_kk)^-1: diagonal blocks (one column per lane); T' rows written as bf16 ----
+                if (warp < 4) {
+                    if (lane < 16) {
+                        const int R = warp, col = lane;
+                        const float *blk = f_akk + pair_of(R, R) * kBlkFloats;
+                        // right-looking forward substitution: x[j] is final once the updates of
+                        // rows < j have been applied; the serial chain is one FMA per row
+                        float x[16];
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float a[16];
+                        for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 t4 = *reinterpret_cast<const float4 *>(blk + r * kBlkPitch + 4 * q4);
-                            a[4 * q4] = t4.x; a[4 * q4 + 1] = t4.y; a[4 * q4 + 2] = t4.z; a[4 * q4 + 3] = t4.w;
+                        for (int j = 0; j < 15; ++j) {
+#pragma unroll
+                            for (int r = j + 1; r < 16; ++r) x[r] -= blk[r * kBlkPitch + j] * x[j];
                         }
-                        float acc = (r == col) ? 1.f : 0.f;
+                        float *tb = f_tm + pair_of(R, R) * kBlkFloats;
+                        const float bc = f_beta[16 * R + col];
 #pragma unroll
-                        for (int jj = 0; jj < r; ++jj) acc -= a[jj] * x[jj];
-                        x[r] = acc;
+                        for (int r = 0; r < 16; ++r) {
+                            tb[r * kBlkPitch + col] = x[r];
+                            const __nv_bfloat16 t1 = __float2bfloat16_rn(x[r] * bc);
+                            *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
+                        }
                     }
-                    float *tb = f_tm + pair_of(R, R) * kBlkFloats;
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) tb[r * kBlkPitch + col] = x[r];
+                } else {
+                    // T' is zero above the block diagonal (warps 4-11)
+                    const int t = tid - 128;
+                    for (int idx = t; idx < 192; idx += 256) {
+                        const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
+                        const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
+                        const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
+                        *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                            make_uint4(0, 0, 0, 0);
+                    }
                 }
                 bar_intra();
-                // ---- off-diagonal blocks by distance d ----
+                // ---- off-diagonal blocks by distance d (tf32 warp MMA), T and T' stored ----
 #pragma unroll 1
                 for (int d = 1; d < 4; ++d) {
                     const int njobs = 2 * (4 - d);
@@ -456,15 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float *ab = f_akk + pair_of(R, J) * kBlkFloats;
                             const float *tb = f_tm + pair_of(J, I) * kBlkFloats;
 #pragma unroll
-                            for (int kb = 0; kb < 16; kb += 8) {
-                                const uint32_t a0 = tf32(ab[gq * kBlkPitch + kb + tq]);
-                                const uint32_t a1 = tf32(ab[(gq + 8) * kBlkPitch + kb + tq]);
-                                const uint32_t a2 = tf32(ab[gq * kBlkPitch + kb + tq + 4]);
-                                const uint32_t a3 = tf32(ab[(gq + 8) * kBlkPitch + kb + tq + 4]);
-                                const uint32_t b0 = tf32(tb[(kb + tq) * kBlkPitch + 8 * nt + gq]);
-                                const uint32_t b1 = tf32(tb[(kb + tq + 4) * kBlkPitch + 8 * nt + gq]);
-                                mma_tf32(xacc, a0, a1, a2, a3, b0, b1);
-                            }
+                            for (int kb = 0; kb < 16; kb += 8)
+                                mma_tf32(xacc, ab[gq * kBlkPitch + kb + tq], ab[(gq + 8) * kBlkPitch + kb + tq],
+                                         ab[gq * kBlkPitch + kb + tq + 4], ab[(gq + 8) * kBlkPitch + kb + tq + 4],
+                                         tb[(kb + tq) * kBlkPitch + 8 * nt + gq], tb[(kb + tq + 4) * kBlkPitch + 8 * nt + gq]);
                         }
                         float *xt = reinterpret_cast<float *>(sm + S::XT) + warp * 128;   // X[16][8]
                         xt[gq * 8 + 2 * tq] = xacc[0];
@@ -475,42 +518,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float *tr = f_tm + pair_of(R, R) * kBlkFloats;
                         float tacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int kb = 0; kb < 16; kb += 8) {
-                            const uint32_t a0 = tf32(tr[gq * kBlkPitch + kb + tq]);
-                            const uint32_t a1 = tf32(tr[(gq + 8) * kBlkPitch + kb + tq]);
-                            const uint32_t a2 = tf32(tr[gq * kBlkPitch + kb + tq + 4]);
-                            const uint32_t a3 = tf32(tr[(gq + 8) * kBlkPitch + kb + tq + 4]);
-                            const uint32_t b0 = tf32(xt[(kb + tq) * 8 + gq]);
-                            const uint32_t b1 = tf32(xt[(kb + tq + 4) * 8 + gq]);
-                            mma_tf32(tacc, a0, a1, a2, a3, b0, b1);
-                        }
+                        for (int kb = 0; kb < 16; kb += 8)
+                            mma_tf32(tacc, tr[gq * kBlkPitch + kb + tq], tr[(gq + 8) * kBlkPitch + kb + tq],
+                                     tr[gq * kBlkPitch + kb + tq + 4], tr[(gq + 8) * kBlkPitch + kb + tq + 4],
+                                     xt[(kb + tq) * 8 + gq], xt[(kb + tq + 4) * 8 + gq]);
                         float *to = f_tm + pair_of(R, I) * kBlkFloats;
-                        *reinterpret_cast<float2 *>(to + gq * kBlkPitch + 8 * nt + 2 * tq) = make_float2(-tacc[0], -tacc[1]);
-                        *reinterpret_cast<float2 *>(to + (gq + 8) * kBlkPitch + 8 * nt + 2 * tq) =
-                            make_float2(-tacc[2], -tacc[3]);
+                        const int cl = 8 * nt + 2 * tq;
+                        *reinterpret_cast<float2 *>(to + gq * kBlkPitch + cl) = make_float2(-tacc[0], -tacc[1]);
+                        *reinterpret_cast<float2 *>(to + (gq + 8) * kBlkPitch + cl) = make_float2(-tacc[2], -tacc[3]);
+                        const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
+                            pack_bf16(-tacc[0] * b0, -tacc[1] * b1);
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
+                            pack_bf16(-tacc[2] * b0, -tacc[3] * b1);
                     }
                     bar_intra();
                 }
-                // ---- T' = T diag(beta) -> bf16 rows 0-63 of A1 ----
-                for (int idx = tid; idx < 512; idx += kIntraThreads) {
-                    const int r = idx >> 3, ch = idx & 7;
-                    const int R = r >> 4, i = r & 15, I = ch >> 1;
-                    uint32_t w4[4];
-                    if (I <= R) {
-                        const float *tb = f_tm + pair_of(R, I) * kBlkFloats + i * kBlkPitch + (ch & 1) * 8;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c0 = ch * 8 + 2 * e;
-                            const float x0 = c0 <= r ? tb[2 * e] * f_beta[c0] : 0.f;
-                            const float x1 = c0 + 1 <= r ? tb[2 * e + 1] * f_beta[c0 + 1] : 0.f;
-                            w4[e] = pack_bf16(x0, x1);
-                        }
-                    } else {
-                        w4[0] = w4[1] = w4[2] = w4[3] = 0u;
-                    }
-                    *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(r, ch)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
-                bar_intra();
                 // ---- A_qk T' -> bf16 rows 64-127 of A1 (warp-level MMA, warps 0-7) ----
                 if (warp < 8) {
                     const int R = warp >> 1, nh = warp & 1;
@@ -555,13 +578,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_wq,
                                 1u);
-                    tc::commit(mbar_wq);
+                    tc::commit(mbar(kMbWQ));
                 }
-                if (!tc::mbar_wait(mbar_wq, (uint32_t)(s & 1), kWaitLimit)) *abort_flag = 1;
+                bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
                 // B2 is free once the previous chunk's state product has read it
-                if (have_state) {
-                    if (!tc::mbar_wait(mbar_2, (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
-                }
+                if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
+                ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
+                if (!ok) *abort_flag = 1;
                 tc::fence_after();
                 if (warp < 8) {
                     const int c = 32 * lq + lane, cg = warp >> 2;
@@ -575,9 +598,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4 *>(sm + S::B2 + tc::mnmaj_chunk(8 * cg + 4 * h2 + e, c, 128)) =
                                 pack8(w + 8 * e, 1.f);
                     }
+                } else if (L < 64) {
+                    // rows of v past the document end are zero (the tile may reach the next document)
+                    for (int idx = tid - 256; idx < (64 - L) * 16; idx += 128) {
+                        const int row = L + (idx >> 4), ch = idx & 15;
+                        *reinterpret_cast<uint4 *>(sm + S::V + (ch >> 3) * 8192 + row * 128 + (ch & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
                 }
-                // v(s) landed (the two groups committed after it may still be in flight)
-                asm volatile("cp.async.wait_group 2;\n" ::: "memory");
                 tc::fence_proxy_async();
                 tc::fence_before();
                 bar_intra();
@@ -589,92 +617,105 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma(tmem + dcol, tc::desc_mnmaj(sbase + S::V, kk, 64), tc::desc_kmaj(sbase + S::KR, kk), id_u,
                                 kk > 0);
-                    tc::commit(mbar_u);
+                    tc::commit(mbar(kMbU));
                 }
-            } else {
-                bar_intra();   // keep the intra barrier count uniform for a step without a chunk
             }
-        } else if (have_state) {
-            // ================= state (chunk s-1), warps 12-15 =================
-            const int n = s - 1, nbuf = n & 1;
-            const int64_t ptok0 = tok0 - 64;
-            const int pL = (int)(doc_end - ptok0 < 64 ? doc_end - ptok0 : 64);
-            const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
-            const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
-            // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_last})
+        } else {
+            // ================= state warps (12-15) =================
+            if (have_state) {
+                // ---- chunk s-1: state update and output ----
+                const int n = s - 1, nbuf = n & 1;
+                const int64_t ptok0 = doc_start + 64 * (int64_t)n;
+                const int pL = chunk_len(n);
+                const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
+                const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
+                // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_last})
 #pragma unroll 1
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                float sv[32];
-                tc::ld32(lane_base + kSF + c0, sv);
-                tc::wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
-                st16(lane_base + kSB + c0 / 2, pk);
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 d4 = *reinterpret_cast<const float4 *>(dc + c0 + i);
-                    sv[i] *= d4.x; sv[i + 1] *= d4.y; sv[i + 2] *= d4.z; sv[i + 3] *= d4.w;
-                }
-                tc::st32(lane_base + kSF + c0, sv);
-            }
-            tc::wait_st();
-            tc::fence_before();
-            bar_state();
-            if (tid == kStateTid0) {
-                tc::fence_after();
-                constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + dcol, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2, kk, 128), id2, 1u);
-                tc::commit(mbar_2);
-            }
-            if (!tc::mbar_wait(mbar_2, (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
-            tc::fence_after();
-            // U~^T (columns 0-63) -> bf16 copy (A operand of the state update)
-            {
-                float u[32];
-                uint32_t pk[16];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    tc::ld32(lane_base + dcol + 32 * h2, u);
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    float sv[32];
+                    tc::ld32(lane_base + kSF + c0, sv);
                     tc::wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(u[2 * i], u[2 * i + 1]);
-                    st16(lane_base + kUB + 16 * h2, pk);
+                    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
+                    st16(lane_base + kSB + c0 / 2, pk);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 d4 = *reinterpret_cast<const float4 *>(dc + c0 + i);
+                        sv[i] *= d4.x; sv[i + 1] *= d4.y; sv[i + 2] *= d4.z; sv[i + 3] *= d4.w;
+                    }
+                    tc::st32(lane_base + kSF + c0, sv);
                 }
                 tc::wait_st();
-            }
-            tc::fence_before();
-            bar_state();
-            if (tid == kStateTid0) {
+                tc::fence_before();
+                bar_state();
+                if (tid == kStateTid0) {
+                    tc::fence_after();
+                    constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + dcol, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2, kk, 128), id2, 1u);
+                    tc::commit(mbar(kMb2));
+                }
+                if (!tc::mbar_wait(mbar(kMb2), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
                 tc::fence_after();
-                constexpr uint32_t id4 = tc::idesc_bf16(128, 128, false, false, false);
+                // U~^T (columns 0-63) -> bf16 copy (A operand of the state update)
+                {
+                    float u[32];
+                    uint32_t pk[16];
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + kSF, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::KDT + nbuf * 16384, kk), id4, 1u);
-                tc::commit(mbar_4);
-            }
-            // O^T (columns 64-127): lane v holds o[r][v] for the 64 rows of chunk s-1
-            {
-                const int vcol = 32 * lq + lane;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        tc::ld32(lane_base + dcol + 32 * h2, u);
+                        tc::wait_ld();
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    float o[32];
-                    tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
-                    tc::wait_ld();
+                        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(u[2 * i], u[2 * i + 1]);
+                        st16(lane_base + kUB + 16 * h2, pk);
+                    }
+                    tc::wait_st();
+                }
+                tc::fence_before();
+                bar_state();
+                if (tid == kStateTid0) {
+                    tc::fence_after();
+                    constexpr uint32_t id4 = tc::idesc_bf16(128, 128, false, false, false);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int r = 32 * h2 + i;
-                        if (r < pL) {
-                            const __nv_bfloat16 b = __float2bfloat16_rn(o[i] * out_scale);
-                            out[((ptok0 + r) * H + h) * kHeadDim + vcol] = *reinterpret_cast<const uint16_t *>(&b);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + kSF, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::KDT + nbuf * 16384, kk), id4, 1u);
+                    tc::commit(mbar(kMb4));
+                }
+                // O^T (columns 64-127): lane v holds o[r][v]; lane pairs swap so each stores (v, v+1)
+                {
+                    const int vcol = 32 * lq + lane;
+                    const bool odd = lane & 1;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        float o[32];
+                        tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
+                        tc::wait_ld();
+                        // even lanes store rows 32h2 + [0,16), odd lanes rows 32h2 + [16,32)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float mine_for_partner = odd ? o[i] : o[16 + i];
+                            const float from_partner = __shfl_xor_sync(0xffffffffu, mine_for_partner, 1);
+                            const int r = 32 * h2 + (odd ? 16 + i : i);
+                            const float lo = odd ? from_partner : o[i];
+                            const float hi = odd ? o[16 + i] : from_partner;
+                            if (r < pL) {
+                                uint32_t *dst = reinterpret_cast<uint32_t *>(
+                                    out + ((ptok0 + r) * H + h) * kHeadDim + (vcol & ~1));
+                                *dst = pack_bf16(lo * out_scale, hi * out_scale);
+                            }
                         }
                     }
                 }
+                if (!tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                tc::fence_after();
             }
-            if (!tc::mbar_wait(mbar_4, (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
-            tc::fence_after();
+            // ---- row norms of chunk s+1 (its raw q, k arrive after this step's A_kk) ----
+            if (have_next) {
+                if (!tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit)) *abort_flag = 1;
+                norms16((warp - 12) * 16, nL);
+            }
         }
         tc::fence_before();
         __syncthreads();
@@ -686,8 +727,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait_all();
     if (aborted) {
         if (tid == 0) atomicExch(status, kStatusTimeout);
-        tc::mbar_wait(mbar_wq, 0, kWaitLimit / 8);
-        tc::mbar_wait(mbar_wq, 1, kWaitLimit / 8);
+        // let any tensor-core work or copy still in flight land before TMEM and shared memory go away
+        for (int i = 0; i < 7; ++i) {
+            tc::mbar_wait(mbar(i), 0u, kWaitLimit / 16);
+            tc::mbar_wait(mbar(i), 1u, kWaitLimit / 16);
+        }
     }
     tc::fence_before();
     __syncthreads();
@@ -695,18 +739,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) tc::dealloc(tmem, kTmemCols);
 }
 
+// ---- host: TMA descriptors ----
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a [rows, cols] row-major tensor (cols contiguous), box [box_rows, box_cols]
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows, uint64_t cols,
+              uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (cuuint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace pipe_path
 
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, uint16_t *out,
                             int *status, cudaStream_t stream) {
-    constexpr int bytes = pipe_path::Smem::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(pipe_path::kda_fwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         bytes);
+    using namespace pipe_path;
+    Maps maps;
+    const uint64_t cols = (uint64_t)H * kHeadDim;
+    if (!make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&maps.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)T, cols, 64, 32, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    constexpr int bytes = Smem::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(kda_fwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (int64_t)n_docs * H;
-    pipe_path::kda_fwd_pipe_kernel<<<(unsigned)blocks, pipe_path::kThreads, bytes, stream>>>(q, k, v, g, beta, cu,
-                                                                                             n_docs, T, H, out, status);
+    kda_fwd_pipe_kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, out, status);
     return cudaGetLastError();
 }
 

@@ -151,5 +151,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long 
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// TMA (no multicast): 2-D tiled bulk copy global -> shared, completion counted
+// in bytes on an mbarrier.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_expect_tx(uint32_t saddr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst_saddr, const void *tmap, int x, int y, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst_saddr),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+
 }  // namespace tc
 }  // namespace kda
