@@ -257,8 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c0 = 0; c0 < 128; c0 += 32) tc::st32(lane_base + kSF + c0, z);
         tc::wait_st();
     }
-    // norms of chunk 0
-    if (!tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit)) *abort_flag = 1;
+    // norms of chunk 0 (one thread polls the barrier; the CTA barrier releases the rest)
+    if (tid == 0 && !tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit)) *abort_flag = 1;
+    __syncthreads();
     if (warp < 4) norms16(warp * 16, chunk_len(0));
     tc::fence_before();
     __syncthreads();
@@ -278,8 +279,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- top: beta(s) landed; the previous step's U product is done (V, KR free) ----
         cp_async_wait_all();
-        if (have_state) {
-            if (!tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
+        if (tid == 0) {
+            bool ok = true;
+            if (have_state) ok = tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit);
+            if (have_intra) {
+                ok = tc::mbar_wait(mbar(kMbQK), par, kWaitLimit) && ok;
+                ok = tc::mbar_wait(mbar(kMbG), par, kWaitLimit) && ok;
+            }
+            if (!ok) *abort_flag = 1;
         }
         tc::fence_before();
         __syncthreads();
@@ -295,22 +302,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pc = tid & 127, pR = tid >> 7;
         if (have_intra) {
             // ---- prep pass 1: thread = (channel c, row block R) ----
-            bool ok = tc::mbar_wait(mbar(kMbQK), par, kWaitLimit);
-            ok = tc::mbar_wait(mbar(kMbG), par, kWaitLimit) && ok;
-            if (!ok) *abort_flag = 1;
-            float lg[16];
+            // per-row decays a_j = 2^{log2e g_j} (one exp2 each); E1 and E2 are running products
+            // inside the 16-row block: E1_j = a_1..a_j, E2_j = a_{j+1}..a_15 (both in [e^-75, 1])
+            float a[16];
             float acc = 0.f;
             const uint8_t *gcol = sm + S::G + (pc >> 5) * 8192 + (pc & 31) * 4;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int r = 16 * pR + j;
                 const float gv = *reinterpret_cast<const float *>(gcol + r * 128);
-                acc += r < L ? gv * kLog2e : 0.f;         // log2-scaled gate cumsum
-                lg[j] = acc;
+                const float gl2 = r < L ? gv * kLog2e : 0.f;      // log2-scaled gate
+                acc += gl2;
+                a[j] = fast_exp2(gl2);
+                if (j == 0) lg0 = acc;
             }
-            lg0 = lg[0];
-            lg15 = lg[15];
+            lg15 = acc;
             f_tot[pR * 128 + pc] = lg15;
+            float e1[16], e2[16];
+            e1[0] = 1.f;
+#pragma unroll
+            for (int j = 1; j < 16; ++j) e1[j] = e1[j - 1] * a[j];
+            e2[15] = 1.f;
+#pragma unroll
+            for (int j = 14; j >= 0; --j) e2[j] = e2[j + 1] * a[j + 1];
             const uint8_t *qcol = sm + S::Q + (pc >> 6) * 8192 + (pc & 63) * 2;
             const uint8_t *kcol = sm + S::K + (pc >> 6) * 8192 + (pc & 63) * 2;
 #pragma unroll
@@ -326,12 +340,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kcol + r * 128));
                     qv = r < L ? qv : 0.f;
                     kv = r < L ? kv : 0.f;
-                    const float e1 = fast_exp2(lg[j] - lg0);
-                    const float e2 = fast_exp2(lg15 - lg[j]);
                     const float qh = qv * rqv[jj], kh = kv * rkv[jj];
-                    ql[j] = qh * e1;
-                    kl[j] = kh * e1;
-                    kr[j] = kh * e2;
+                    ql[j] = qh * e1[j];
+                    kl[j] = kh * e1[j];
+                    kr[j] = kh * e2[j];
                 }
             }
         }
@@ -368,16 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4 *>(sm + S::KGT + off) = pack8(kl + j0, P);
                 *reinterpret_cast<uint4 *>(sm + S::KDT + buf * 16384 + off) = pack8(kr + j0, Dk);
             }
-            // D_WQ init in TMEM (lane c): columns 16R.. = 0, columns 64+16R.. = Q~ rows 16R..16R+15
+            // Q~ into TMEM (lane c, columns 64+16R..): the accumulator of the Q' product
             {
-                float qt[16], z[16];
+                float qt[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    qt[j] = ql[j] * P;
-                    z[j] = 0.f;
-                }
+                for (int j = 0; j < 16; ++j) qt[j] = ql[j] * P;
                 const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
-                st16f(lane_base + dcol + 16 * pR, z);
                 st16f(lane_base + dcol + 64 + 16 * pR, qt);
                 tc::wait_st();
             }
@@ -399,6 +407,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float ak[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                     float aq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                     const int j = lane >> 3;
+                    // the pair scale of this thread's fragment channels, as bf16x2, for all 8 k-steps
+                    __nv_bfloat162 hs[8][2];
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int cb = kk * 16 + 2 * tq;
+                        const float2 s0 = *reinterpret_cast<const float2 *>(ps + cb);
+                        const float2 s8 = *reinterpret_cast<const float2 *>(ps + cb + 8);
+                        hs[kk][0] = __floats2bfloat162_rn(s0.x, s0.y);
+                        hs[kk][1] = __floats2bfloat162_rn(s8.x, s8.y);
+                    }
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t aoff = tc::kmaj_chunk(16 * kk + (lane & 7) + 8 * (j >> 1), 2 * R + (j & 1));
@@ -407,14 +425,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ldsm_x4_t(qbase + aoff, fq[0], fq[1], fq[2], fq[3]);
                         ldsm_x4_t(rbase + tc::kmaj_chunk(16 * kk + (lane & 7) + 8 * (j & 1), 2 * I + (j >> 1)), b0, b1,
                                   b2, b3);
-                        const int cb = kk * 16 + 2 * tq;
-                        const float2 s0 = *reinterpret_cast<const float2 *>(ps + cb);
-                        const float2 s8 = *reinterpret_cast<const float2 *>(ps + cb + 8);
-                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(s0.x, s0.y);
-                        const __nv_bfloat162 h8 = __floats2bfloat162_rn(s8.x, s8.y);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 sc = e < 2 ? h0 : h8;
+                            const __nv_bfloat162 sc = hs[kk][e >> 1];
                             __nv_bfloat162 x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fk[e]), sc);
                             fk[e] = *reinterpret_cast<uint32_t *>(&x);
                             x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fq[e]), sc);
@@ -573,18 +586,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
                 if (tid == 0) {
                     tc::fence_after();
-                    constexpr uint32_t id_wq = tc::idesc_bf16(128, 128, false, false, true);
+                    // columns 0-63: -W^T (fresh); columns 64-127: Q~^T - (A_qk W)^T (accumulate)
+                    constexpr uint32_t id_wq = tc::idesc_bf16(128, 64, false, false, true);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_wq,
-                                1u);
+                                kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma(tmem + dcol + 64, tc::desc_kmaj(sbase + S::KGT, kk),
+                                tc::desc_kmaj(sbase + S::KR + 8192, kk), id_wq, 1u);
                     tc::commit(mbar(kMbWQ));
                 }
-                bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
-                // B2 is free once the previous chunk's state product has read it
-                if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
-                ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
-                if (!ok) *abort_flag = 1;
+                if (tid == 0) {
+                    bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
+                    // B2 is free once the previous chunk's state product has read it
+                    if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
+                    ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
+                    if (!ok) *abort_flag = 1;
+                    tc::fence_before();
+                }
+                bar_intra();
                 tc::fence_after();
                 if (warp < 8) {
                     const int c = 32 * lq + lane, cg = warp >> 2;
@@ -657,7 +679,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ts(tmem + dcol, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2, kk, 128), id2, 1u);
                     tc::commit(mbar(kMb2));
                 }
-                if (!tc::mbar_wait(mbar(kMb2), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                if (tid == kStateTid0) {
+                    if (!tc::mbar_wait(mbar(kMb2), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                    tc::fence_before();
+                }
+                bar_state();
                 tc::fence_after();
                 // U~^T (columns 0-63) -> bf16 copy (A operand of the state update)
                 {
@@ -708,12 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (!tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
-                tc::fence_after();
+                if (tid == kStateTid0 && !tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
             }
             // ---- row norms of chunk s+1 (its raw q, k arrive after this step's A_kk) ----
             if (have_next) {
-                if (!tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit)) *abort_flag = 1;
+                if (tid == kStateTid0 && !tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit))
+                    *abort_flag = 1;
+                bar_state();
                 norms16((warp - 12) * 16, nL);
             }
         }

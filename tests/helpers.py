@@ -28,6 +28,12 @@ def out_to_f64(o) -> np.ndarray:
     return bf16_bits_to_f32(bits).reshape(bits.shape).astype(np.float64)
 
 
+def bf16_out(bits_i16: np.ndarray) -> np.ndarray:
+    """int16 view of bf16 output bits -> float64."""
+    b = np.ascontiguousarray(bits_i16).view(np.uint16)
+    return bf16_bits_to_f32(b).reshape(b.shape).astype(np.float64)
+
+
 def oracle_out(d: dict, chains=None, **kw) -> np.ndarray:
     f = lambda key: bf16_bits_to_f32(d[key]).reshape(d[key].shape)
     return oracle.kda_fwd(f("q"), f("k"), f("v"), d["g"], d["beta"], d["cu_seqlens"], chains=chains, **kw)

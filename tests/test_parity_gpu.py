@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 from chunked_gated_delta_12_b200.inputs import custom_workload, generate, workload
-from tests.helpers import ATOL_MAX, RTOL_L2, compare, oracle_out, out_to_f64, to_device
+from tests.helpers import ATOL_MAX, RTOL_L2, bf16_out, compare, oracle_out, out_to_f64, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -159,3 +159,50 @@ def test_rejects_wrong_dtype(kda):
     cu = torch.tensor([0, 64], dtype=torch.int32, device="cuda")
     with pytest.raises(kda.KdaError):
         kda.kda_chunk_fwd(x, x, x, g, b, cu)
+
+
+def test_pipelined_path_isolation_bitwise(kda):
+    """Same isolation check on a launch large enough for the pipelined kernel
+    (>= 112 chains): its TMA tiles read past document ends, so poisoned rows of
+    the next document must be masked, never used."""
+    import torch
+    lens = [1, 64, 65, 129, 63, 200, 64, 14]
+    w = custom_workload("iso_pipe", lens, 16, seed=37)       # 8 docs x 16 heads = 128 chains
+    d = generate(w)
+    cu = d["cu_seqlens"]
+    T, H = w.T, w.H
+    guard = 4096
+    buf = torch.full((guard + T * H * 128 + guard,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = buf[guard:guard + T * H * 128].view(T, H, 128)
+    run(kda, d, out=out)
+    assert not torch.isnan(out).any(), "some output row was not written"
+    assert torch.isnan(buf[:guard]).all() and torch.isnan(buf[-guard:]).all(), "write outside out"
+    base = out.view(torch.int16).cpu().numpy()
+    ref = oracle_out(d, chains=list(range(0, 128, 5)))
+    rel, mx = compare(bf16_out(base), ref, cu, w.H, list(range(0, 128, 5)))
+    assert rel <= RTOL_L2 and mx <= ATOL_MAX, (rel, mx)
+    for victim in (1, 3, 6):
+        e = dict(d)
+        s0, s1 = int(cu[victim]), int(cu[victim + 1])
+        for key in ("q", "k", "v", "g", "beta"):
+            e[key] = d[key].copy()
+        e["q"][s0:s1] = 0x7FC0
+        e["k"][s0:s1] = 0x7F80
+        e["v"][s0:s1] = 0x7FC0
+        e["g"][s0:s1] = np.nan
+        e["beta"][s0:s1] = np.inf
+        got = run(kda, e).view(torch.int16).cpu().numpy()
+        assert np.array_equal(got[:s0], base[:s0]), f"doc {victim} leaked backwards"
+        assert np.array_equal(got[s1:], base[s1:]), f"doc {victim} leaked forwards"
+
+
+@pytest.mark.parametrize("lens", [[64] * 8, [1] * 8, [65, 63, 128, 127, 1, 64, 192, 2]])
+def test_pipelined_path_lengths(kda, lens):
+    """Chunk-aligned, single-token and mixed documents on the pipelined kernel."""
+    w = custom_workload("pipe_lens", lens, 16, seed=38)
+    d = generate(w)
+    got = out_to_f64(run(kda, d))
+    chains = list(range(0, 8 * 16, 3))
+    ref = oracle_out(d, chains=chains)
+    rel, mx = compare(got, ref, d["cu_seqlens"], w.H, chains)
+    assert rel <= RTOL_L2 and mx <= ATOL_MAX, (rel, mx)
