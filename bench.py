@@ -128,6 +128,24 @@ def dist_setup(n_gpus: int):
     return world, rank, local
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` across the ranks of the default process group (the
+    value itself when not distributed).  Used for device times, so the slowest
+    rank sets the whole-job throughput."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Mtokens/s of the whole job: every rank processes its own replica of the workload."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3) / 1e6
+
+
 def oracle_sample_rate(w, d, tokens: int, n_threads: int):
     """Time the fp64 oracle on the first `tokens` tokens of document 0 (all heads)."""
     import oracle
@@ -268,12 +286,7 @@ def main():
     barrier()
     kda.device_status(stream)
     per_launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    elapsed_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dev)
 
     # end to end through the public API: pinned host inputs -> device, forward, result -> host
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -291,15 +304,11 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps) if not args.no_e2e else float("nan")
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
 
     tokens_all = w.T * world
     ms_step = elapsed_ms / args.steps
-    value = tokens_all / (ms_step * 1e-3) / 1e6
+    value = whole_job_rate(w.T, world, ms_step)
     hbm_peak, tc_peak, peak_kind = peaks()
     launch_ms = float(np.mean(per_launch_ms))
     alg_bytes = w.T * w.H * BYTES_PER_TOKEN_HEAD

@@ -40,6 +40,8 @@ def lib() -> ctypes.CDLL:
         L.kda_last_error.argtypes = []
         L.kda_device_status.restype = i32
         L.kda_device_status.argtypes = [vp]
+        L.kda_wait_selftest.restype = i32
+        L.kda_wait_selftest.argtypes = [vp]
         L.kda_abi_version.restype = i32
         L.kda_abi_version.argtypes = []
         _lib = L
@@ -88,6 +90,11 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                              cu_seqlens.numel() - 1, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
     return out
+
+
+def wait_selftest(stream: torch.cuda.Stream | None = None) -> None:
+    """Enqueue the self-test whose device wait must time out (see kda_wait_selftest)."""
+    _check(lib().kda_wait_selftest(ctypes.c_void_p(_stream_handle(stream))))
 
 
 def device_status(stream: torch.cuda.Stream | None = None) -> None:

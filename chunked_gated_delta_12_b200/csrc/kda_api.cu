@@ -117,6 +117,19 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return KDA_OK;
 }
 
+kda_status kda_wait_selftest(void *stream) {
+    g_err[0] = '\0';
+    int dev = -1;
+    kda_status s = check_device(&dev);
+    if (s != KDA_OK) return s;
+    int *status = nullptr;
+    s = status_ptr(dev, &status);
+    if (s != KDA_OK) return s;
+    cudaError_t e = kda::launch_wait_selftest(status, 20000000LL, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+    return KDA_OK;
+}
+
 kda_status kda_device_status(void *stream) {
     g_err[0] = '\0';
     int dev = -1;

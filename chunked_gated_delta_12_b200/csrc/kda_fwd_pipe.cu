@@ -390,6 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::wait_st();
             }
         }
+        // operand tiles written through the generic proxy are read by the tensor core
+        tc::fence_proxy_async();
         tc::fence_before();
         __syncthreads();
         tc::fence_after();
@@ -494,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
                         }
                     }
+                    tc::fence_proxy_async();
                 } else {
                     // T' is zero above the block diagonal (warps 4-11)
                     const int t = tid - 128;
@@ -504,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
                             make_uint4(0, 0, 0, 0);
                     }
+                    tc::fence_proxy_async();
                 }
                 bar_intra();
                 // ---- off-diagonal blocks by distance d (tf32 warp MMA), T and T' stored ----
@@ -544,8 +548,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pack_bf16(-tacc[0] * b0, -tacc[1] * b1);
                         *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
                             pack_bf16(-tacc[2] * b0, -tacc[3] * b1);
+                        tc::fence_proxy_async();
                     }
                     bar_intra();
+                }
+                // T' is complete: the W half of the W/Q' product can start now
+                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
+                if (tid == 0) {
+                    tc::fence_after();
+                    constexpr uint32_t id_w = tc::idesc_bf16(128, 64, false, false, true);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_w,
+                                kk > 0);
                 }
                 // ---- A_qk T' -> bf16 rows 64-127 of A1 (warp-level MMA, warps 0-7) ----
                 if (warp < 8) {
@@ -582,16 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_proxy_async();
                 tc::fence_before();
                 bar_intra();
-                // ---- tcgen05: D_WQ = [0 | Q~^T] - KG^T A1^T ----
-                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
+                // ---- tcgen05: Q' half, columns 64-127: Q~^T - (A_qk W)^T (accumulate) ----
                 if (tid == 0) {
                     tc::fence_after();
-                    // columns 0-63: -W^T (fresh); columns 64-127: Q~^T - (A_qk W)^T (accumulate)
                     constexpr uint32_t id_wq = tc::idesc_bf16(128, 64, false, false, true);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_wq,
-                                kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma(tmem + dcol + 64, tc::desc_kmaj(sbase + S::KGT, kk),

@@ -22,4 +22,8 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
                             uint16_t *out, int *status, cudaStream_t stream);
 
+// Runs one time-limited mbarrier wait that can never complete (self-test of the
+// timeout path): records kStatusTimeout in *status after about limit_cycles.
+cudaError_t launch_wait_selftest(int *status, long long limit_cycles, cudaStream_t stream);
+
 }  // namespace kda

@@ -87,6 +87,17 @@ const char *kda_last_error(void);
  */
 kda_status kda_device_status(void *stream);
 
+/*
+ * kda_wait_selftest -- enqueue on `stream` a one-warp kernel whose time-limited
+ * device wait can never be satisfied, so that it gives up (after ~10 ms of SM
+ * clock) and records KDA_ERR_TIMEOUT exactly as the forward kernels do when a
+ * tensor-core or TMA completion never arrives.  A following kda_device_status()
+ * returns KDA_ERR_TIMEOUT and clears it; the CUDA context stays usable.  This is
+ * a diagnostic of the failure-reporting path (the kda_fused page's rule: report
+ * the condition, never hang or fall back), not part of the forward.
+ */
+kda_status kda_wait_selftest(void *stream);
+
 /* ABI version of this header (bumped on any signature change). */
 int kda_abi_version(void);
 

@@ -206,3 +206,19 @@ def test_pipelined_path_lengths(kda, lens):
     ref = oracle_out(d, chains=chains)
     rel, mx = compare(got, ref, d["cu_seqlens"], w.H, chains)
     assert rel <= RTOL_L2 and mx <= ATOL_MAX, (rel, mx)
+
+
+def test_device_wait_timeout_is_reported_and_context_survives(kda):
+    """A device wait that can never complete gives up, reports KDA_ERR_TIMEOUT
+    through kda_device_status, and the next forward runs normally."""
+    kda.wait_selftest()
+    with pytest.raises(kda.KdaError) as ei:
+        kda.device_status()
+    assert ei.value.code == 5
+    kda.device_status()                      # cleared
+    w = workload(0)
+    d = generate(w)
+    got = out_to_f64(run(kda, d))
+    ref = oracle_out(d)
+    rel, mx = compare(got, ref, d["cu_seqlens"], w.H)
+    assert rel <= RTOL_L2 and mx <= ATOL_MAX, (rel, mx)
