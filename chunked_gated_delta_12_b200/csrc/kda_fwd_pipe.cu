@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint16_t *__restrict__ out, int *__restrict__ status) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    // align by offsetting the shared array itself, so every access stays in the shared window (LDS/STS)
+    uint8_t *sm = sm_raw + (((smem_u32(sm_raw) + 1023u) & ~1023u) - smem_u32(sm_raw));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
@@ -496,7 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
                         }
                     }
-                    tc::fence_proxy_async();
                 } else {
                     // T' is zero above the block diagonal (warps 4-11)
                     const int t = tid - 128;
@@ -507,7 +507,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
                             make_uint4(0, 0, 0, 0);
                     }
-                    tc::fence_proxy_async();
                 }
                 bar_intra();
                 // ---- off-diagonal blocks by distance d (tf32 warp MMA), T and T' stored ----
@@ -548,8 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pack_bf16(-tacc[0] * b0, -tacc[1] * b1);
                         *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
                             pack_bf16(-tacc[2] * b0, -tacc[3] * b1);
-                        tc::fence_proxy_async();
                     }
+                    if (d == 3) tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
                     bar_intra();
                 }
                 // T' is complete: the W half of the W/Q' product can start now

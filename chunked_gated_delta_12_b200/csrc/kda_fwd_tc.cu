@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int CW = VS / 4;            // TMEM columns per warp in the U~ / O passes
     static_assert(CW == 32 || CW == 16, "VS must be 128 or 64");
     extern __shared__ __align__(1024) uint8_t sm_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    // align by offsetting the shared array itself, so every access stays in the shared window (LDS/STS)
+    uint8_t *sm = sm_raw + (((smem_u32(sm_raw) + 1023u) & ~1023u) - smem_u32(sm_raw));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
