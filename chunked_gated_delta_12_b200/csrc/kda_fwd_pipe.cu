@@ -79,7 +79,7 @@ struct Smem {
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
 
-enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV };
+enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kMbO };   // kMbO: thread-arrived, B2 free again
 
 __device__ __forceinline__ void bar_intra() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void bar_state() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
@@ -135,7 +135,7 @@ __device__ __forceinline__ void load_beta(uint8_t *sm, const float *beta, int64_
 }
 
 struct Maps {
-    CUtensorMap q, k, g, v;
+    CUtensorMap q, k, g, v, o;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- setup ----
     if (warp == 0) tc::alloc(smem_u32(sm + S::TBASE), kTmemCols);
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) tc::mbar_init(mbar(i), 1);
+        for (int i = 0; i < 8; ++i) tc::mbar_init(mbar(i), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -366,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float ge = offs[pR + 1];
             const float gl = offs[4];
             const float P = fast_exp2(gm);
+            const float Pq = P * out_scale;          // the output scale rides on Q~ and A_qk
             const float Dk = fast_exp2(gl - ge);
 #pragma unroll
             for (int I = 0; I < 4; ++I)
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 float qt[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) qt[j] = ql[j] * P;
+                for (int j = 0; j < 16; ++j) qt[j] = ql[j] * Pq;
                 const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
                 st16f(lane_base + dcol + 64 + 16 * pR, qt);
                 tc::wait_st();
@@ -452,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float x0 = col < row ? ak[nt][2 * hh] * br : 0.f;
                             const float x1 = col + 1 < row ? ak[nt][2 * hh + 1] * br : 0.f;
                             *reinterpret_cast<float2 *>(blk + i * kBlkPitch + jj) = make_float2(x0, x1);
-                            const float y0 = col <= row ? aq[nt][2 * hh] : 0.f;
-                            const float y1 = col + 1 <= row ? aq[nt][2 * hh + 1] : 0.f;
+                            const float y0 = col <= row ? aq[nt][2 * hh] * out_scale : 0.f;
+                            const float y1 = col + 1 <= row ? aq[nt][2 * hh + 1] * out_scale : 0.f;
                             *reinterpret_cast<uint32_t *>(sm + S::AQK + tc::kmaj_off(row, col)) = pack_bf16(y0, y1);
                         }
                 } else {
@@ -608,8 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (tid == 0) {
                     bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
-                    // B2 is free once the previous chunk's state product has read it
-                    if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
+                    // B2 is free once the previous chunk's state product has read it and its
+                    // output tile, staged there, has been read by the TMA store
+                    if (have_state) ok = tc::mbar_wait(mbar(kMbO), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
                     ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
                     if (!ok) *abort_flag = 1;
                     tc::fence_before();
@@ -717,27 +719,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ts(tmem + kSF, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::KDT + nbuf * 16384, kk), id4, 1u);
                     tc::commit(mbar(kMb4));
                 }
-                // O^T (columns 64-127): lane v holds o[r][v]; lane pairs swap so each stores (v, v+1)
+                // O^T (columns 64-127; the output scale is already applied): lane v holds o[r][v].
+                // Lane pairs swap values so that each thread writes the pair (v, v+1) of one row.
                 {
                     const int vcol = 32 * lq + lane;
                     const bool odd = lane & 1;
+                    if (pL == 64) {
+                        // whole chunk: stage o[r][v] as bf16 in B2 (two 64-channel boxes, 128-B swizzled
+                        // rows) and write it with one TMA store per box.  Even lanes take rows with
+                        // (r & 4) == 0, odd lanes the row 4 below, so one store instruction covers 32 banks.
+                        const uint32_t vb = (uint32_t)(vcol & 62) * 2;          // byte of the pair in its row
+                        uint8_t *stage = sm + S::B2 + (vcol >> 6) * 8192;
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        float o[32];
-                        tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
-                        tc::wait_ld();
-                        // even lanes store rows 32h2 + [0,16), odd lanes rows 32h2 + [16,32)
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float o[32];
+                            tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
+                            tc::wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float mine_for_partner = odd ? o[i] : o[16 + i];
-                            const float from_partner = __shfl_xor_sync(0xffffffffu, mine_for_partner, 1);
-                            const int r = 32 * h2 + (odd ? 16 + i : i);
-                            const float lo = odd ? from_partner : o[i];
-                            const float hi = odd ? o[16 + i] : from_partner;
-                            if (r < pL) {
-                                uint32_t *dst = reinterpret_cast<uint32_t *>(
-                                    out + ((ptok0 + r) * H + h) * kHeadDim + (vcol & ~1));
-                                *dst = pack_bf16(lo * out_scale, hi * out_scale);
+                            for (int i = 0; i < 16; ++i) {
+                                const int ja = (i & 3) + 8 * (i >> 2), jb = ja + 4;
+                                const float send = odd ? o[ja] : o[jb];
+                                const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                                const float lo = odd ? recv : o[ja];
+                                const float hi = odd ? o[jb] : recv;
+                                const int r = 32 * h2 + (odd ? jb : ja);
+                                const uint32_t off = (uint32_t)r * 128u + ((((vb >> 4) ^ (uint32_t)(r & 7)) << 4) | (vb & 15u));
+                                *reinterpret_cast<uint32_t *>(stage + off) = pack_bf16(lo, hi);
+                            }
+                        }
+                        tc::fence_proxy_async();
+                        bar_state();
+                        if (tid == kStateTid0) {
+                            tc::tma_store_2d(&maps.o, xq, (int)ptok0, sbase + S::B2);
+                            tc::tma_store_2d(&maps.o, xq + 64, (int)ptok0, sbase + S::B2 + 8192);
+                            tc::bulk_commit();
+                            tc::bulk_wait_read();
+                            tc::mbar_arrive(mbar(kMbO));
+                        }
+                    } else {
+                        // partial chunk: rows past the document end belong to the next document, so
+                        // store the valid rows directly
+                        if (tid == kStateTid0) tc::mbar_arrive(mbar(kMbO));
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float o[32];
+                            tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
+                            tc::wait_ld();
+                            // even lanes store rows 32h2 + [0,16), odd lanes rows 32h2 + [16,32)
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float mine_for_partner = odd ? o[i] : o[16 + i];
+                                const float from_partner = __shfl_xor_sync(0xffffffffu, mine_for_partner, 1);
+                                const int r = 32 * h2 + (odd ? 16 + i : i);
+                                const float lo = odd ? from_partner : o[i];
+                                const float hi = odd ? o[16 + i] : from_partner;
+                                if (r < pL) {
+                                    uint32_t *dst = reinterpret_cast<uint32_t *>(
+                                        out + ((ptok0 + r) * H + h) * kHeadDim + (vcol & ~1));
+                                    *dst = pack_bf16(lo, hi);
+                                }
                             }
                         }
                     }
@@ -760,6 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- teardown ----
     cp_async_wait_all();
+    if (tid == kStateTid0) tc::bulk_wait();   // output tiles written before shared memory goes away
     if (aborted) {
         if (tid == 0) atomicExch(status, kStatusTimeout);
         // let any tensor-core work or copy still in flight land before TMEM and shared memory go away
@@ -812,7 +853,8 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
     if (!make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&maps.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)T, cols, 64, 32, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps.o, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     constexpr int bytes = Smem::ALLOC;
     cudaError_t e = cudaFuncSetAttribute(kda_fwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

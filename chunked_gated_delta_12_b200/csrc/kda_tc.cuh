@@ -158,6 +158,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long 
 __device__ __forceinline__ void mbar_expect_tx(uint32_t saddr, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr), "r"(bytes) : "memory");
 }
+// TMA store of one 2-D box from shared memory, tracked by the issuing thread's bulk group
+// (no multicast; x * element size must be a multiple of 16 bytes, x and y non-negative)
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uint32_t src_saddr) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(src_saddr)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the source shared memory of every committed bulk store has been read
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed bulk store has completed
+__device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr) : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst_saddr, const void *tmap, int x, int y, uint32_t mbar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
