@@ -11,14 +11,16 @@
 // Per chunk (rows r, i; Gamma = in-chunk cumsum of g):
 //   A_kk[r,i] = beta_r k^_r.(k^_i e^{Gamma_r - Gamma_i}) (i < r),  A_qk (i <= r)
 //   T' = (I + A_kk)^-1 diag(beta)
-//   W  = T' K^e^Gamma,  U = T' V,  Q' = Q^e^Gamma - A_qk W,  U' = A_qk U
-//   U~ = U - W S,  O = Q'S + U'  (= Q^e^Gamma S + A_qk U~)
+//   W  = T' K^e^Gamma,  U = T' V,  U~ = U - W S
+//   O  = Q^e^Gamma S + A_qk U~
 //   S <- Diag(e^{Gamma_last}) S + (K^ e^{Gamma_last - Gamma})^T U~
 // and on the tensor cores (M = 128 everywhere):
-//   intra  D_WQ = [0 | Q~^T] - (K^e^Gamma)^T [T'; A_qk T']^T      -> [-W^T | Q'^T]   (B2, shared)
-//          D    = V^T [T'; A_qk T']^T                              -> [U^T | U'^T]
-//   state  D   += S^T_bf16 (TMEM) B2                               -> [U~^T | O^T]
-//          S^T += U~^T_bf16 (TMEM) Kd                               (after S^T <- S^T Diag(e^{Gamma_last}))
+//   intra  D[:, 0:64] = -(K^e^Gamma)^T T'^T = -W^T, next to Q~^T (written by the prep)
+//          -> B2 = [-W^T | Q~^T] (bf16, shared);  then D[:, 0:64] = V^T T'^T = U^T
+//   state  D   += S^T_bf16 (TMEM) B2                -> [U~^T | (Q~ S)^T]
+//          O^T += U~^T_bf16 (TMEM) A_qk^T
+//          S^T += U~^T_bf16 (TMEM) Kd               (after S^T <- S^T Diag(e^{Gamma_last}))
+// The output scale is carried by Q~ and A_qk.
 // q, k, g and v tiles arrive by TMA (2-D tensor maps over [T, H*128], no
 // multicast); rows past the document end are masked with selects (and v rows
 // zeroed) because a tile may reach into the next document.  The gate exponent
@@ -56,11 +58,11 @@ struct Smem {
     static constexpr int K = 16384;        // raw k                                                -> k^E1 [c][r] SW128
     static constexpr int G = 32768;        // raw g: four TMA boxes [64 rows][32 ch] fp32
     static constexpr int V = 65536;        // raw v: two TMA boxes, 128B-swizzled = MN-major SW128 atoms
-    static constexpr int KR = 81920;       // k^E2 [c][r] SW128 -> A1 = [T'; A_qk T'] (K-major, 128 rows)
+    static constexpr int KR = 81920;       // k^E2 [c][r] SW128 -> T' (rows 0-63) and the A_qk staging tile
     static constexpr int KGT = 98304;      // (k^ e^Gamma)^T, K-major [c][r]
     static constexpr int KDT = 114688;     // two buffers: (k^ e^{Gamma_last-Gamma})^T, K-major [c][r]
     static constexpr int B2 = 147456;      // [-W^T | Q'^T], MN-major [c][n], two 64-wide atoms
-    static constexpr int AQK = 180224;     // A_qk [r][i], K-major (64 rows)
+    static constexpr int AQK = 180224;     // A_qk [r][i], K-major (64 rows), read by the state side's O product
     static constexpr int AKK = 188416;     // A_kk blocks fp32
     static constexpr int TM = AKK + 10 * kBlkFloats * 4;   // T blocks fp32
     static constexpr int SMALL = TM + 10 * kBlkFloats * 4;
@@ -71,15 +73,16 @@ struct Smem {
     static constexpr int PS = TOT + 2048;            // fp32 [10][128]
     static constexpr int DC = PS + 5120;             // fp32 [2][128]
     static constexpr int XT = DC + 1024;             // fp32 [6][16][8]
-    static constexpr int MBAR = XT + 3072;           // u64 [8]
-    static constexpr int TBASE = MBAR + 64;
+    static constexpr int MBAR = XT + 3072;           // u64 [16]
+    static constexpr int TBASE = MBAR + 128;
     static constexpr int ABORT = TBASE + 16;
     static constexpr int BYTES = ABORT + 16;
     static constexpr int ALLOC = BYTES + 1024;
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
 
-enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kMbO };   // kMbO: thread-arrived, B2 free again
+// kMbO is arrived by a thread (B2 free again); the others complete by tcgen05.commit or TMA bytes
+enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kMbO, kMbOq, kNumMbar };
 
 __device__ __forceinline__ void bar_intra() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void bar_state() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- setup ----
     if (warp == 0) tc::alloc(smem_u32(sm + S::TBASE), kTmemCols);
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) tc::mbar_init(mbar(i), 1);
+        for (int i = 0; i < kNumMbar; ++i) tc::mbar_init(mbar(i), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -278,25 +281,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = s & 1;
         const uint32_t par = (uint32_t)(s & 1);
 
-        // ---- top: beta(s) landed; the previous step's U product is done (V, KR free) ----
+        // ---- top: beta(s), q, k and g of chunk s landed ----
         cp_async_wait_all();
-        if (tid == 0) {
-            bool ok = true;
-            if (have_state) ok = tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit);
-            if (have_intra) {
-                ok = tc::mbar_wait(mbar(kMbQK), par, kWaitLimit) && ok;
-                ok = tc::mbar_wait(mbar(kMbG), par, kWaitLimit) && ok;
-            }
+        if (tid == 0 && have_intra) {
+            bool ok = tc::mbar_wait(mbar(kMbQK), par, kWaitLimit);
+            ok = tc::mbar_wait(mbar(kMbG), par, kWaitLimit) && ok;
             if (!ok) *abort_flag = 1;
         }
-        tc::fence_before();
         __syncthreads();
-        tc::fence_after();
         if (*abort_flag) { aborted = true; break; }
-        if (tid == 0 && have_intra) {
-            tc::fence_proxy_async();
-            issue_v(s);
-        }
 
         float ql[16], kl[16], kr[16];
         float lg0 = 0.f, lg15 = 0.f;
@@ -348,11 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        // the previous step's U product is done: V, KR and its accumulator are free
+        if (tid == 0 && have_state && !tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
+        tc::fence_before();
         __syncthreads();   // raw q, k, g read; block sums published
-        // raw g, beta(s+1) buffer are free: the next chunk's g and beta
-        if (tid == 0 && have_next) {
+        tc::fence_after();
+        if (*abort_flag) { aborted = true; break; }
+        // raw g, beta(s+1) buffer are free: the next chunk's g and beta; v of chunk s
+        if (tid == 0) {
             tc::fence_proxy_async();
-            issue_g(s + 1);
+            if (have_next) issue_g(s + 1);
+            if (have_intra) issue_v(s);
         }
         if (have_next) load_beta(sm, beta, doc_start + 64 * (int64_t)(s + 1), nL, H, h, buf ^ 1);
         cp_async_commit();
@@ -403,6 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (have_intra) {
                 const float *f_beta = reinterpret_cast<const float *>(sm + S::BETA + buf * 256);
                 // ---- A_kk and A_qk, one 16x16 block pair per warp ----
+                uint32_t aq_pk[4];
+                constexpr int kAqs = S::KR + 8192;
                 if (warp < 10) {
                     const int p = warp;
                     const int R = pair_R(p), I = p - R * (R + 1) / 2;
@@ -455,39 +456,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<float2 *>(blk + i * kBlkPitch + jj) = make_float2(x0, x1);
                             const float y0 = col <= row ? aq[nt][2 * hh] * out_scale : 0.f;
                             const float y1 = col + 1 <= row ? aq[nt][2 * hh + 1] * out_scale : 0.f;
-                            *reinterpret_cast<uint32_t *>(sm + S::AQK + tc::kmaj_off(row, col)) = pack_bf16(y0, y1);
+                            aq_pk[2 * nt + hh] = pack_bf16(y0, y1);
                         }
+                }
+                bar_intra();
+                // A_qk of chunk s -> its staging tile (the k^E2 half at KR + 8192, free now); it moves to
+                // AQK at the end of the step, once the state side has finished with the previous one
+                if (warp < 10) {
+                    const int R = pair_R(warp), I = warp - R * (R + 1) / 2;
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh)
+                            *reinterpret_cast<uint32_t *>(sm + kAqs + tc::kmaj_off(16 * R + gq + 8 * hh, 16 * I + 8 * nt + 2 * tq)) =
+                                aq_pk[2 * nt + hh];
                 } else {
                     // warps 10, 11: A_qk is zero above the block diagonal
-                    const int t = tid - 320;
-                    for (int idx = t; idx < 192; idx += 64) {
+                    for (int idx = tid - 320; idx < 192; idx += 64) {
                         const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
                         const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
                         const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-                        *reinterpret_cast<uint4 *>(sm + S::AQK + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                        *reinterpret_cast<uint4 *>(sm + kAqs + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
                             make_uint4(0, 0, 0, 0);
                     }
                 }
-                bar_intra();
                 // q^E1 / k^E1 consumed: the next chunk's raw q, k
                 if (tid == 0 && have_next) {
                     tc::fence_proxy_async();
                     issue_qk(s + 1);
                 }
-                // ---- T = (I + A_kk)^-1: diagonal blocks (one column per lane); T' rows written as bf16 ----
+                // ---- T = (I + A_kk)^-1, diagonal blocks: lane = column, left-looking substitution
+                // x[r] = delta_rc - sum_{j<r} A[r][j] x[j] with the rows of A read as float4.
+                // T (fp32) is kept for the off-diagonal pass, T' = T diag(beta) is written as bf16.
                 if (warp < 4) {
                     if (lane < 16) {
                         const int R = warp, col = lane;
                         const float *blk = f_akk + pair_of(R, R) * kBlkFloats;
-                        // right-looking forward substitution: x[j] is final once the updates of
-                        // rows < j have been applied; the serial chain is one FMA per row
                         float x[16];
 #pragma unroll
-                        for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
+                        for (int r = 0; r < 16; ++r) {
+                            float acc = (r == col) ? 1.f : 0.f;
 #pragma unroll
-                        for (int j = 0; j < 15; ++j) {
-#pragma unroll
-                            for (int r = j + 1; r < 16; ++r) x[r] -= blk[r * kBlkPitch + j] * x[j];
+                            for (int j4 = 0; j4 < r; j4 += 4) {
+                                const float4 a = *reinterpret_cast<const float4 *>(blk + r * kBlkPitch + j4);
+                                acc -= a.x * x[j4];
+                                if (j4 + 1 < r) acc -= a.y * x[j4 + 1];
+                                if (j4 + 2 < r) acc -= a.z * x[j4 + 2];
+                                if (j4 + 3 < r) acc -= a.w * x[j4 + 3];
+                            }
+                            x[r] = acc;
                         }
                         float *tb = f_tm + pair_of(R, R) * kBlkFloats;
                         const float bc = f_beta[16 * R + col];
@@ -510,48 +527,73 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 bar_intra();
-                // ---- off-diagonal blocks by distance d (tf32 warp MMA), T and T' stored ----
-#pragma unroll 1
-                for (int d = 1; d < 4; ++d) {
-                    const int njobs = 2 * (4 - d);
-                    if (warp < njobs) {
-                        const int R = d + (warp >> 1), I = R - d, nt = warp & 1;
-                        float xacc[4] = {0.f, 0.f, 0.f, 0.f};
-                        for (int J = I; J < R; ++J) {
-                            const float *ab = f_akk + pair_of(R, J) * kBlkFloats;
-                            const float *tb = f_tm + pair_of(J, I) * kBlkFloats;
+                // ---- off-diagonal blocks: warp (I, nt) walks down its 16x8 column strip of T ----
+                // T_RI = -T_RR sum_{J=I}^{R-1} A_RJ T_JI (tf32 warp MMA).  The strip blocks stay in
+                // registers as B fragments (rows tq, tq+4, 8+tq, 12+tq; column gq); an accumulator
+                // becomes a B fragment by two shuffles per register.
+                if (warp < 6) {
+                    const int I = warp >> 1, nt = warp & 1;
+                    const int src_lo = 4 * tq + (gq >> 1);          // holder of rows tq (and 8+tq), column gq
+                    const int src_hi = 4 * (tq + 4) + (gq >> 1);    // holder of rows tq+4 (and 12+tq)
+                    const bool odd_col = gq & 1;
+                    auto to_bfrag = [&](const float (&c)[4], float (&b)[4], float sign) {
 #pragma unroll
-                            for (int kb = 0; kb < 16; kb += 8)
-                                mma_tf32(xacc, ab[gq * kBlkPitch + kb + tq], ab[(gq + 8) * kBlkPitch + kb + tq],
-                                         ab[gq * kBlkPitch + kb + tq + 4], ab[(gq + 8) * kBlkPitch + kb + tq + 4],
-                                         tb[(kb + tq) * kBlkPitch + 8 * nt + gq], tb[(kb + tq + 4) * kBlkPitch + 8 * nt + gq]);
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const float e0 = __shfl_sync(0xffffffffu, c[2 * ks], src_lo);
+                            const float o0 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_lo);
+                            const float e1 = __shfl_sync(0xffffffffu, c[2 * ks], src_hi);
+                            const float o1 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_hi);
+                            b[2 * ks] = sign * (odd_col ? o0 : e0);
+                            b[2 * ks + 1] = sign * (odd_col ? o1 : e1);
                         }
-                        float *xt = reinterpret_cast<float *>(sm + S::XT) + warp * 128;   // X[16][8]
-                        xt[gq * 8 + 2 * tq] = xacc[0];
-                        xt[gq * 8 + 2 * tq + 1] = xacc[1];
-                        xt[(gq + 8) * 8 + 2 * tq] = xacc[2];
-                        xt[(gq + 8) * 8 + 2 * tq + 1] = xacc[3];
-                        __syncwarp();
-                        const float *tr = f_tm + pair_of(R, R) * kBlkFloats;
-                        float tacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                        for (int kb = 0; kb < 16; kb += 8)
-                            mma_tf32(tacc, tr[gq * kBlkPitch + kb + tq], tr[(gq + 8) * kBlkPitch + kb + tq],
-                                     tr[gq * kBlkPitch + kb + tq + 4], tr[(gq + 8) * kBlkPitch + kb + tq + 4],
-                                     xt[(kb + tq) * 8 + gq], xt[(kb + tq + 4) * 8 + gq]);
-                        float *to = f_tm + pair_of(R, I) * kBlkFloats;
-                        const int cl = 8 * nt + 2 * tq;
-                        *reinterpret_cast<float2 *>(to + gq * kBlkPitch + cl) = make_float2(-tacc[0], -tacc[1]);
-                        *reinterpret_cast<float2 *>(to + (gq + 8) * kBlkPitch + cl) = make_float2(-tacc[2], -tacc[3]);
-                        const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
-                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
-                            pack_bf16(-tacc[0] * b0, -tacc[1] * b1);
-                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
-                            pack_bf16(-tacc[2] * b0, -tacc[3] * b1);
+                    };
+                    float tb[3][4];
+                    {
+                        const float *t = f_tm + pair_of(I, I) * kBlkFloats + 8 * nt + gq;
+                        tb[0][0] = t[tq * kBlkPitch];
+                        tb[0][1] = t[(tq + 4) * kBlkPitch];
+                        tb[0][2] = t[(8 + tq) * kBlkPitch];
+                        tb[0][3] = t[(12 + tq) * kBlkPitch];
                     }
-                    if (d == 3) tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
-                    bar_intra();
+                    const int cl = 8 * nt + 2 * tq;
+                    const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
+#pragma unroll
+                    for (int d = 1; d < 4; ++d) {
+                        if (I + d > 3) break;
+                        const int R = I + d;
+                        float xacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int jo = d - 1; jo >= 0; --jo) {       // the newest strip block last
+                            const float *ab = f_akk + pair_of(R, I + jo) * kBlkFloats;
+#pragma unroll
+                            for (int ks = 0; ks < 2; ++ks) {
+                                const int k0 = 8 * ks;
+                                mma_tf32(xacc, ab[gq * kBlkPitch + k0 + tq], ab[(gq + 8) * kBlkPitch + k0 + tq],
+                                         ab[gq * kBlkPitch + k0 + tq + 4], ab[(gq + 8) * kBlkPitch + k0 + tq + 4],
+                                         tb[jo][2 * ks], tb[jo][2 * ks + 1]);
+                            }
+                        }
+                        float xb[4];
+                        to_bfrag(xacc, xb, 1.f);
+                        const float *tr = f_tm + pair_of(R, R) * kBlkFloats;
+                        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const int k0 = 8 * ks;
+                            mma_tf32(y, tr[gq * kBlkPitch + k0 + tq], tr[(gq + 8) * kBlkPitch + k0 + tq],
+                                     tr[gq * kBlkPitch + k0 + tq + 4], tr[(gq + 8) * kBlkPitch + k0 + tq + 4], xb[2 * ks],
+                                     xb[2 * ks + 1]);
+                        }
+                        // T_RI = -y
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
+                            pack_bf16(-y[0] * b0, -y[1] * b1);
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
+                            pack_bf16(-y[2] * b0, -y[3] * b1);
+                        if (d < 3) to_bfrag(y, tb[d], -1.f);
+                    }
                 }
+                tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
+                bar_intra();
                 // T' is complete: the W half of the W/Q' product can start now
                 const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
                 if (tid == 0) {
@@ -561,50 +603,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_w,
                                 kk > 0);
-                }
-                // ---- A_qk T' -> bf16 rows 64-127 of A1 (warp-level MMA, warps 0-7) ----
-                if (warp < 8) {
-                    const int R = warp >> 1, nh = warp & 1;
-                    const uint32_t abase = sbase + S::AQK, tbase2 = sbase + S::KR;
-                    float acc[4][4];
-#pragma unroll
-                    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
-                    const int j = lane >> 3;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        uint32_t fa[4];
-                        ldsm_x4(abase + tc::kmaj_chunk(16 * R + (lane & 7) + 8 * (j & 1), 2 * kk + (j >> 1)), fa[0], fa[1],
-                                fa[2], fa[3]);
-#pragma unroll
-                        for (int np = 0; np < 2; ++np) {
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4_t(tbase2 + tc::kmaj_chunk(16 * kk + (lane & 7) + 8 * (j & 1), 4 * nh + 2 * np + (j >> 1)),
-                                      b0, b1, b2, b3);
-                            mma_bf16(acc[2 * np], fa, b0, b1);
-                            mma_bf16(acc[2 * np + 1], fa, b2, b3);
-                        }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int row = 64 + 16 * R + gq + 8 * hh;
-                            const int col = 32 * nh + 8 * nt + 2 * tq;
-                            *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(row, col)) =
-                                pack_bf16(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
-                        }
-                }
-                tc::fence_proxy_async();
-                tc::fence_before();
-                bar_intra();
-                // ---- tcgen05: Q' half, columns 64-127: Q~^T - (A_qk W)^T (accumulate) ----
-                if (tid == 0) {
-                    tc::fence_after();
-                    constexpr uint32_t id_wq = tc::idesc_bf16(128, 64, false, false, true);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma(tmem + dcol + 64, tc::desc_kmaj(sbase + S::KGT, kk),
-                                tc::desc_kmaj(sbase + S::KR + 8192, kk), id_wq, 1u);
                     tc::commit(mbar(kMbWQ));
                 }
                 if (tid == 0) {
@@ -641,16 +639,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_proxy_async();
                 tc::fence_before();
                 bar_intra();
-                // ---- tcgen05: D = V^T A1^T = [U^T | (A_qk U)^T] ----
+                // ---- tcgen05: D[:, 0:64] = V^T T'^T = U^T ----
                 if (tid == 0) {
                     tc::fence_after();
-                    constexpr uint32_t id_u = tc::idesc_bf16(128, 128, true, false, false);
+                    constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma(tmem + dcol, tc::desc_mnmaj(sbase + S::V, kk, 64), tc::desc_kmaj(sbase + S::KR, kk), id_u,
                                 kk > 0);
                     tc::commit(mbar(kMbU));
                 }
+                // A_qk of chunk s -> AQK, once the state side's output product of chunk s-1 has read it
+                if (tid == 0 && have_state && !tc::mbar_wait(mbar(kMbOq), (uint32_t)((s - 1) & 1), kWaitLimit))
+                    *abort_flag = 1;
+                bar_intra();
+                for (int idx = tid; idx < 512; idx += 384)
+                    *reinterpret_cast<uint4 *>(sm + S::AQK + 16 * idx) = *reinterpret_cast<const uint4 *>(sm + kAqs + 16 * idx);
+                tc::fence_proxy_async();
             }
         } else {
             // ================= state warps (12-15) =================
@@ -683,10 +688,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bar_state();
                 if (tid == kStateTid0) {
                     tc::fence_after();
-                    constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
+                    // [U~^T | (Q~ S)^T]: the first half accumulates onto U^T, the second starts fresh
+                    constexpr uint32_t id2 = tc::idesc_bf16(128, 64, false, true, false);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
+                    for (int kk = 0; kk < 8; ++kk) {
                         mma_ts(tmem + dcol, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2, kk, 128), id2, 1u);
+                        mma_ts(tmem + dcol + 64, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2 + 16384, kk, 128), id2,
+                               kk > 0 ? 1u : 0u);
+                    }
                     tc::commit(mbar(kMb2));
                 }
                 if (tid == kStateTid0) {
@@ -713,12 +722,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bar_state();
                 if (tid == kStateTid0) {
                     tc::fence_after();
+                    // O^T += U~^T A_qk^T (A_qk [r][i] is the K-major B operand), then the state update
+                    constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + dcol + 64, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::AQK, kk), id_o, 1u);
+                    tc::commit(mbar(kMbOq));
                     constexpr uint32_t id4 = tc::idesc_bf16(128, 128, false, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ts(tmem + kSF, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::KDT + nbuf * 16384, kk), id4, 1u);
                     tc::commit(mbar(kMb4));
+                    if (!tc::mbar_wait(mbar(kMbOq), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                    tc::fence_before();
                 }
+                bar_state();
+                tc::fence_after();
                 // O^T (columns 64-127; the output scale is already applied): lane v holds o[r][v].
                 // Lane pairs swap values so that each thread writes the pair (v, v+1) of one row.
                 {
@@ -804,7 +823,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (aborted) {
         if (tid == 0) atomicExch(status, kStatusTimeout);
         // let any tensor-core work or copy still in flight land before TMEM and shared memory go away
-        for (int i = 0; i < 7; ++i) {
+        for (int i = 0; i < kNumMbar; ++i) {
+            if (i == kMbO) continue;
             tc::mbar_wait(mbar(i), 0u, kWaitLimit / 16);
             tc::mbar_wait(mbar(i), 1u, kWaitLimit / 16);
         }
