@@ -91,5 +91,14 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 
 // 2^x through the SFU (CUDA's exp2f intrinsic path).
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+// 2^x by the hardware approximation (PTX ex2.approx.ftz): results below 2^-126 flush to zero,
+// which only drops decay factors that are negligible anyway (every exponent here is <= 0)
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// bf16 bit pattern -> fp32 (exact)
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 }  // namespace kda

@@ -62,18 +62,17 @@ struct Smem {
     static constexpr int KGT = 98304;      // (k^ e^Gamma)^T, K-major [c][r]
     static constexpr int KDT = 114688;     // two buffers: (k^ e^{Gamma_last-Gamma})^T, K-major [c][r]
     static constexpr int B2 = 147456;      // [-W^T | Q'^T], MN-major [c][n], two 64-wide atoms
-    static constexpr int AQK = 180224;     // A_qk [r][i], K-major (64 rows), read by the state side's O product
-    static constexpr int AKK = 188416;     // A_kk blocks fp32
+    static constexpr int AQK = 180224;     // two buffers: A_qk [r][i], K-major (64 rows), read by the state side
+    static constexpr int AKK = 196608;     // A_kk blocks fp32
     static constexpr int TM = AKK + 10 * kBlkFloats * 4;   // T blocks fp32
     static constexpr int SMALL = TM + 10 * kBlkFloats * 4;
     static constexpr int BETA = SMALL;               // fp32 [2][64]
     static constexpr int RQ = BETA + 512;            // fp32 [64]
     static constexpr int RK = RQ + 256;              // fp32 [64]
     static constexpr int TOT = RK + 256;             // fp32 [4][128]
-    static constexpr int PS = TOT + 2048;            // fp32 [10][128]
-    static constexpr int DC = PS + 5120;             // fp32 [2][128]
-    static constexpr int XT = DC + 1024;             // fp32 [6][16][8]
-    static constexpr int MBAR = XT + 3072;           // u64 [16]
+    static constexpr int PS = TOT + 2048;            // bf16 [10][128] pair scales
+    static constexpr int DC = PS + 2560;             // fp32 [2][128]
+    static constexpr int MBAR = DC + 1024;           // u64 [16]
     static constexpr int TBASE = MBAR + 128;
     static constexpr int ABORT = TBASE + 16;
     static constexpr int BYTES = ABORT + 16;
@@ -81,11 +80,12 @@ struct Smem {
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
 
-// kMbO is arrived by a thread (B2 free again); the others complete by tcgen05.commit or TMA bytes
-enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kMbO, kMbOq, kNumMbar };
+// every barrier completes by tcgen05.commit or by TMA transaction bytes
+enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kNumMbar };
 
 __device__ __forceinline__ void bar_intra() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void bar_state() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_solve() { asm volatile("bar.sync 3, 256;" ::: "memory"); }   // warps 0-7
 
 // tf32 warp MMA on fp32 bit patterns (the tensor core ignores the low mantissa bits)
 __device__ __forceinline__ void mma_tf32(float (&d)[4], float a0, float a1, float a2, float a3, float b0, float b1) {
@@ -121,13 +121,22 @@ __device__ __forceinline__ uint4 pack8(const float *x, float s) {
     return make_uint4(pack_bf16(x[0] * s, x[1] * s), pack_bf16(x[2] * s, x[3] * s), pack_bf16(x[4] * s, x[5] * s),
                       pack_bf16(x[6] * s, x[7] * s));
 }
+// eight values held as four row pairs, as bf16 (optionally scaled by a packed multiply)
+__device__ __forceinline__ uint4 pack8x2(const float2 *x) {
+    return make_uint4(pack_bf16(x[0].x, x[0].y), pack_bf16(x[1].x, x[1].y), pack_bf16(x[2].x, x[2].y),
+                      pack_bf16(x[3].x, x[3].y));
+}
+__device__ __forceinline__ uint4 pack8x2s(const float2 *x, float2 s) {
+    const float2 a = __fmul2_rn(x[0], s), b = __fmul2_rn(x[1], s), c = __fmul2_rn(x[2], s), d = __fmul2_rn(x[3], s);
+    return make_uint4(pack_bf16(a.x, a.y), pack_bf16(b.x, b.y), pack_bf16(c.x, c.y), pack_bf16(d.x, d.y));
+}
 __device__ __forceinline__ int pair_R(int p) { return p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0; }
 __device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
 
-// beta rows [tok0, tok0 + L) of head h (threads 0-63; rows >= L zero-filled)
-__device__ __forceinline__ void load_beta(uint8_t *sm, const float *beta, int64_t tok0, int L, int H, int h, int buf) {
-    if (threadIdx.x < 64) {
-        const int row = threadIdx.x;
+// beta rows [tok0, tok0 + L) of head h, one row per calling thread (row in [0, 64); rows >= L zero-filled)
+__device__ __forceinline__ void load_beta(uint8_t *sm, const float *beta, int64_t tok0, int L, int H, int h, int buf,
+                                          int row) {
+    {
         const bool ok = row < L;
         const float *src = ok ? beta + (tok0 + row) * H + h : beta;
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *f_rq = reinterpret_cast<float *>(sm + S::RQ);
     float *f_rk = reinterpret_cast<float *>(sm + S::RK);
     float *f_tot = reinterpret_cast<float *>(sm + S::TOT);
-    float *f_ps = reinterpret_cast<float *>(sm + S::PS);
+    __nv_bfloat16 *f_ps = reinterpret_cast<__nv_bfloat16 *>(sm + S::PS);
     float *f_akk = reinterpret_cast<float *>(sm + S::AKK);
     float *f_tm = reinterpret_cast<float *>(sm + S::TM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::ABORT);
@@ -245,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_qk(0);
         issue_g(0);
     }
-    load_beta(sm, beta, doc_start, chunk_len(0), H, h, 0);
+    if (tid < 64) load_beta(sm, beta, doc_start, chunk_len(0), H, h, 0, tid);
     cp_async_commit();
     tc::fence_before();
     __syncthreads();
@@ -261,8 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c0 = 0; c0 < 128; c0 += 32) tc::st32(lane_base + kSF + c0, z);
         tc::wait_st();
     }
-    // norms of chunk 0 (one thread polls the barrier; the CTA barrier releases the rest)
-    if (tid == 0 && !tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit)) *abort_flag = 1;
+    // chunk 0's inputs (one thread polls the barriers; the CTA barrier releases the rest), then its norms
+    cp_async_wait_all();
+    if (tid == 0) {
+        bool ok = tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit);
+        ok = tc::mbar_wait(mbar(kMbG), 0u, kWaitLimit) && ok;
+        if (!ok) *abort_flag = 1;
+    }
     __syncthreads();
     if (warp < 4) norms16(warp * 16, chunk_len(0));
     tc::fence_before();
@@ -281,63 +295,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = s & 1;
         const uint32_t par = (uint32_t)(s & 1);
 
-        // ---- top: beta(s), q, k and g of chunk s landed ----
-        cp_async_wait_all();
-        if (tid == 0 && have_intra) {
-            bool ok = tc::mbar_wait(mbar(kMbQK), par, kWaitLimit);
-            ok = tc::mbar_wait(mbar(kMbG), par, kWaitLimit) && ok;
-            if (!ok) *abort_flag = 1;
-        }
-        __syncthreads();
-        if (*abort_flag) { aborted = true; break; }
+        // beta(s), q, k and g of chunk s landed before the previous step's closing barrier
 
-        float ql[16], kl[16], kr[16];
-        float lg0 = 0.f, lg15 = 0.f;
+        // a partial last chunk: rows past the document end (the TMA tile reaches into the next
+        // document) are zeroed, so the prep below needs no per-element masks
+        if (have_intra && L < 64) {
+            for (int idx = tid; idx < (64 - L) * 16; idx += kThreads) {
+                const int row = L + (idx >> 4), ch = idx & 15;             // 16 chunks of 16 B per row
+                const uint32_t o = (uint32_t)row * 128u + (uint32_t)(ch & 7) * 16u;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sm + S::Q + (ch >> 3) * 8192 + o) = z;
+                *reinterpret_cast<uint4 *>(sm + S::K + (ch >> 3) * 8192 + o) = z;
+                *reinterpret_cast<uint4 *>(sm + S::G + (ch >> 3) * 16384 + o) = z;
+                *reinterpret_cast<uint4 *>(sm + S::G + (ch >> 3) * 16384 + 8192 + o) = z;
+            }
+            __syncthreads();
+        }
+        float2 ql[8], kl[8], kr[8];      // row pairs (2j, 2j+1) of this thread's 16-row block
+        float lg0 = 0.f;
         const int pc = tid & 127, pR = tid >> 7;
         if (have_intra) {
             // ---- prep pass 1: thread = (channel c, row block R) ----
             // per-row decays a_j = 2^{log2e g_j} (one exp2 each); E1 and E2 are running products
             // inside the 16-row block: E1_j = a_1..a_j, E2_j = a_{j+1}..a_15 (both in [e^-75, 1])
-            float a[16];
-            float acc = 0.f;
+            float2 a[8];
+            float gsum = 0.f;
             const uint8_t *gcol = sm + S::G + (pc >> 5) * 8192 + (pc & 31) * 4;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int r = 16 * pR + j;
-                const float gv = *reinterpret_cast<const float *>(gcol + r * 128);
-                const float gl2 = r < L ? gv * kLog2e : 0.f;      // log2-scaled gate
-                acc += gl2;
-                a[j] = fast_exp2(gl2);
-                if (j == 0) lg0 = acc;
+            for (int j2 = 0; j2 < 8; ++j2) {
+                const int r = 16 * pR + 2 * j2;
+                const float g0 = *reinterpret_cast<const float *>(gcol + r * 128);
+                const float g1 = *reinterpret_cast<const float *>(gcol + (r + 1) * 128);
+                gsum += g0;
+                gsum += g1;
+                const float2 gl2 = __fmul2_rn(make_float2(g0, g1), make_float2(kLog2e, kLog2e));   // log2-scaled
+                if (j2 == 0) lg0 = gl2.x;
+                a[j2] = make_float2(ex2_ftz(gl2.x), ex2_ftz(gl2.y));
             }
-            lg15 = acc;
-            f_tot[pR * 128 + pc] = lg15;
-            float e1[16], e2[16];
-            e1[0] = 1.f;
+            f_tot[pR * 128 + pc] = gsum * kLog2e;
+            float2 e1[8], e2[8];
+            e1[0] = make_float2(1.f, a[0].y);
 #pragma unroll
-            for (int j = 1; j < 16; ++j) e1[j] = e1[j - 1] * a[j];
-            e2[15] = 1.f;
+            for (int j2 = 1; j2 < 8; ++j2) {
+                e1[j2].x = e1[j2 - 1].y * a[j2].x;
+                e1[j2].y = e1[j2].x * a[j2].y;
+            }
+            e2[7] = make_float2(a[7].y, 1.f);
 #pragma unroll
-            for (int j = 14; j >= 0; --j) e2[j] = e2[j + 1] * a[j + 1];
+            for (int j2 = 6; j2 >= 0; --j2) {
+                e2[j2].y = e2[j2 + 1].x * a[j2 + 1].x;
+                e2[j2].x = e2[j2].y * a[j2].y;
+            }
             const uint8_t *qcol = sm + S::Q + (pc >> 6) * 8192 + (pc & 63) * 2;
             const uint8_t *kcol = sm + S::K + (pc >> 6) * 8192 + (pc & 63) * 2;
 #pragma unroll
-            for (int j4 = 0; j4 < 16; j4 += 4) {
-                const float4 rq4 = *reinterpret_cast<const float4 *>(f_rq + 16 * pR + j4);
-                const float4 rk4 = *reinterpret_cast<const float4 *>(f_rk + 16 * pR + j4);
-                const float rqv[4] = {rq4.x, rq4.y, rq4.z, rq4.w};
-                const float rkv[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
+            for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 rq4 = *reinterpret_cast<const float4 *>(f_rq + 16 * pR + 4 * j4);
+                const float4 rk4 = *reinterpret_cast<const float4 *>(f_rk + 16 * pR + 4 * j4);
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = j4 + jj, r = 16 * pR + j;
-                    float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qcol + r * 128));
-                    float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kcol + r * 128));
-                    qv = r < L ? qv : 0.f;
-                    kv = r < L ? kv : 0.f;
-                    const float qh = qv * rqv[jj], kh = kv * rkv[jj];
-                    ql[j] = qh * e1[j];
-                    kl[j] = kh * e1[j];
-                    kr[j] = kh * e2[j];
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int j2 = 2 * j4 + h2, r = 16 * pR + 2 * j2;
+                    const float2 qv = make_float2(bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(qcol + r * 128)),
+                                                  bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(qcol + (r + 1) * 128)));
+                    const float2 kv = make_float2(bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(kcol + r * 128)),
+                                                  bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(kcol + (r + 1) * 128)));
+                    const float2 qh = __fmul2_rn(qv, h2 ? make_float2(rq4.z, rq4.w) : make_float2(rq4.x, rq4.y));
+                    const float2 kh = __fmul2_rn(kv, h2 ? make_float2(rk4.z, rk4.w) : make_float2(rk4.x, rk4.y));
+                    ql[j2] = __fmul2_rn(qh, e1[j2]);
+                    kl[j2] = __fmul2_rn(kh, e1[j2]);
+                    kr[j2] = __fmul2_rn(kh, e2[j2]);
                 }
             }
         }
@@ -347,14 +373,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();   // raw q, k, g read; block sums published
         tc::fence_after();
         if (*abort_flag) { aborted = true; break; }
-        // raw g, beta(s+1) buffer are free: the next chunk's g and beta; v of chunk s
-        if (tid == 0) {
-            tc::fence_proxy_async();
-            if (have_next) issue_g(s + 1);
-            if (have_intra) issue_v(s);
-        }
-        if (have_next) load_beta(sm, beta, doc_start + 64 * (int64_t)(s + 1), nL, H, h, buf ^ 1);
-        cp_async_commit();
         if (have_intra) {
             // ---- prep pass 2 (log2-scaled Gamma) ----
             float offs[5];
@@ -364,32 +382,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float gm = offs[pR] + lg0;
             const float ge = offs[pR + 1];
             const float gl = offs[4];
-            const float P = fast_exp2(gm);
-            const float Pq = P * out_scale;          // the output scale rides on Q~ and A_qk
-            const float Dk = fast_exp2(gl - ge);
+            const float P = ex2_ftz(gm);
+            const float2 Pq = make_float2(P * out_scale, P * out_scale);   // the output scale rides on Q~ and A_qk
+            // Q~ into TMEM first (lane c, columns 64+16R..), next to -W^T of the W product
+            {
+                float qtf[16];
+#pragma unroll
+                for (int j2 = 0; j2 < 8; ++j2) {
+                    const float2 t = __fmul2_rn(ql[j2], Pq);
+                    qtf[2 * j2] = t.x;
+                    qtf[2 * j2 + 1] = t.y;
+                }
+                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
+                st16f(lane_base + dcol + 64 + 16 * pR, qtf);
+            }
+            const float2 P2 = make_float2(P, P);
+            const float Dkv = ex2_ftz(gl - ge);
+            const float2 Dk = make_float2(Dkv, Dkv);
 #pragma unroll
             for (int I = 0; I < 4; ++I)
-                if (I <= pR) f_ps[pair_of(pR, I) * 128 + pc] = fast_exp2(gm - offs[I + 1]);
-            if (pR == 0) reinterpret_cast<float *>(sm + S::DC)[buf * 128 + pc] = fast_exp2(gl);
+                if (I <= pR) f_ps[pair_of(pR, I) * 128 + pc] = __float2bfloat16_rn(ex2_ftz(gm - offs[I + 1]));
+            if (pR == 0) reinterpret_cast<float *>(sm + S::DC)[buf * 128 + pc] = ex2_ftz(gl);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const int j0 = half * 8;
+                const int j0 = half * 4;
                 const uint32_t off = tc::kmaj_chunk(pc, 2 * pR + half);
-                *reinterpret_cast<uint4 *>(sm + S::Q + off) = pack8(ql + j0, 1.f);
-                *reinterpret_cast<uint4 *>(sm + S::K + off) = pack8(kl + j0, 1.f);
-                *reinterpret_cast<uint4 *>(sm + S::KR + off) = pack8(kr + j0, 1.f);
-                *reinterpret_cast<uint4 *>(sm + S::KGT + off) = pack8(kl + j0, P);
-                *reinterpret_cast<uint4 *>(sm + S::KDT + buf * 16384 + off) = pack8(kr + j0, Dk);
+                *reinterpret_cast<uint4 *>(sm + S::Q + off) = pack8x2(ql + j0);
+                *reinterpret_cast<uint4 *>(sm + S::K + off) = pack8x2(kl + j0);
+                *reinterpret_cast<uint4 *>(sm + S::KR + off) = pack8x2(kr + j0);
+                *reinterpret_cast<uint4 *>(sm + S::KGT + off) = pack8x2s(kl + j0, P2);
+                *reinterpret_cast<uint4 *>(sm + S::KDT + buf * 16384 + off) = pack8x2s(kr + j0, Dk);
             }
-            // Q~ into TMEM (lane c, columns 64+16R..): the accumulator of the Q' product
-            {
-                float qt[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) qt[j] = ql[j] * Pq;
-                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
-                st16f(lane_base + dcol + 64 + 16 * pR, qt);
-                tc::wait_st();
-            }
+            tc::wait_st();
         }
         // operand tiles written through the generic proxy are read by the tensor core
         tc::fence_proxy_async();
@@ -402,13 +426,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (have_intra) {
                 const float *f_beta = reinterpret_cast<const float *>(sm + S::BETA + buf * 256);
                 // ---- A_kk and A_qk, one 16x16 block pair per warp ----
-                uint32_t aq_pk[4];
-                constexpr int kAqs = S::KR + 8192;
+                const int aqk = S::AQK + buf * 8192;      // A_qk(s); the other buffer holds A_qk(s-1)
                 if (warp < 10) {
                     const int p = warp;
                     const int R = pair_R(p), I = p - R * (R + 1) / 2;
                     const uint32_t kbase = sbase + S::K, qbase = sbase + S::Q, rbase = sbase + S::KR;
-                    const float *ps = f_ps + p * 128;
+                    const __nv_bfloat16 *ps = f_ps + p * 128;
                     float ak[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                     float aq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                     const int j = lane >> 3;
@@ -417,10 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const int cb = kk * 16 + 2 * tq;
-                        const float2 s0 = *reinterpret_cast<const float2 *>(ps + cb);
-                        const float2 s8 = *reinterpret_cast<const float2 *>(ps + cb + 8);
-                        hs[kk][0] = __floats2bfloat162_rn(s0.x, s0.y);
-                        hs[kk][1] = __floats2bfloat162_rn(s8.x, s8.y);
+                        hs[kk][0] = *reinterpret_cast<const __nv_bfloat162 *>(ps + cb);
+                        hs[kk][1] = *reinterpret_cast<const __nv_bfloat162 *>(ps + cb + 8);
                     }
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -456,160 +477,168 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<float2 *>(blk + i * kBlkPitch + jj) = make_float2(x0, x1);
                             const float y0 = col <= row ? aq[nt][2 * hh] * out_scale : 0.f;
                             const float y1 = col + 1 <= row ? aq[nt][2 * hh + 1] * out_scale : 0.f;
-                            aq_pk[2 * nt + hh] = pack_bf16(y0, y1);
+                            *reinterpret_cast<uint32_t *>(sm + aqk + tc::kmaj_off(row, col)) = pack_bf16(y0, y1);
                         }
-                }
-                bar_intra();
-                // A_qk of chunk s -> its staging tile (the k^E2 half at KR + 8192, free now); it moves to
-                // AQK at the end of the step, once the state side has finished with the previous one
-                if (warp < 10) {
-                    const int R = pair_R(warp), I = warp - R * (R + 1) / 2;
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh)
-                            *reinterpret_cast<uint32_t *>(sm + kAqs + tc::kmaj_off(16 * R + gq + 8 * hh, 16 * I + 8 * nt + 2 * tq)) =
-                                aq_pk[2 * nt + hh];
                 } else {
-                    // warps 10, 11: A_qk is zero above the block diagonal
+                    // warps 10-11 have no A_kk block: raw g and the beta(s+1) buffer are free (prep pass 1
+                    // is done) and so is V (the previous U product is done): the next chunk's g and
+                    // beta, this chunk's v
+                    if (tid == 320) {
+                        tc::fence_proxy_async();
+                        if (have_next) issue_g(s + 1);
+                        issue_v(s);
+                    }
+                    if (have_next) load_beta(sm, beta, doc_start + 64 * (int64_t)(s + 1), nL, H, h, buf ^ 1, tid - 320);
+                    cp_async_commit();
+                    // A_qk is zero above the block diagonal
                     for (int idx = tid - 320; idx < 192; idx += 64) {
                         const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
                         const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
                         const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-                        *reinterpret_cast<uint4 *>(sm + kAqs + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                        *reinterpret_cast<uint4 *>(sm + aqk + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
                             make_uint4(0, 0, 0, 0);
                     }
                 }
+                bar_intra();
                 // q^E1 / k^E1 consumed: the next chunk's raw q, k
-                if (tid == 0 && have_next) {
+                if (tid == 320 && have_next) {
                     tc::fence_proxy_async();
                     issue_qk(s + 1);
                 }
-                // ---- T = (I + A_kk)^-1, diagonal blocks: lane = column, left-looking substitution
-                // x[r] = delta_rc - sum_{j<r} A[r][j] x[j] with the rows of A read as float4.
-                // T (fp32) is kept for the off-diagonal pass, T' = T diag(beta) is written as bf16.
-                if (warp < 4) {
-                    if (lane < 16) {
-                        const int R = warp, col = lane;
-                        const float *blk = f_akk + pair_of(R, R) * kBlkFloats;
-                        float x[16];
-#pragma unroll
-                        for (int r = 0; r < 16; ++r) {
-                            float acc = (r == col) ? 1.f : 0.f;
-#pragma unroll
-                            for (int j4 = 0; j4 < r; j4 += 4) {
-                                const float4 a = *reinterpret_cast<const float4 *>(blk + r * kBlkPitch + j4);
-                                acc -= a.x * x[j4];
-                                if (j4 + 1 < r) acc -= a.y * x[j4 + 1];
-                                if (j4 + 2 < r) acc -= a.z * x[j4 + 2];
-                                if (j4 + 3 < r) acc -= a.w * x[j4 + 3];
-                            }
-                            x[r] = acc;
-                        }
-                        float *tb = f_tm + pair_of(R, R) * kBlkFloats;
-                        const float bc = f_beta[16 * R + col];
-#pragma unroll
-                        for (int r = 0; r < 16; ++r) {
-                            tb[r * kBlkPitch + col] = x[r];
-                            const __nv_bfloat16 t1 = __float2bfloat16_rn(x[r] * bc);
-                            *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
-                        }
+                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
+                // warps 8-11: row norms of chunk s+1 while warps 0-7 solve for T (they rejoin at the
+                // barrier before the W readback)
+                if (warp >= 8) {
+                    if (have_next) {
+                        if (lane == 0 && !tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit)) *abort_flag = 1;
+                        __syncwarp();
+                        norms16((warp - 8) * 16, nL);
                     }
                 } else {
-                    // T' is zero above the block diagonal (warps 4-11)
-                    const int t = tid - 128;
-                    for (int idx = t; idx < 192; idx += 256) {
-                        const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
-                        const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
-                        const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-                        *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                }
-                bar_intra();
-                // ---- off-diagonal blocks: warp (I, nt) walks down its 16x8 column strip of T ----
-                // T_RI = -T_RR sum_{J=I}^{R-1} A_RJ T_JI (tf32 warp MMA).  The strip blocks stay in
-                // registers as B fragments (rows tq, tq+4, 8+tq, 12+tq; column gq); an accumulator
-                // becomes a B fragment by two shuffles per register.
-                if (warp < 6) {
-                    const int I = warp >> 1, nt = warp & 1;
-                    const int src_lo = 4 * tq + (gq >> 1);          // holder of rows tq (and 8+tq), column gq
-                    const int src_hi = 4 * (tq + 4) + (gq >> 1);    // holder of rows tq+4 (and 12+tq)
-                    const bool odd_col = gq & 1;
-                    auto to_bfrag = [&](const float (&c)[4], float (&b)[4], float sign) {
-#pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {
-                            const float e0 = __shfl_sync(0xffffffffu, c[2 * ks], src_lo);
-                            const float o0 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_lo);
-                            const float e1 = __shfl_sync(0xffffffffu, c[2 * ks], src_hi);
-                            const float o1 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_hi);
-                            b[2 * ks] = sign * (odd_col ? o0 : e0);
-                            b[2 * ks + 1] = sign * (odd_col ? o1 : e1);
-                        }
-                    };
-                    float tb[3][4];
-                    {
-                        const float *t = f_tm + pair_of(I, I) * kBlkFloats + 8 * nt + gq;
-                        tb[0][0] = t[tq * kBlkPitch];
-                        tb[0][1] = t[(tq + 4) * kBlkPitch];
-                        tb[0][2] = t[(8 + tq) * kBlkPitch];
-                        tb[0][3] = t[(12 + tq) * kBlkPitch];
-                    }
-                    const int cl = 8 * nt + 2 * tq;
-                    const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
-#pragma unroll
-                    for (int d = 1; d < 4; ++d) {
-                        if (I + d > 3) break;
-                        const int R = I + d;
-                        float xacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                        for (int jo = d - 1; jo >= 0; --jo) {       // the newest strip block last
-                            const float *ab = f_akk + pair_of(R, I + jo) * kBlkFloats;
-#pragma unroll
-                            for (int ks = 0; ks < 2; ++ks) {
-                                const int k0 = 8 * ks;
-                                mma_tf32(xacc, ab[gq * kBlkPitch + k0 + tq], ab[(gq + 8) * kBlkPitch + k0 + tq],
-                                         ab[gq * kBlkPitch + k0 + tq + 4], ab[(gq + 8) * kBlkPitch + k0 + tq + 4],
-                                         tb[jo][2 * ks], tb[jo][2 * ks + 1]);
+                    // ---- T = (I + A_kk)^-1, diagonal blocks: lane = column, left-looking substitution
+                    // x[r] = delta_rc - sum_{j<r} A[r][j] x[j] with the rows of A read as float4.
+                    // T (fp32) is kept for the off-diagonal pass, T' = T diag(beta) is written as bf16.
+                    if (warp < 4) {
+                        if (lane < 16) {
+                            const int R = warp, col = lane;
+                            const float *blk = f_akk + pair_of(R, R) * kBlkFloats;
+                            float x[16];
+    #pragma unroll
+                            for (int r = 0; r < 16; ++r) {
+                                float acc = (r == col) ? 1.f : 0.f;
+    #pragma unroll
+                                for (int j4 = 0; j4 < r; j4 += 4) {
+                                    const float4 a = *reinterpret_cast<const float4 *>(blk + r * kBlkPitch + j4);
+                                    acc -= a.x * x[j4];
+                                    if (j4 + 1 < r) acc -= a.y * x[j4 + 1];
+                                    if (j4 + 2 < r) acc -= a.z * x[j4 + 2];
+                                    if (j4 + 3 < r) acc -= a.w * x[j4 + 3];
+                                }
+                                x[r] = acc;
+                            }
+                            float *tb = f_tm + pair_of(R, R) * kBlkFloats;
+                            const float bc = f_beta[16 * R + col];
+    #pragma unroll
+                            for (int r = 0; r < 16; ++r) {
+                                tb[r * kBlkPitch + col] = x[r];
+                                const __nv_bfloat16 t1 = __float2bfloat16_rn(x[r] * bc);
+                                *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
                             }
                         }
-                        float xb[4];
-                        to_bfrag(xacc, xb, 1.f);
-                        const float *tr = f_tm + pair_of(R, R) * kBlkFloats;
-                        float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {
-                            const int k0 = 8 * ks;
-                            mma_tf32(y, tr[gq * kBlkPitch + k0 + tq], tr[(gq + 8) * kBlkPitch + k0 + tq],
-                                     tr[gq * kBlkPitch + k0 + tq + 4], tr[(gq + 8) * kBlkPitch + k0 + tq + 4], xb[2 * ks],
-                                     xb[2 * ks + 1]);
+                    } else {
+                        // T' is zero above the block diagonal (warps 4-7)
+                        const int t = tid - 128;
+                        for (int idx = t; idx < 192; idx += 128) {
+                            const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
+                            const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
+                            const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
+                            *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                                make_uint4(0, 0, 0, 0);
                         }
-                        // T_RI = -y
-                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
-                            pack_bf16(-y[0] * b0, -y[1] * b1);
-                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
-                            pack_bf16(-y[2] * b0, -y[3] * b1);
-                        if (d < 3) to_bfrag(y, tb[d], -1.f);
                     }
-                }
-                tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
-                bar_intra();
-                // T' is complete: the W half of the W/Q' product can start now
-                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
-                if (tid == 0) {
-                    tc::fence_after();
-                    constexpr uint32_t id_w = tc::idesc_bf16(128, 64, false, false, true);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_w,
-                                kk > 0);
-                    tc::commit(mbar(kMbWQ));
-                }
+                    bar_solve();
+                    // ---- off-diagonal blocks: warp (I, nt) walks down its 16x8 column strip of T ----
+                    // T_RI = -T_RR sum_{J=I}^{R-1} A_RJ T_JI (tf32 warp MMA).  The strip blocks stay in
+                    // registers as B fragments (rows tq, tq+4, 8+tq, 12+tq; column gq); an accumulator
+                    // becomes a B fragment by two shuffles per register.
+                    if (warp < 6) {
+                        const int I = warp >> 1, nt = warp & 1;
+                        const int src_lo = 4 * tq + (gq >> 1);          // holder of rows tq (and 8+tq), column gq
+                        const int src_hi = 4 * (tq + 4) + (gq >> 1);    // holder of rows tq+4 (and 12+tq)
+                        const bool odd_col = gq & 1;
+                        auto to_bfrag = [&](const float (&c)[4], float (&b)[4], float sign) {
+    #pragma unroll
+                            for (int ks = 0; ks < 2; ++ks) {
+                                const float e0 = __shfl_sync(0xffffffffu, c[2 * ks], src_lo);
+                                const float o0 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_lo);
+                                const float e1 = __shfl_sync(0xffffffffu, c[2 * ks], src_hi);
+                                const float o1 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_hi);
+                                b[2 * ks] = sign * (odd_col ? o0 : e0);
+                                b[2 * ks + 1] = sign * (odd_col ? o1 : e1);
+                            }
+                        };
+                        float tb[3][4];
+                        {
+                            const float *t = f_tm + pair_of(I, I) * kBlkFloats + 8 * nt + gq;
+                            tb[0][0] = t[tq * kBlkPitch];
+                            tb[0][1] = t[(tq + 4) * kBlkPitch];
+                            tb[0][2] = t[(8 + tq) * kBlkPitch];
+                            tb[0][3] = t[(12 + tq) * kBlkPitch];
+                        }
+                        const int cl = 8 * nt + 2 * tq;
+                        const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
+    #pragma unroll
+                        for (int d = 1; d < 4; ++d) {
+                            if (I + d > 3) break;
+                            const int R = I + d;
+                            float xacc[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                            for (int jo = d - 1; jo >= 0; --jo) {       // the newest strip block last
+                                const float *ab = f_akk + pair_of(R, I + jo) * kBlkFloats;
+    #pragma unroll
+                                for (int ks = 0; ks < 2; ++ks) {
+                                    const int k0 = 8 * ks;
+                                    mma_tf32(xacc, ab[gq * kBlkPitch + k0 + tq], ab[(gq + 8) * kBlkPitch + k0 + tq],
+                                             ab[gq * kBlkPitch + k0 + tq + 4], ab[(gq + 8) * kBlkPitch + k0 + tq + 4],
+                                             tb[jo][2 * ks], tb[jo][2 * ks + 1]);
+                                }
+                            }
+                            float xb[4];
+                            to_bfrag(xacc, xb, 1.f);
+                            const float *tr = f_tm + pair_of(R, R) * kBlkFloats;
+                            float y[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                            for (int ks = 0; ks < 2; ++ks) {
+                                const int k0 = 8 * ks;
+                                mma_tf32(y, tr[gq * kBlkPitch + k0 + tq], tr[(gq + 8) * kBlkPitch + k0 + tq],
+                                         tr[gq * kBlkPitch + k0 + tq + 4], tr[(gq + 8) * kBlkPitch + k0 + tq + 4], xb[2 * ks],
+                                         xb[2 * ks + 1]);
+                            }
+                            // T_RI = -y
+                            *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
+                                pack_bf16(-y[0] * b0, -y[1] * b1);
+                            *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
+                                pack_bf16(-y[2] * b0, -y[3] * b1);
+                            if (d < 3) to_bfrag(y, tb[d], -1.f);
+                        }
+                    }
+                    tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
+                    bar_solve();
+                    // T' is complete: the W product can start now
+                    if (tid == 0) {
+                        tc::fence_after();
+                        constexpr uint32_t id_w = tc::idesc_bf16(128, 64, false, false, true);
+    #pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma(tmem + dcol, tc::desc_kmaj(sbase + S::KGT, kk), tc::desc_kmaj(sbase + S::KR, kk), id_w,
+                                    kk > 0);
+                        tc::commit(mbar(kMbWQ));
+                    }
+                }   // warps 0-7
                 if (tid == 0) {
                     bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
-                    // B2 is free once the previous chunk's state product has read it and its
-                    // output tile, staged there, has been read by the TMA store
-                    if (have_state) ok = tc::mbar_wait(mbar(kMbO), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
+                    // B2 is free once the previous chunk's state product has read it
+                    if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
                     ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
                     if (!ok) *abort_flag = 1;
                     tc::fence_before();
@@ -649,14 +678,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 kk > 0);
                     tc::commit(mbar(kMbU));
                 }
-                // A_qk of chunk s -> AQK, once the state side's output product of chunk s-1 has read it
-                if (tid == 0 && have_state && !tc::mbar_wait(mbar(kMbOq), (uint32_t)((s - 1) & 1), kWaitLimit))
-                    *abort_flag = 1;
-                bar_intra();
-                for (int idx = tid; idx < 512; idx += 384)
-                    *reinterpret_cast<uint4 *>(sm + S::AQK + 16 * idx) = *reinterpret_cast<const uint4 *>(sm + kAqs + 16 * idx);
-                tc::fence_proxy_async();
             }
+            // the beta rows of chunk s+1 (issued by warps 10-11) have landed before the step ends
+            cp_async_wait_all();
         } else {
             // ================= state warps (12-15) =================
             if (have_state) {
@@ -667,11 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
                 const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
                 // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_last})
-#pragma unroll 1
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    float sv[32];
-                    tc::ld32(lane_base + kSF + c0, sv);
-                    tc::wait_ld();
+                auto sprep = [&](float (&sv)[32], int c0) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
@@ -679,9 +699,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
                         const float4 d4 = *reinterpret_cast<const float4 *>(dc + c0 + i);
-                        sv[i] *= d4.x; sv[i + 1] *= d4.y; sv[i + 2] *= d4.z; sv[i + 3] *= d4.w;
+                        const float2 x = __fmul2_rn(make_float2(sv[i], sv[i + 1]), make_float2(d4.x, d4.y));
+                        const float2 y = __fmul2_rn(make_float2(sv[i + 2], sv[i + 3]), make_float2(d4.z, d4.w));
+                        sv[i] = x.x; sv[i + 1] = x.y; sv[i + 2] = y.x; sv[i + 3] = y.y;
                     }
                     tc::st32(lane_base + kSF + c0, sv);
+                };
+#pragma unroll 1
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    float sv[32];
+                    tc::ld32(lane_base + kSF + c0, sv);
+                    tc::wait_ld();
+                    sprep(sv, c0);
                 }
                 tc::wait_st();
                 tc::fence_before();
@@ -726,14 +755,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + dcol + 64, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::AQK, kk), id_o, 1u);
-                    tc::commit(mbar(kMbOq));
+                        mma_ts(tmem + dcol + 64, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::AQK + nbuf * 8192, kk), id_o,
+                               1u);
                     constexpr uint32_t id4 = tc::idesc_bf16(128, 128, false, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ts(tmem + kSF, tmem + kUB + 8 * kk, tc::desc_kmaj(sbase + S::KDT + nbuf * 16384, kk), id4, 1u);
                     tc::commit(mbar(kMb4));
-                    if (!tc::mbar_wait(mbar(kMbOq), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                    // the output tile is staged in Kd's buffer, which the state update reads
+                    if (!tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
                     tc::fence_before();
                 }
                 bar_state();
@@ -744,11 +774,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int vcol = 32 * lq + lane;
                     const bool odd = lane & 1;
                     if (pL == 64) {
-                        // whole chunk: stage o[r][v] as bf16 in B2 (two 64-channel boxes, 128-B swizzled
-                        // rows) and write it with one TMA store per box.  Even lanes take rows with
+                        // whole chunk: stage o[r][v] as bf16 in Kd's buffer (free now, rewritten only by the
+                        // next step's prep; two 64-channel boxes, 128-B swizzled rows) and write it with one
+                        // TMA store per box.  Even lanes take rows with
                         // (r & 4) == 0, odd lanes the row 4 below, so one store instruction covers 32 banks.
                         const uint32_t vb = (uint32_t)(vcol & 62) * 2;          // byte of the pair in its row
-                        uint8_t *stage = sm + S::B2 + (vcol >> 6) * 8192;
+                        const uint32_t stage_off = S::KDT + (uint32_t)nbuf * 16384u;
+                        uint8_t *stage = sm + stage_off + (vcol >> 6) * 8192;
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
                             float o[32];
@@ -769,16 +801,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::fence_proxy_async();
                         bar_state();
                         if (tid == kStateTid0) {
-                            tc::tma_store_2d(&maps.o, xq, (int)ptok0, sbase + S::B2);
-                            tc::tma_store_2d(&maps.o, xq + 64, (int)ptok0, sbase + S::B2 + 8192);
+                            tc::tma_store_2d(&maps.o, xq, (int)ptok0, sbase + stage_off);
+                            tc::tma_store_2d(&maps.o, xq + 64, (int)ptok0, sbase + stage_off + 8192);
                             tc::bulk_commit();
-                            tc::bulk_wait_read();
-                            tc::mbar_arrive(mbar(kMbO));
+                            tc::bulk_wait_read();   // the staging buffer is read before the step ends
                         }
                     } else {
                         // partial chunk: rows past the document end belong to the next document, so
                         // store the valid rows directly
-                        if (tid == kStateTid0) tc::mbar_arrive(mbar(kMbO));
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
                             float o[32];
@@ -801,14 +831,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (tid == kStateTid0 && !tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
             }
-            // ---- row norms of chunk s+1 (its raw q, k arrive after this step's A_kk) ----
-            if (have_next) {
-                if (tid == kStateTid0 && !tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit))
-                    *abort_flag = 1;
-                bar_state();
-                norms16((warp - 12) * 16, nL);
+            // the raw q, k and g of chunk s+1 have landed before the step ends
+            if (tid == kStateTid0 && have_next) {
+                bool ok = tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit);
+                ok = tc::mbar_wait(mbar(kMbG), (uint32_t)((s + 1) & 1), kWaitLimit) && ok;
+                if (!ok) *abort_flag = 1;
             }
         }
         tc::fence_before();
@@ -824,7 +852,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) atomicExch(status, kStatusTimeout);
         // let any tensor-core work or copy still in flight land before TMEM and shared memory go away
         for (int i = 0; i < kNumMbar; ++i) {
-            if (i == kMbO) continue;
             tc::mbar_wait(mbar(i), 0u, kWaitLimit / 16);
             tc::mbar_wait(mbar(i), 1u, kWaitLimit / 16);
         }
