@@ -3,6 +3,7 @@
 The compute lives in libkda.so (CUDA, C ABI in include/kda.h); this package
 only marshals torch tensors into that ABI.
 """
-from ._lib import KdaError, device_status, kda_chunk_fwd, lib, wait_selftest
+from ._lib import KdaError, bwd_workspace_bytes, device_status, kda_chunk_bwd, kda_chunk_fwd, lib, wait_selftest
 
-__all__ = ["kda_chunk_fwd", "device_status", "wait_selftest", "KdaError", "lib"]
+__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "bwd_workspace_bytes", "device_status", "wait_selftest", "KdaError",
+           "lib"]

@@ -42,6 +42,11 @@ def lib() -> ctypes.CDLL:
         L.kda_device_status.argtypes = [vp]
         L.kda_wait_selftest.restype = i32
         L.kda_wait_selftest.argtypes = [vp]
+        L.kda_chunk_bwd_workspace_size.restype = ctypes.c_size_t
+        L.kda_chunk_bwd_workspace_size.argtypes = [i32, i64, i32]
+        L.kda_chunk_bwd.restype = i32
+        L.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp,
+                                    ctypes.c_size_t, vp]
         L.kda_abi_version.restype = i32
         L.kda_abi_version.argtypes = []
         _lib = L
@@ -90,6 +95,42 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                              cu_seqlens.numel() - 1, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
     return out
+
+
+def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                  cu_seqlens: torch.Tensor, dout: torch.Tensor, workspace: torch.Tensor | None = None,
+                  stream: torch.cuda.Stream | None = None):
+    """Recompute backward through libkda's kda_chunk_bwd.
+
+    Same inputs as ``kda_chunk_fwd`` plus dout [T, H, 128] bf16.  Returns (dq, dk, dv, dg, dbeta):
+    bf16 [T, H, 128] x3, fp32 [T, H, 128], fp32 [T, H].  ``workspace`` (a CUDA uint8 tensor of at
+    least ``bwd_workspace_bytes`` bytes) is allocated by torch when not given.
+    """
+    T, H, D = q.shape
+    for name, t, dt, shape in (("q", q, torch.bfloat16, (T, H, D)), ("k", k, torch.bfloat16, (T, H, D)),
+                               ("v", v, torch.bfloat16, (T, H, D)), ("g", g, torch.float32, (T, H, D)),
+                               ("beta", beta, torch.float32, (T, H)), ("dout", dout, torch.bfloat16, (T, H, D))):
+        if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or not t.is_cuda:
+            raise KdaError(1, f"{name} must be a contiguous CUDA {dt} tensor of shape {shape} "
+                              f"(got {t.dtype} {tuple(t.shape)})")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise KdaError(1, "cu_seqlens must be a 1-d int32 CUDA tensor")
+    n_docs = cu_seqlens.numel() - 1
+    need = bwd_workspace_bytes(n_docs, T, H)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg, dbeta = torch.empty_like(g), torch.empty_like(beta)
+    rc = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
+                             _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_handle(stream)))
+    _check(rc)
+    return dq, dk, dv, dg, dbeta
+
+
+def bwd_workspace_bytes(n_docs: int, T: int, H: int) -> int:
+    """Device workspace bytes kda_chunk_bwd needs (kda_chunk_bwd_workspace_size)."""
+    return int(lib().kda_chunk_bwd_workspace_size(n_docs, T, H))
 
 
 def wait_selftest(stream: torch.cuda.Stream | None = None) -> None:

@@ -117,6 +117,60 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return KDA_OK;
 }
 
+size_t kda_chunk_bwd_workspace_size(int n_docs, int64_t T, int H) {
+    if (n_docs < 1 || H < 1 || T < 0) return 0;
+    return kda::bwd_workspace_floats(n_docs, T, H) * sizeof(float);
+}
+
+kda_status kda_chunk_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                         const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                         const uint16_t *dout, uint16_t *dq, uint16_t *dk, uint16_t *dv, float *dg,
+                         float *dbeta, void *workspace, size_t workspace_bytes, void *stream) {
+    g_err[0] = '\0';
+    if (n_docs < 1) return fail(KDA_ERR_INVALID_ARG, "n_docs must be >= 1 (got %d)", n_docs);
+    if (H < 1) return fail(KDA_ERR_INVALID_ARG, "H must be >= 1 (got %d)", H);
+    if (T < 0) return fail(KDA_ERR_INVALID_ARG, "T must be >= 0 (got %lld)", (long long)T);
+    if (T > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "T must fit int32 (cu_seqlens is int32)");
+    if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if (T == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
+        return fail(KDA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(dg, 16))
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, dout, dq, dk, dv and dg must be 16-byte aligned");
+    if (!aligned(beta, 4) || !aligned(cu_seqlens, 4) || !aligned(dbeta, 4))
+        return fail(KDA_ERR_INVALID_ARG, "beta, dbeta and cu_seqlens must be 4-byte aligned");
+    if (!workspace || !aligned(workspace, 16))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be a 16-byte aligned device buffer");
+    const size_t need = kda_chunk_bwd_workspace_size(n_docs, T, H);
+    if (workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+    const size_t nel = (size_t)T * (size_t)H * KDA_HEAD_DIM;
+    const void *ins[7] = {q, k, v, dout, g, beta, workspace};
+    const size_t insz[7] = {nel * 2, nel * 2, nel * 2, nel * 2, nel * 4, (size_t)T * H * 4, need};
+    const void *outs[5] = {dq, dk, dv, dg, dbeta};
+    const size_t outsz[5] = {nel * 2, nel * 2, nel * 2, nel * 4, (size_t)T * H * 4};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 7; ++j)
+            if (overlaps(outs[i], outsz[i], ins[j], insz[j]))
+                return fail(KDA_ERR_INVALID_ARG, "gradient outputs must not alias an input or the workspace");
+        for (int j = i + 1; j < 5; ++j)
+            if (overlaps(outs[i], outsz[i], outs[j], outsz[j]))
+                return fail(KDA_ERR_INVALID_ARG, "gradient outputs must not alias each other");
+    }
+    if ((int64_t)n_docs * H > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large");
+    int dev = -1;
+    kda_status s = check_device(&dev);
+    if (s != KDA_OK) return s;
+    int *status = nullptr;
+    s = status_ptr(dev, &status);
+    if (s != KDA_OK) return s;
+    cudaError_t e = kda::launch_bwd(q, k, v, g, beta, cu_seqlens, n_docs, T, H, dout, dq, dk, dv, dg, dbeta,
+                                    static_cast<float *>(workspace), status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+    return KDA_OK;
+}
+
 kda_status kda_wait_selftest(void *stream) {
     g_err[0] = '\0';
     int dev = -1;

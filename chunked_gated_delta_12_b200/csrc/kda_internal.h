@@ -22,6 +22,15 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
                             uint16_t *out, int *status, cudaStream_t stream);
 
+// Recompute backward: dq, dk, dv (bf16), dg, dbeta (fp32) from the forward inputs and dout.
+// workspace holds bwd_workspace_floats(n_docs, T, H) floats (entering states of every chunk
+// and per-chain scratch).
+size_t bwd_workspace_floats(int n_docs, int64_t T, int H);
+cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g, const float *beta,
+                       const int32_t *cu, int n_docs, int64_t T, int H, const uint16_t *dout, uint16_t *dq,
+                       uint16_t *dk, uint16_t *dv, float *dg, float *dbeta, float *workspace, int *status,
+                       cudaStream_t stream);
+
 // Runs one time-limited mbarrier wait that can never complete (self-test of the
 // timeout path): records kStatusTimeout in *status after about limit_cycles.
 cudaError_t launch_wait_selftest(int *status, long long limit_cycles, cudaStream_t stream);

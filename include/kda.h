@@ -22,6 +22,7 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -76,6 +77,40 @@ typedef enum {
 kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          const float *g, const float *beta, const int32_t *cu_seqlens,
                          int n_docs, int64_t T, int H, uint16_t *out, void *stream);
+
+/*
+ * kda_chunk_bwd_workspace_size -- bytes of device workspace kda_chunk_bwd needs for a call
+ * with these sizes (an upper bound that does not depend on the cu_seqlens content).
+ */
+size_t kda_chunk_bwd_workspace_size(int n_docs, int64_t T, int H);
+
+/*
+ * kda_chunk_bwd -- recompute-from-inputs backward of kda_chunk_fwd.
+ *
+ * Operation: the gradients of L = sum(dout * o), o = KDA(q, k, v, g, beta) per document as in
+ * kda_chunk_fwd, with respect to the raw (un-normalised) q and k, to v, g and beta.  This is the
+ * backward of fused_chunk_kda on the kda_fused page: nothing is saved by the forward, every
+ * intermediate is recomputed from the inputs.  Evaluated chunk-wise in exact algebra (64-token
+ * chunks from each document start); equal to the reverse-mode derivative of the token
+ * recurrence up to rounding.
+ *
+ * Arguments (DEVICE memory, C-contiguous):
+ *   q, k, v, g, beta, cu_seqlens, n_docs, T, H   exactly as for kda_chunk_fwd
+ *   dout       [T, H, 128] bf16 (uint16 bit patterns): the upstream gradient of o
+ *   dq, dk, dv [T, H, 128] bf16 outputs; dg [T, H, 128] fp32; dbeta [T, H] fp32.  Every row in
+ *              [0, T) is written.  Outputs must not alias an input or each other.
+ *   workspace  device buffer of at least kda_chunk_bwd_workspace_size(n_docs, T, H) bytes,
+ *              16-byte aligned, owned by the caller; its content on entry is ignored and on
+ *              return is unspecified (it holds the state entering every chunk and per-chain
+ *              scratch).  libkda allocates no memory of its own.
+ *   stream     cudaStream_t (NULL = legacy default stream); the call is asynchronous
+ *
+ * Errors: as kda_chunk_fwd; a workspace smaller than required is KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_chunk_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                         const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                         const uint16_t *dout, uint16_t *dq, uint16_t *dk, uint16_t *dv, float *dg,
+                         float *dbeta, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Thread-local description of the first violated condition of the last failing call. */
 const char *kda_last_error(void);

@@ -19,6 +19,8 @@ def to_device(d: dict):
     t["g"] = torch.from_numpy(np.ascontiguousarray(d["g"])).to(dev)
     t["beta"] = torch.from_numpy(np.ascontiguousarray(d["beta"])).to(dev)
     t["cu_seqlens"] = torch.from_numpy(np.ascontiguousarray(d["cu_seqlens"], dtype=np.int32)).to(dev)
+    if "do" in d:
+        t["do"] = torch.from_numpy(np.ascontiguousarray(d["do"]).view(np.int16)).view(torch.bfloat16).to(dev)
     return t
 
 
@@ -60,3 +62,26 @@ def compare(got: np.ndarray, ref: np.ndarray, cu, H, chains=None) -> tuple[float
         den += float((b ** 2).sum())
         mx = max(mx, float(np.abs(a - b).max()))
     return (num ** 0.5) / max(den ** 0.5, 1e-300), mx
+
+
+def oracle_grads(d: dict, chains=None) -> dict:
+    """fp64 reverse-mode gradients of the oracle on the exact input values of `d`."""
+    f = lambda key: bf16_bits_to_f32(d[key]).reshape(d[key].shape)
+    return oracle.kda_bwd(f("q"), f("k"), f("v"), d["g"], d["beta"], f("do"), d["cu_seqlens"], chains=chains)
+
+
+def compare_grad(got: np.ndarray, ref: np.ndarray, cu, H, chains=None) -> tuple[float, float]:
+    """rel-L2 error and max-abs error relative to max |ref|, over the rows of `chains`."""
+    if chains is None:
+        chains = range((len(cu) - 1) * H)
+    num = den = mx = top = 0.0
+    for s, e, h in chain_slices(cu, H, chains):
+        if e == s:
+            continue
+        a, b = got[s:e, h], ref[s:e, h]
+        assert np.isfinite(a).all(), "non-finite gradient"
+        num += float(((a - b) ** 2).sum())
+        den += float((b ** 2).sum())
+        mx = max(mx, float(np.abs(a - b).max()))
+        top = max(top, float(np.abs(b).max()))
+    return (num / den) ** 0.5 if den > 0 else num ** 0.5, mx / top if top > 0 else mx
