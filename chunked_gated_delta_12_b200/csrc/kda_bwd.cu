@@ -48,8 +48,9 @@ struct Ws {
                             KG = EG + CD, QG = KG + CD, KD = QG + CD, BK = KD + CD, BV = BK + CD, W = BV + CD,
                             U = W + CD, UT = U + CD, DUT = UT + CD, DQG = DUT + CD, DKD = DQG + CD, DW = DKD + CD,
                             DBK = DW + CD, DBV = DBK + CD, DKN = DBV + CD, DQN = DKN + CD, DG = DQN + CD,
-                            X1 = DG + CD, Y1 = X1 + CD, Q1 = Y1 + CD, E1 = Q1 + CD, E2 = E1 + CD;
-    static constexpr size_t TM = E2 + CD, AH = TM + CC, AQ = AH + CC, DT = AQ + CC, XM = DT + CC, DAH = XM + CC,
+                            X1 = DG + CD, Y1 = X1 + CD, Q1 = Y1 + CD, E1 = Q1 + CD, E2 = E1 + CD,
+                            A24 = E2 + CD;
+    static constexpr size_t TM = A24 + CD, AH = TM + CC, AQ = AH + CC, DT = AQ + CC, XM = DT + CC, DAH = XM + CC,
                             DAQ = DAH + CC;
     static constexpr size_t SP = DAQ + CC;    // pair scales [10][128]
     static constexpr size_t RQ = SP + 10 * D, RK = RQ + C, BB = RK + C, DB = BB + C, DL = DB + C, DGL = DL + D;
@@ -72,21 +73,41 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// C(M x N) = alpha * op(A) op(B) + (accumulate ? C : 0), CTA-wide.  op(A)(i, k) = A[i*ar + k*ac],
-// op(B)(k, j) = B[k*br + j*bc], C(i, j) = Cm[i*ldc + j].  M % 16 == N % 8 == K % 8 == 0.  Each
-// warp owns 16x8 output tiles; both operands are split into tf32 hi + lo parts and the tile is
-// accumulated as hi*hi + hi*lo + lo*hi.  Ends with a CTA barrier.
-__device__ void gemm(int M, int N, int K, float alpha, const float *A, int ar, int ac, const float *B, int br,
-                     int bc, bool accumulate, float *Cm, int ldc) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+// shared-memory operand buffers of gemm: two matrices of up to 128 rows, rows padded by 8 floats
+// (with that pitch the fragment reads of both layouts hit 32 distinct banks)
+constexpr int kPad = 8;
+constexpr int kOpFloats = 128 * (128 + kPad);
+
+// C(M x N) = alpha * op(A) op(B) + (accumulate ? C : 0), CTA-wide.  A is stored row-major as
+// [M][K] (or [K][M] when transA), B as [K][N] (or [N][K] when transB), both contiguous; C(i, j)
+// = Cm[i*ldc + j].  M % 16 == N % 8 == K % 8 == 0.  Both operands are first copied to shared
+// memory (float4, padded rows); each warp then owns 16x8 output tiles, splitting both operands
+// into tf32 hi + lo parts and accumulating hi*hi + hi*lo + lo*hi.  Ends with a CTA barrier.
+__device__ void gemm(int M, int N, int K, float alpha, const float *A, bool transA, const float *B, bool transB,
+                     bool accumulate, float *Cm, int ldc, float *sa, float *sb) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const int acols = transA ? M : K, arows = transA ? K : M;
+    const int bcols = transB ? K : N, brows = transB ? N : K;
+    const int ald = acols + kPad, bld = bcols + kPad;
+    for (int idx = tid; idx < arows * acols / 4; idx += kThreads) {
+        const int r = (idx * 4) / acols, c = (idx * 4) % acols;
+        *reinterpret_cast<float4 *>(sa + r * ald + c) = reinterpret_cast<const float4 *>(A)[idx];
+    }
+    for (int idx = tid; idx < brows * bcols / 4; idx += kThreads) {
+        const int r = (idx * 4) / bcols, c = (idx * 4) % bcols;
+        *reinterpret_cast<float4 *>(sb + r * bld + c) = reinterpret_cast<const float4 *>(B)[idx];
+    }
+    __syncthreads();
+    const int ar = transA ? 1 : ald, ac = transA ? ald : 1;
+    const int br = transB ? 1 : bld, bc = transB ? bld : 1;
     const int nt = N / 8, tiles = (M / 16) * nt;
     for (int t = warp; t < tiles; t += kWarps) {
         const int i0 = (t / nt) * 16, j0 = (t % nt) * 8;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         for (int k0 = 0; k0 < K; k0 += 8) {
-            const float av[4] = {A[(i0 + gq) * ar + (k0 + tq) * ac], A[(i0 + gq + 8) * ar + (k0 + tq) * ac],
-                                 A[(i0 + gq) * ar + (k0 + tq + 4) * ac], A[(i0 + gq + 8) * ar + (k0 + tq + 4) * ac]};
-            const float bv0 = B[(k0 + tq) * br + (j0 + gq) * bc], bv1 = B[(k0 + tq + 4) * br + (j0 + gq) * bc];
+            const float av[4] = {sa[(i0 + gq) * ar + (k0 + tq) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq) * ac],
+                                 sa[(i0 + gq) * ar + (k0 + tq + 4) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq + 4) * ac]};
+            const float bv0 = sb[(k0 + tq) * br + (j0 + gq) * bc], bv1 = sb[(k0 + tq + 4) * br + (j0 + gq) * bc];
             uint32_t ah[4], al[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -111,6 +132,139 @@ __device__ void gemm(int M, int N, int K, float alpha, const float *A, int ar, i
     __syncthreads();
 }
 
+// acc(16x8) += op(A)(16 x 8k) op(B)(8k x 8) with tf32 hi/lo splits (see gemm); a[e], b[e] fp32
+__device__ __forceinline__ void mma3(float (&acc)[4], const float (&av)[4], float bv0, float bv1) {
+    uint32_t ah[4], al[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        ah[e] = to_tf32(av[e]);
+        al[e] = to_tf32(av[e] - __uint_as_float(ah[e]));
+    }
+    const uint32_t bh0 = to_tf32(bv0), bh1 = to_tf32(bv1);
+    const uint32_t bl0 = to_tf32(bv0 - __uint_as_float(bh0)), bl1 = to_tf32(bv1 - __uint_as_float(bh1));
+    mma_tf32(acc, al, bh0, bh1);
+    mma_tf32(acc, ah, bl0, bl1);
+    mma_tf32(acc, ah, bh0, bh1);
+}
+
+// A_hat (strictly lower) and, if full, A_qk (lower incl.), block pair by block pair:
+// block (R, I) = (X_R diag(s_RI)) Y_I^T with X = k^ e^{G-G_16R} (or q^ ...), Y = k^ e^{G_16I+15-G}.
+__device__ void pair_products(float *w, bool full) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const int items = full ? 40 : 20;          // (pair, 8-column half, which)
+    for (int t = warp; t < items; t += kWarps) {
+        const int which = t / 20, p = (t % 20) >> 1, nh = t & 1;
+        const int R = p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0, I = p - R * (R + 1) / 2;
+        const float *X = w + (which ? Ws::Q1 : Ws::X1) + (16 * R) * D, *Y = w + Ws::Y1 + (16 * I + 8 * nh) * D;
+        const float *sp = w + Ws::SP + p * D;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 0; k0 < D; k0 += 8) {
+            const float s0 = sp[k0 + tq], s1 = sp[k0 + tq + 4];
+            const float av[4] = {X[gq * D + k0 + tq] * s0, X[(gq + 8) * D + k0 + tq] * s0,
+                                 X[gq * D + k0 + tq + 4] * s1, X[(gq + 8) * D + k0 + tq + 4] * s1};
+            mma3(acc, av, Y[gq * D + k0 + tq], Y[gq * D + k0 + tq + 4]);
+        }
+        float *out = w + (which ? Ws::AQ : Ws::AH);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = 16 * R + gq + 8 * (e >> 1), col = 16 * I + 8 * nh + 2 * tq + (e & 1);
+            out[row * C + col] = (which ? col <= row : col < row) ? acc[e] : 0.f;
+        }
+    }
+    // blocks above the diagonal are zero
+    for (int idx = threadIdx.x; idx < 6 * 256; idx += kThreads) {
+        const int b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
+        const int R = b < 3 ? 0 : b < 5 ? 1 : 2, I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
+        w[Ws::AH + (16 * R + rr) * C + 16 * I + cc] = 0.f;
+        if (full) w[Ws::AQ + (16 * R + rr) * C + 16 * I + cc] = 0.f;
+    }
+    __syncthreads();
+}
+
+// Pairwise-decay sums of the reverse sweep, block pair by block pair (dA = dA_hat*beta, dA_qk):
+//   row side    (r in block R):  a1 = E1 sum_{I<=R} s_RI (dA_RI Y_I),   a3 = same with dA_qk
+//   column side (i in block I):  a24 = E2 sum_{R>=I} s_RI (dA_RI^T X_R + dA_qk,RI^T Q_R)
+// a1 -> DKN, a3 -> DQN, a24 -> A24.
+__device__ void pair_grads(float *w) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const float *dah = w + Ws::DAH, *daq = w + Ws::DAQ;
+    for (int t = warp; t < 128; t += kWarps) {
+        const bool col_side = t >= 64;
+        const int B = (t & 63) >> 4, c0 = (t & 15) * 8;      // block (R or I) and 8-channel tile
+        float acc1[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+        const int lo = col_side ? B : 0, hi = col_side ? 3 : B;
+        for (int o = lo; o <= hi; ++o) {
+            const int R = col_side ? o : B, I = col_side ? B : o, p = pair_of(R, I);
+            float t1[4] = {0.f, 0.f, 0.f, 0.f}, t2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+                if (!col_side) {
+                    // A(row, k) = dA[16R + row][16I + k], B(k, j) = Y[16I + k][c0 + j]
+                    const float *a1p = dah + (16 * R) * C + 16 * I, *a3p = daq + (16 * R) * C + 16 * I;
+                    const float *Y = w + Ws::Y1 + (16 * I) * D + c0;
+                    const float b0 = Y[(k0 + tq) * D + gq], b1 = Y[(k0 + tq + 4) * D + gq];
+                    const float av1[4] = {a1p[gq * C + k0 + tq], a1p[(gq + 8) * C + k0 + tq], a1p[gq * C + k0 + tq + 4],
+                                          a1p[(gq + 8) * C + k0 + tq + 4]};
+                    const float av3[4] = {a3p[gq * C + k0 + tq], a3p[(gq + 8) * C + k0 + tq], a3p[gq * C + k0 + tq + 4],
+                                          a3p[(gq + 8) * C + k0 + tq + 4]};
+                    mma3(t1, av1, b0, b1);
+                    mma3(t2, av3, b0, b1);
+                } else {
+                    // A(row, k) = dA[16R + k][16I + row], B(k, j) = X[16R + k][c0 + j]
+                    const float *a1p = dah + (16 * R) * C + 16 * I, *a3p = daq + (16 * R) * C + 16 * I;
+                    const float *X = w + Ws::X1 + (16 * R) * D + c0, *Q = w + Ws::Q1 + (16 * R) * D + c0;
+                    const float av1[4] = {a1p[(k0 + tq) * C + gq], a1p[(k0 + tq) * C + gq + 8], a1p[(k0 + tq + 4) * C + gq],
+                                          a1p[(k0 + tq + 4) * C + gq + 8]};
+                    const float av3[4] = {a3p[(k0 + tq) * C + gq], a3p[(k0 + tq) * C + gq + 8], a3p[(k0 + tq + 4) * C + gq],
+                                          a3p[(k0 + tq + 4) * C + gq + 8]};
+                    mma3(t1, av1, X[(k0 + tq) * D + gq], X[(k0 + tq + 4) * D + gq]);
+                    mma3(t2, av3, Q[(k0 + tq) * D + gq], Q[(k0 + tq + 4) * D + gq]);
+                }
+            }
+            const float s0 = w[Ws::SP + p * D + c0 + 2 * tq], s1 = w[Ws::SP + p * D + c0 + 2 * tq + 1];
+            acc1[0] += s0 * t1[0]; acc1[1] += s1 * t1[1]; acc1[2] += s0 * t1[2]; acc1[3] += s1 * t1[3];
+            acc2[0] += s0 * t2[0]; acc2[1] += s1 * t2[1]; acc2[2] += s0 * t2[2]; acc2[3] += s1 * t2[3];
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = 16 * B + gq + 8 * (e >> 1), c = c0 + 2 * tq + (e & 1);
+            const int idx = row * D + c;
+            if (!col_side) {
+                const float e1 = w[Ws::E1 + idx];
+                w[Ws::DKN + idx] = e1 * acc1[e];
+                w[Ws::DQN + idx] = e1 * acc2[e];
+            } else {
+                w[Ws::A24 + idx] = w[Ws::E2 + idx] * (acc1[e] + acc2[e]);
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// T = (I + diag(beta) A_hat)^-1 (unit lower), rows in order through shared memory:
+// T[r][j] = delta_rj - beta_r sum_{j<=i<r} A_hat[r][i] T[i][j]; 8 threads per (r, j).
+__device__ void tri_inverse(float *w, float *sA, float *sT) {
+    const int tid = threadIdx.x;
+    for (int idx = tid; idx < CC; idx += kThreads) {
+        const int r = idx / C, i = idx % C;
+        sA[r * (C + 1) + i] = w[Ws::BB + r] * w[Ws::AH + idx];
+        sT[r * (C + 1) + i] = 0.f;
+    }
+    __syncthreads();
+    const int j = tid >> 3, part = tid & 7;
+    for (int r = 0; r < C; ++r) {
+        float acc = 0.f;
+        for (int i = j + part; i < r; i += 8) acc += sA[r * (C + 1) + i] * sT[i * (C + 1) + j];
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        if (part == 0 && j <= r) sT[r * (C + 1) + j] = (r == j ? 1.f : 0.f) - acc;
+        __syncthreads();
+    }
+    for (int idx = tid; idx < CC; idx += kThreads) w[Ws::TM + idx] = sT[(idx / C) * (C + 1) + idx % C];
+    __syncthreads();
+}
+
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 __device__ __forceinline__ uint16_t f2bf(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
@@ -131,7 +285,8 @@ struct Args {
 };
 
 // Loads and recomputes everything a chunk needs.  full: also A_qk and Q^e^G (reverse sweep).
-__device__ void recompute_chunk(const Args &a, float *w, int64_t tok0, int L, int h, bool full) {
+__device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, float *ga, float *gb, int64_t tok0, int L,
+                                int h, bool full) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *qn = w + Ws::QN, *kn = w + Ws::KN, *vv = w + Ws::VV, *G = w + Ws::G, *eg = w + Ws::EG;
     float *rq = w + Ws::RQ, *rk = w + Ws::RK, *bb = w + Ws::BB;
@@ -207,41 +362,12 @@ __device__ void recompute_chunk(const Args &a, float *w, int64_t tok0, int L, in
     }
     __syncthreads();
     // A_hat[r][i] = sum_c k^_rc k^_ic e^{G_rc - G_ic} (i < r); A_qk the same with q^ (i <= r)
-    for (int idx = tid; idx < CC; idx += kThreads) {
-        const int r = idx / C, i = idx % C;
-        float ah = 0.f, aq = 0.f;
-        if (i <= r) {
-            const float *x = w + Ws::X1 + r * D, *y = w + Ws::Y1 + i * D, *xq = w + Ws::Q1 + r * D;
-            const float *sp = w + Ws::SP + pair_of(r >> 4, i >> 4) * D;
-            for (int c = 0; c < D; ++c) {
-                const float ys = y[c] * sp[c];
-                ah += x[c] * ys;
-                if (full) aq += xq[c] * ys;
-            }
-        }
-        w[Ws::AH + idx] = i < r ? ah : 0.f;
-        if (full) w[Ws::AQ + idx] = aq;
-    }
-    __syncthreads();
-    // T = (I + diag(beta) A_hat)^-1 (unit lower): one thread per column, forward substitution
-    if (tid < C) {
-        const int j = tid;
-        float *tm = w + Ws::TM;
-        const float *ah = w + Ws::AH;
-        float x[C];
-#pragma unroll
-        for (int r = 0; r < C; ++r) {
-            float acc = r == j ? 1.f : 0.f;
-            for (int i = j; i < r; ++i) acc -= bb[r] * ah[r * C + i] * x[i];
-            x[r] = r < j ? 0.f : acc;
-        }
-#pragma unroll
-        for (int r = 0; r < C; ++r) tm[r * C + j] = x[r];
-    }
-    __syncthreads();
+    pair_products(w, full);
+    // T = (I + diag(beta) A_hat)^-1
+    tri_inverse(w, sA, sT);
     // W = T (beta K^e^G), U = T (beta V)
-    gemm(C, D, C, 1.f, w + Ws::TM, C, 1, w + Ws::BK, D, 1, false, w + Ws::W, D);
-    gemm(C, D, C, 1.f, w + Ws::TM, C, 1, w + Ws::BV, D, 1, false, w + Ws::U, D);
+    gemm(C, D, C, 1.f, w + Ws::TM, false, w + Ws::BK, false, false, w + Ws::W, D, ga, gb);
+    gemm(C, D, C, 1.f, w + Ws::TM, false, w + Ws::BV, false, false, w + Ws::U, D, ga, gb);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
@@ -259,6 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     const int64_t slot0 = d0 / C + doc;                     // checkpoint slots of this document
     float *w = a.scratch + (size_t)chain * Ws::TOTAL;
     float *S = w + Ws::S;
+    extern __shared__ __align__(16) float smem[];
+    float *ga = smem, *gb = smem + kOpFloats;                 // gemm operand buffers
+    float *sA = gb + kOpFloats, *sT = sA + C * (C + 1);       // triangular inverse
 
     // ---------------- forward sweep: entering states ----------------
     for (int idx = tid; idx < DD; idx += kThreads) S[idx] = 0.f;
@@ -266,17 +395,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     for (int n = 0; n < nch; ++n) {
         const int64_t tok0 = d0 + (int64_t)n * C;
         const int L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
-        recompute_chunk(a, w, tok0, L, h, false);
+        recompute_chunk(a, w, sA, sT, ga, gb, tok0, L, h, false);
         float *ck = a.ckpt + ((size_t)(slot0 + n) * H + h) * DD;
         for (int idx = tid; idx < DD; idx += kThreads) ck[idx] = S[idx];
         // U~ = U - W S
         for (int idx = tid; idx < CD; idx += kThreads) w[Ws::UT + idx] = w[Ws::U + idx];
         __syncthreads();
-        gemm(C, D, D, -1.f, w + Ws::W, D, 1, S, D, 1, true, w + Ws::UT, D);
+        gemm(C, D, D, -1.f, w + Ws::W, false, S, false, true, w + Ws::UT, D, ga, gb);
         // S <- Diag(e^{G_last}) S + Kd^T U~
         for (int idx = tid; idx < DD; idx += kThreads) S[idx] *= w[Ws::DL + idx / D];
         __syncthreads();
-        gemm(D, D, C, 1.f, w + Ws::KD, 1, D, w + Ws::UT, D, 1, true, S, D);
+        gemm(D, D, C, 1.f, w + Ws::KD, true, w + Ws::UT, false, true, S, D, ga, gb);
     }
 
     // ---------------- reverse sweep ----------------
@@ -286,25 +415,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     for (int n = nch - 1; n >= 0; --n) {
         const int64_t tok0 = d0 + (int64_t)n * C;
         const int L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
-        recompute_chunk(a, w, tok0, L, h, true);
+        recompute_chunk(a, w, sA, sT, ga, gb, tok0, L, h, true);
         const float *Sin = a.ckpt + ((size_t)(slot0 + n) * H + h) * DD;
         float *Ut = w + Ws::UT, *dUt = w + Ws::DUT, *dO = w + Ws::DO;
         for (int idx = tid; idx < CD; idx += kThreads) Ut[idx] = w[Ws::U + idx];
         __syncthreads();
-        gemm(C, D, D, -1.f, w + Ws::W, D, 1, Sin, D, 1, true, Ut, D);
+        gemm(C, D, D, -1.f, w + Ws::W, false, Sin, false, true, Ut, D, ga, gb);
         // dU~ = A_qk^T dO + Kd dS
-        gemm(C, D, C, 1.f, w + Ws::AQ, 1, C, dO, D, 1, false, dUt, D);
-        gemm(C, D, D, 1.f, w + Ws::KD, D, 1, dS, D, 1, true, dUt, D);
+        gemm(C, D, C, 1.f, w + Ws::AQ, true, dO, false, false, dUt, D, ga, gb);
+        gemm(C, D, D, 1.f, w + Ws::KD, false, dS, false, true, dUt, D, ga, gb);
         // dS_in = QG^T dO + Diag(e^{G_last}) dS - W^T dU~
-        gemm(D, D, C, 1.f, w + Ws::QG, 1, D, dO, D, 1, false, dSn, D);
+        gemm(D, D, C, 1.f, w + Ws::QG, true, dO, false, false, dSn, D, ga, gb);
         for (int idx = tid; idx < DD; idx += kThreads) dSn[idx] += w[Ws::DL + idx / D] * dS[idx];
         __syncthreads();
-        gemm(D, D, C, -1.f, w + Ws::W, 1, D, dUt, D, 1, true, dSn, D);
+        gemm(D, D, C, -1.f, w + Ws::W, true, dUt, false, true, dSn, D, ga, gb);
         // dQG = dO S^T, dA_qk = lower(dO U~^T), dKd = U~ dS^T, dW = -dU~ S^T
-        gemm(C, D, D, 1.f, dO, D, 1, Sin, 1, D, false, w + Ws::DQG, D);
-        gemm(C, C, D, 1.f, dO, D, 1, Ut, 1, D, false, w + Ws::DAQ, C);
-        gemm(C, D, D, 1.f, Ut, D, 1, dS, 1, D, false, w + Ws::DKD, D);
-        gemm(C, D, D, -1.f, dUt, D, 1, Sin, 1, D, false, w + Ws::DW, D);
+        gemm(C, D, D, 1.f, dO, false, Sin, true, false, w + Ws::DQG, D, ga, gb);
+        gemm(C, C, D, 1.f, dO, false, Ut, true, false, w + Ws::DAQ, C, ga, gb);
+        gemm(C, D, D, 1.f, Ut, false, dS, true, false, w + Ws::DKD, D, ga, gb);
+        gemm(C, D, D, -1.f, dUt, false, Sin, true, false, w + Ws::DW, D, ga, gb);
         // dG_last (from Diag(e^{G_last}) S) and the lower mask of dA_qk
         if (tid < D) {
             float acc = 0.f;
@@ -315,13 +444,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
             if (idx % C > idx / C) w[Ws::DAQ + idx] = 0.f;
         __syncthreads();
         // dT = dW (beta KG)^T + dU~ (beta V)^T;  dBk = T^T dW, dBv = T^T dU~
-        gemm(C, C, D, 1.f, w + Ws::DW, D, 1, w + Ws::BK, 1, D, false, w + Ws::DT, C);
-        gemm(C, C, D, 1.f, dUt, D, 1, w + Ws::BV, 1, D, true, w + Ws::DT, C);
-        gemm(C, D, C, 1.f, w + Ws::TM, 1, C, w + Ws::DW, D, 1, false, w + Ws::DBK, D);
-        gemm(C, D, C, 1.f, w + Ws::TM, 1, C, dUt, D, 1, false, w + Ws::DBV, D);
+        gemm(C, C, D, 1.f, w + Ws::DW, false, w + Ws::BK, true, false, w + Ws::DT, C, ga, gb);
+        gemm(C, C, D, 1.f, dUt, false, w + Ws::BV, true, true, w + Ws::DT, C, ga, gb);
+        gemm(C, D, C, 1.f, w + Ws::TM, true, w + Ws::DW, false, false, w + Ws::DBK, D, ga, gb);
+        gemm(C, D, C, 1.f, w + Ws::TM, true, dUt, false, false, w + Ws::DBV, D, ga, gb);
         // dA_kk = strict_lower(-T^T dT T^T)
-        gemm(C, C, C, 1.f, w + Ws::TM, 1, C, w + Ws::DT, C, 1, false, w + Ws::XM, C);
-        gemm(C, C, C, -1.f, w + Ws::XM, C, 1, w + Ws::TM, 1, C, false, w + Ws::DAH, C);
+        gemm(C, C, C, 1.f, w + Ws::TM, true, w + Ws::DT, false, false, w + Ws::XM, C, ga, gb);
+        gemm(C, C, C, -1.f, w + Ws::XM, false, w + Ws::TM, true, false, w + Ws::DAH, C, ga, gb);
         // dbeta (rows), dv, dKG = beta dBk, dA_hat = beta dA_kk
         for (int r = warp; r < C; r += kWarps) {
             float acc = 0.f;
@@ -345,33 +474,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
             w[Ws::DBK + idx] *= b;                              // now dKG
         }
         __syncthreads();
-        // pairwise-decay terms and the elementwise chain rule, per (row r, channel c)
+        // pairwise-decay sums (block MMA), then the elementwise chain rule per (row r, channel c)
+        pair_grads(w);
         for (int idx = tid; idx < CD; idx += kThreads) {
-            const int r = idx / D, c = idx % D, R = r >> 4;
-            float s1 = 0.f, s3 = 0.f;          // row sides:  sum_i dA[r][i] (k^_i e^{G_16I+15-G_i}) s_RI
-            for (int i = 0; i <= r; ++i) {
-                const float y = w[Ws::Y1 + i * D + c] * w[Ws::SP + pair_of(R, i >> 4) * D + c];
-                s1 += w[Ws::DAH + r * C + i] * y;
-                s3 += w[Ws::DAQ + r * C + i] * y;
-            }
-            float s2 = 0.f, s4 = 0.f;          // column sides: sum_r' dA[r'][r] (x_r' e^{G_r'-G_16R'}) s_R'I
-            for (int rr = r; rr < C; ++rr) {
-                const float sp = w[Ws::SP + pair_of(rr >> 4, R) * D + c];
-                s2 += w[Ws::DAH + rr * C + r] * w[Ws::X1 + rr * D + c] * sp;
-                s4 += w[Ws::DAQ + rr * C + r] * w[Ws::Q1 + rr * D + c] * sp;
-            }
-            const float e1 = w[Ws::E1 + idx], e2 = w[Ws::E2 + idx];
-            const float a1 = e1 * s1, a2 = e2 * s2, a3 = e1 * s3, a4 = e2 * s4;
+            const int c = idx % D;
+            const float a1 = w[Ws::DKN + idx], a3 = w[Ws::DQN + idx], a24 = w[Ws::A24 + idx];
             const float knv = w[Ws::KN + idx], qnv = w[Ws::QN + idx], eg = w[Ws::EG + idx];
             const float dKG = w[Ws::DBK + idx], dQG = w[Ws::DQG + idx], dKd = w[Ws::DKD + idx];
             const float e3 = expf(w[Ws::G + (C - 1) * D + c] - w[Ws::G + idx]);
-            float dkn = a1 + a2 + a4 + dKG * eg + dKd * e3;
-            float dqn = a3 + dQG * eg;
-            float dG = knv * (a1 - a2 - a4) + qnv * a3 + dKG * w[Ws::KG + idx] + dQG * w[Ws::QG + idx] -
-                       dKd * w[Ws::KD + idx];
-            w[Ws::DKN + idx] = dkn;
-            w[Ws::DQN + idx] = dqn;
-            w[Ws::DG + idx] = dG;
+            w[Ws::DKN + idx] = a1 + a24 + dKG * eg + dKd * e3;
+            w[Ws::DQN + idx] = a3 + dQG * eg;
+            w[Ws::DG + idx] = knv * (a1 - a24) + qnv * a3 + dKG * w[Ws::KG + idx] + dQG * w[Ws::QG + idx] -
+                              dKd * w[Ws::KD + idx];
         }
         __syncthreads();
         // dg: reverse cumsum per channel (+ the G_last terms at the last row)
@@ -430,7 +544,10 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     a.ckpt = workspace;
     a.scratch = workspace + ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * bwd::DD;
     a.status = status;
-    bwd::kda_bwd_kernel<<<n_docs * H, bwd::kThreads, 0, stream>>>(a);
+    constexpr int smem = (2 * bwd::kOpFloats + 2 * bwd::C * (bwd::C + 1)) * (int)sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(bwd::kda_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    bwd::kda_bwd_kernel<<<n_docs * H, bwd::kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
