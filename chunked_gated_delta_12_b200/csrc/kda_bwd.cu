@@ -59,11 +59,11 @@ struct Ws {
 
 __device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+// tf32 split x = hi + lo: hi keeps the top 19 bits of x (exactly representable in tf32), lo = x - hi
+// is exact in fp32; the tensor core reads lo's top 19 bits.  hi*hi + hi*lo + lo*hi then carries
+// about 2^-21 relative error per product.
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
+__device__ __forceinline__ uint32_t tf32_lo(float x, uint32_t hi) { return __float_as_uint(x - __uint_as_float(hi)); }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -71,6 +71,21 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc(16x8) += op(A)(16 x 8k) op(B)(8k x 8) with tf32 hi/lo splits (see gemm); a[e], b[e] fp32
+__device__ __forceinline__ void mma3(float (&acc)[4], const float (&av)[4], float bv0, float bv1) {
+    uint32_t ah[4], al[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        ah[e] = tf32_hi(av[e]);
+        al[e] = tf32_lo(av[e], ah[e]);
+    }
+    const uint32_t bh0 = tf32_hi(bv0), bh1 = tf32_hi(bv1);
+    const uint32_t bl0 = tf32_lo(bv0, bh0), bl1 = tf32_lo(bv1, bh1);
+    mma_tf32(acc, al, bh0, bh1);
+    mma_tf32(acc, ah, bl0, bl1);
+    mma_tf32(acc, ah, bh0, bh1);
 }
 
 // shared-memory operand buffers of gemm: two matrices of up to 128 rows, rows padded by 8 floats
@@ -83,12 +98,13 @@ constexpr int kOpFloats = 128 * (128 + kPad);
 // = Cm[i*ldc + j].  M % 16 == N % 8 == K % 8 == 0.  Both operands are first copied to shared
 // memory (float4, padded rows); each warp then owns 16x8 output tiles, splitting both operands
 // into tf32 hi + lo parts and accumulating hi*hi + hi*lo + lo*hi.  Ends with a CTA barrier.
-__device__ void gemm(int M, int N, int K, float alpha, const float *A, bool transA, const float *B, bool transB,
-                     bool accumulate, float *Cm, int ldc, float *sa, float *sb) {
+template <int M, int N, int K, bool transA, bool transB>
+__device__ void gemm(float alpha, const float *A, const float *B, bool accumulate, float *Cm, int ldc, float *sa,
+                     float *sb) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const int acols = transA ? M : K, arows = transA ? K : M;
-    const int bcols = transB ? K : N, brows = transB ? N : K;
-    const int ald = acols + kPad, bld = bcols + kPad;
+    constexpr int acols = transA ? M : K, arows = transA ? K : M;
+    constexpr int bcols = transB ? K : N, brows = transB ? N : K;
+    constexpr int ald = acols + kPad, bld = bcols + kPad;
     for (int idx = tid; idx < arows * acols / 4; idx += kThreads) {
         const int r = (idx * 4) / acols, c = (idx * 4) % acols;
         *reinterpret_cast<float4 *>(sa + r * ald + c) = reinterpret_cast<const float4 *>(A)[idx];
@@ -98,27 +114,18 @@ __device__ void gemm(int M, int N, int K, float alpha, const float *A, bool tran
         *reinterpret_cast<float4 *>(sb + r * bld + c) = reinterpret_cast<const float4 *>(B)[idx];
     }
     __syncthreads();
-    const int ar = transA ? 1 : ald, ac = transA ? ald : 1;
-    const int br = transB ? 1 : bld, bc = transB ? bld : 1;
-    const int nt = N / 8, tiles = (M / 16) * nt;
+    constexpr int ar = transA ? 1 : ald, ac = transA ? ald : 1;
+    constexpr int br = transB ? 1 : bld, bc = transB ? bld : 1;
+    constexpr int nt = N / 8, tiles = (M / 16) * nt;
     for (int t = warp; t < tiles; t += kWarps) {
         const int i0 = (t / nt) * 16, j0 = (t % nt) * 8;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
         for (int k0 = 0; k0 < K; k0 += 8) {
             const float av[4] = {sa[(i0 + gq) * ar + (k0 + tq) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq) * ac],
                                  sa[(i0 + gq) * ar + (k0 + tq + 4) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq + 4) * ac]};
             const float bv0 = sb[(k0 + tq) * br + (j0 + gq) * bc], bv1 = sb[(k0 + tq + 4) * br + (j0 + gq) * bc];
-            uint32_t ah[4], al[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ah[e] = to_tf32(av[e]);
-                al[e] = to_tf32(av[e] - __uint_as_float(ah[e]));
-            }
-            const uint32_t bh0 = to_tf32(bv0), bh1 = to_tf32(bv1);
-            const uint32_t bl0 = to_tf32(bv0 - __uint_as_float(bh0)), bl1 = to_tf32(bv1 - __uint_as_float(bh1));
-            mma_tf32(acc, al, bh0, bh1);
-            mma_tf32(acc, ah, bl0, bl1);
-            mma_tf32(acc, ah, bh0, bh1);
+            mma3(acc, av, bv0, bv1);
         }
         float *c0 = Cm + (i0 + gq) * ldc + j0 + 2 * tq, *c1 = c0 + 8 * ldc;
         if (accumulate) {
@@ -132,37 +139,38 @@ __device__ void gemm(int M, int N, int K, float alpha, const float *A, bool tran
     __syncthreads();
 }
 
-// acc(16x8) += op(A)(16 x 8k) op(B)(8k x 8) with tf32 hi/lo splits (see gemm); a[e], b[e] fp32
-__device__ __forceinline__ void mma3(float (&acc)[4], const float (&av)[4], float bv0, float bv1) {
-    uint32_t ah[4], al[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        ah[e] = to_tf32(av[e]);
-        al[e] = to_tf32(av[e] - __uint_as_float(ah[e]));
+// copy a contiguous [rows][cols] fp32 matrix to shared memory with row pitch `pitch` (no barrier)
+__device__ __forceinline__ void stage(float *dst, const float *src, int rows, int cols, int pitch) {
+    for (int idx = threadIdx.x; idx < rows * cols / 4; idx += kThreads) {
+        const int r = (idx * 4) / cols, c = (idx * 4) % cols;
+        *reinterpret_cast<float4 *>(dst + r * pitch + c) = reinterpret_cast<const float4 *>(src)[idx];
     }
-    const uint32_t bh0 = to_tf32(bv0), bh1 = to_tf32(bv1);
-    const uint32_t bl0 = to_tf32(bv0 - __uint_as_float(bh0)), bl1 = to_tf32(bv1 - __uint_as_float(bh1));
-    mma_tf32(acc, al, bh0, bh1);
-    mma_tf32(acc, ah, bl0, bl1);
-    mma_tf32(acc, ah, bh0, bh1);
 }
 
 // A_hat (strictly lower) and, if full, A_qk (lower incl.), block pair by block pair:
 // block (R, I) = (X_R diag(s_RI)) Y_I^T with X = k^ e^{G-G_16R} (or q^ ...), Y = k^ e^{G_16I+15-G}.
-__device__ void pair_products(float *w, bool full) {
+__device__ void pair_products(float *w, bool full, float *sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    constexpr int P = D + 4;                    // pitch: row-wise fragment reads hit 32 banks
+    float *sx = sm, *sq = sm + C * P, *sy = sm + 2 * C * P, *ss = sm + 3 * C * P;
+    stage(sx, w + Ws::X1, C, D, P);
+    if (full) stage(sq, w + Ws::Q1, C, D, P);
+    stage(sy, w + Ws::Y1, C, D, P);
+    stage(ss, w + Ws::SP, 10, D, D);
+    __syncthreads();
     const int items = full ? 40 : 20;          // (pair, 8-column half, which)
     for (int t = warp; t < items; t += kWarps) {
         const int which = t / 20, p = (t % 20) >> 1, nh = t & 1;
         const int R = p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0, I = p - R * (R + 1) / 2;
-        const float *X = w + (which ? Ws::Q1 : Ws::X1) + (16 * R) * D, *Y = w + Ws::Y1 + (16 * I + 8 * nh) * D;
-        const float *sp = w + Ws::SP + p * D;
+        const float *X = (which ? sq : sx) + (16 * R) * P, *Y = sy + (16 * I + 8 * nh) * P;
+        const float *sp = ss + p * D;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
         for (int k0 = 0; k0 < D; k0 += 8) {
             const float s0 = sp[k0 + tq], s1 = sp[k0 + tq + 4];
-            const float av[4] = {X[gq * D + k0 + tq] * s0, X[(gq + 8) * D + k0 + tq] * s0,
-                                 X[gq * D + k0 + tq + 4] * s1, X[(gq + 8) * D + k0 + tq + 4] * s1};
-            mma3(acc, av, Y[gq * D + k0 + tq], Y[gq * D + k0 + tq + 4]);
+            const float av[4] = {X[gq * P + k0 + tq] * s0, X[(gq + 8) * P + k0 + tq] * s0,
+                                 X[gq * P + k0 + tq + 4] * s1, X[(gq + 8) * P + k0 + tq + 4] * s1};
+            mma3(acc, av, Y[gq * P + k0 + tq], Y[gq * P + k0 + tq + 4]);
         }
         float *out = w + (which ? Ws::AQ : Ws::AH);
 #pragma unroll
@@ -178,16 +186,23 @@ __device__ void pair_products(float *w, bool full) {
         w[Ws::AH + (16 * R + rr) * C + 16 * I + cc] = 0.f;
         if (full) w[Ws::AQ + (16 * R + rr) * C + 16 * I + cc] = 0.f;
     }
-    __syncthreads();
+    __syncthreads();   // also frees the staging buffers
 }
 
 // Pairwise-decay sums of the reverse sweep, block pair by block pair (dA = dA_hat*beta, dA_qk):
 //   row side    (r in block R):  a1 = E1 sum_{I<=R} s_RI (dA_RI Y_I),   a3 = same with dA_qk
 //   column side (i in block I):  a24 = E2 sum_{R>=I} s_RI (dA_RI^T X_R + dA_qk,RI^T Q_R)
 // a1 -> DKN, a3 -> DQN, a24 -> A24.
-__device__ void pair_grads(float *w) {
+__device__ void pair_grads(float *w, float *sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    const float *dah = w + Ws::DAH, *daq = w + Ws::DAQ;
+    constexpr int PA = C + 4, PB = D + 8;       // pitches for the fragment read patterns below
+    float *dah = sm, *daq = sm + C * PA, *sx = sm + 2 * C * PA, *sy = sx + C * PB, *sq = sy + C * PB;
+    stage(dah, w + Ws::DAH, C, C, PA);
+    stage(daq, w + Ws::DAQ, C, C, PA);
+    stage(sx, w + Ws::X1, C, D, PB);
+    stage(sy, w + Ws::Y1, C, D, PB);
+    stage(sq, w + Ws::Q1, C, D, PB);
+    __syncthreads();
     for (int t = warp; t < 128; t += kWarps) {
         const bool col_side = t >= 64;
         const int B = (t & 63) >> 4, c0 = (t & 15) * 8;      // block (R or I) and 8-channel tile
@@ -200,25 +215,25 @@ __device__ void pair_grads(float *w) {
             for (int k0 = 0; k0 < 16; k0 += 8) {
                 if (!col_side) {
                     // A(row, k) = dA[16R + row][16I + k], B(k, j) = Y[16I + k][c0 + j]
-                    const float *a1p = dah + (16 * R) * C + 16 * I, *a3p = daq + (16 * R) * C + 16 * I;
-                    const float *Y = w + Ws::Y1 + (16 * I) * D + c0;
-                    const float b0 = Y[(k0 + tq) * D + gq], b1 = Y[(k0 + tq + 4) * D + gq];
-                    const float av1[4] = {a1p[gq * C + k0 + tq], a1p[(gq + 8) * C + k0 + tq], a1p[gq * C + k0 + tq + 4],
-                                          a1p[(gq + 8) * C + k0 + tq + 4]};
-                    const float av3[4] = {a3p[gq * C + k0 + tq], a3p[(gq + 8) * C + k0 + tq], a3p[gq * C + k0 + tq + 4],
-                                          a3p[(gq + 8) * C + k0 + tq + 4]};
+                    const float *a1p = dah + (16 * R) * PA + 16 * I, *a3p = daq + (16 * R) * PA + 16 * I;
+                    const float *Y = sy + (16 * I) * PB + c0;
+                    const float b0 = Y[(k0 + tq) * PB + gq], b1 = Y[(k0 + tq + 4) * PB + gq];
+                    const float av1[4] = {a1p[gq * PA + k0 + tq], a1p[(gq + 8) * PA + k0 + tq], a1p[gq * PA + k0 + tq + 4],
+                                          a1p[(gq + 8) * PA + k0 + tq + 4]};
+                    const float av3[4] = {a3p[gq * PA + k0 + tq], a3p[(gq + 8) * PA + k0 + tq], a3p[gq * PA + k0 + tq + 4],
+                                          a3p[(gq + 8) * PA + k0 + tq + 4]};
                     mma3(t1, av1, b0, b1);
                     mma3(t2, av3, b0, b1);
                 } else {
                     // A(row, k) = dA[16R + k][16I + row], B(k, j) = X[16R + k][c0 + j]
-                    const float *a1p = dah + (16 * R) * C + 16 * I, *a3p = daq + (16 * R) * C + 16 * I;
-                    const float *X = w + Ws::X1 + (16 * R) * D + c0, *Q = w + Ws::Q1 + (16 * R) * D + c0;
-                    const float av1[4] = {a1p[(k0 + tq) * C + gq], a1p[(k0 + tq) * C + gq + 8], a1p[(k0 + tq + 4) * C + gq],
-                                          a1p[(k0 + tq + 4) * C + gq + 8]};
-                    const float av3[4] = {a3p[(k0 + tq) * C + gq], a3p[(k0 + tq) * C + gq + 8], a3p[(k0 + tq + 4) * C + gq],
-                                          a3p[(k0 + tq + 4) * C + gq + 8]};
-                    mma3(t1, av1, X[(k0 + tq) * D + gq], X[(k0 + tq + 4) * D + gq]);
-                    mma3(t2, av3, Q[(k0 + tq) * D + gq], Q[(k0 + tq + 4) * D + gq]);
+                    const float *a1p = dah + (16 * R) * PA + 16 * I, *a3p = daq + (16 * R) * PA + 16 * I;
+                    const float *X = sx + (16 * R) * PB + c0, *Q = sq + (16 * R) * PB + c0;
+                    const float av1[4] = {a1p[(k0 + tq) * PA + gq], a1p[(k0 + tq) * PA + gq + 8], a1p[(k0 + tq + 4) * PA + gq],
+                                          a1p[(k0 + tq + 4) * PA + gq + 8]};
+                    const float av3[4] = {a3p[(k0 + tq) * PA + gq], a3p[(k0 + tq) * PA + gq + 8], a3p[(k0 + tq + 4) * PA + gq],
+                                          a3p[(k0 + tq + 4) * PA + gq + 8]};
+                    mma3(t1, av1, X[(k0 + tq) * PB + gq], X[(k0 + tq + 4) * PB + gq]);
+                    mma3(t2, av3, Q[(k0 + tq) * PB + gq], Q[(k0 + tq + 4) * PB + gq]);
                 }
             }
             const float s0 = w[Ws::SP + p * D + c0 + 2 * tq], s1 = w[Ws::SP + p * D + c0 + 2 * tq + 1];
@@ -285,8 +300,8 @@ struct Args {
 };
 
 // Loads and recomputes everything a chunk needs.  full: also A_qk and Q^e^G (reverse sweep).
-__device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, float *ga, float *gb, int64_t tok0, int L,
-                                int h, bool full) {
+__device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, float *ga, float *gb, float *sred,
+                                int64_t tok0, int L, int h, bool full) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *qn = w + Ws::QN, *kn = w + Ws::KN, *vv = w + Ws::VV, *G = w + Ws::G, *eg = w + Ws::EG;
     float *rq = w + Ws::RQ, *rk = w + Ws::RK, *bb = w + Ws::BB;
@@ -326,16 +341,24 @@ __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, f
             rk[r] = ik;
         }
     }
-    // in-chunk cumsum per channel
-    if (tid < D) {
-        float acc = 0.f;
-        for (int r = 0; r < C; ++r) {
-            acc += G[r * D + tid];
-            G[r * D + tid] = acc;
-        }
-        w[Ws::DL + tid] = expf(acc);          // e^{G_last}
+    // in-chunk cumsum per channel: thread (c, quarter) scans 16 rows in registers, then adds the
+    // totals of the quarters above it
+    {
+        const int c = tid & (D - 1), qr = tid >> 7;
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) x[j] = G[(16 * qr + j) * D + c];
+#pragma unroll
+        for (int j = 1; j < 16; ++j) x[j] += x[j - 1];
+        sred[qr * D + c] = x[15];
+        __syncthreads();
+        float off = 0.f;
+        for (int q2 = 0; q2 < qr; ++q2) off += sred[q2 * D + c];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) G[(16 * qr + j) * D + c] = x[j] + off;
+        if (qr == 3) w[Ws::DL + c] = expf(x[15] + off);          // e^{G_last}
+        __syncthreads();
     }
-    __syncthreads();
     // decay factors: E1 = e^{G_r - G_16R}, E2 = e^{G_16R+15 - G_r}, pair scales s_RI = e^{G_16R - G_16I+15}
     for (int idx = tid; idx < CD; idx += kThreads) {
         const int r = idx / D, c = idx % D, R = r >> 4;
@@ -362,12 +385,12 @@ __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, f
     }
     __syncthreads();
     // A_hat[r][i] = sum_c k^_rc k^_ic e^{G_rc - G_ic} (i < r); A_qk the same with q^ (i <= r)
-    pair_products(w, full);
+    pair_products(w, full, ga);
     // T = (I + diag(beta) A_hat)^-1
     tri_inverse(w, sA, sT);
     // W = T (beta K^e^G), U = T (beta V)
-    gemm(C, D, C, 1.f, w + Ws::TM, false, w + Ws::BK, false, false, w + Ws::W, D, ga, gb);
-    gemm(C, D, C, 1.f, w + Ws::TM, false, w + Ws::BV, false, false, w + Ws::U, D, ga, gb);
+    gemm<C, D, C, false, false>(1.f, w + Ws::TM, w + Ws::BK, false, w + Ws::W, D, ga, gb);
+    gemm<C, D, C, false, false>(1.f, w + Ws::TM, w + Ws::BV, false, w + Ws::U, D, ga, gb);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
@@ -388,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     extern __shared__ __align__(16) float smem[];
     float *ga = smem, *gb = smem + kOpFloats;                 // gemm operand buffers
     float *sA = gb + kOpFloats, *sT = sA + C * (C + 1);       // triangular inverse
+    float *sred = sT + C * (C + 1);                           // [4][128] partial sums
 
     // ---------------- forward sweep: entering states ----------------
     for (int idx = tid; idx < DD; idx += kThreads) S[idx] = 0.f;
@@ -395,17 +419,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     for (int n = 0; n < nch; ++n) {
         const int64_t tok0 = d0 + (int64_t)n * C;
         const int L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
-        recompute_chunk(a, w, sA, sT, ga, gb, tok0, L, h, false);
+        recompute_chunk(a, w, sA, sT, ga, gb, sred, tok0, L, h, false);
         float *ck = a.ckpt + ((size_t)(slot0 + n) * H + h) * DD;
         for (int idx = tid; idx < DD; idx += kThreads) ck[idx] = S[idx];
         // U~ = U - W S
         for (int idx = tid; idx < CD; idx += kThreads) w[Ws::UT + idx] = w[Ws::U + idx];
         __syncthreads();
-        gemm(C, D, D, -1.f, w + Ws::W, false, S, false, true, w + Ws::UT, D, ga, gb);
+        gemm<C, D, D, false, false>(-1.f, w + Ws::W, S, true, w + Ws::UT, D, ga, gb);
         // S <- Diag(e^{G_last}) S + Kd^T U~
         for (int idx = tid; idx < DD; idx += kThreads) S[idx] *= w[Ws::DL + idx / D];
         __syncthreads();
-        gemm(D, D, C, 1.f, w + Ws::KD, true, w + Ws::UT, false, true, S, D, ga, gb);
+        gemm<D, D, C, true, false>(1.f, w + Ws::KD, w + Ws::UT, true, S, D, ga, gb);
     }
 
     // ---------------- reverse sweep ----------------
@@ -415,42 +439,46 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     for (int n = nch - 1; n >= 0; --n) {
         const int64_t tok0 = d0 + (int64_t)n * C;
         const int L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
-        recompute_chunk(a, w, sA, sT, ga, gb, tok0, L, h, true);
+        recompute_chunk(a, w, sA, sT, ga, gb, sred, tok0, L, h, true);
         const float *Sin = a.ckpt + ((size_t)(slot0 + n) * H + h) * DD;
         float *Ut = w + Ws::UT, *dUt = w + Ws::DUT, *dO = w + Ws::DO;
         for (int idx = tid; idx < CD; idx += kThreads) Ut[idx] = w[Ws::U + idx];
         __syncthreads();
-        gemm(C, D, D, -1.f, w + Ws::W, false, Sin, false, true, Ut, D, ga, gb);
+        gemm<C, D, D, false, false>(-1.f, w + Ws::W, Sin, true, Ut, D, ga, gb);
         // dU~ = A_qk^T dO + Kd dS
-        gemm(C, D, C, 1.f, w + Ws::AQ, true, dO, false, false, dUt, D, ga, gb);
-        gemm(C, D, D, 1.f, w + Ws::KD, false, dS, false, true, dUt, D, ga, gb);
+        gemm<C, D, C, true, false>(1.f, w + Ws::AQ, dO, false, dUt, D, ga, gb);
+        gemm<C, D, D, false, false>(1.f, w + Ws::KD, dS, true, dUt, D, ga, gb);
         // dS_in = QG^T dO + Diag(e^{G_last}) dS - W^T dU~
-        gemm(D, D, C, 1.f, w + Ws::QG, true, dO, false, false, dSn, D, ga, gb);
+        gemm<D, D, C, true, false>(1.f, w + Ws::QG, dO, false, dSn, D, ga, gb);
         for (int idx = tid; idx < DD; idx += kThreads) dSn[idx] += w[Ws::DL + idx / D] * dS[idx];
         __syncthreads();
-        gemm(D, D, C, -1.f, w + Ws::W, true, dUt, false, true, dSn, D, ga, gb);
+        gemm<D, D, C, true, false>(-1.f, w + Ws::W, dUt, true, dSn, D, ga, gb);
         // dQG = dO S^T, dA_qk = lower(dO U~^T), dKd = U~ dS^T, dW = -dU~ S^T
-        gemm(C, D, D, 1.f, dO, false, Sin, true, false, w + Ws::DQG, D, ga, gb);
-        gemm(C, C, D, 1.f, dO, false, Ut, true, false, w + Ws::DAQ, C, ga, gb);
-        gemm(C, D, D, 1.f, Ut, false, dS, true, false, w + Ws::DKD, D, ga, gb);
-        gemm(C, D, D, -1.f, dUt, false, Sin, true, false, w + Ws::DW, D, ga, gb);
+        gemm<C, D, D, false, true>(1.f, dO, Sin, false, w + Ws::DQG, D, ga, gb);
+        gemm<C, C, D, false, true>(1.f, dO, Ut, false, w + Ws::DAQ, C, ga, gb);
+        gemm<C, D, D, false, true>(1.f, Ut, dS, false, w + Ws::DKD, D, ga, gb);
+        gemm<C, D, D, false, true>(-1.f, dUt, Sin, false, w + Ws::DW, D, ga, gb);
         // dG_last (from Diag(e^{G_last}) S) and the lower mask of dA_qk
-        if (tid < D) {
+        {
+            const int c = tid >> 2, part = tid & 3;
             float acc = 0.f;
-            for (int x = 0; x < D; ++x) acc += Sin[tid * D + x] * dS[tid * D + x];
-            w[Ws::DGL + tid] = w[Ws::DL + tid] * acc;
+#pragma unroll 8
+            for (int x = part; x < D; x += 4) acc += Sin[c * D + x] * dS[c * D + x];
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (part == 0) w[Ws::DGL + c] = w[Ws::DL + c] * acc;
         }
         for (int idx = tid; idx < CC; idx += kThreads)
             if (idx % C > idx / C) w[Ws::DAQ + idx] = 0.f;
         __syncthreads();
         // dT = dW (beta KG)^T + dU~ (beta V)^T;  dBk = T^T dW, dBv = T^T dU~
-        gemm(C, C, D, 1.f, w + Ws::DW, false, w + Ws::BK, true, false, w + Ws::DT, C, ga, gb);
-        gemm(C, C, D, 1.f, dUt, false, w + Ws::BV, true, true, w + Ws::DT, C, ga, gb);
-        gemm(C, D, C, 1.f, w + Ws::TM, true, w + Ws::DW, false, false, w + Ws::DBK, D, ga, gb);
-        gemm(C, D, C, 1.f, w + Ws::TM, true, dUt, false, false, w + Ws::DBV, D, ga, gb);
+        gemm<C, C, D, false, true>(1.f, w + Ws::DW, w + Ws::BK, false, w + Ws::DT, C, ga, gb);
+        gemm<C, C, D, false, true>(1.f, dUt, w + Ws::BV, true, w + Ws::DT, C, ga, gb);
+        gemm<C, D, C, true, false>(1.f, w + Ws::TM, w + Ws::DW, false, w + Ws::DBK, D, ga, gb);
+        gemm<C, D, C, true, false>(1.f, w + Ws::TM, dUt, false, w + Ws::DBV, D, ga, gb);
         // dA_kk = strict_lower(-T^T dT T^T)
-        gemm(C, C, C, 1.f, w + Ws::TM, true, w + Ws::DT, false, false, w + Ws::XM, C, ga, gb);
-        gemm(C, C, C, -1.f, w + Ws::XM, false, w + Ws::TM, true, false, w + Ws::DAH, C, ga, gb);
+        gemm<C, C, C, true, false>(1.f, w + Ws::TM, w + Ws::DT, false, w + Ws::XM, C, ga, gb);
+        gemm<C, C, C, false, true>(-1.f, w + Ws::XM, w + Ws::TM, false, w + Ws::DAH, C, ga, gb);
         // dbeta (rows), dv, dKG = beta dBk, dA_hat = beta dA_kk
         for (int r = warp; r < C; r += kWarps) {
             float acc = 0.f;
@@ -475,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
         }
         __syncthreads();
         // pairwise-decay sums (block MMA), then the elementwise chain rule per (row r, channel c)
-        pair_grads(w);
+        pair_grads(w, ga);
         for (int idx = tid; idx < CD; idx += kThreads) {
             const int c = idx % D;
             const float a1 = w[Ws::DKN + idx], a3 = w[Ws::DQN + idx], a24 = w[Ws::A24 + idx];
@@ -488,15 +516,34 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
                               dKd * w[Ws::KD + idx];
         }
         __syncthreads();
-        // dg: reverse cumsum per channel (+ the G_last terms at the last row)
-        if (tid < D) {
-            const int c = tid;
-            float gl = w[Ws::DGL + c];
-            for (int r = 0; r < C; ++r) gl += w[Ws::DKD + r * D + c] * w[Ws::KD + r * D + c];
-            float acc = gl;
-            for (int r = C - 1; r >= 0; --r) {
-                acc += w[Ws::DG + r * D + c];
-                if (r < L) a.dg[((tok0 + r) * H + h) * D + c] = acc;
+        // dg: reverse cumsum of dG per channel, plus the G_last terms (which reach every row):
+        // thread (c, quarter) holds 16 rows in registers; quarter sums go through shared memory
+        {
+            const int c = tid & (D - 1), qr = tid >> 7;
+            float x[16];
+            float gl = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int idx = (16 * qr + j) * D + c;
+                x[j] = w[Ws::DG + idx];
+                gl += w[Ws::DKD + idx] * w[Ws::KD + idx];
+            }
+#pragma unroll
+            for (int j = 14; j >= 0; --j) x[j] += x[j + 1];
+            sred[qr * D + c] = x[0];
+            __syncthreads();
+            float off = w[Ws::DGL + c];
+            for (int q2 = 0; q2 < 4; ++q2) {
+                if (q2 > qr) off += sred[q2 * D + c];
+            }
+            __syncthreads();
+            sred[qr * D + c] = gl;
+            __syncthreads();
+            for (int q2 = 0; q2 < 4; ++q2) off += sred[q2 * D + c];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int r = 16 * qr + j;
+                if (r < L) a.dg[((tok0 + r) * H + h) * D + c] = x[j] + off;
             }
         }
         // dq, dk through the l2 norms; dbeta
@@ -544,7 +591,7 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     a.ckpt = workspace;
     a.scratch = workspace + ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * bwd::DD;
     a.status = status;
-    constexpr int smem = (2 * bwd::kOpFloats + 2 * bwd::C * (bwd::C + 1)) * (int)sizeof(float);
+    constexpr int smem = (2 * bwd::kOpFloats + 2 * bwd::C * (bwd::C + 1) + 4 * bwd::D) * (int)sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd::kda_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     bwd::kda_bwd_kernel<<<n_docs * H, bwd::kThreads, smem, stream>>>(a);
