@@ -213,6 +213,40 @@ def run_reference(args, w, d):
     print(json.dumps(line), flush=True)
 
 
+def bench_backward(kda, steps: int, dev, stream, barrier) -> dict:
+    """Device time of kda_chunk_bwd on the packed forward+backward workload (16 documents,
+    H = 32), inputs resident, workspace allocated once; max over ranks."""
+    import torch
+    from chunked_gated_delta_12_b200.inputs import generate, workload
+    wb = workload(4)
+    db = generate(wb, with_grad=True)
+    t = {}
+    for key in ("q", "k", "v", "do"):
+        t[key] = torch.from_numpy(db[key].view(np.int16)).view(torch.bfloat16).to(dev)
+    for key in ("g", "beta", "cu_seqlens"):
+        t[key] = torch.from_numpy(db[key]).to(dev)
+    ws = torch.empty(kda.bwd_workspace_bytes(wb.n_docs, wb.T, wb.H), dtype=torch.uint8, device=dev)
+
+    def run():
+        kda.kda_chunk_bwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"], t["do"], workspace=ws,
+                          stream=stream)
+
+    run()
+    kda.device_status(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    kda.device_status(stream)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+    return {"workload": wb.name, "T": wb.T, "H": wb.H, "ms_per_launch": ms, "launches": steps,
+            "Mtokens_per_s": wb.T / (ms * 1e-3) / 1e6, "workspace_bytes": ws.numel()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -223,6 +257,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bwd-steps", type=int, default=3,
+                    help="timed launches of the recompute backward on the packed forward+backward "
+                         "workload, reported under 'backward' (0 skips it)")
     ap.add_argument("--shape", default=None,
                     help="DOCSxLEN:H -- a custom dense workload with the same distributions "
                          "(e.g. 4x2048:32 for a profiling case larger than L2)")
@@ -333,6 +370,8 @@ def main():
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
     }
+    if args.bwd_steps > 0:
+        line["backward"] = bench_backward(kda, args.bwd_steps, dev, stream, barrier)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, d)
     if rank == 0:

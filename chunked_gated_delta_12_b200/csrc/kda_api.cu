@@ -102,17 +102,12 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
     int *status = nullptr;
     s = status_ptr(dev, &status);
     if (s != KDA_OK) return s;
-    // one CTA per (document, head, value slice): split the value columns in two
-    // when there are too few chains to cover the 148 SMs
+    // one CTA per (document, head): the pipelined kernel.  (Splitting the value columns over two
+    // CTAs when chains are few does not pay: its serial step is about twice as long.)
     const int64_t chains = (int64_t)n_docs * H;
-    const int v_slice = chains >= 112 ? 128 : 64;
-    if (chains * (KDA_HEAD_DIM / v_slice) > (int64_t)INT32_MAX)
-        return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large for one launch");
-    cudaError_t e = v_slice == 128
-                        ? kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status,
-                                               static_cast<cudaStream_t>(stream))
-                        : kda::launch_fwd_tc(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status, v_slice,
-                                             static_cast<cudaStream_t>(stream));
+    if (chains > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large for one launch");
+    cudaError_t e = kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status,
+                                         static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return KDA_OK;
 }

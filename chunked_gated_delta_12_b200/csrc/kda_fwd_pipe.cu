@@ -1,5 +1,5 @@
 // kda_fwd_pipe.cu -- pipelined fused chunk-KDA forward (one CTA per (document, head),
-// all 128 value columns), for launches with enough chains to cover the SMs.
+// all 128 value columns); kda_chunk_fwd launches it for every call.
 //
 // Two chunks are in flight per CTA.  In step s all 16 warps first prepare chunk
 // s; then warps 0-11 finish chunk s's intra-chunk work while warps 12-15 run
@@ -24,7 +24,8 @@
 // q, k, g and v tiles arrive by TMA (2-D tensor maps over [T, H*128], no
 // multicast); rows past the document end are masked with selects (and v rows
 // zeroed) because a tile may reach into the next document.  The gate exponent
-// is split at 16-row sub-block boundaries exactly as in kda_fwd_tc.cu.  Every
+// is split at 16-row sub-block boundaries (e^{G_r - G_i} = E1_r s_RI E2_i, every factor within
+// the fp32/bf16 range).  Every
 // wait is time-limited and reports KDA_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cuda_runtime.h>

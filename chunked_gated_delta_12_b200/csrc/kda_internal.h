@@ -10,11 +10,6 @@ namespace kda {
 constexpr int kStatusBadSeqlens = 6;
 constexpr int kStatusTimeout = 5;
 
-// Fused forward on tcgen05 tensor cores with the state in TMEM.  v_slice in {64, 128}.
-cudaError_t launch_fwd_tc(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                          const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
-                          uint16_t *out, int *status, int v_slice, cudaStream_t stream);
-
 // Pipelined fused forward: one CTA per (document, head) covering all 128 value
 // columns, two chunks in flight (intra-chunk work of chunk s overlapped with the
 // state update of chunk s-1).

@@ -62,8 +62,8 @@ def test_edge_lengths_and_empty_docs(kda):
     assert rel <= RTOL_L2 and mx <= ATOL_MAX, (rel, mx)
 
 
-def test_many_chains_full_slice_path(kda):
-    """Enough chains that one CTA covers all 128 value columns."""
+def test_many_chains(kda):
+    """60 documents x 2 heads: 120 chains, several waves of CTAs."""
     lens = [70] * 60
     w = custom_workload("many", lens, 2, seed=32)
     d = generate(w)
@@ -162,9 +162,9 @@ def test_rejects_wrong_dtype(kda):
 
 
 def test_pipelined_path_isolation_bitwise(kda):
-    """Same isolation check on a launch large enough for the pipelined kernel
-    (>= 112 chains): its TMA tiles read past document ends, so poisoned rows of
-    the next document must be masked, never used."""
+    """Same isolation check on a launch with 128 chains: the TMA tiles read
+    past document ends, so poisoned rows of the next document must be zeroed,
+    never used."""
     import torch
     lens = [1, 64, 65, 129, 63, 200, 64, 14]
     w = custom_workload("iso_pipe", lens, 16, seed=37)       # 8 docs x 16 heads = 128 chains
