@@ -44,10 +44,14 @@ def peaks():
     return FALLBACK_HBM_GBS, 1590.0, "fallback"
 
 
+FWD_KERNEL_SOURCES = ("kda_fwd_pipe.cu", "kda_tc.cuh", "kda_common.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the sources of the forward kernel whose DRAM traffic profiles/traffic.json records."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_gated_delta_12_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in FWD_KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
