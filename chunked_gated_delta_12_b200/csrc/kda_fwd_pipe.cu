@@ -558,70 +558,91 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     bar_solve();
-                    // ---- off-diagonal blocks: warp (I, nt) walks down its 16x8 column strip of T ----
-                    // T_RI = -T_RR sum_{J=I}^{R-1} A_RJ T_JI (tf32 warp MMA).  The strip blocks stay in
-                    // registers as B fragments (rows tq, tq+4, 8+tq, 12+tq; column gq); an accumulator
-                    // becomes a B fragment by two shuffles per register.
-                    if (warp < 6) {
-                        const int I = warp >> 1, nt = warp & 1;
-                        const int src_lo = 4 * tq + (gq >> 1);          // holder of rows tq (and 8+tq), column gq
-                        const int src_hi = 4 * (tq + 4) + (gq >> 1);    // holder of rows tq+4 (and 12+tq)
-                        const bool odd_col = gq & 1;
-                        auto to_bfrag = [&](const float (&c)[4], float (&b)[4], float sign) {
-    #pragma unroll
-                            for (int ks = 0; ks < 2; ++ks) {
-                                const float e0 = __shfl_sync(0xffffffffu, c[2 * ks], src_lo);
-                                const float o0 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_lo);
-                                const float e1 = __shfl_sync(0xffffffffu, c[2 * ks], src_hi);
-                                const float o1 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_hi);
-                                b[2 * ks] = sign * (odd_col ? o0 : e0);
-                                b[2 * ks + 1] = sign * (odd_col ? o1 : e1);
-                            }
-                        };
-                        float tb[3][4];
-                        {
-                            const float *t = f_tm + pair_of(I, I) * kBlkFloats + 8 * nt + gq;
-                            tb[0][0] = t[tq * kBlkPitch];
-                            tb[0][1] = t[(tq + 4) * kBlkPitch];
-                            tb[0][2] = t[(8 + tq) * kBlkPitch];
-                            tb[0][3] = t[(12 + tq) * kBlkPitch];
+                    // ---- off-diagonal blocks of T as a two-level block inverse (tf32 warp MMA) ----
+                    // T = [[T_a, 0], [-T_b A_ba T_a, T_b]] with T_a, T_b the 32x32 inverses, each
+                    // [[T_00, 0], [-T_11 A_10 T_00, T_11]] at the 16-row level.  Level 32: T_10 and T_32
+                    // (warps 0-3, one 16x8 strip each); level 64: the lower-left 32x32 block (warps 0-3,
+                    // one 32x8 column strip each).  Accumulators become B fragments (rows tq, tq+4,
+                    // 8+tq, 12+tq; column gq) by two shuffles per register.
+                    const int src_lo = 4 * tq + (gq >> 1);          // holder of rows tq (and 8+tq), column gq
+                    const int src_hi = 4 * (tq + 4) + (gq >> 1);    // holder of rows tq+4 (and 12+tq)
+                    const bool odd_col = gq & 1;
+                    auto to_bfrag = [&](const float (&c)[4], float (&b)[4]) {
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const float e0 = __shfl_sync(0xffffffffu, c[2 * ks], src_lo);
+                            const float o0 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_lo);
+                            const float e1 = __shfl_sync(0xffffffffu, c[2 * ks], src_hi);
+                            const float o1 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src_hi);
+                            b[2 * ks] = odd_col ? o0 : e0;
+                            b[2 * ks + 1] = odd_col ? o1 : e1;
                         }
+                    };
+                    // B fragment of column strip 8nt..8nt+7 of an fp32 16x16 block
+                    auto load_bfrag = [&](const float *blk, int nt, float (&b)[4]) {
+                        const float *t = blk + 8 * nt + gq;
+                        b[0] = t[tq * kBlkPitch];
+                        b[1] = t[(tq + 4) * kBlkPitch];
+                        b[2] = t[(8 + tq) * kBlkPitch];
+                        b[3] = t[(12 + tq) * kBlkPitch];
+                    };
+                    // acc += blk (16x16, fp32 A fragment) * b (16x8 B fragment)
+                    auto mma16 = [&](float (&acc)[4], const float *blk, const float (&b)[4]) {
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const int k0 = 8 * ks;
+                            mma_tf32(acc, blk[gq * kBlkPitch + k0 + tq], blk[(gq + 8) * kBlkPitch + k0 + tq],
+                                     blk[gq * kBlkPitch + k0 + tq + 4], blk[(gq + 8) * kBlkPitch + k0 + tq + 4],
+                                     b[2 * ks], b[2 * ks + 1]);
+                        }
+                    };
+                    // T'_RI strip = -y diag(beta), bf16, into the B operand of the W and U products
+                    auto store_tp = [&](int R, int I, int nt, const float (&y)[4]) {
                         const int cl = 8 * nt + 2 * tq;
                         const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
-    #pragma unroll
-                        for (int d = 1; d < 4; ++d) {
-                            if (I + d > 3) break;
-                            const int R = I + d;
-                            float xacc[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
-                            for (int jo = d - 1; jo >= 0; --jo) {       // the newest strip block last
-                                const float *ab = f_akk + pair_of(R, I + jo) * kBlkFloats;
-    #pragma unroll
-                                for (int ks = 0; ks < 2; ++ks) {
-                                    const int k0 = 8 * ks;
-                                    mma_tf32(xacc, ab[gq * kBlkPitch + k0 + tq], ab[(gq + 8) * kBlkPitch + k0 + tq],
-                                             ab[gq * kBlkPitch + k0 + tq + 4], ab[(gq + 8) * kBlkPitch + k0 + tq + 4],
-                                             tb[jo][2 * ks], tb[jo][2 * ks + 1]);
-                                }
-                            }
-                            float xb[4];
-                            to_bfrag(xacc, xb, 1.f);
-                            const float *tr = f_tm + pair_of(R, R) * kBlkFloats;
-                            float y[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
-                            for (int ks = 0; ks < 2; ++ks) {
-                                const int k0 = 8 * ks;
-                                mma_tf32(y, tr[gq * kBlkPitch + k0 + tq], tr[(gq + 8) * kBlkPitch + k0 + tq],
-                                         tr[gq * kBlkPitch + k0 + tq + 4], tr[(gq + 8) * kBlkPitch + k0 + tq + 4], xb[2 * ks],
-                                         xb[2 * ks + 1]);
-                            }
-                            // T_RI = -y
-                            *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
-                                pack_bf16(-y[0] * b0, -y[1] * b1);
-                            *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
-                                pack_bf16(-y[2] * b0, -y[3] * b1);
-                            if (d < 3) to_bfrag(y, tb[d], -1.f);
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
+                            pack_bf16(-y[0] * b0, -y[1] * b1);
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
+                            pack_bf16(-y[2] * b0, -y[3] * b1);
+                    };
+                    if (warp < 4) {
+                        // level 32: T_RI = -T_RR (A_RI T_II), (R, I) = (1, 0) or (3, 2)
+                        const int R = warp < 2 ? 1 : 3, I = R - 1, nt = warp & 1;
+                        float tb[4], xacc[4] = {0.f, 0.f, 0.f, 0.f}, xb[4], y[4] = {0.f, 0.f, 0.f, 0.f};
+                        load_bfrag(f_tm + pair_of(I, I) * kBlkFloats, nt, tb);
+                        mma16(xacc, f_akk + pair_of(R, I) * kBlkFloats, tb);
+                        to_bfrag(xacc, xb);
+                        mma16(y, f_tm + pair_of(R, R) * kBlkFloats, xb);
+                        store_tp(R, I, nt, y);
+                        float *to = f_tm + pair_of(R, I) * kBlkFloats;
+                        const int cl = 8 * nt + 2 * tq;
+                        *reinterpret_cast<float2 *>(to + gq * kBlkPitch + cl) = make_float2(-y[0], -y[1]);
+                        *reinterpret_cast<float2 *>(to + (gq + 8) * kBlkPitch + cl) = make_float2(-y[2], -y[3]);
+                    }
+                    bar_solve();
+                    if (warp < 4) {
+                        // level 64: column strip (I, nt) of rows 32..63:
+                        //   X = A_ba T_a[:, strip]:  X_2 = A_20 T_0I + A_21 T_1I,  X_3 = A_30 T_0I + A_31 T_1I
+                        //   Y = T_b X:               Y_2 = T_22 X_2,  Y_3 = T_32 X_2 + T_33 X_3;  T_RI = -Y_R
+                        const int I = warp >> 1, nt = warp & 1;
+                        float t1[4], x2[4] = {0.f, 0.f, 0.f, 0.f}, x3[4] = {0.f, 0.f, 0.f, 0.f};
+                        load_bfrag(f_tm + pair_of(1, I) * kBlkFloats, nt, t1);
+                        if (I == 0) {
+                            float t0[4];
+                            load_bfrag(f_tm + pair_of(0, 0) * kBlkFloats, nt, t0);
+                            mma16(x2, f_akk + pair_of(2, 0) * kBlkFloats, t0);
+                            mma16(x3, f_akk + pair_of(3, 0) * kBlkFloats, t0);
                         }
+                        mma16(x2, f_akk + pair_of(2, 1) * kBlkFloats, t1);
+                        mma16(x3, f_akk + pair_of(3, 1) * kBlkFloats, t1);
+                        float xb2[4], xb3[4], y2[4] = {0.f, 0.f, 0.f, 0.f}, y3[4] = {0.f, 0.f, 0.f, 0.f};
+                        to_bfrag(x2, xb2);
+                        to_bfrag(x3, xb3);
+                        mma16(y2, f_tm + pair_of(2, 2) * kBlkFloats, xb2);
+                        mma16(y3, f_tm + pair_of(3, 2) * kBlkFloats, xb2);
+                        mma16(y3, f_tm + pair_of(3, 3) * kBlkFloats, xb3);
+                        store_tp(2, I, nt, y2);
+                        store_tp(3, I, nt, y3);
                     }
                     tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
                     bar_solve();
