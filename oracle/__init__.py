@@ -49,7 +49,7 @@ def _load():
                                               ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                               ctypes.c_double, ctypes.c_int, ctypes.c_void_p,
                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
-                                              ctypes.c_int]
+                                              ctypes.c_void_p, ctypes.c_int]
         f = lib.kda_oracle_fwd64
         f.restype = ctypes.c_int
         f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
@@ -75,14 +75,15 @@ def _ptr(a: np.ndarray | None):
 
 def kda_fwd(q, k, v, g, beta, cu_seqlens, scale: float | None = None, eps: float = 1e-6,
             erase: bool = True, chains=None, n_threads: int | None = None,
-            return_state: bool = False):
+            return_state: bool = False, initial_state=None):
     """Token-recurrence KDA forward in fp64.
 
     q, k, g: [T, H, K] (any float dtype; widened exactly to fp32 then fp64 inside)
     v: [T, H, V]; beta: [T, H]; cu_seqlens: [n_docs + 1] int.
     chains: optional list of chain ids (doc * H + head) to compute; other rows of
-    the result are NaN.  Returns o [T, H, V] fp64 (and the final states
-    [n_chains, K, V] if ``return_state``).
+    the result are NaN.  initial_state: optional [n_docs, H, K, V] starting states (zero if
+    None).  Returns o [T, H, V] fp64 (and the final states [n_chains, K, V] if
+    ``return_state``).
     """
     q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
     beta = _f32(beta)
@@ -100,9 +101,12 @@ def kda_fwd(q, k, v, g, beta, cu_seqlens, scale: float | None = None, eps: float
     fs = np.zeros((n_chains, K, V), dtype=np.float64) if return_state else None
     if n_threads is None:
         n_threads = os.cpu_count() or 1
+    h0 = None
+    if initial_state is not None:
+        h0 = _f32(initial_state).reshape(n_docs * H, K, V)
     rc = _load().kda_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu),
                                 n_docs, T, H, K, V, float(scale), float(eps), int(bool(erase)),
-                                _ptr(ch), n_chains, _ptr(out), _ptr(fs), int(n_threads))
+                                _ptr(ch), n_chains, _ptr(out), _ptr(fs), _ptr(h0), int(n_threads))
     if rc != 0:
         raise ValueError("oracle rejected the arguments (cu_seqlens or sizes malformed)")
     return (out, fs) if return_state else out

@@ -26,6 +26,12 @@
  * threads; inside a chain the loop over tokens is strictly sequential, so the
  * result does not depend on the thread count.
  *
+ * The state may start from a given S_0 (initial_state, one K x V matrix per
+ * (document, head) chain) instead of zero, and the state after a document's
+ * last token can be returned (final_state): FLA's initial/final state
+ * convention, which the fused contract leaves out and the library offers as
+ * an extension.
+ *
  * erase = 0 drops the "- S'^T k^" term (test-only switch): the recurrence then
  * becomes gated linear attention, which has an independent closed form that
  * the tests use to pin the decay bookkeeping.
@@ -50,6 +56,7 @@ typedef struct {
     int n_chains;
     double *out;             /* [T, H, V] */
     double *final_state;     /* [n_chains, K, V] or NULL */
+    const float *initial_state;  /* [n_docs * H, K, V] by chain id, or NULL (zero) */
     int next;                /* work counter */
     pthread_mutex_t mu;
 } job_t;
@@ -60,6 +67,8 @@ static void run_chain(job_t *j, int idx) {
     const int K = j->K, V = j->V, H = j->H;
     const int64_t t0 = j->cu[doc], t1 = j->cu[doc + 1];
     double *S = calloc((size_t)K * V, sizeof(double));
+    if (j->initial_state)
+        for (size_t e = 0; e < (size_t)K * V; ++e) S[e] = j->initial_state[(size_t)chain * K * V + e];
     double *qn = malloc(sizeof(double) * K), *kn = malloc(sizeof(double) * K);
     double *p = malloc(sizeof(double) * V);
     for (int64_t t = t0; t < t1; ++t) {
@@ -125,13 +134,13 @@ int kda_oracle_fwd(const float *q, const float *k, const float *v, const float *
                    const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T,
                    int H, int K, int V, double scale, double eps, int erase,
                    const int32_t *chains, int n_chains, double *out, double *final_state,
-                   int n_threads) {
+                   const float *initial_state, int n_threads) {
     if (n_docs < 1 || H < 1 || K < 1 || V < 1 || T < 0) return -1;
     if (cu_seqlens[0] != 0 || cu_seqlens[n_docs] != T) return -1;
     for (int d = 0; d < n_docs; ++d)
         if (cu_seqlens[d + 1] < cu_seqlens[d]) return -1;
     job_t j = {q, k, v, g, beta, cu_seqlens, n_docs, T, H, K, V, scale, eps, erase,
-               chains, chains ? n_chains : n_docs * H, out, final_state, 0};
+               chains, chains ? n_chains : n_docs * H, out, final_state, initial_state, 0};
     for (int i = 0; chains && i < n_chains; ++i)
         if (chains[i] < 0 || chains[i] >= n_docs * H) return -1;
     pthread_mutex_init(&j.mu, NULL);

@@ -232,3 +232,56 @@ def test_empty_documents_allowed():
     o = oracle.kda_fwd(q, k, v, g, b, [0, 0, 4, 4, 10])
     o2 = oracle.kda_fwd(q, k, v, g, b, [0, 4, 10])
     assert np.array_equal(o, o2)
+
+
+# ---- initial / final state (FLA's convention, an extension of the fused contract) ----
+
+def _rand_inputs(rng, T, H, K, V, decay_scale=5.0):
+    return dict(q=rng.normal(size=(T, H, K)), k=rng.normal(size=(T, H, K)), v=rng.normal(size=(T, H, V)),
+                g=-decay_scale / (1.0 + np.exp(-rng.normal(size=(T, H, K)))),
+                beta=1.0 / (1.0 + np.exp(-rng.normal(size=(T, H)))))
+
+
+def test_zero_initial_state_is_the_default():
+    rng = np.random.default_rng(11)
+    x = _rand_inputs(rng, 40, 2, 8, 6)
+    cu = np.array([0, 15, 40], np.int32)
+    a, sa = oracle.kda_fwd(**x, cu_seqlens=cu, return_state=True)
+    b, sb = oracle.kda_fwd(**x, cu_seqlens=cu, return_state=True, initial_state=np.zeros((2, 2, 8, 6), np.float32))
+    assert np.array_equal(a, b) and np.array_equal(sa, sb)
+
+
+def test_state_hand_off_equals_one_run():
+    """Running tokens [0, L1) and handing the final state to a second run over [L1, L) gives the
+    outputs and final state of one run over [0, L) (up to the fp32 rounding of the handed state).
+    Mild decay keeps the handed state significant."""
+    rng = np.random.default_rng(12)
+    T, H, K, V, L1 = 90, 2, 8, 6, 37
+    x = _rand_inputs(rng, T, H, K, V, decay_scale=0.05)
+    o, s = oracle.kda_fwd(**x, cu_seqlens=np.array([0, T], np.int32), return_state=True)
+    oa, sa = oracle.kda_fwd(**{k: v[:L1] for k, v in x.items()}, cu_seqlens=np.array([0, L1], np.int32),
+                            return_state=True)
+    ob, sb = oracle.kda_fwd(**{k: v[L1:] for k, v in x.items()}, cu_seqlens=np.array([0, T - L1], np.int32),
+                            return_state=True, initial_state=sa.reshape(1, H, K, V))
+    assert np.abs(sa).max() > 0.1
+    np.testing.assert_allclose(np.concatenate([oa, ob]), o, rtol=0, atol=1e-6)
+    np.testing.assert_allclose(sb, s, rtol=0, atol=1e-6)
+
+
+def test_initial_state_one_token_closed_form():
+    """S_1 = (I - b k^ k^T) Diag(e^g) S_0 + b k^ v^T, o = scale S_1^T q^ with S_0 given (K x V:
+    rows are key channels)."""
+    rng = np.random.default_rng(13)
+    K, V = 6, 5
+    x = _rand_inputs(rng, 1, 1, K, V)
+    S0 = rng.normal(size=(K, V)).astype(np.float32).astype(np.float64)
+    o, s = oracle.kda_fwd(**x, cu_seqlens=np.array([0, 1], np.int32), return_state=True,
+                          initial_state=S0.reshape(1, 1, K, V))
+    q, k, v, g, b = (x["q"][0, 0], x["k"][0, 0], x["v"][0, 0], x["g"][0, 0], x["beta"][0, 0])
+    eps = 1e-6
+    q32, k32, v32, g32 = (np.float64(np.float32(t)) for t in (q, k, v, g))
+    b32 = np.float64(np.float32(b))
+    qn, kn = q32 / np.sqrt(q32 @ q32 + eps), k32 / np.sqrt(k32 @ k32 + eps)
+    S1 = (np.eye(K) - b32 * np.outer(kn, kn)) @ (np.exp(g32)[:, None] * S0) + b32 * np.outer(kn, v32)
+    np.testing.assert_allclose(s[0], S1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(o[0, 0], S1.T @ qn / np.sqrt(K), rtol=1e-12, atol=1e-13)
