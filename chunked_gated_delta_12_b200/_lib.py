@@ -36,6 +36,8 @@ def lib() -> ctypes.CDLL:
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         L.kda_chunk_fwd.restype = i32
         L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp]
+        L.kda_chunk_fwd_state.restype = i32
+        L.kda_chunk_fwd_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp]
         L.kda_last_error.restype = ctypes.c_char_p
         L.kda_last_error.argtypes = []
         L.kda_device_status.restype = i32
@@ -70,12 +72,15 @@ def _ptr(t):
 
 def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                   beta: torch.Tensor, cu_seqlens: torch.Tensor, out: torch.Tensor | None = None,
-                  stream: torch.cuda.Stream | None = None) -> torch.Tensor:
-    """Chunked KDA forward through libkda's kda_chunk_fwd.
+                  stream: torch.cuda.Stream | None = None, initial_state: torch.Tensor | None = None,
+                  output_final_state: bool = False, final_state: torch.Tensor | None = None):
+    """Chunked KDA forward through libkda's kda_chunk_fwd (kda_chunk_fwd_state with states).
 
     q, k, v: [T, H, 128] bf16 (a leading batch dim of 1 is accepted); g: [T, H, 128] fp32;
     beta: [T, H] fp32; cu_seqlens: [n_docs + 1] int32, all on the same CUDA device.
-    Returns out [T, H, 128] bf16 (allocated by torch if not given).
+    initial_state: optional [n_docs, H, 128, 128] fp32 starting states (zero if None).
+    Returns out [T, H, 128] bf16 (allocated by torch if not given), or (out, final_state
+    [n_docs, H, 128, 128] fp32) when output_final_state (or a final_state buffer) is given.
     """
     if q.dim() == 4:
         q, k, v, g = (x.squeeze(0) for x in (q, k, v, g))
@@ -91,10 +96,24 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
         raise KdaError(1, "cu_seqlens must be a 1-d int32 CUDA tensor")
     if out is None:
         out = torch.empty_like(q)
-    rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
-                             cu_seqlens.numel() - 1, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))
+    n_docs = cu_seqlens.numel() - 1
+    shape_s = (n_docs, H, D, D)
+    for name, t in (("initial_state", initial_state), ("final_state", final_state)):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape_s or not t.is_contiguous()
+                              or not t.is_cuda):
+            raise KdaError(1, f"{name} must be a contiguous CUDA float32 tensor of shape {shape_s}")
+    if initial_state is None and final_state is None and not output_final_state:
+        rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                 n_docs, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))
+        _check(rc)
+        return out
+    if final_state is None and output_final_state:
+        final_state = torch.empty(shape_s, dtype=torch.float32, device=q.device)
+    rc = lib().kda_chunk_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
+                                   _ptr(initial_state), _ptr(final_state), _ptr(out),
+                                   ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
-    return out
+    return (out, final_state) if final_state is not None else out
 
 
 def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,

@@ -76,16 +76,36 @@ const char *kda_last_error(void) { return g_err; }
 
 int kda_abi_version(void) { return 1; }
 
-kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                         const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
-                         uint16_t *out, void *stream) {
+kda_status kda_chunk_fwd_state(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                               const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                               const float *initial_state, float *final_state, uint16_t *out, void *stream) {
     g_err[0] = '\0';
     if (n_docs < 1) return fail(KDA_ERR_INVALID_ARG, "n_docs must be >= 1 (got %d)", n_docs);
     if (H < 1) return fail(KDA_ERR_INVALID_ARG, "H must be >= 1 (got %d)", H);
     if (T < 0) return fail(KDA_ERR_INVALID_ARG, "T must be >= 0 (got %lld)", (long long)T);
     if (T > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "T must fit int32 (cu_seqlens is int32)");
     if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL");
-    if (T == 0) return KDA_OK;
+    const int64_t chains = (int64_t)n_docs * H;
+    if (chains > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large for one launch");
+    const size_t state_bytes = (size_t)chains * KDA_HEAD_DIM * KDA_HEAD_DIM * sizeof(float);
+    if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+        return fail(KDA_ERR_INVALID_ARG, "initial_state and final_state must be 16-byte aligned");
+    if (initial_state && final_state && initial_state != final_state &&
+        overlaps(initial_state, state_bytes, final_state, state_bytes))
+        return fail(KDA_ERR_INVALID_ARG, "initial_state and final_state must be the same buffer or disjoint");
+    if (T == 0) {
+        // no tokens: the final states are the initial ones
+        if (!final_state || final_state == initial_state) return KDA_OK;
+        int dev = -1;
+        kda_status s = check_device(&dev);
+        if (s != KDA_OK) return s;
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        cudaError_t e = initial_state
+                            ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, st)
+                            : cudaMemsetAsync(final_state, 0, state_bytes, st);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "final state copy: %s", cudaGetErrorString(e));
+        return KDA_OK;
+    }
     if (!q || !k || !v || !g || !beta || !out) return fail(KDA_ERR_INVALID_ARG, "a tensor pointer is NULL");
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) || !aligned(out, 16))
         return fail(KDA_ERR_INVALID_ARG, "q, k, v, g and out must be 16-byte aligned");
@@ -96,20 +116,30 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
     if (overlaps(out, ob, q, ob) || overlaps(out, ob, k, ob) || overlaps(out, ob, v, ob) ||
         overlaps(out, ob, g, nel * 4) || overlaps(out, ob, beta, (size_t)T * H * 4))
         return fail(KDA_ERR_INVALID_ARG, "out must not alias an input");
+    if (final_state) {
+        const void *ins[6] = {q, k, v, g, beta, out};
+        const size_t insz[6] = {ob, ob, ob, nel * 4, (size_t)T * H * 4, ob};
+        for (int i = 0; i < 6; ++i)
+            if (overlaps(final_state, state_bytes, ins[i], insz[i]))
+                return fail(KDA_ERR_INVALID_ARG, "final_state must not alias an input or out");
+    }
     int dev = -1;
     kda_status s = check_device(&dev);
     if (s != KDA_OK) return s;
     int *status = nullptr;
     s = status_ptr(dev, &status);
     if (s != KDA_OK) return s;
-    // one CTA per (document, head): the pipelined kernel.  (Splitting the value columns over two
-    // CTAs when chains are few does not pay: its serial step is about twice as long.)
-    const int64_t chains = (int64_t)n_docs * H;
-    if (chains > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "n_docs * H too large for one launch");
-    cudaError_t e = kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, out, status,
-                                         static_cast<cudaStream_t>(stream));
+    // one CTA per (document, head): the pipelined kernel
+    cudaError_t e = kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, initial_state, final_state, out,
+                                         status, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return KDA_OK;
+}
+
+kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                         const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                         uint16_t *out, void *stream) {
+    return kda_chunk_fwd_state(q, k, v, g, beta, cu_seqlens, n_docs, T, H, nullptr, nullptr, out, stream);
 }
 
 size_t kda_chunk_bwd_workspace_size(int n_docs, int64_t T, int H) {

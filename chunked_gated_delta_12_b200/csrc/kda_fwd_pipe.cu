@@ -154,7 +154,8 @@ struct Maps {
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
                         const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
-                        uint16_t *__restrict__ out, int *__restrict__ status) {
+                        const float *__restrict__ h0, float *ht, uint16_t *__restrict__ out,
+                        int *__restrict__ status) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     // align by offsetting the shared array itself, so every access stays in the shared window (LDS/STS)
@@ -172,7 +173,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) atomicExch(status, kStatusBadSeqlens);
         return;
     }
-    if (doc_end == doc_start) return;
+    // initial / final state of this chain: [n_docs * H][128 key channels][128 value columns] fp32
+    const size_t state_off = (size_t)blockIdx.x * kHeadDim * kHeadDim;
+    if (doc_end == doc_start) {
+        // nothing to process: the final state is the initial one
+        if (ht)
+            for (int idx = tid; idx < kHeadDim * kHeadDim; idx += kThreads)
+                ht[state_off + idx] = h0 ? h0[state_off + idx] : 0.f;
+        return;
+    }
     const int nchunks = (int)((doc_end - doc_start + 63) / 64);
     auto chunk_len = [&](int i) -> int {
         const int64_t rem = doc_end - (doc_start + 64 * (int64_t)i);
@@ -264,11 +273,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lq = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * lq) << 16);
     if (warp >= 12) {
-        float z[32];
+        // S^T[v][c] (lane v) = h0[c][v], or zero
+        const int vcol = 32 * lq + lane;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            float z[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = 0.f;
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) tc::st32(lane_base + kSF + c0, z);
+            for (int i = 0; i < 32; ++i) z[i] = h0 ? h0[state_off + (size_t)(c0 + i) * kHeadDim + vcol] : 0.f;
+            tc::st32(lane_base + kSF + c0, z);
+        }
         tc::wait_st();
     }
     // chunk 0's inputs (one thread polls the barriers; the CTA barrier releases the rest), then its norms
@@ -867,6 +880,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag) { aborted = true; break; }
     }
 
+    // ---- final state: ht[c][v] = S^T[v][c] (the last state update has completed) ----
+    if (!aborted && ht && warp >= 12) {
+        const int vcol = 32 * lq + lane;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            float z[32];
+            tc::ld32(lane_base + kSF + c0, z);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ht[state_off + (size_t)(c0 + i) * kHeadDim + vcol] = z[i];
+        }
+    }
+
     // ---- teardown ----
     cp_async_wait_all();
     if (tid == kStateTid0) tc::bulk_wait();   // output tiles written before shared memory goes away
@@ -914,8 +940,8 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
 }  // namespace pipe_path
 
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                            const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, uint16_t *out,
-                            int *status, cudaStream_t stream) {
+                            const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, const float *h0,
+                            float *ht, uint16_t *out, int *status, cudaStream_t stream) {
     using namespace pipe_path;
     Maps maps;
     const uint64_t cols = (uint64_t)H * kHeadDim;
@@ -929,7 +955,8 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
     cudaError_t e = cudaFuncSetAttribute(kda_fwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (int64_t)n_docs * H;
-    kda_fwd_pipe_kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, out, status);
+    kda_fwd_pipe_kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, out,
+                                                                        status);
     return cudaGetLastError();
 }
 

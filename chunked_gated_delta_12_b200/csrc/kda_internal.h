@@ -13,9 +13,10 @@ constexpr int kStatusTimeout = 5;
 // Pipelined fused forward: one CTA per (document, head) covering all 128 value
 // columns, two chunks in flight (intra-chunk work of chunk s overlapped with the
 // state update of chunk s-1).
+// h0 / ht: optional initial / final states, [n_docs * H][128][128] fp32 (NULL: zero / not written).
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
-                            uint16_t *out, int *status, cudaStream_t stream);
+                            const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream);
 
 // Recompute backward: dq, dk, dv (bf16), dg, dbeta (fp32) from the forward inputs and dout.
 // workspace holds bwd_workspace_floats(n_docs, T, H) floats (entering states of every chunk

@@ -79,6 +79,29 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          int n_docs, int64_t T, int H, uint16_t *out, void *stream);
 
 /*
+ * kda_chunk_fwd_state -- kda_chunk_fwd with an initial and a final state per chain.
+ *
+ * The same forward, except that the state of each (document, head) chain starts from
+ * initial_state instead of zero, and the state after the document's last token is written
+ * to final_state.  This is FLA's initial/final state convention, which the fused-kernel
+ * contract of the kda_fused page leaves out (it fixes "no initial or final state"); it makes
+ * stateful use possible (a long sequence in pieces, or decoding after a prefill).
+ *
+ * Arguments: as kda_chunk_fwd, plus
+ *   initial_state [n_docs, H, 128, 128] fp32 DEVICE memory: S_0 of chain (doc, head), rows are
+ *                 key channels, columns value columns; NULL means zero.
+ *   final_state   [n_docs, H, 128, 128] fp32 DEVICE memory, written for every chain (an empty
+ *                 document gets its initial state); NULL means not written.  It may be the same
+ *                 buffer as initial_state (updated in place) but must not overlap it otherwise,
+ *                 nor any input or out.  Both 16-byte aligned.
+ * With T = 0 only final_state is written (a copy of initial_state, or zero).
+ * Errors: as kda_chunk_fwd.
+ */
+kda_status kda_chunk_fwd_state(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                               const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                               const float *initial_state, float *final_state, uint16_t *out, void *stream);
+
+/*
  * kda_chunk_bwd_workspace_size -- bytes of device workspace kda_chunk_bwd needs for a call
  * with these sizes (an upper bound that does not depend on the cu_seqlens content).
  */
