@@ -251,6 +251,53 @@ def bench_backward(kda, steps: int, dev, stream, barrier) -> dict:
             "Mtokens_per_s": wb.T / (ms * 1e-3) / 1e6, "workspace_bytes": ws.numel()}
 
 
+DECODE_DOCS = 256                    # one decoding step of 256 sequences x 32 heads, states in place
+STATE_BYTES = 2 * 128 * 128 * 4      # fp32 state read and written per chain
+
+
+def bench_decode(kda, steps: int, dev, stream, barrier) -> dict:
+    """Device time of kda_recurrent_fwd for one decoding step (one token for each of 256
+    documents, H = 32) with the 128 x 128 fp32 states updated in place; the states (537 MB) are
+    larger than L2.  Bound: HBM, STATE_BYTES + BYTES_PER_TOKEN_HEAD per chain."""
+    import torch
+    from chunked_gated_delta_12_b200.inputs import custom_workload, generate
+    wd = custom_workload("decode_256x1_H32", [1] * DECODE_DOCS, 32, seed=20265)
+    dd = generate(wd)
+    t = {}
+    for key in ("q", "k", "v"):
+        t[key] = torch.from_numpy(dd[key].view(np.int16)).view(torch.bfloat16).to(dev)
+    for key in ("g", "beta", "cu_seqlens"):
+        t[key] = torch.from_numpy(dd[key]).to(dev)
+    gen = torch.Generator(device=dev).manual_seed(20266)
+    state = torch.randn(wd.n_docs, wd.H, 128, 128, device=dev, generator=gen) * 0.1
+    out = torch.empty_like(t["q"])
+
+    def run():
+        kda.kda_recurrent_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"], out=out, stream=stream,
+                              initial_state=state, final_state=state)
+
+    for _ in range(3):
+        run()
+    kda.device_status(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    kda.device_status(stream)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+    hbm_peak, _, peak_kind = peaks()
+    alg = wd.n_docs * wd.H * (STATE_BYTES + BYTES_PER_TOKEN_HEAD)
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {"workload": wd.name, "T": wd.T, "H": wd.H, "ms_per_launch": ms, "launches": steps,
+            "Mtokens_per_s": wd.T / (ms * 1e-3) / 1e6,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -264,6 +311,9 @@ def main():
     ap.add_argument("--bwd-steps", type=int, default=3,
                     help="timed launches of the recompute backward on the packed forward+backward "
                          "workload, reported under 'backward' (0 skips it)")
+    ap.add_argument("--dec-steps", type=int, default=20,
+                    help="timed launches of the token-by-token kernel on one decoding step of 256 "
+                         "sequences, reported under 'decode' (0 skips it)")
     ap.add_argument("--shape", default=None,
                     help="DOCSxLEN:H -- a custom dense workload with the same distributions "
                          "(e.g. 4x2048:32 for a profiling case larger than L2)")
@@ -376,6 +426,8 @@ def main():
     }
     if args.bwd_steps > 0:
         line["backward"] = bench_backward(kda, args.bwd_steps, dev, stream, barrier)
+    if args.dec_steps > 0:
+        line["decode"] = bench_decode(kda, args.dec_steps, dev, stream, barrier)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, d)
     if rank == 0:

@@ -1,9 +1,10 @@
-"""chunked_gated_delta_12_b200: chunk-KDA forward for B200 (sm_100a).
+"""chunked_gated_delta_12_b200: chunk-KDA forward (and its recurrent and backward companions) for B200.
 
 The compute lives in libkda.so (CUDA, C ABI in include/kda.h); this package
 only marshals torch tensors into that ABI.
 """
-from ._lib import KdaError, bwd_workspace_bytes, device_status, kda_chunk_bwd, kda_chunk_fwd, lib, wait_selftest
+from ._lib import (RECURRENT_MAX_LEN, KdaError, bwd_workspace_bytes, device_status, kda_chunk_bwd, kda_chunk_fwd,
+                   kda_recurrent_fwd, lib, resolve_mode, wait_selftest)
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "bwd_workspace_bytes", "device_status", "wait_selftest", "KdaError",
-           "lib"]
+__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "resolve_mode", "RECURRENT_MAX_LEN", "kda_chunk_bwd",
+           "bwd_workspace_bytes", "device_status", "wait_selftest", "KdaError", "lib"]

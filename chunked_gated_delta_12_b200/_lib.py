@@ -38,6 +38,8 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp]
         L.kda_chunk_fwd_state.restype = i32
         L.kda_chunk_fwd_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp]
+        L.kda_recurrent_fwd.restype = i32
+        L.kda_recurrent_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp]
         L.kda_last_error.restype = ctypes.c_char_p
         L.kda_last_error.argtypes = []
         L.kda_device_status.restype = i32
@@ -70,18 +72,8 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
-                  beta: torch.Tensor, cu_seqlens: torch.Tensor, out: torch.Tensor | None = None,
-                  stream: torch.cuda.Stream | None = None, initial_state: torch.Tensor | None = None,
-                  output_final_state: bool = False, final_state: torch.Tensor | None = None):
-    """Chunked KDA forward through libkda's kda_chunk_fwd (kda_chunk_fwd_state with states).
-
-    q, k, v: [T, H, 128] bf16 (a leading batch dim of 1 is accepted); g: [T, H, 128] fp32;
-    beta: [T, H] fp32; cu_seqlens: [n_docs + 1] int32, all on the same CUDA device.
-    initial_state: optional [n_docs, H, 128, 128] fp32 starting states (zero if None).
-    Returns out [T, H, 128] bf16 (allocated by torch if not given), or (out, final_state
-    [n_docs, H, 128, 128] fp32) when output_final_state (or a final_state buffer) is given.
-    """
+def _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state, output_final_state, final_state):
+    """Shape/dtype checks shared by both forwards; returns the marshalled tensors and sizes."""
     if q.dim() == 4:
         q, k, v, g = (x.squeeze(0) for x in (q, k, v, g))
         beta = beta.squeeze(0)
@@ -102,18 +94,69 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
         if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape_s or not t.is_contiguous()
                               or not t.is_cuda):
             raise KdaError(1, f"{name} must be a contiguous CUDA float32 tensor of shape {shape_s}")
-    if initial_state is None and final_state is None and not output_final_state:
+    if final_state is None and output_final_state:
+        final_state = torch.empty(shape_s, dtype=torch.float32, device=q.device)
+    return q, k, v, g, beta, out, n_docs, T, H, final_state
+
+
+def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, cu_seqlens: torch.Tensor, out: torch.Tensor | None = None,
+                  stream: torch.cuda.Stream | None = None, initial_state: torch.Tensor | None = None,
+                  output_final_state: bool = False, final_state: torch.Tensor | None = None):
+    """Chunked KDA forward through libkda's kda_chunk_fwd (kda_chunk_fwd_state with states).
+
+    q, k, v: [T, H, 128] bf16 (a leading batch dim of 1 is accepted); g: [T, H, 128] fp32;
+    beta: [T, H] fp32; cu_seqlens: [n_docs + 1] int32, all on the same CUDA device.
+    initial_state: optional [n_docs, H, 128, 128] fp32 starting states (zero if None).
+    Returns out [T, H, 128] bf16 (allocated by torch if not given), or (out, final_state
+    [n_docs, H, 128, 128] fp32) when output_final_state (or a final_state buffer) is given.
+    """
+    want_state = initial_state is not None or final_state is not None or output_final_state
+    q, k, v, g, beta, out, n_docs, T, H, final_state = _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state,
+                                                                     output_final_state, final_state)
+    if not want_state:
         rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
                                  n_docs, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))
         _check(rc)
         return out
-    if final_state is None and output_final_state:
-        final_state = torch.empty(shape_s, dtype=torch.float32, device=q.device)
     rc = lib().kda_chunk_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
                                    _ptr(initial_state), _ptr(final_state), _ptr(out),
                                    ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
     return (out, final_state) if final_state is not None else out
+
+
+def kda_recurrent_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                      beta: torch.Tensor, cu_seqlens: torch.Tensor, out: torch.Tensor | None = None,
+                      stream: torch.cuda.Stream | None = None, initial_state: torch.Tensor | None = None,
+                      output_final_state: bool = False, final_state: torch.Tensor | None = None):
+    """Token-by-token KDA forward through libkda's kda_recurrent_fwd (decode, short inputs).
+
+    Same arguments and return convention as ``kda_chunk_fwd``.
+    """
+    q, k, v, g, beta, out, n_docs, T, H, final_state = _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state,
+                                                                     output_final_state, final_state)
+    rc = lib().kda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
+                                 _ptr(initial_state), _ptr(final_state), _ptr(out),
+                                 ctypes.c_void_p(_stream_handle(stream)))
+    _check(rc)
+    return (out, final_state) if final_state is not None else out
+
+
+# Longest document (tokens) for which the token-by-token kernel beats the chunked one.  Measured
+# on B200 with 64 documents x 32 heads and states in and out: 4 tokens 124 us vs 229 us, 16
+# tokens 378 us vs 236 us; the crossover lies near 8.
+RECURRENT_MAX_LEN = 8
+
+
+def resolve_mode(seq_len: int) -> str:
+    """Kernel for documents of at most ``seq_len`` tokens: "recurrent" (kda_recurrent_fwd) for
+    short inputs such as decoding, "chunk" (kda_chunk_fwd) otherwise.  The same choice as
+    KimiDeltaAttention._resolve_mode on the kimi_linear model page, with the threshold measured
+    here (the page does not print one)."""
+    if seq_len < 0:
+        raise ValueError("seq_len must be >= 0")
+    return "recurrent" if seq_len <= RECURRENT_MAX_LEN else "chunk"
 
 
 def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,

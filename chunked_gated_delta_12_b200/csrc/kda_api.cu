@@ -76,9 +76,17 @@ const char *kda_last_error(void) { return g_err; }
 
 int kda_abi_version(void) { return 1; }
 
-kda_status kda_chunk_fwd_state(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                               const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
-                               const float *initial_state, float *final_state, uint16_t *out, void *stream) {
+}  // extern "C"
+
+namespace {
+
+enum class FwdKernel { kChunk, kRecurrent };
+
+// Validation and launch shared by the chunked and the recurrent forward (same arguments,
+// same contract); `which` selects the kernel.
+kda_status fwd_common(FwdKernel which, const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                      const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                      const float *initial_state, float *final_state, uint16_t *out, void *stream) {
     g_err[0] = '\0';
     if (n_docs < 1) return fail(KDA_ERR_INVALID_ARG, "n_docs must be >= 1 (got %d)", n_docs);
     if (H < 1) return fail(KDA_ERR_INVALID_ARG, "H must be >= 1 (got %d)", H);
@@ -129,11 +137,33 @@ kda_status kda_chunk_fwd_state(const uint16_t *q, const uint16_t *k, const uint1
     int *status = nullptr;
     s = status_ptr(dev, &status);
     if (s != KDA_OK) return s;
-    // one CTA per (document, head): the pipelined kernel
-    cudaError_t e = kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, initial_state, final_state, out,
-                                         status, static_cast<cudaStream_t>(stream));
+    // one CTA per (document, head) in both kernels
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = which == FwdKernel::kChunk
+                        ? kda::launch_fwd_pipe(q, k, v, g, beta, cu_seqlens, n_docs, T, H, initial_state,
+                                               final_state, out, status, st)
+                        : kda::launch_fwd_recurrent(q, k, v, g, beta, cu_seqlens, n_docs, T, H, initial_state,
+                                                    final_state, out, status, st);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd_state(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                               const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                               const float *initial_state, float *final_state, uint16_t *out, void *stream) {
+    return fwd_common(FwdKernel::kChunk, q, k, v, g, beta, cu_seqlens, n_docs, T, H, initial_state, final_state,
+                      out, stream);
+}
+
+kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                             const float *initial_state, float *final_state, uint16_t *out, void *stream) {
+    return fwd_common(FwdKernel::kRecurrent, q, k, v, g, beta, cu_seqlens, n_docs, T, H, initial_state,
+                      final_state, out, stream);
 }
 
 kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,

@@ -154,7 +154,7 @@ struct Maps {
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
                         const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
-                        const float *__restrict__ h0, float *ht, uint16_t *__restrict__ out,
+                        const float *h0, float *ht, uint16_t *__restrict__ out,
                         int *__restrict__ status) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];

@@ -18,6 +18,12 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
                             const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream);
 
+// Token-by-token forward (the recurrence itself, no chunking): one CTA of 128 threads per
+// (document, head), the state in registers.  Same arguments and contract as launch_fwd_pipe.
+cudaError_t launch_fwd_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                                 const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
+                                 const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream);
+
 // Recompute backward: dq, dk, dv (bf16), dg, dbeta (fp32) from the forward inputs and dout.
 // workspace holds bwd_workspace_floats(n_docs, T, H) floats (entering states of every chunk
 // and per-chain scratch).

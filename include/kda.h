@@ -15,9 +15,14 @@
  * cu_seqlens; a dense batch of B equal-length sequences is passed as B packed
  * documents with cu_seqlens = [0, L, 2L, ..., BL]), q/k l2-normalised inside
  * the kernel, a bounded log gate, no initial or final state, no context
- * parallelism, chunk mode only.  Like fused_kda_unsupported_reason on that
- * page, every call that falls outside this scope is rejected with the first
- * violated condition (kda_last_error); there is no fallback path of any kind.
+ * parallelism, chunk mode only (kda_chunk_fwd).  Two entry points widen it:
+ * kda_chunk_fwd_state adds an initial and a final state per chain, and
+ * kda_recurrent_fwd is the token-by-token mode (the "recurrent" alternative to
+ * "chunk" that the kda_mode setting and KimiDeltaAttention._resolve_mode of
+ * the kimi_linear model page choose between) for decoding and short inputs.
+ * Like fused_kda_unsupported_reason on the kda_fused page, every call that
+ * falls outside this scope is rejected with the first violated condition
+ * (kda_last_error); there is no fallback path of any kind.
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -100,6 +105,26 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
 kda_status kda_chunk_fwd_state(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                                const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
                                const float *initial_state, float *final_state, uint16_t *out, void *stream);
+
+/*
+ * kda_recurrent_fwd -- token-by-token KDA forward (recurrent mode), with optional states.
+ *
+ * Operation: the recurrence in the header comment taken one token at a time, no chunking
+ * (the "recurrent" kernel choice of the kda_mode setting on the kimi_linear model page, which
+ * KimiDeltaAttention._resolve_mode picks by sequence length).  The result is the same as
+ * kda_chunk_fwd_state's up to rounding; the state stays fp32 throughout.  One CTA of 128
+ * threads per (document, head) chain; its cost per token is a fixed 128 x 128 state update,
+ * so it suits few tokens per document (decoding a token after a prefill, short documents),
+ * while kda_chunk_fwd is far faster on long documents.
+ *
+ * Arguments, layouts, ownership and errors: exactly as kda_chunk_fwd_state (initial_state and
+ * final_state optional, final_state may be initial_state for an in-place update).  Only
+ * 2-byte alignment is needed by this kernel, but the same 16-byte rule is enforced so that a
+ * buffer valid for one mode is valid for the other.
+ */
+kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                             const float *initial_state, float *final_state, uint16_t *out, void *stream);
 
 /*
  * kda_chunk_bwd_workspace_size -- bytes of device workspace kda_chunk_bwd needs for a call

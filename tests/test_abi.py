@@ -68,3 +68,31 @@ def test_no_device_is_an_error_not_a_fallback(L):
     rc = call(L)
     assert rc in (2, 3), rc            # UNSUPPORTED_DEVICE or CUDA error, never OK
     assert L.kda_last_error()
+
+
+def call_rec(L, q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, n_docs=1, T=64, H=1, h0=None, ht=None,
+             out=FAKE + (1 << 30)):
+    vp = ctypes.c_void_p
+    return L.kda_recurrent_fwd(vp(q), vp(k), vp(v), vp(g), vp(beta), vp(cu), n_docs, T, H, vp(h0), vp(ht), vp(out),
+                               None)
+
+
+def test_recurrent_entry_validates_like_the_chunked_one(L):
+    assert call_rec(L, n_docs=0) == 1 and b"n_docs" in L.kda_last_error()
+    assert call_rec(L, H=0) == 1 and b"H must" in L.kda_last_error()
+    assert call_rec(L, q=0) == 1 and b"NULL" in L.kda_last_error()
+    assert call_rec(L, v=FAKE + 8) == 1 and b"aligned" in L.kda_last_error()
+    assert call_rec(L, out=FAKE) == 1 and b"alias" in L.kda_last_error()
+    st = FAKE + (2 << 30)
+    assert call_rec(L, h0=st, ht=st + 64) == 1 and b"same buffer or disjoint" in L.kda_last_error()
+    assert call_rec(L, h0=st + 4) == 1 and b"16-byte" in L.kda_last_error()
+    assert call_rec(L, ht=FAKE) == 1 and b"alias" in L.kda_last_error()
+    assert call_rec(L, T=0) == 0                       # no tokens and no final state: nothing to do
+
+
+def test_resolve_mode():
+    from chunked_gated_delta_12_b200 import RECURRENT_MAX_LEN, resolve_mode
+    assert resolve_mode(1) == "recurrent" and resolve_mode(RECURRENT_MAX_LEN) == "recurrent"
+    assert resolve_mode(RECURRENT_MAX_LEN + 1) == "chunk" and resolve_mode(65536) == "chunk"
+    with pytest.raises(ValueError):
+        resolve_mode(-1)
