@@ -3,8 +3,9 @@
 The compute lives in libkda.so (CUDA, C ABI in include/kda.h); this package
 only marshals torch tensors into that ABI.
 """
-from ._lib import (RECURRENT_MAX_LEN, KdaError, bwd_workspace_bytes, device_status, kda_chunk_bwd, kda_chunk_fwd,
-                   kda_recurrent_fwd, lib, resolve_mode, wait_selftest)
+from ._lib import (NOALLOC_SCRATCH_BYTES, RECURRENT_MAX_LEN, KdaError, bwd_workspace_bytes, device_status,
+                   kda_chunk_bwd, kda_chunk_bwd_noalloc, kda_chunk_fwd, kda_recurrent_fwd, lib, resolve_mode,
+                   wait_selftest)
 
 __all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "resolve_mode", "RECURRENT_MAX_LEN", "kda_chunk_bwd",
-           "bwd_workspace_bytes", "device_status", "wait_selftest", "KdaError", "lib"]
+           "kda_chunk_bwd_noalloc", "NOALLOC_SCRATCH_BYTES", "bwd_workspace_bytes", "device_status", "wait_selftest", "KdaError", "lib"]

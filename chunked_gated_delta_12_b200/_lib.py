@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_bwd.restype = i32
         L.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp,
                                     ctypes.c_size_t, vp]
+        L.kda_chunk_bwd_noalloc.restype = i32
+        L.kda_chunk_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         L.kda_abi_version.restype = i32
         L.kda_abi_version.argtypes = []
         _lib = L
@@ -188,6 +190,37 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                              workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
     return dq, dk, dv, dg, dbeta
+
+
+def kda_chunk_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                          cu_seqlens: torch.Tensor, dout: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor,
+                          dv: torch.Tensor, dg: torch.Tensor, dbeta: torch.Tensor,
+                          stream: torch.cuda.Stream | None = None) -> None:
+    """Recompute backward through libkda's kda_chunk_bwd_noalloc, for callers that cannot
+    allocate device memory: the caller passes every input and output (dq, dk, dv bf16
+    [T, H, 128]; dg fp32 [T, H, 128]; dbeta fp32 [T, H]) and the library's own fixed scratch
+    (``NOALLOC_SCRATCH_BYTES``) serves as the workspace.  Nothing is allocated here either.
+    Calls on one device share that scratch, so calls that overlap on the GPU race."""
+    T, H, D = q.shape
+    for name, t, dt, shape in (("q", q, torch.bfloat16, (T, H, D)), ("k", k, torch.bfloat16, (T, H, D)),
+                               ("v", v, torch.bfloat16, (T, H, D)), ("g", g, torch.float32, (T, H, D)),
+                               ("beta", beta, torch.float32, (T, H)), ("dout", dout, torch.bfloat16, (T, H, D)),
+                               ("dq", dq, torch.bfloat16, (T, H, D)), ("dk", dk, torch.bfloat16, (T, H, D)),
+                               ("dv", dv, torch.bfloat16, (T, H, D)), ("dg", dg, torch.float32, (T, H, D)),
+                               ("dbeta", dbeta, torch.float32, (T, H))):
+        if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or not t.is_cuda:
+            raise KdaError(1, f"{name} must be a contiguous CUDA {dt} tensor of shape {shape} "
+                              f"(got {t.dtype} {tuple(t.shape)})")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise KdaError(1, "cu_seqlens must be a 1-d int32 CUDA tensor")
+    rc = lib().kda_chunk_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                     cu_seqlens.numel() - 1, T, H, _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _ptr(dg), _ptr(dbeta), ctypes.c_void_p(_stream_handle(stream)))
+    _check(rc)
+
+
+# Scratch bytes kda_chunk_bwd_noalloc holds per GPU (KDA_BWD_NOALLOC_SCRATCH_BYTES in kda.h).
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 def bwd_workspace_bytes(n_docs: int, T: int, H: int) -> int:

@@ -70,6 +70,12 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 }  // namespace
 
+namespace kda {
+
+int set_last_error(int status, const char *msg) { return (int)fail((kda_status)status, "%s", msg); }
+
+}  // namespace kda
+
 extern "C" {
 
 const char *kda_last_error(void) { return g_err; }

@@ -33,6 +33,10 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
                        uint16_t *dk, uint16_t *dv, float *dg, float *dbeta, float *workspace, int *status,
                        cudaStream_t stream);
 
+// Records `msg` as the thread's kda_last_error() text and returns `status` (for entry points
+// defined outside kda_api.cu).
+int set_last_error(int status, const char *msg);
+
 // Runs one time-limited mbarrier wait that can never complete (self-test of the
 // timeout path): records kStatusTimeout in *status after about limit_cycles.
 cudaError_t launch_wait_selftest(int *status, long long limit_cycles, cudaStream_t stream);

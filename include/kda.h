@@ -160,6 +160,45 @@ kda_status kda_chunk_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          const uint16_t *dout, uint16_t *dq, uint16_t *dk, uint16_t *dv, float *dg,
                          float *dbeta, void *workspace, size_t workspace_bytes, void *stream);
 
+/* Bytes of device scratch that kda_chunk_bwd_noalloc holds on each GPU (64 MiB). */
+#define KDA_BWD_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * kda_chunk_bwd_noalloc -- kda_chunk_bwd for callers that cannot allocate device memory.
+ *
+ * The reference pages have no counterpart to this entry point; it is a convenience of this
+ * library.  Some callers cannot call cudaMalloc when they run the backward: their device
+ * memory is owned by another allocator (for instance a framework's caching pool that has
+ * already reserved the free memory, so a fresh cudaMalloc fails), or they must not allocate
+ * after start-up because cudaMalloc and cudaFree synchronise the device and can stall the
+ * work of every other stream.  This entry point computes exactly what kda_chunk_bwd computes,
+ * with the same kernel, but takes its workspace from a fixed scratch array of
+ * KDA_BWD_NOALLOC_SCRATCH_BYTES that lives in the library's own device image.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layouts and errors: as kda_chunk_bwd without the workspace pair.  The caller
+ * still provides every input and output buffer.
+ *
+ * Limit: calls whose kda_chunk_bwd_workspace_size(n_docs, T, H) exceeds
+ * KDA_BWD_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_INVALID_ARG and a message naming
+ * the sizes (for example 1 document of 2048 tokens with 8 heads fits; 4096 tokens with 32
+ * heads does not); those callers need kda_chunk_bwd.
+ *
+ * Memory held: every GPU that loads libkda's device code keeps the array until the process
+ * exits.  Its device address is looked up on the first call made on each device (with that
+ * device current), so make that first call before any stream capture.
+ *
+ * Sharing: every call on a device uses the same array, which keeps the last call's contents
+ * (the kernel sets every value it reads, so nothing needs clearing between calls).  Calls
+ * whose executions overlap on the GPU -- on different streams, or from different host
+ * threads without ordering -- race on the array and give wrong results; order them on one
+ * stream or use kda_chunk_bwd with separate workspaces.
+ */
+kda_status kda_chunk_bwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                                 const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                                 const uint16_t *dout, uint16_t *dq, uint16_t *dk, uint16_t *dv, float *dg,
+                                 float *dbeta, void *stream);
+
 /* Thread-local description of the first violated condition of the last failing call. */
 const char *kda_last_error(void);
 
