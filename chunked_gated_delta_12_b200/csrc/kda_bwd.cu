@@ -395,7 +395,11 @@ __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, f
 
 __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = a.H, chain = blockIdx.x, doc = chain / H, h = chain % H;
+    extern __shared__ __align__(16) float smem[];
+    // CTA -> (document, head), longest documents first (the shared memory is not in use yet);
+    // `chain` indexes this CTA's scratch
+    const int H = a.H, chain = blockIdx.x, h = chain % H;
+    const int doc = doc_at_rank(a.cu, a.n_docs, chain / H, reinterpret_cast<int *>(smem));
     if (blockIdx.x == 0 && tid == 0 && (a.cu[0] != 0 || (int64_t)a.cu[a.n_docs] != a.T))
         atomicExch(a.status, kStatusBadSeqlens);
     const int64_t d0 = a.cu[doc], d1 = a.cu[doc + 1];
@@ -408,7 +412,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     const int64_t slot0 = d0 / C + doc;                     // checkpoint slots of this document
     float *w = a.scratch + (size_t)chain * Ws::TOTAL;
     float *S = w + Ws::S;
-    extern __shared__ __align__(16) float smem[];
     float *ga = smem, *gb = smem + kOpFloats;                 // gemm operand buffers
     float *sA = gb + kOpFloats, *sT = sA + C * (C + 1);       // triangular inverse
     float *sred = sT + C * (C + 1);                           // [4][128] partial sums

@@ -98,6 +98,33 @@ __device__ __forceinline__ float ex2_ftz(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// Longest-first document order for grids of one CTA per (document, head), CTA b covering
+// (document doc_at_rank(b / H), head b % H).  The hardware starts CTAs in index order, so the
+// longest chains start in the first wave and the short ones fill the tail (list scheduling in
+// decreasing order).  Ranks documents by (length descending, index ascending), a permutation for
+// any cu_seqlens content; with more than kLongestFirstMaxDocs documents the order is the identity.
+// Every thread of the CTA must call it (it holds a CTA barrier); `scratch` is n_docs + 2 ints of
+// shared memory that the caller does not use yet.
+constexpr int kLongestFirstMaxDocs = 256;
+__device__ __forceinline__ int doc_at_rank(const int32_t *cu, int n_docs, int rank, int *scratch) {
+    if (n_docs <= 1 || n_docs > kLongestFirstMaxDocs) return rank;
+    for (int i = threadIdx.x; i <= n_docs; i += blockDim.x) scratch[1 + i] = cu[i];
+    __syncthreads();
+    for (int d = threadIdx.x; d < n_docs; d += blockDim.x) {
+        const int len = scratch[2 + d] - scratch[1 + d];
+        int r = 0;
+        for (int e = 0; e < n_docs; ++e) {
+            const int le = scratch[2 + e] - scratch[1 + e];
+            r += (le > len) || (le == len && e < d);
+        }
+        if (r == rank) scratch[0] = d;
+    }
+    __syncthreads();
+    const int doc = scratch[0];
+    __syncthreads();   // scratch may be reused by the caller
+    return doc;
+}
+
 // bf16 bit pattern -> fp32 (exact)
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 

@@ -112,6 +112,11 @@ __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t (&r)[16]) {
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+__device__ __forceinline__ void st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
 __device__ __forceinline__ void st16f(uint32_t taddr, const float (&v)[16]) {
     uint32_t r[16];
 #pragma unroll
@@ -130,6 +135,13 @@ __device__ __forceinline__ uint4 pack8x2(const float2 *x) {
 __device__ __forceinline__ uint4 pack8x2s(const float2 *x, float2 s) {
     const float2 a = __fmul2_rn(x[0], s), b = __fmul2_rn(x[1], s), c = __fmul2_rn(x[2], s), d = __fmul2_rn(x[3], s);
     return make_uint4(pack_bf16(a.x, a.y), pack_bf16(b.x, b.y), pack_bf16(c.x, c.y), pack_bf16(d.x, d.y));
+}
+// registers filled by tcgen05.ld are valid only after tcgen05.wait::ld: this empty asm, placed after
+// the wait, keeps the compiler from moving their first use above it
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
 __device__ __forceinline__ int pair_R(int p) { return p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0; }
 __device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
@@ -163,7 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
-    const int doc = blockIdx.x / H, h = blockIdx.x % H;
+    // CTA -> (document, head), longest documents first; the Q tile area is free until the first TMA load
+    const int doc = doc_at_rank(cu_seqlens, n_docs, blockIdx.x / H, reinterpret_cast<int *>(sm)), h = blockIdx.x % H;
 
     if (blockIdx.x == 0 && tid == 0) {
         if (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[n_docs] != T) atomicExch(status, kStatusBadSeqlens);
@@ -174,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     // initial / final state of this chain: [n_docs * H][128 key channels][128 value columns] fp32
-    const size_t state_off = (size_t)blockIdx.x * kHeadDim * kHeadDim;
+    const size_t state_off = ((size_t)doc * H + h) * kHeadDim * kHeadDim;
     if (doc_end == doc_start) {
         // nothing to process: the final state is the initial one
         if (ht)
@@ -383,6 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the previous step's U product is done: V, KR and its accumulator are free
         if (tid == 0 && have_state && !tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
+        // the previous step's output store has read its staging buffer (Kd's buffer, rewritten below)
+        if (tid == kStateTid0) tc::bulk_wait_read();
         tc::fence_before();
         __syncthreads();   // raw q, k, g read; block sums published
         tc::fence_after();
@@ -501,6 +516,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::fence_proxy_async();
                         if (have_next) issue_g(s + 1);
                         issue_v(s);
+                        // warm L2 with the tiles of the next steps' loads (v of chunk s+1; q, k, g of s+2)
+                        if (have_next) {
+                            const int y1 = (int)(doc_start + 64 * (int64_t)(s + 1));
+                            tc::tma_prefetch_2d(&maps.v, xq, y1);
+                            tc::tma_prefetch_2d(&maps.v, xq + 64, y1);
+                        }
+                        if (s + 2 < nchunks) {
+                            const int y2 = (int)(doc_start + 64 * (int64_t)(s + 2));
+                            tc::tma_prefetch_2d(&maps.q, xq, y2);
+                            tc::tma_prefetch_2d(&maps.q, xq + 64, y2);
+                            tc::tma_prefetch_2d(&maps.k, xq, y2);
+                            tc::tma_prefetch_2d(&maps.k, xq + 64, y2);
+#pragma unroll
+                            for (int b = 0; b < 4; ++b) tc::tma_prefetch_2d(&maps.g, xq + 32 * b, y2);
+                        }
                     }
                     if (have_next) load_beta(sm, beta, doc_start + 64 * (int64_t)(s + 1), nL, H, h, buf ^ 1, tid - 320);
                     cp_async_commit();
@@ -514,6 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 bar_intra();
+                // the state side's tcgen05 product waits for the warp-level A_kk products to finish
+                if (have_state && warp == 0) asm volatile("bar.arrive 4, 160;" ::: "memory");
                 // q^E1 / k^E1 consumed: the next chunk's raw q, k
                 if (tid == 320 && have_next) {
                     tc::fence_proxy_async();
@@ -692,6 +724,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4 *>(sm + S::B2 + tc::mnmaj_chunk(8 * cg + 4 * h2 + e, c, 128)) =
                                 pack8(w + 8 * e, 1.f);
                     }
+                    if (cg == 1) {
+                        // Q~ has been read: zero its columns, so that the state product can accumulate
+                        // [U~^T | (Q~ S)^T] onto [U^T | 0] with one N = 128 instruction per k-step
+                        float z[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+                        tc::st32(lane_base + dcol + 64, z);
+                        tc::st32(lane_base + dcol + 96, z);
+                        tc::wait_st();
+                    }
                 } else if (L < 64) {
                     // rows of v past the document end are zero (the tile may reach the next document)
                     for (int idx = tid - 256; idx < (64 - L) * 16; idx += 128) {
@@ -726,41 +768,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
                 const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
                 // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_last})
-                auto sprep = [&](float (&sv)[32], int c0) {
-                    uint32_t pk[16];
+                auto sprep = [&](float (&sv)[16], int c0) {
+                    uint32_t pk[8];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
-                    st16(lane_base + kSB + c0 / 2, pk);
+                    for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
+                    st8(lane_base + kSB + c0 / 2, pk);
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
+                    for (int i = 0; i < 16; i += 4) {
                         const float4 d4 = *reinterpret_cast<const float4 *>(dc + c0 + i);
                         const float2 x = __fmul2_rn(make_float2(sv[i], sv[i + 1]), make_float2(d4.x, d4.y));
                         const float2 y = __fmul2_rn(make_float2(sv[i + 2], sv[i + 3]), make_float2(d4.z, d4.w));
                         sv[i] = x.x; sv[i + 1] = x.y; sv[i + 2] = y.x; sv[i + 3] = y.y;
                     }
-                    tc::st32(lane_base + kSF + c0, sv);
+                    st16f(lane_base + kSF + c0, sv);
                 };
-#pragma unroll 1
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    float sv[32];
-                    tc::ld32(lane_base + kSF + c0, sv);
-                    tc::wait_ld();
-                    sprep(sv, c0);
-                }
-                tc::wait_st();
-                tc::fence_before();
-                bar_state();
-                if (tid == kStateTid0) {
-                    tc::fence_after();
-                    // [U~^T | (Q~ S)^T]: the first half accumulates onto U^T, the second starts fresh
-                    constexpr uint32_t id2 = tc::idesc_bf16(128, 64, false, true, false);
+                // two loads in flight: the next 32 columns are read while the current ones are converted;
+                // the product's first four k-steps (key channels 0-63) start once their bf16 copy is in
+                // place, while the second half is converted
+                constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
+                auto state_mma = [&](int kk0) {   // [U~^T | (Q~ S)^T] accumulated onto [U^T | 0]
+                    if (kk0 == 0 && have_intra) asm volatile("bar.sync 4, 160;" ::: "memory");
+                    tc::wait_st();
+                    tc::fence_before();
+                    bar_state();
+                    if (tid == kStateTid0) {
+                        tc::fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        mma_ts(tmem + dcol, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2, kk, 128), id2, 1u);
-                        mma_ts(tmem + dcol + 64, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2 + 16384, kk, 128), id2,
-                               kk > 0 ? 1u : 0u);
+                        for (int kk = kk0; kk < kk0 + 4; ++kk)
+                            mma_ts(tmem + dcol, tmem + kSB + 8 * kk, tc::desc_mnmaj(sbase + S::B2, kk, 128), id2, 1u);
                     }
-                    tc::commit(mbar(kMb2));
+                };
+                {
+                    float sa[16], sb[16];
+                    tc::ld16(lane_base + kSF, sa);
+                    tc::wait_ld();
+                    reg_fence(sa);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float(&cur)[16] = (ch & 1) ? sb : sa;
+                        float(&nxt)[16] = (ch & 1) ? sa : sb;
+                        if (ch < 7) tc::ld16(lane_base + kSF + 16 * (ch + 1), nxt);
+                        sprep(cur, 16 * ch);
+                        if (ch == 3) state_mma(0);
+                        if (ch < 7) {
+                            tc::wait_ld();
+                            reg_fence(nxt);
+                        }
+                    }
+                    state_mma(4);
+                    if (tid == kStateTid0) tc::commit(mbar(kMb2));
                 }
                 if (tid == kStateTid0) {
                     if (!tc::mbar_wait(mbar(kMb2), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
@@ -838,8 +894,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (tid == kStateTid0) {
                             tc::tma_store_2d(&maps.o, xq, (int)ptok0, sbase + stage_off);
                             tc::tma_store_2d(&maps.o, xq + 64, (int)ptok0, sbase + stage_off + 8192);
-                            tc::bulk_commit();
-                            tc::bulk_wait_read();   // the staging buffer is read before the step ends
+                            tc::bulk_commit();   // its reads of the staging buffer are awaited in the next step
                         }
                     } else {
                         // partial chunk: rows past the document end belong to the next document, so
