@@ -6,10 +6,11 @@
 //
 //   S' = Diag(e^{g_t}) S,  p = S'^T k^,  S = S' + beta_t k^ (v_t - p)^T,  o_t = scale S^T q^
 //
-// One CTA of 256 threads per (document, head); two threads share value column v and keep
-// 64 rows each of the fp32 state column S[:, v] in registers, so a token costs 4 x 64
-// multiply-adds per thread, with the token's q, k and decays broadcast from shared memory, one
-// barrier, and the next token's inputs loaded while this one computes.  The norms are applied
+// A chain's 128 value columns are split over 4 CTAs of 128 threads (the columns of S evolve
+// independently given q, k, g and beta, so the split needs no exchange).  Four adjacent lanes
+// share value column v and keep 32 rows each of the fp32 state column S[:, v] in registers, so a
+// token costs 4 x 32 multiply-adds per thread, with the token's q, k and decays broadcast from
+// shared memory, one barrier, and the next token's inputs loaded while this one computes.  The norms are applied
 // to the dot products rather than to the vectors: S'^T k^ = rk S'^T k and likewise for q.
 // The state may start from an initial state and be written out at the end, as in
 // kda_chunk_fwd_state.  Meant for few tokens per document (decode after a prefill); the chunked
