@@ -57,6 +57,15 @@ def test_edge_lengths_and_empty_docs(kda):
     check(got, oracle_grads(d), d["cu_seqlens"], w.H)
 
 
+def test_many_short_documents(kda):
+    """More documents than the grid ranks longest-first (256), including empty ones: every chain is
+    computed once, in index order."""
+    w = custom_workload("bwd_many", [(5 * i) % 7 for i in range(260)], 1, seed=43)
+    d = generate(w, with_grad=True)
+    got, _ = run_bwd(kda, d)
+    check(got, oracle_grads(d), d["cu_seqlens"], w.H)
+
+
 def test_packed_forward_backward_workload_sampled_chains(kda):
     """16 packed documents, H = 32 (the forward + backward workload); the oracle recomputes a
     sample of whole (document, head) chains."""
