@@ -93,6 +93,27 @@ __device__ __forceinline__ void mma3(float (&acc)[4], const float (&av)[4], floa
 constexpr int kPad = 8;
 constexpr int kOpFloats = 128 * (128 + kPad);
 
+// copy a contiguous [ROWS][COLS] fp32 matrix to shared memory with row pitch PITCH (no barrier):
+// every load of the thread is issued before its first store, so they are in flight together
+template <int ROWS, int COLS, int PITCH>
+__device__ __forceinline__ void stage(float *dst, const float *src) {
+    constexpr int n4 = ROWS * COLS / 4, it = (n4 + kThreads - 1) / kThreads;
+    float4 r[it];
+#pragma unroll
+    for (int i = 0; i < it; ++i) {
+        const int idx = threadIdx.x + i * kThreads;
+        if (n4 % kThreads == 0 || idx < n4) r[i] = reinterpret_cast<const float4 *>(src)[idx];
+    }
+#pragma unroll
+    for (int i = 0; i < it; ++i) {
+        const int idx = threadIdx.x + i * kThreads;
+        if (n4 % kThreads == 0 || idx < n4) {
+            const int row = (idx * 4) / COLS, c = (idx * 4) % COLS;
+            *reinterpret_cast<float4 *>(dst + row * PITCH + c) = r[i];
+        }
+    }
+}
+
 // C(M x N) = alpha * op(A) op(B) + (accumulate ? C : 0), CTA-wide.  A is stored row-major as
 // [M][K] (or [K][M] when transA), B as [K][N] (or [N][K] when transB), both contiguous; C(i, j)
 // = Cm[i*ldc + j].  M % 16 == N % 8 == K % 8 == 0.  Both operands are first copied to shared
@@ -105,20 +126,21 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
     constexpr int acols = transA ? M : K, arows = transA ? K : M;
     constexpr int bcols = transB ? K : N, brows = transB ? N : K;
     constexpr int ald = acols + kPad, bld = bcols + kPad;
-    for (int idx = tid; idx < arows * acols / 4; idx += kThreads) {
-        const int r = (idx * 4) / acols, c = (idx * 4) % acols;
-        *reinterpret_cast<float4 *>(sa + r * ald + c) = reinterpret_cast<const float4 *>(A)[idx];
-    }
-    for (int idx = tid; idx < brows * bcols / 4; idx += kThreads) {
-        const int r = (idx * 4) / bcols, c = (idx * 4) % bcols;
-        *reinterpret_cast<float4 *>(sb + r * bld + c) = reinterpret_cast<const float4 *>(B)[idx];
-    }
+    stage<arows, acols, ald>(sa, A);
+    stage<brows, bcols, bld>(sb, B);
     __syncthreads();
     constexpr int ar = transA ? 1 : ald, ac = transA ? ald : 1;
     constexpr int br = transB ? 1 : bld, bc = transB ? bld : 1;
     constexpr int nt = N / 8, tiles = (M / 16) * nt;
     for (int t = warp; t < tiles; t += kWarps) {
         const int i0 = (t / nt) * 16, j0 = (t % nt) * 8;
+        float *c0 = Cm + (i0 + gq) * ldc + j0 + 2 * tq, *c1 = c0 + 8 * ldc;
+        // the values accumulated onto are fetched before the products, so their latency overlaps them
+        float2 p0 = make_float2(0.f, 0.f), p1 = p0;
+        if (accumulate) {
+            p0 = *reinterpret_cast<const float2 *>(c0);
+            p1 = *reinterpret_cast<const float2 *>(c1);
+        }
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
         for (int k0 = 0; k0 < K; k0 += 8) {
@@ -127,24 +149,10 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
             const float bv0 = sb[(k0 + tq) * br + (j0 + gq) * bc], bv1 = sb[(k0 + tq + 4) * br + (j0 + gq) * bc];
             mma3(acc, av, bv0, bv1);
         }
-        float *c0 = Cm + (i0 + gq) * ldc + j0 + 2 * tq, *c1 = c0 + 8 * ldc;
-        if (accumulate) {
-            c0[0] += alpha * acc[0]; c0[1] += alpha * acc[1];
-            c1[0] += alpha * acc[2]; c1[1] += alpha * acc[3];
-        } else {
-            c0[0] = alpha * acc[0]; c0[1] = alpha * acc[1];
-            c1[0] = alpha * acc[2]; c1[1] = alpha * acc[3];
-        }
+        *reinterpret_cast<float2 *>(c0) = make_float2(fmaf(alpha, acc[0], p0.x), fmaf(alpha, acc[1], p0.y));
+        *reinterpret_cast<float2 *>(c1) = make_float2(fmaf(alpha, acc[2], p1.x), fmaf(alpha, acc[3], p1.y));
     }
     __syncthreads();
-}
-
-// copy a contiguous [rows][cols] fp32 matrix to shared memory with row pitch `pitch` (no barrier)
-__device__ __forceinline__ void stage(float *dst, const float *src, int rows, int cols, int pitch) {
-    for (int idx = threadIdx.x; idx < rows * cols / 4; idx += kThreads) {
-        const int r = (idx * 4) / cols, c = (idx * 4) % cols;
-        *reinterpret_cast<float4 *>(dst + r * pitch + c) = reinterpret_cast<const float4 *>(src)[idx];
-    }
 }
 
 // A_hat (strictly lower) and, if full, A_qk (lower incl.), block pair by block pair:
@@ -153,10 +161,10 @@ __device__ void pair_products(float *w, bool full, float *sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
     constexpr int P = D + 4;                    // pitch: row-wise fragment reads hit 32 banks
     float *sx = sm, *sq = sm + C * P, *sy = sm + 2 * C * P, *ss = sm + 3 * C * P;
-    stage(sx, w + Ws::X1, C, D, P);
-    if (full) stage(sq, w + Ws::Q1, C, D, P);
-    stage(sy, w + Ws::Y1, C, D, P);
-    stage(ss, w + Ws::SP, 10, D, D);
+    stage<C, D, P>(sx, w + Ws::X1);
+    if (full) stage<C, D, P>(sq, w + Ws::Q1);
+    stage<C, D, P>(sy, w + Ws::Y1);
+    stage<10, D, D>(ss, w + Ws::SP);
     __syncthreads();
     const int items = full ? 40 : 20;          // (pair, 8-column half, which)
     for (int t = warp; t < items; t += kWarps) {
@@ -197,11 +205,11 @@ __device__ void pair_grads(float *w, float *sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
     constexpr int PA = C + 4, PB = D + 8;       // pitches for the fragment read patterns below
     float *dah = sm, *daq = sm + C * PA, *sx = sm + 2 * C * PA, *sy = sx + C * PB, *sq = sy + C * PB;
-    stage(dah, w + Ws::DAH, C, C, PA);
-    stage(daq, w + Ws::DAQ, C, C, PA);
-    stage(sx, w + Ws::X1, C, D, PB);
-    stage(sy, w + Ws::Y1, C, D, PB);
-    stage(sq, w + Ws::Q1, C, D, PB);
+    stage<C, C, PA>(dah, w + Ws::DAH);
+    stage<C, C, PA>(daq, w + Ws::DAQ);
+    stage<C, D, PB>(sx, w + Ws::X1);
+    stage<C, D, PB>(sy, w + Ws::Y1);
+    stage<C, D, PB>(sq, w + Ws::Q1);
     __syncthreads();
     for (int t = warp; t < 128; t += kWarps) {
         const bool col_side = t >= 64;
@@ -256,27 +264,62 @@ __device__ void pair_grads(float *w, float *sm) {
     __syncthreads();
 }
 
-// T = (I + diag(beta) A_hat)^-1 (unit lower), rows in order through shared memory:
-// T[r][j] = delta_rj - beta_r sum_{j<=i<r} A_hat[r][i] T[i][j]; 8 threads per (r, j).
-__device__ void tri_inverse(float *w, float *sA, float *sT) {
-    const int tid = threadIdx.x;
+// T = (I + B)^-1 with B = diag(beta) A_hat strictly lower (T unit lower), by 16 x 16 blocks:
+//   diagonal blocks  T_RR = (I + B_RR)^-1, lane = column, row-by-row substitution (warps 0-3);
+//   off-diagonal     T_RI = -T_RR sum_{J=I..R-1} B_RJ T_JI, by block distance R - I = 1, 2, 3,
+//                    each level as X = sum B T into `sx`, then -T_RR X (one element per thread).
+// fp32 throughout; seven CTA barriers.  `sx` is 3 * 256 floats of free shared memory.
+__device__ void tri_inverse(float *w, float *sA, float *sT, float *sx) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int P = C + 1;
     for (int idx = tid; idx < CC; idx += kThreads) {
         const int r = idx / C, i = idx % C;
-        sA[r * (C + 1) + i] = w[Ws::BB + r] * w[Ws::AH + idx];
-        sT[r * (C + 1) + i] = 0.f;
+        sA[r * P + i] = w[Ws::BB + r] * w[Ws::AH + idx];
+        sT[r * P + i] = 0.f;
     }
     __syncthreads();
-    const int j = tid >> 3, part = tid & 7;
-    for (int r = 0; r < C; ++r) {
-        float acc = 0.f;
-        for (int i = j + part; i < r; i += 8) acc += sA[r * (C + 1) + i] * sT[i * (C + 1) + j];
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-        if (part == 0 && j <= r) sT[r * (C + 1) + j] = (r == j ? 1.f : 0.f) - acc;
+    if (warp < 4 && lane < 16) {
+        const int R = warp, c = lane;
+        const float *b = sA + (16 * R) * P + 16 * R;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < r; ++i) acc = fmaf(-b[r * P + i], x[i], acc);
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[(16 * R + r) * P + 16 * R + c] = x[r];
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        const int nblk = 4 - d;   // blocks (R, I) = (I + d, I), I = 0 .. 3 - d
+        for (int e = tid; e < nblk * 256; e += kThreads) {
+            const int I = e >> 8, R = I + d, r = (e >> 4) & 15, c = e & 15;
+            float acc = 0.f;
+            for (int J = I; J < R; ++J) {
+                const float *brow = sA + (16 * R + r) * P + 16 * J;
+                const float *tcol = sT + (16 * J) * P + 16 * I + c;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc = fmaf(brow[i], tcol[i * P], acc);
+            }
+            sx[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nblk * 256; e += kThreads) {
+            const int I = e >> 8, R = I + d, r = (e >> 4) & 15, c = e & 15;
+            const float *trow = sT + (16 * R + r) * P + 16 * R;
+            const float *xc = sx + (I << 8) + c;
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) acc = fmaf(trow[m], xc[m * 16], acc);
+            sT[(16 * R + r) * P + 16 * I + c] = -acc;
+        }
         __syncthreads();
     }
-    for (int idx = tid; idx < CC; idx += kThreads) w[Ws::TM + idx] = sT[(idx / C) * (C + 1) + idx % C];
+    for (int idx = tid; idx < CC; idx += kThreads) w[Ws::TM + idx] = sT[(idx / C) * P + idx % C];
     __syncthreads();
 }
 
@@ -306,36 +349,53 @@ __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, f
     float *qn = w + Ws::QN, *kn = w + Ws::KN, *vv = w + Ws::VV, *G = w + Ws::G, *eg = w + Ws::EG;
     float *rq = w + Ws::RQ, *rk = w + Ws::RK, *bb = w + Ws::BB;
     const int H = a.H;
-    // raw rows (rows >= L are zero: they then add nothing to any product)
-    for (int idx = tid; idx < CD; idx += kThreads) {
-        const int r = idx / D, c = idx % D;
-        const bool ok = r < L;
-        const int64_t off = ((tok0 + r) * H + h) * D + c;
-        qn[idx] = ok ? bf2f(a.q[off]) : 0.f;
-        kn[idx] = ok ? bf2f(a.k[off]) : 0.f;
-        vv[idx] = ok ? bf2f(a.v[off]) : 0.f;
-        G[idx] = ok ? a.g[off] : 0.f;
-        if (full) w[Ws::DO + idx] = ok ? bf2f(a.dout[off]) * rsqrtf((float)D) : 0.f;   // dO = scale dout
+    // raw rows, four channels per access (rows >= L are zero: they then add nothing to any product)
+    {
+        constexpr int it = CD / 4 / kThreads;
+        uint2 rq4[it], rk4[it], rv4[it], rd4[it];
+        float4 rg4[it];
+#pragma unroll
+        for (int i = 0; i < it; ++i) {
+            const int idx = 4 * (tid + i * kThreads), r = idx / D, c = idx % D;
+            const int64_t off = ((tok0 + r) * H + h) * D + c;
+            const uint2 z2 = make_uint2(0u, 0u);
+            const bool ok = r < L;
+            rq4[i] = ok ? *reinterpret_cast<const uint2 *>(a.q + off) : z2;
+            rk4[i] = ok ? *reinterpret_cast<const uint2 *>(a.k + off) : z2;
+            rv4[i] = ok ? *reinterpret_cast<const uint2 *>(a.v + off) : z2;
+            rg4[i] = ok ? *reinterpret_cast<const float4 *>(a.g + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (full) rd4[i] = ok ? *reinterpret_cast<const uint2 *>(a.dout + off) : z2;
+        }
+        auto f4 = [](uint2 u, float sc) {
+            return make_float4(bf2f((uint16_t)(u.x & 0xffffu)) * sc, bf2f((uint16_t)(u.x >> 16)) * sc,
+                               bf2f((uint16_t)(u.y & 0xffffu)) * sc, bf2f((uint16_t)(u.y >> 16)) * sc);
+        };
+#pragma unroll
+        for (int i = 0; i < it; ++i) {
+            const int idx = 4 * (tid + i * kThreads);
+            *reinterpret_cast<float4 *>(qn + idx) = f4(rq4[i], 1.f);
+            *reinterpret_cast<float4 *>(kn + idx) = f4(rk4[i], 1.f);
+            *reinterpret_cast<float4 *>(vv + idx) = f4(rv4[i], 1.f);
+            *reinterpret_cast<float4 *>(G + idx) = rg4[i];
+            if (full) *reinterpret_cast<float4 *>(w + Ws::DO + idx) = f4(rd4[i], rsqrtf((float)D));   // dO = scale dout
+        }
     }
     if (tid < C) bb[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
     __syncthreads();
     // l2 norms: one warp per row
     for (int r = warp; r < C; r += kWarps) {
-        float sq = 0.f, sk = 0.f;
-        for (int c = lane; c < D; c += 32) {
-            sq += qn[r * D + c] * qn[r * D + c];
-            sk += kn[r * D + c] * kn[r * D + c];
-        }
+        const float4 q4 = *reinterpret_cast<const float4 *>(qn + r * D + 4 * lane);
+        const float4 k4 = *reinterpret_cast<const float4 *>(kn + r * D + 4 * lane);
+        float sq = q4.x * q4.x + q4.y * q4.y + q4.z * q4.z + q4.w * q4.w;
+        float sk = k4.x * k4.x + k4.y * k4.y + k4.z * k4.z + k4.w * k4.w;
 #pragma unroll
         for (int o = 16; o; o >>= 1) {
             sq += __shfl_xor_sync(0xffffffffu, sq, o);
             sk += __shfl_xor_sync(0xffffffffu, sk, o);
         }
         const float iq = rsqrtf(sq + 1e-6f), ik = rsqrtf(sk + 1e-6f);
-        for (int c = lane; c < D; c += 32) {
-            qn[r * D + c] *= iq;
-            kn[r * D + c] *= ik;
-        }
+        *reinterpret_cast<float4 *>(qn + r * D + 4 * lane) = make_float4(q4.x * iq, q4.y * iq, q4.z * iq, q4.w * iq);
+        *reinterpret_cast<float4 *>(kn + r * D + 4 * lane) = make_float4(k4.x * ik, k4.y * ik, k4.z * ik, k4.w * ik);
         if (lane == 0) {
             rq[r] = iq;
             rk[r] = ik;
@@ -360,23 +420,50 @@ __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, f
         __syncthreads();
     }
     // decay factors: E1 = e^{G_r - G_16R}, E2 = e^{G_16R+15 - G_r}, pair scales s_RI = e^{G_16R - G_16I+15}
-    for (int idx = tid; idx < CD; idx += kThreads) {
+    // (four channels per thread and step, every operand read and written as float4)
+    for (int idx = 4 * tid; idx < CD; idx += 4 * kThreads) {
         const int r = idx / D, c = idx % D, R = r >> 4;
-        const float gr = G[idx], gl = G[(C - 1) * D + c];
-        const float e1 = expf(gr - G[(16 * R) * D + c]);
-        const float e2 = expf(G[(16 * R + 15) * D + c] - gr);
-        w[Ws::E1 + idx] = e1;
-        w[Ws::E2 + idx] = e2;
-        w[Ws::X1 + idx] = kn[idx] * e1;
-        w[Ws::Y1 + idx] = kn[idx] * e2;
-        if (full) w[Ws::Q1 + idx] = qn[idx] * e1;
-        const float e = expf(gr);
-        eg[idx] = e;
-        w[Ws::KG + idx] = kn[idx] * e;
-        w[Ws::BK + idx] = bb[r] * kn[idx] * e;
-        w[Ws::BV + idx] = bb[r] * vv[idx];
-        w[Ws::KD + idx] = kn[idx] * expf(gl - gr);
-        if (full) w[Ws::QG + idx] = qn[idx] * e;
+        const float4 gr4 = *reinterpret_cast<const float4 *>(G + idx);
+        const float4 gl4 = *reinterpret_cast<const float4 *>(G + (C - 1) * D + c);
+        const float4 g04 = *reinterpret_cast<const float4 *>(G + (16 * R) * D + c);
+        const float4 g14 = *reinterpret_cast<const float4 *>(G + (16 * R + 15) * D + c);
+        const float4 k4 = *reinterpret_cast<const float4 *>(kn + idx);
+        const float4 q4 = *reinterpret_cast<const float4 *>(qn + idx);
+        const float4 v4 = *reinterpret_cast<const float4 *>(vv + idx);
+        const float br = bb[r];
+        const float grv[4] = {gr4.x, gr4.y, gr4.z, gr4.w}, glv[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
+        const float g0v[4] = {g04.x, g04.y, g04.z, g04.w}, g1v[4] = {g14.x, g14.y, g14.z, g14.w};
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
+        const float vvv[4] = {v4.x, v4.y, v4.z, v4.w};
+        float e1[4], e2[4], x1[4], y1[4], q1[4], ev[4], kg[4], bk[4], bv[4], kd[4], qg[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            e1[j] = expf(grv[j] - g0v[j]);
+            e2[j] = expf(g1v[j] - grv[j]);
+            x1[j] = kv[j] * e1[j];
+            y1[j] = kv[j] * e2[j];
+            q1[j] = qv[j] * e1[j];
+            ev[j] = expf(grv[j]);
+            kg[j] = kv[j] * ev[j];
+            bk[j] = br * kv[j] * ev[j];
+            bv[j] = br * vvv[j];
+            kd[j] = kv[j] * expf(glv[j] - grv[j]);
+            qg[j] = qv[j] * ev[j];
+        }
+        auto st4 = [&](size_t off, const float (&x)[4]) {
+            *reinterpret_cast<float4 *>(w + off + idx) = make_float4(x[0], x[1], x[2], x[3]);
+        };
+        st4(Ws::E1, e1);
+        st4(Ws::E2, e2);
+        st4(Ws::X1, x1);
+        st4(Ws::Y1, y1);
+        if (full) st4(Ws::Q1, q1);
+        st4(Ws::EG, ev);
+        st4(Ws::KG, kg);
+        st4(Ws::BK, bk);
+        st4(Ws::BV, bv);
+        st4(Ws::KD, kd);
+        if (full) st4(Ws::QG, qg);
     }
     for (int idx = tid; idx < 10 * D; idx += kThreads) {
         const int p = idx / D, c = idx % D;
@@ -387,7 +474,7 @@ __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, f
     // A_hat[r][i] = sum_c k^_rc k^_ic e^{G_rc - G_ic} (i < r); A_qk the same with q^ (i <= r)
     pair_products(w, full, ga);
     // T = (I + diag(beta) A_hat)^-1
-    tri_inverse(w, sA, sT);
+    tri_inverse(w, sA, sT, ga);
     // W = T (beta K^e^G), U = T (beta V)
     gemm<C, D, C, false, false>(1.f, w + Ws::TM, w + Ws::BK, false, w + Ws::W, D, ga, gb);
     gemm<C, D, C, false, false>(1.f, w + Ws::TM, w + Ws::BV, false, w + Ws::U, D, ga, gb);
