@@ -117,8 +117,9 @@ __device__ __forceinline__ void stage(float *dst, const float *src) {
 // C(M x N) = alpha * op(A) op(B) + (accumulate ? C : 0), CTA-wide.  A is stored row-major as
 // [M][K] (or [K][M] when transA), B as [K][N] (or [N][K] when transB), both contiguous; C(i, j)
 // = Cm[i*ldc + j].  M % 16 == N % 8 == K % 8 == 0.  Both operands are first copied to shared
-// memory (float4, padded rows); each warp then owns 16x8 output tiles, splitting both operands
-// into tf32 hi + lo parts and accumulating hi*hi + hi*lo + lo*hi.  Ends with a CTA barrier.
+// memory (float4, padded rows); each warp then owns a strip of 16x8 output tiles of one 16-row
+// block, splitting both operands into tf32 hi + lo parts and accumulating hi*hi + hi*lo + lo*hi.
+// Ends with a CTA barrier.
 template <int M, int N, int K, bool transA, bool transB>
 __device__ void gemm(float alpha, const float *A, const float *B, bool accumulate, float *Cm, int ldc, float *sa,
                      float *sb) {
@@ -131,26 +132,53 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
     __syncthreads();
     constexpr int ar = transA ? 1 : ald, ac = transA ? ald : 1;
     constexpr int br = transB ? 1 : bld, bc = transB ? bld : 1;
-    constexpr int nt = N / 8, tiles = (M / 16) * nt;
-    for (int t = warp; t < tiles; t += kWarps) {
-        const int i0 = (t / nt) * 16, j0 = (t % nt) * 8;
-        float *c0 = Cm + (i0 + gq) * ldc + j0 + 2 * tq, *c1 = c0 + 8 * ldc;
+    // each warp owns a 16-row strip of kTpw consecutive 16x8 tiles, taken kSub at a time, so that
+    // one split A fragment serves kSub tiles
+    constexpr int nt = N / 8, tiles = (M / 16) * nt, kTpw = tiles / kWarps, kSub = kTpw < 4 ? kTpw : 4;
+    static_assert(tiles % kWarps == 0 && nt % kTpw == 0 && kTpw % kSub == 0, "tile split");
+    const int t0 = warp * kTpw, i0 = (t0 / nt) * 16;
+#pragma unroll 1
+    for (int sub = 0; sub < kTpw; sub += kSub) {
+        const int jb = (t0 % nt + sub) * 8;
+        float *c0 = Cm + (i0 + gq) * ldc + jb + 2 * tq, *c1 = c0 + 8 * ldc;
         // the values accumulated onto are fetched before the products, so their latency overlaps them
-        float2 p0 = make_float2(0.f, 0.f), p1 = p0;
-        if (accumulate) {
-            p0 = *reinterpret_cast<const float2 *>(c0);
-            p1 = *reinterpret_cast<const float2 *>(c1);
+        float2 p0[kSub], p1[kSub];
+#pragma unroll
+        for (int j = 0; j < kSub; ++j) {
+            p0[j] = accumulate ? *reinterpret_cast<const float2 *>(c0 + 8 * j) : make_float2(0.f, 0.f);
+            p1[j] = accumulate ? *reinterpret_cast<const float2 *>(c1 + 8 * j) : make_float2(0.f, 0.f);
         }
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+        float acc[kSub][4];
+#pragma unroll
+        for (int j = 0; j < kSub; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll 2
         for (int k0 = 0; k0 < K; k0 += 8) {
             const float av[4] = {sa[(i0 + gq) * ar + (k0 + tq) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq) * ac],
                                  sa[(i0 + gq) * ar + (k0 + tq + 4) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq + 4) * ac]};
-            const float bv0 = sb[(k0 + tq) * br + (j0 + gq) * bc], bv1 = sb[(k0 + tq + 4) * br + (j0 + gq) * bc];
-            mma3(acc, av, bv0, bv1);
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ah[e] = tf32_hi(av[e]);
+                al[e] = tf32_lo(av[e], ah[e]);
+            }
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                const float bv0 = sb[(k0 + tq) * br + (jb + 8 * j + gq) * bc];
+                const float bv1 = sb[(k0 + tq + 4) * br + (jb + 8 * j + gq) * bc];
+                const uint32_t bh0 = tf32_hi(bv0), bh1 = tf32_hi(bv1);
+                const uint32_t bl0 = tf32_lo(bv0, bh0), bl1 = tf32_lo(bv1, bh1);
+                mma_tf32(acc[j], al, bh0, bh1);
+                mma_tf32(acc[j], ah, bl0, bl1);
+                mma_tf32(acc[j], ah, bh0, bh1);
+            }
         }
-        *reinterpret_cast<float2 *>(c0) = make_float2(fmaf(alpha, acc[0], p0.x), fmaf(alpha, acc[1], p0.y));
-        *reinterpret_cast<float2 *>(c1) = make_float2(fmaf(alpha, acc[2], p1.x), fmaf(alpha, acc[3], p1.y));
+#pragma unroll
+        for (int j = 0; j < kSub; ++j) {
+            *reinterpret_cast<float2 *>(c0 + 8 * j) =
+                make_float2(fmaf(alpha, acc[j][0], p0[j].x), fmaf(alpha, acc[j][1], p0[j].y));
+            *reinterpret_cast<float2 *>(c1 + 8 * j) =
+                make_float2(fmaf(alpha, acc[j][2], p1[j].x), fmaf(alpha, acc[j][3], p1[j].y));
+        }
     }
     __syncthreads();
 }
