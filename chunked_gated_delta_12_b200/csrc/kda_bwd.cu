@@ -73,7 +73,18 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// acc(16x8) += op(A)(16 x 8k) op(B)(8k x 8) with tf32 hi/lo splits (see gemm); a[e], b[e] fp32
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for two values packed as bf16x2 (the lower
+// k index in the low half); hi*hi + hi*lo + lo*hi then carries about 2^-17 relative error per
+// product, with twice the k-depth of a tf32 instruction per bf16 one
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// acc(16x8) += op(A)(16 x 8k) op(B)(8k x 8) with tf32 hi/lo splits; a[e], b[e] fp32
 __device__ __forceinline__ void mma3(float (&acc)[4], const float (&av)[4], float bv0, float bv1) {
     uint32_t ah[4], al[4];
 #pragma unroll
@@ -116,10 +127,10 @@ __device__ __forceinline__ void stage(float *dst, const float *src) {
 
 // C(M x N) = alpha * op(A) op(B) + (accumulate ? C : 0), CTA-wide.  A is stored row-major as
 // [M][K] (or [K][M] when transA), B as [K][N] (or [N][K] when transB), both contiguous; C(i, j)
-// = Cm[i*ldc + j].  M % 16 == N % 8 == K % 8 == 0.  Both operands are first copied to shared
+// = Cm[i*ldc + j].  M % 16 == N % 8 == 0.  Both operands are first copied to shared
 // memory (float4, padded rows); each warp then owns a strip of 16x8 output tiles of one 16-row
-// block, splitting both operands into tf32 hi + lo parts and accumulating hi*hi + hi*lo + lo*hi.
-// Ends with a CTA barrier.
+// block, splitting both operands into bf16 hi + lo parts (split_bf16) and accumulating
+// hi*hi + hi*lo + lo*hi with m16n8k16 warp MMAs.  K % 16 == 0.  Ends with a CTA barrier.
 template <int M, int N, int K, bool transA, bool transB>
 __device__ void gemm(float alpha, const float *A, const float *B, bool accumulate, float *Cm, int ldc, float *sa,
                      float *sb) {
@@ -136,6 +147,7 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
     // one split A fragment serves kSub tiles
     constexpr int nt = N / 8, tiles = (M / 16) * nt, kTpw = tiles / kWarps, kSub = kTpw < 4 ? kTpw : 4;
     static_assert(tiles % kWarps == 0 && nt % kTpw == 0 && kTpw % kSub == 0, "tile split");
+    static_assert(K % 16 == 0, "k-steps of 16");
     const int t0 = warp * kTpw, i0 = (t0 / nt) * 16;
 #pragma unroll 1
     for (int sub = 0; sub < kTpw; sub += kSub) {
@@ -152,24 +164,27 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
 #pragma unroll
         for (int j = 0; j < kSub; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 #pragma unroll 2
-        for (int k0 = 0; k0 < K; k0 += 8) {
-            const float av[4] = {sa[(i0 + gq) * ar + (k0 + tq) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq) * ac],
-                                 sa[(i0 + gq) * ar + (k0 + tq + 4) * ac], sa[(i0 + gq + 8) * ar + (k0 + tq + 4) * ac]};
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            // A fragment of m16n8k16: rows gq, gq+8; k pairs (2tq, 2tq+1) and (2tq+8, 2tq+9)
+            const int ka = k0 + 2 * tq;
+            const float x00 = sa[(i0 + gq) * ar + ka * ac], x01 = sa[(i0 + gq) * ar + (ka + 1) * ac];
+            const float x10 = sa[(i0 + gq + 8) * ar + ka * ac], x11 = sa[(i0 + gq + 8) * ar + (ka + 1) * ac];
+            const float x02 = sa[(i0 + gq) * ar + (ka + 8) * ac], x03 = sa[(i0 + gq) * ar + (ka + 9) * ac];
+            const float x12 = sa[(i0 + gq + 8) * ar + (ka + 8) * ac], x13 = sa[(i0 + gq + 8) * ar + (ka + 9) * ac];
             uint32_t ah[4], al[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ah[e] = tf32_hi(av[e]);
-                al[e] = tf32_lo(av[e], ah[e]);
-            }
+            split_bf16(x00, x01, ah[0], al[0]);
+            split_bf16(x10, x11, ah[1], al[1]);
+            split_bf16(x02, x03, ah[2], al[2]);
+            split_bf16(x12, x13, ah[3], al[3]);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
-                const float bv0 = sb[(k0 + tq) * br + (jb + 8 * j + gq) * bc];
-                const float bv1 = sb[(k0 + tq + 4) * br + (jb + 8 * j + gq) * bc];
-                const uint32_t bh0 = tf32_hi(bv0), bh1 = tf32_hi(bv1);
-                const uint32_t bl0 = tf32_lo(bv0, bh0), bl1 = tf32_lo(bv1, bh1);
-                mma_tf32(acc[j], al, bh0, bh1);
-                mma_tf32(acc[j], ah, bl0, bl1);
-                mma_tf32(acc[j], ah, bh0, bh1);
+                const int col = jb + 8 * j + gq;
+                uint32_t bh0, bl0, bh1, bl1;
+                split_bf16(sb[ka * br + col * bc], sb[(ka + 1) * br + col * bc], bh0, bl0);
+                split_bf16(sb[(ka + 8) * br + col * bc], sb[(ka + 9) * br + col * bc], bh1, bl1);
+                mma_bf16(acc[j], al, bh0, bh1);
+                mma_bf16(acc[j], ah, bl0, bl1);
+                mma_bf16(acc[j], ah, bh0, bh1);
             }
         }
 #pragma unroll
