@@ -595,8 +595,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
         {
             const int c = tid >> 2, part = tid & 3;
             float acc = 0.f;
-#pragma unroll 8
-            for (int x = part; x < D; x += 4) acc += Sin[c * D + x] * dS[c * D + x];
+#pragma unroll
+            for (int x = 32 * part; x < 32 * part + 32; x += 4) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(Sin + c * D + x);
+                const float4 d4 = *reinterpret_cast<const float4 *>(dS + c * D + x);
+                acc += s4.x * d4.x + s4.y * d4.y + s4.z * d4.z + s4.w * d4.w;
+            }
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             if (part == 0) w[Ws::DGL + c] = w[Ws::DL + c] * acc;
@@ -614,39 +618,73 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
         gemm<C, C, C, false, true>(-1.f, w + Ws::XM, w + Ws::TM, false, w + Ws::DAH, C, ga, gb);
         // dbeta (rows), dv, dKG = beta dBk, dA_hat = beta dA_kk
         for (int r = warp; r < C; r += kWarps) {
-            float acc = 0.f;
-            for (int c = lane; c < D; c += 32)
-                acc += w[Ws::DBV + r * D + c] * w[Ws::VV + r * D + c] + w[Ws::DBK + r * D + c] * w[Ws::KG + r * D + c];
-            for (int i = lane; i < C; i += 32)
-                if (i < r) acc += w[Ws::DAH + r * C + i] * w[Ws::AH + r * C + i];
+            const int c4 = r * D + 4 * lane;
+            const float4 dbv = *reinterpret_cast<const float4 *>(w + Ws::DBV + c4);
+            const float4 vv4 = *reinterpret_cast<const float4 *>(w + Ws::VV + c4);
+            const float4 dbk = *reinterpret_cast<const float4 *>(w + Ws::DBK + c4);
+            const float4 kg4 = *reinterpret_cast<const float4 *>(w + Ws::KG + c4);
+            float acc = dbv.x * vv4.x + dbv.y * vv4.y + dbv.z * vv4.z + dbv.w * vv4.w + dbk.x * kg4.x + dbk.y * kg4.y +
+                        dbk.z * kg4.z + dbk.w * kg4.w;
+            const float2 dah = *reinterpret_cast<const float2 *>(w + Ws::DAH + r * C + 2 * lane);
+            const float2 ah = *reinterpret_cast<const float2 *>(w + Ws::AH + r * C + 2 * lane);
+            if (2 * lane < r) acc += dah.x * ah.x;
+            if (2 * lane + 1 < r) acc += dah.y * ah.y;
 #pragma unroll
             for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
             if (lane == 0) w[Ws::DB + r] = acc;
         }
         __syncthreads();
-        for (int idx = tid; idx < CC; idx += kThreads) {
+        for (int idx = 4 * tid; idx < CC; idx += 4 * kThreads) {
             const int r = idx / C, i = idx % C;
-            w[Ws::DAH + idx] = i < r ? w[Ws::BB + r] * w[Ws::DAH + idx] : 0.f;
+            const float b = w[Ws::BB + r];
+            const float4 x = *reinterpret_cast<const float4 *>(w + Ws::DAH + idx);
+            *reinterpret_cast<float4 *>(w + Ws::DAH + idx) =
+                make_float4(i < r ? b * x.x : 0.f, i + 1 < r ? b * x.y : 0.f, i + 2 < r ? b * x.z : 0.f,
+                            i + 3 < r ? b * x.w : 0.f);
         }
-        for (int idx = tid; idx < CD; idx += kThreads) {
+        for (int idx = 4 * tid; idx < CD; idx += 4 * kThreads) {
             const int r = idx / D;
             const float b = w[Ws::BB + r];
-            if (r < L) a.dv[((tok0 + r) * H + h) * D + idx % D] = f2bf(b * w[Ws::DBV + idx]);
-            w[Ws::DBK + idx] *= b;                              // now dKG
+            const float4 dbv = *reinterpret_cast<const float4 *>(w + Ws::DBV + idx);
+            if (r < L)
+                *reinterpret_cast<uint2 *>(a.dv + ((tok0 + r) * H + h) * D + idx % D) =
+                    make_uint2((uint32_t)f2bf(b * dbv.x) | ((uint32_t)f2bf(b * dbv.y) << 16),
+                               (uint32_t)f2bf(b * dbv.z) | ((uint32_t)f2bf(b * dbv.w) << 16));
+            const float4 dbk = *reinterpret_cast<const float4 *>(w + Ws::DBK + idx);
+            *reinterpret_cast<float4 *>(w + Ws::DBK + idx) = make_float4(b * dbk.x, b * dbk.y, b * dbk.z, b * dbk.w);   // now dKG
         }
         __syncthreads();
         // pairwise-decay sums (block MMA), then the elementwise chain rule per (row r, channel c)
         pair_grads(w, ga);
-        for (int idx = tid; idx < CD; idx += kThreads) {
+        for (int idx = 4 * tid; idx < CD; idx += 4 * kThreads) {
             const int c = idx % D;
-            const float a1 = w[Ws::DKN + idx], a3 = w[Ws::DQN + idx], a24 = w[Ws::A24 + idx];
-            const float knv = w[Ws::KN + idx], qnv = w[Ws::QN + idx], eg = w[Ws::EG + idx];
-            const float dKG = w[Ws::DBK + idx], dQG = w[Ws::DQG + idx], dKd = w[Ws::DKD + idx];
-            const float e3 = expf(w[Ws::G + (C - 1) * D + c] - w[Ws::G + idx]);
-            w[Ws::DKN + idx] = a1 + a24 + dKG * eg + dKd * e3;
-            w[Ws::DQN + idx] = a3 + dQG * eg;
-            w[Ws::DG + idx] = knv * (a1 - a24) + qnv * a3 + dKG * w[Ws::KG + idx] + dQG * w[Ws::QG + idx] -
-                              dKd * w[Ws::KD + idx];
+            auto ld4 = [&](size_t off) {
+                const float4 x = *reinterpret_cast<const float4 *>(w + off + idx);
+                return x;
+            };
+            const float4 a1 = ld4(Ws::DKN), a3 = ld4(Ws::DQN), a24 = ld4(Ws::A24), knv = ld4(Ws::KN), qnv = ld4(Ws::QN);
+            const float4 eg = ld4(Ws::EG), dKG = ld4(Ws::DBK), dQG = ld4(Ws::DQG), dKd = ld4(Ws::DKD), kg = ld4(Ws::KG);
+            const float4 qg = ld4(Ws::QG), kd = ld4(Ws::KD), gr = ld4(Ws::G);
+            const float4 gl = *reinterpret_cast<const float4 *>(w + Ws::G + (C - 1) * D + c);
+            const float a1v[4] = {a1.x, a1.y, a1.z, a1.w}, a3v[4] = {a3.x, a3.y, a3.z, a3.w};
+            const float a24v[4] = {a24.x, a24.y, a24.z, a24.w}, knvv[4] = {knv.x, knv.y, knv.z, knv.w};
+            const float qnvv[4] = {qnv.x, qnv.y, qnv.z, qnv.w}, egv[4] = {eg.x, eg.y, eg.z, eg.w};
+            const float dkgv[4] = {dKG.x, dKG.y, dKG.z, dKG.w}, dqgv[4] = {dQG.x, dQG.y, dQG.z, dQG.w};
+            const float dkdv[4] = {dKd.x, dKd.y, dKd.z, dKd.w}, kgv[4] = {kg.x, kg.y, kg.z, kg.w};
+            const float qgv[4] = {qg.x, qg.y, qg.z, qg.w}, kdv[4] = {kd.x, kd.y, kd.z, kd.w};
+            const float grv[4] = {gr.x, gr.y, gr.z, gr.w}, glv[4] = {gl.x, gl.y, gl.z, gl.w};
+            float dkn[4], dqn[4], dg[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float e3 = expf(glv[j] - grv[j]);
+                dkn[j] = a1v[j] + a24v[j] + dkgv[j] * egv[j] + dkdv[j] * e3;
+                dqn[j] = a3v[j] + dqgv[j] * egv[j];
+                dg[j] = knvv[j] * (a1v[j] - a24v[j]) + qnvv[j] * a3v[j] + dkgv[j] * kgv[j] + dqgv[j] * qgv[j] -
+                        dkdv[j] * kdv[j];
+            }
+            *reinterpret_cast<float4 *>(w + Ws::DKN + idx) = make_float4(dkn[0], dkn[1], dkn[2], dkn[3]);
+            *reinterpret_cast<float4 *>(w + Ws::DQN + idx) = make_float4(dqn[0], dqn[1], dqn[2], dqn[3]);
+            *reinterpret_cast<float4 *>(w + Ws::DG + idx) = make_float4(dg[0], dg[1], dg[2], dg[3]);
         }
         __syncthreads();
         // dg: reverse cumsum of dG per channel, plus the G_last terms (which reach every row):
@@ -682,11 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
         // dq, dk through the l2 norms; dbeta
         for (int r = warp; r < C; r += kWarps) {
             if (r >= L) continue;
-            float sq = 0.f, sk = 0.f;
-            for (int c = lane; c < D; c += 32) {
-                sq += w[Ws::QN + r * D + c] * w[Ws::DQN + r * D + c];
-                sk += w[Ws::KN + r * D + c] * w[Ws::DKN + r * D + c];
-            }
+            const int c4 = r * D + 4 * lane;
+            const float4 qn4 = *reinterpret_cast<const float4 *>(w + Ws::QN + c4);
+            const float4 dqn4 = *reinterpret_cast<const float4 *>(w + Ws::DQN + c4);
+            const float4 kn4 = *reinterpret_cast<const float4 *>(w + Ws::KN + c4);
+            const float4 dkn4 = *reinterpret_cast<const float4 *>(w + Ws::DKN + c4);
+            float sq = qn4.x * dqn4.x + qn4.y * dqn4.y + qn4.z * dqn4.z + qn4.w * dqn4.w;
+            float sk = kn4.x * dkn4.x + kn4.y * dkn4.y + kn4.z * dkn4.z + kn4.w * dkn4.w;
 #pragma unroll
             for (int o = 16; o; o >>= 1) {
                 sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -694,10 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
             }
             const float iq = w[Ws::RQ + r], ik = w[Ws::RK + r];
             const int64_t row = ((tok0 + r) * H + h) * D;
-            for (int c = lane; c < D; c += 32) {
-                a.dq[row + c] = f2bf(iq * (w[Ws::DQN + r * D + c] - w[Ws::QN + r * D + c] * sq));
-                a.dk[row + c] = f2bf(ik * (w[Ws::DKN + r * D + c] - w[Ws::KN + r * D + c] * sk));
-            }
+            auto pk = [](float x0, float x1) { return (uint32_t)f2bf(x0) | ((uint32_t)f2bf(x1) << 16); };
+            *reinterpret_cast<uint2 *>(a.dq + row + 4 * lane) =
+                make_uint2(pk(iq * (dqn4.x - qn4.x * sq), iq * (dqn4.y - qn4.y * sq)),
+                           pk(iq * (dqn4.z - qn4.z * sq), iq * (dqn4.w - qn4.w * sq)));
+            *reinterpret_cast<uint2 *>(a.dk + row + 4 * lane) =
+                make_uint2(pk(ik * (dkn4.x - kn4.x * sk), ik * (dkn4.y - kn4.y * sk)),
+                           pk(ik * (dkn4.z - kn4.z * sk), ik * (dkn4.w - kn4.w * sk)));
             if (lane == 0) a.dbeta[(tok0 + r) * H + h] = w[Ws::DB + r];
         }
         __syncthreads();
