@@ -5,13 +5,13 @@
 // recompute backward with these outputs (kda_fused page of
 // nemo_automodel.components.models.kimi_k3, the backward of fused_chunk_kda).
 //
-// One CTA per (document, head) chain, two sweeps over the chain's 64-token chunks:
+// First the pipelined forward kernel (kda_fwd_pipe.cu) runs over the same inputs and writes the
+// state entering every chunk into the workspace's checkpoint slots (its output o goes to dq, which is
+// overwritten here).  Then one CTA per (document, head) chain walks the chain's 64-token chunks in
+// reverse, carrying dS (the gradient of the state leaving the chunk):
 //
-//  forward sweep   per chunk: recompute A_kk, T = (I + A_kk)^-1, W = T diag(beta) K^e^G,
-//                  U = T diag(beta) V; store the entering state S in the workspace;
-//                  U~ = U - W S;  S <- Diag(e^{G_last}) S + Kd^T U~
-//  reverse sweep   per chunk, carrying dS (gradient of the state leaving the chunk):
-//                  recompute the chunk's factors, then
+//  reverse sweep   per chunk: recompute A_kk, T = (I + A_kk)^-1, W = T diag(beta) K^e^G,
+//                  U = T diag(beta) V, then
 //                  dU~ = A_qk^T dO + Kd dS,  dS_in = (Q^e^G)^T dO + Diag(e^{G_last}) dS - W^T dU~,
 //                  dQG = dO S^T, dA_qk = lower(dO U~^T), dKd = U~ dS^T, dW = -dU~ S^T,
 //                  dT = dW (beta KG)^T + dU~ (beta V)^T, dA_kk = strict_lower(-T^T dT T^T),
@@ -20,11 +20,11 @@
 //
 // G is the in-chunk inclusive cumsum of g.  Pairwise decays e^{G_r - G_i} (r >= i) are
 // split at 16-row blocks, e^{G_r - G_16R} s_RI e^{G_16I+15 - G_i} with
-// s_RI = e^{G_16R - G_16I+15}, so no factor leaves the fp32 range.  Matrix products run
-// on tf32 warp MMA with a hi/lo split of both operands (three products per tile, close
-// to fp32 accuracy); the triangular inverse, the pairwise-decay sums and all elementwise
-// work are fp32.  Per-chain scratch lives in the caller's workspace (L2-resident for the
-// chains that run at once); libkda allocates nothing.
+// s_RI = e^{G_16R - G_16I+15}, so no factor leaves the fp32 range.  The chunk products run
+// on bf16 warp MMA with a hi/lo split of both operands (gemm), the pairwise-decay products on
+// tf32 warp MMA with a hi/lo split (three products per tile in both, about 2^-17 and 2^-21
+// relative error per product); the triangular inverse and all elementwise work are fp32.
+// Per-chain scratch lives in the caller's workspace; libkda allocates nothing.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -389,7 +389,7 @@ struct Args {
 __device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, float *ga, float *gb, float *sred,
                                 int64_t tok0, int L, int h, bool full) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float *qn = w + Ws::QN, *kn = w + Ws::KN, *vv = w + Ws::VV, *G = w + Ws::G, *eg = w + Ws::EG;
+    float *qn = w + Ws::QN, *kn = w + Ws::KN, *vv = w + Ws::VV, *G = w + Ws::G;
     float *rq = w + Ws::RQ, *rk = w + Ws::RK, *bb = w + Ws::BB;
     const int H = a.H;
     // raw rows, four channels per access (rows >= L are zero: they then add nothing to any product)
@@ -541,29 +541,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
     const int nch = (int)((d1 - d0 + C - 1) / C);
     const int64_t slot0 = d0 / C + doc;                     // checkpoint slots of this document
     float *w = a.scratch + (size_t)chain * Ws::TOTAL;
-    float *S = w + Ws::S;
     float *ga = smem, *gb = smem + kOpFloats;                 // gemm operand buffers
     float *sA = gb + kOpFloats, *sT = sA + C * (C + 1);       // triangular inverse
     float *sred = sT + C * (C + 1);                           // [4][128] partial sums
 
-    // ---------------- forward sweep: entering states ----------------
-    for (int idx = tid; idx < DD; idx += kThreads) S[idx] = 0.f;
-    __syncthreads();
-    for (int n = 0; n < nch; ++n) {
-        const int64_t tok0 = d0 + (int64_t)n * C;
-        const int L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
-        recompute_chunk(a, w, sA, sT, ga, gb, sred, tok0, L, h, false);
-        float *ck = a.ckpt + ((size_t)(slot0 + n) * H + h) * DD;
-        for (int idx = tid; idx < DD; idx += kThreads) ck[idx] = S[idx];
-        // U~ = U - W S
-        for (int idx = tid; idx < CD; idx += kThreads) w[Ws::UT + idx] = w[Ws::U + idx];
-        __syncthreads();
-        gemm<C, D, D, false, false>(-1.f, w + Ws::W, S, true, w + Ws::UT, D, ga, gb);
-        // S <- Diag(e^{G_last}) S + Kd^T U~
-        for (int idx = tid; idx < DD; idx += kThreads) S[idx] *= w[Ws::DL + idx / D];
-        __syncthreads();
-        gemm<D, D, C, true, false>(1.f, w + Ws::KD, w + Ws::UT, true, S, D, ga, gb);
-    }
+    // The state entering every chunk is in the checkpoint slots: the pipelined forward kernel wrote
+    // them (launch_bwd runs it first).
 
     // ---------------- reverse sweep ----------------
     float *dS = w + Ws::DS, *dSn = w + Ws::DSN;
@@ -767,6 +750,10 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     a.ckpt = workspace;
     a.scratch = workspace + ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * bwd::DD;
     a.status = status;
+    // forward pass first: the pipelined forward kernel writes the state entering every chunk into the
+    // checkpoint slots; its output o goes to dq, which the backward overwrites
+    cudaError_t e0 = launch_fwd_pipe(q, k, v, g, beta, cu, n_docs, T, H, nullptr, nullptr, dq, status, stream, a.ckpt);
+    if (e0 != cudaSuccess) return e0;
     constexpr int smem = (2 * bwd::kOpFloats + 2 * bwd::C * (bwd::C + 1) + 4 * bwd::D) * (int)sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd::kda_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

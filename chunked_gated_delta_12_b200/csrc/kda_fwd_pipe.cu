@@ -166,7 +166,7 @@ struct Maps {
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
                         const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
-                        const float *h0, float *ht, uint16_t *__restrict__ out,
+                        const float *h0, float *ht, float *ckpt, uint16_t *__restrict__ out,
                         int *__restrict__ status) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
@@ -808,6 +808,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float(&cur)[16] = (ch & 1) ? sb : sa;
                         float(&nxt)[16] = (ch & 1) ? sa : sb;
                         if (ch < 7) tc::ld16(lane_base + kSF + 16 * (ch + 1), nxt);
+                        if (ckpt) {
+                            // the state entering chunk n, S[c][v] fp32, into its checkpoint slot
+                            float *ck = ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) * (kHeadDim * kHeadDim) +
+                                        (size_t)(16 * ch) * kHeadDim + 32 * lq + lane;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) ck[(size_t)i * kHeadDim] = cur[i];
+                        }
                         sprep(cur, 16 * ch);
                         if (ch == 3) state_mma(0);
                         if (ch < 7) {
@@ -996,7 +1003,7 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
 
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, const float *h0,
-                            float *ht, uint16_t *out, int *status, cudaStream_t stream) {
+                            float *ht, uint16_t *out, int *status, cudaStream_t stream, float *ckpt) {
     using namespace pipe_path;
     Maps maps;
     const uint64_t cols = (uint64_t)H * kHeadDim;
@@ -1010,8 +1017,8 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
     cudaError_t e = cudaFuncSetAttribute(kda_fwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (int64_t)n_docs * H;
-    kda_fwd_pipe_kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, out,
-                                                                        status);
+    kda_fwd_pipe_kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt,
+                                                                        out, status);
     return cudaGetLastError();
 }
 

@@ -14,9 +14,12 @@ constexpr int kStatusTimeout = 5;
 // columns, two chunks in flight (intra-chunk work of chunk s overlapped with the
 // state update of chunk s-1).
 // h0 / ht: optional initial / final states, [n_docs * H][128][128] fp32 (NULL: zero / not written).
+// ckpt: optional, receives the state entering every chunk, S[c][v] fp32, in slot
+// (cu[d] / 64 + d + j) * H + h for chunk j of document d (the backward's checkpoint layout).
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
-                            const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream);
+                            const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream,
+                            float *ckpt = nullptr);
 
 // Token-by-token forward (the recurrence itself, no chunking): one CTA of 128 threads per
 // (document, head), the state in registers.  Same arguments and contract as launch_fwd_pipe.
