@@ -217,12 +217,18 @@ def run_reference(args, w, d):
     print(json.dumps(line), flush=True)
 
 
-def bench_backward(kda, steps: int, dev, stream, barrier) -> dict:
+def bench_backward(kda, steps: int, dev, stream, barrier, shape=None) -> dict:
     """Device time of kda_chunk_bwd on the packed forward+backward workload (16 documents,
-    H = 32), inputs resident, workspace allocated once; max over ranks."""
+    H = 32), or on a dense DOCSxLEN:H `shape`, inputs resident, workspace allocated once; max over
+    ranks."""
     import torch
-    from chunked_gated_delta_12_b200.inputs import generate, workload
-    wb = workload(4)
+    from chunked_gated_delta_12_b200.inputs import custom_workload, generate, workload
+    if shape:
+        docs_len, heads = shape.split(":")
+        n_docs, doc_len = (int(x) for x in docs_len.split("x"))
+        wb = custom_workload(f"dense_{n_docs}x{doc_len}_H{heads}", [doc_len] * n_docs, int(heads), seed=20264)
+    else:
+        wb = workload(4)
     db = generate(wb, with_grad=True)
     t = {}
     for key in ("q", "k", "v", "do"):
@@ -314,6 +320,8 @@ def main():
     ap.add_argument("--dec-steps", type=int, default=20,
                     help="timed launches of the token-by-token kernel on one decoding step of 256 "
                          "sequences, reported under 'decode' (0 skips it)")
+    ap.add_argument("--bwd-shape", default=None,
+                    help="DOCSxLEN:H -- run the backward on a custom dense workload instead (profiling)")
     ap.add_argument("--shape", default=None,
                     help="DOCSxLEN:H -- a custom dense workload with the same distributions "
                          "(e.g. 4x2048:32 for a profiling case larger than L2)")
@@ -425,7 +433,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
     }
     if args.bwd_steps > 0:
-        line["backward"] = bench_backward(kda, args.bwd_steps, dev, stream, barrier)
+        line["backward"] = bench_backward(kda, args.bwd_steps, dev, stream, barrier, args.bwd_shape)
     if args.dec_steps > 0:
         line["decode"] = bench_decode(kda, args.dec_steps, dev, stream, barrier)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

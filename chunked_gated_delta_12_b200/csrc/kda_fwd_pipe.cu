@@ -163,6 +163,9 @@ struct Maps {
     CUtensorMap q, k, g, v, o;
 };
 
+// kCkpt: also store the state entering every chunk into `ckpt` (the backward's checkpoints); a
+// separate instance, so that the plain forward carries no trace of it
+template <bool kCkpt>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
                         const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
@@ -808,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float(&cur)[16] = (ch & 1) ? sb : sa;
                         float(&nxt)[16] = (ch & 1) ? sa : sb;
                         if (ch < 7) tc::ld16(lane_base + kSF + 16 * (ch + 1), nxt);
-                        if (ckpt) {
+                        if constexpr (kCkpt) {
                             // the state entering chunk n, S[c][v] fp32, into its checkpoint slot
                             float *ck = ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) * (kHeadDim * kHeadDim) +
                                         (size_t)(16 * ch) * kHeadDim + 32 * lq + lane;
@@ -1014,11 +1017,11 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
         !make_map(&maps.o, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     constexpr int bytes = Smem::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(kda_fwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    auto kernel = ckpt ? kda_fwd_pipe_kernel<true> : kda_fwd_pipe_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (int64_t)n_docs * H;
-    kda_fwd_pipe_kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt,
-                                                                        out, status);
+    kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt, out, status);
     return cudaGetLastError();
 }
 
