@@ -43,7 +43,7 @@ constexpr int CD = C * D, CC = C * C, DD = D * D;
 
 // per-chain scratch, in floats
 struct Ws {
-    static constexpr size_t S = 0, DS = S + DD, DSN = DS + DD;
+    static constexpr size_t DS = 0, DSN = DS + DD;
     static constexpr size_t QN = DSN + DD, KN = QN + CD, VV = KN + CD, DO = VV + CD, G = DO + CD, EG = G + CD,
                             KG = EG + CD, QG = KG + CD, KD = QG + CD, BK = KD + CD, BV = BK + CD, W = BV + CD,
                             U = W + CD, UT = U + CD, DUT = UT + CD, DQG = DUT + CD, DKD = DQG + CD, DW = DKD + CD,
@@ -137,12 +137,12 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
     constexpr int acols = transA ? M : K, arows = transA ? K : M;
     constexpr int bcols = transB ? K : N, brows = transB ? N : K;
-    constexpr int ald = acols + kPad, bld = bcols + kPad;
+    // row pads: an operand read along its rows (k pairs contiguous) is read as float2 and padded by 8
+    // floats; one read across its rows is padded by 4; both patterns are then free of bank conflicts
+    constexpr int ald = acols + (transA ? 4 : kPad), bld = bcols + (transB ? kPad : 4);
     stage<arows, acols, ald>(sa, A);
     stage<brows, bcols, bld>(sb, B);
     __syncthreads();
-    constexpr int ar = transA ? 1 : ald, ac = transA ? ald : 1;
-    constexpr int br = transB ? 1 : bld, bc = transB ? bld : 1;
     // each warp owns a 16-row strip of kTpw consecutive 16x8 tiles, taken kSub at a time, so that
     // one split A fragment serves kSub tiles
     constexpr int nt = N / 8, tiles = (M / 16) * nt, kTpw = tiles / kWarps, kSub = kTpw < 4 ? kTpw : 4;
@@ -167,21 +167,35 @@ __device__ void gemm(float alpha, const float *A, const float *B, bool accumulat
         for (int k0 = 0; k0 < K; k0 += 16) {
             // A fragment of m16n8k16: rows gq, gq+8; k pairs (2tq, 2tq+1) and (2tq+8, 2tq+9)
             const int ka = k0 + 2 * tq;
-            const float x00 = sa[(i0 + gq) * ar + ka * ac], x01 = sa[(i0 + gq) * ar + (ka + 1) * ac];
-            const float x10 = sa[(i0 + gq + 8) * ar + ka * ac], x11 = sa[(i0 + gq + 8) * ar + (ka + 1) * ac];
-            const float x02 = sa[(i0 + gq) * ar + (ka + 8) * ac], x03 = sa[(i0 + gq) * ar + (ka + 9) * ac];
-            const float x12 = sa[(i0 + gq + 8) * ar + (ka + 8) * ac], x13 = sa[(i0 + gq + 8) * ar + (ka + 9) * ac];
             uint32_t ah[4], al[4];
-            split_bf16(x00, x01, ah[0], al[0]);
-            split_bf16(x10, x11, ah[1], al[1]);
-            split_bf16(x02, x03, ah[2], al[2]);
-            split_bf16(x12, x13, ah[3], al[3]);
+            if constexpr (!transA) {
+                const float2 x0 = *reinterpret_cast<const float2 *>(sa + (i0 + gq) * ald + ka);
+                const float2 x1 = *reinterpret_cast<const float2 *>(sa + (i0 + gq + 8) * ald + ka);
+                const float2 x2 = *reinterpret_cast<const float2 *>(sa + (i0 + gq) * ald + ka + 8);
+                const float2 x3 = *reinterpret_cast<const float2 *>(sa + (i0 + gq + 8) * ald + ka + 8);
+                split_bf16(x0.x, x0.y, ah[0], al[0]);
+                split_bf16(x1.x, x1.y, ah[1], al[1]);
+                split_bf16(x2.x, x2.y, ah[2], al[2]);
+                split_bf16(x3.x, x3.y, ah[3], al[3]);
+            } else {
+                split_bf16(sa[ka * ald + i0 + gq], sa[(ka + 1) * ald + i0 + gq], ah[0], al[0]);
+                split_bf16(sa[ka * ald + i0 + gq + 8], sa[(ka + 1) * ald + i0 + gq + 8], ah[1], al[1]);
+                split_bf16(sa[(ka + 8) * ald + i0 + gq], sa[(ka + 9) * ald + i0 + gq], ah[2], al[2]);
+                split_bf16(sa[(ka + 8) * ald + i0 + gq + 8], sa[(ka + 9) * ald + i0 + gq + 8], ah[3], al[3]);
+            }
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
                 const int col = jb + 8 * j + gq;
                 uint32_t bh0, bl0, bh1, bl1;
-                split_bf16(sb[ka * br + col * bc], sb[(ka + 1) * br + col * bc], bh0, bl0);
-                split_bf16(sb[(ka + 8) * br + col * bc], sb[(ka + 9) * br + col * bc], bh1, bl1);
+                if constexpr (transB) {
+                    const float2 y0 = *reinterpret_cast<const float2 *>(sb + col * bld + ka);
+                    const float2 y1 = *reinterpret_cast<const float2 *>(sb + col * bld + ka + 8);
+                    split_bf16(y0.x, y0.y, bh0, bl0);
+                    split_bf16(y1.x, y1.y, bh1, bl1);
+                } else {
+                    split_bf16(sb[ka * bld + col], sb[(ka + 1) * bld + col], bh0, bl0);
+                    split_bf16(sb[(ka + 8) * bld + col], sb[(ka + 9) * bld + col], bh1, bl1);
+                }
                 mma_bf16(acc[j], al, bh0, bh1);
                 mma_bf16(acc[j], ah, bl0, bl1);
                 mma_bf16(acc[j], ah, bh0, bh1);
