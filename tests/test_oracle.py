@@ -268,6 +268,34 @@ def test_state_hand_off_equals_one_run():
     np.testing.assert_allclose(sb, s, rtol=0, atol=1e-6)
 
 
+def test_segment_transition_is_affine():
+    """A segment maps its entering state affinely: S_out = M S_in + N, where N is the segment run
+    from the zero state and M the same run with v = 0 from the identity state (the key-channel
+    transition product).  Three segments chained this way give the outputs and final state of one
+    run (up to the fp32 rounding of the handed states).  Mild decay keeps M significant."""
+    rng = np.random.default_rng(14)
+    T, H, K, b1, b2 = 120, 2, 8, 40, 85
+    x = _rand_inputs(rng, T, H, K, K, decay_scale=0.05)
+    one = lambda a, b: np.array([0, b - a], np.int32)
+    seg = lambda a, b, **kw: {key: (val[a:b] if key != "v" else kw.get("v", val)[a:b]) for key, val in x.items()}
+    o, s = oracle.kda_fwd(**x, cu_seqlens=np.array([0, T], np.int32), return_state=True)
+    _, n0 = oracle.kda_fwd(**seg(0, b1), cu_seqlens=one(0, b1), return_state=True)
+    _, n1 = oracle.kda_fwd(**seg(b1, b2), cu_seqlens=one(b1, b2), return_state=True)
+    eye = np.broadcast_to(np.eye(K), (1, H, K, K)).astype(np.float32)
+    _, m1 = oracle.kda_fwd(**seg(b1, b2, v=np.zeros_like(x["v"])), cu_seqlens=one(b1, b2), return_state=True,
+                           initial_state=eye)
+    assert 0.05 < np.abs(m1).max() < 1.0 + 1e-9 and np.abs(m1 - np.eye(K)).max() > 0.05
+    s2 = np.einsum("hij,hjv->hiv", m1, n0) + n1             # state entering the third segment
+    o2, s_end = oracle.kda_fwd(**seg(b2, T), cu_seqlens=one(b2, T), return_state=True,
+                               initial_state=s2.reshape(1, H, K, K))
+    np.testing.assert_allclose(o2, o[b2:], rtol=0, atol=1e-6)
+    np.testing.assert_allclose(s_end, s, rtol=0, atol=1e-6)
+    # the homogeneous part is linear: from the true entering state with v = 0 the run gives M S_in
+    _, ms = oracle.kda_fwd(**seg(b1, b2, v=np.zeros_like(x["v"])), cu_seqlens=one(b1, b2), return_state=True,
+                           initial_state=n0.reshape(1, H, K, K))
+    np.testing.assert_allclose(ms, np.einsum("hij,hjv->hiv", m1, n0.astype(np.float32)), rtol=0, atol=1e-12)
+
+
 def test_initial_state_one_token_closed_form():
     """S_1 = (I - b k^ k^T) Diag(e^g) S_0 + b k^ v^T, o = scale S_1^T q^ with S_0 given (K x V:
     rows are key channels)."""
