@@ -257,6 +257,50 @@ def bench_backward(kda, steps: int, dev, stream, barrier, shape=None) -> dict:
             "Mtokens_per_s": wb.T / (ms * 1e-3) / 1e6, "workspace_bytes": ws.numel()}
 
 
+def bench_long(kda, steps: int, dev, stream, barrier) -> dict:
+    """Device time of one document of 65536 tokens, H = 32 (32 chains), through kda_chunk_fwd and
+    through kda_chunk_fwd_long with its default segment count; inputs resident, workspace
+    allocated once; max over ranks."""
+    import torch
+    from chunked_gated_delta_12_b200.inputs import generate, workload
+    wl = workload(3)
+    dl = generate(wl)
+    t = {}
+    for key in ("q", "k", "v"):
+        t[key] = torch.from_numpy(dl[key].view(np.int16)).view(torch.bfloat16).to(dev)
+    for key in ("g", "beta", "cu_seqlens"):
+        t[key] = torch.from_numpy(dl[key]).to(dev)
+    out = torch.empty_like(t["q"])
+    P = kda.long_segments(wl.T, wl.H)
+    ws = torch.empty(max(kda.long_workspace_bytes(wl.T, wl.H, P), 256), dtype=torch.uint8, device=dev)
+    runs = {
+        "kda_chunk_fwd": lambda: kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"],
+                                                   out=out, stream=stream),
+        "kda_chunk_fwd_long": lambda: kda.kda_chunk_fwd_long(t["q"], t["k"], t["v"], t["g"], t["beta"], out=out,
+                                                             segments=P, workspace=ws, stream=stream),
+    }
+    res = {"workload": wl.name, "T": wl.T, "H": wl.H, "segments": P, "workspace_bytes": ws.numel()}
+    hbm_peak, _, peak_kind = peaks()
+    for name, run in runs.items():
+        for _ in range(3):
+            run()
+        kda.device_status(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        kda.device_status(stream)
+        ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+        gbs = wl.T * wl.H * BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
+        res[name] = {"ms_per_call": ms, "Mtokens_per_s": wl.T / (ms * 1e-3) / 1e6,
+                     "frac_of_hbm": gbs / hbm_peak, "peak_source": peak_kind}
+    return res
+
+
 DECODE_DOCS = 256                    # one decoding step of 256 sequences x 32 heads, states in place
 STATE_BYTES = 2 * 128 * 128 * 4      # fp32 state read and written per chain
 
@@ -320,6 +364,10 @@ def main():
     ap.add_argument("--dec-steps", type=int, default=20,
                     help="timed launches of the token-by-token kernel on one decoding step of 256 "
                          "sequences, reported under 'decode' (0 skips it)")
+    ap.add_argument("--long-steps", type=int, default=0,
+                    help="timed calls of one 65536-token document (H = 32) through kda_chunk_fwd and "
+                         "kda_chunk_fwd_long, reported under 'long_document' (0 skips it; its inputs take "
+                         "about half a minute to generate)")
     ap.add_argument("--bwd-shape", default=None,
                     help="DOCSxLEN:H -- run the backward on a custom dense workload instead (profiling)")
     ap.add_argument("--shape", default=None,
@@ -436,6 +484,8 @@ def main():
         line["backward"] = bench_backward(kda, args.bwd_steps, dev, stream, barrier, args.bwd_shape)
     if args.dec_steps > 0:
         line["decode"] = bench_decode(kda, args.dec_steps, dev, stream, barrier)
+    if args.long_steps > 0:
+        line["long_document"] = bench_long(kda, args.long_steps, dev, stream, barrier)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, d)
     if rank == 0:

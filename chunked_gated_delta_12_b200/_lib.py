@@ -53,6 +53,12 @@ def lib() -> ctypes.CDLL:
                                     ctypes.c_size_t, vp]
         L.kda_chunk_bwd_noalloc.restype = i32
         L.kda_chunk_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.kda_chunk_fwd_long.restype = i32
+        L.kda_chunk_fwd_long.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.kda_chunk_fwd_long_workspace_size.restype = ctypes.c_size_t
+        L.kda_chunk_fwd_long_workspace_size.argtypes = [i64, i32, i32]
+        L.kda_chunk_fwd_long_segments.restype = i32
+        L.kda_chunk_fwd_long_segments.argtypes = [i64, i32, i32]
         L.kda_abi_version.restype = i32
         L.kda_abi_version.argtypes = []
         _lib = L
@@ -75,7 +81,8 @@ def _ptr(t):
 
 
 def _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state, output_final_state, final_state):
-    """Shape/dtype checks shared by both forwards; returns the marshalled tensors and sizes."""
+    """Shape/dtype checks shared by the forwards; returns the marshalled tensors and sizes.
+    cu_seqlens None means one document [0, T) (kda_chunk_fwd_long)."""
     if q.dim() == 4:
         q, k, v, g = (x.squeeze(0) for x in (q, k, v, g))
         beta = beta.squeeze(0)
@@ -86,11 +93,12 @@ def _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state, output_final_
         if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or not t.is_cuda:
             raise KdaError(1, f"{name} must be a contiguous CUDA {dt} tensor of shape {shape} "
                               f"(got {t.dtype} {tuple(t.shape)})")
-    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+    if cu_seqlens is not None and (cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda
+                                   or cu_seqlens.dim() != 1):
         raise KdaError(1, "cu_seqlens must be a 1-d int32 CUDA tensor")
     if out is None:
         out = torch.empty_like(q)
-    n_docs = cu_seqlens.numel() - 1
+    n_docs = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
     shape_s = (n_docs, H, D, D)
     for name, t in (("initial_state", initial_state), ("final_state", final_state)):
         if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape_s or not t.is_contiguous()
@@ -141,6 +149,47 @@ def kda_recurrent_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     rc = lib().kda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
                                  _ptr(initial_state), _ptr(final_state), _ptr(out),
                                  ctypes.c_void_p(_stream_handle(stream)))
+    _check(rc)
+    return (out, final_state) if final_state is not None else out
+
+
+def long_segments(T: int, H: int, num_sms: int | None = None) -> int:
+    """Segment count kda_chunk_fwd_long uses by default (kda_chunk_fwd_long_segments) on a GPU with
+    ``num_sms`` SMs (the current device's if None)."""
+    if num_sms is None:
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return int(lib().kda_chunk_fwd_long_segments(T, H, num_sms))
+
+
+def long_workspace_bytes(T: int, H: int, segments: int) -> int:
+    """Device workspace bytes kda_chunk_fwd_long needs (kda_chunk_fwd_long_workspace_size)."""
+    return int(lib().kda_chunk_fwd_long_workspace_size(T, H, segments))
+
+
+def kda_chunk_fwd_long(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                       beta: torch.Tensor, out: torch.Tensor | None = None, segments: int | None = None,
+                       initial_state: torch.Tensor | None = None, output_final_state: bool = False,
+                       final_state: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                       stream: torch.cuda.Stream | None = None):
+    """Forward of ONE document [0, T) through libkda's kda_chunk_fwd_long: its chunk chain is split
+    into ``segments`` pieces (``long_segments`` if None) that run side by side, joined through the
+    state hand-off S_out = M S_in + N.
+
+    Tensors as ``kda_chunk_fwd`` with one document (no cu_seqlens); states [1, H, 128, 128] fp32.
+    ``workspace`` (a CUDA uint8 tensor of at least ``long_workspace_bytes`` bytes) is allocated by
+    torch when not given.  Returns out, or (out, final_state) as ``kda_chunk_fwd`` does.
+    """
+    q, k, v, g, beta, out, _, T, H, final_state = _fwd_checked(q, k, v, g, beta, None, out, initial_state,
+                                                               output_final_state, final_state)
+    if segments is None:
+        segments = long_segments(T, H)
+    need = long_workspace_bytes(T, H, segments)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib().kda_chunk_fwd_long(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, H, segments,
+                                  _ptr(initial_state), _ptr(final_state), _ptr(out), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
     return (out, final_state) if final_state is not None else out
 

@@ -74,6 +74,12 @@ namespace kda {
 
 int set_last_error(int status, const char *msg) { return (int)fail((kda_status)status, "%s", msg); }
 
+int device_context(int *dev, int **status) {
+    kda_status s = check_device(dev);
+    if (s != KDA_OK) return s;
+    return status_ptr(*dev, status);
+}
+
 }  // namespace kda
 
 extern "C" {

@@ -40,6 +40,11 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
 // defined outside kda_api.cu).
 int set_last_error(int status, const char *msg);
 
+// Checks that the current device is sm_100 and returns it with its device status word (the
+// word kernels record KDA_ERR_BAD_SEQLENS / KDA_ERR_TIMEOUT in); a kda_status, with the
+// message recorded on failure.
+int device_context(int *dev, int **status);
+
 // Runs one time-limited mbarrier wait that can never complete (self-test of the
 // timeout path): records kStatusTimeout in *status after about limit_cycles.
 cudaError_t launch_wait_selftest(int *status, long long limit_cycles, cudaStream_t stream);

@@ -127,6 +127,65 @@ kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_
                              const float *initial_state, float *final_state, uint16_t *out, void *stream);
 
 /*
+ * kda_chunk_fwd_long -- kda_chunk_fwd_state for ONE document, its chunk chain split into
+ * `segments` pieces that run side by side.
+ *
+ * Why: the chunked kernel runs one CTA per (document, head) chain, so one long document with H
+ * heads occupies only H SMs and takes as long as its serial chain of T/64 chunk steps.
+ *
+ * Operation: the same result as kda_chunk_fwd_state with cu_seqlens = [0, T], up to rounding.
+ * The recurrence in the header comment is affine in the state: a segment of tokens maps its
+ * entering state to S_out = M S_in + N, where N is the segment run from the zero state and M the
+ * product of its per-token maps (I - beta k k^T) Diag(exp(g)) (the same run with v = 0 from the
+ * identity state).  The document is cut at chunk boundaries into P segments (segment p covers
+ * chunks [floor(n p / P), floor(n (p + 1) / P)) of its n = ceil(T / 64) chunks) and run as
+ *   1. N_p of segments 0..P-2, segment 0 from initial_state (its outputs are final), while a
+ *      second, library-owned stream computes M_p of the middle segments 1..P-2;
+ *   2. the hand-off, in fp32: S_in(1) = N_0, S_in(p + 1) = M_p S_in(p) + N_p;
+ *   3. segments 1..P-1 from their entering states: their outputs and the final state.
+ * Each stage's chains are at most ceil(n / P) chunks long, so the document takes about 2 n / P
+ * chunk steps instead of n.  The state hand-off between pieces of one sequence is how the kimi_k3
+ * model page runs KDA under context parallelism (KimiDeltaAttention._forward_with_cp passes the
+ * recurrent state from one shard to the next); the transition map M lets the pieces run at the
+ * same time on one GPU.  Outputs of segment 0 are bit-identical to kda_chunk_fwd_state's.
+ *
+ * Arguments: q, k, v, g, beta, out, T, H, initial_state, final_state and stream as
+ * kda_chunk_fwd_state with n_docs = 1 (states [1, H, 128, 128]; no cu_seqlens: the document is
+ * [0, T)), plus
+ *   segments        P, 1..16 and at most ceil(T / 64); 1 runs the document unsplit.
+ *                   kda_chunk_fwd_long_segments gives the choice that fits the GPU.
+ *   workspace       DEVICE memory, 256-byte aligned, at least
+ *                   kda_chunk_fwd_long_workspace_size(T, H, segments) bytes, overlapping no
+ *                   other argument; its contents on entry do not matter.  Calls that share a
+ *                   workspace must be ordered (one stream).
+ * Streams: stage 1's M pass runs on a non-blocking stream that libkda creates, with two events,
+ * once per device at the first call with P >= 3 with that device current; `stream` forks to it
+ * and joins it through the events, so the call stays asynchronous and ordered on `stream`.
+ * Ownership and errors: as kda_chunk_fwd_state; bad sizes, pointers, alignment, aliasing or a
+ * small workspace return KDA_ERR_INVALID_ARG and launch nothing.
+ */
+kda_status kda_chunk_fwd_long(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                              const float *beta, int64_t T, int H, int segments, const float *initial_state,
+                              float *final_state, uint16_t *out, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * kda_chunk_fwd_long_workspace_size -- bytes of workspace kda_chunk_fwd_long needs for these
+ * sizes (0 for invalid sizes): 256 bytes of cu_seqlens tables; for P >= 2, per head
+ * 3 (P - 1) states of 64 KB; for P >= 3, per head 2 (P - 2) more states and two bf16
+ * [tokens of segments 1..P-2, H, 128] buffers (zero values and the M pass's unused outputs).
+ */
+size_t kda_chunk_fwd_long_workspace_size(int64_t T, int H, int segments);
+
+/*
+ * kda_chunk_fwd_long_segments -- the segment count for kda_chunk_fwd_long on a GPU with
+ * num_sms SMs: the largest P <= 16 whose stage 1, (2 P - 3) H chains of one CTA each, fits on
+ * the SMs at once and whose segments keep at least 8 chunks; 1 (no split) when that P is below
+ * 3, where splitting does not shorten the chain (P = 2 takes n / 2 + n / 2 steps).
+ */
+int kda_chunk_fwd_long_segments(int64_t T, int H, int num_sms);
+
+/*
  * kda_chunk_bwd_workspace_size -- bytes of device workspace kda_chunk_bwd needs for a call
  * with these sizes (an upper bound that does not depend on the cu_seqlens content).
  */
