@@ -15,11 +15,13 @@
  * cu_seqlens; a dense batch of B equal-length sequences is passed as B packed
  * documents with cu_seqlens = [0, L, 2L, ..., BL]), q/k l2-normalised inside
  * the kernel, a bounded log gate, no initial or final state, no context
- * parallelism, chunk mode only (kda_chunk_fwd).  Two entry points widen it:
- * kda_chunk_fwd_state adds an initial and a final state per chain, and
+ * parallelism, chunk mode only (kda_chunk_fwd).  Entry points that widen it:
+ * kda_chunk_fwd_state adds an initial and a final state per chain;
  * kda_recurrent_fwd is the token-by-token mode (the "recurrent" alternative to
  * "chunk" that the kda_mode setting and KimiDeltaAttention._resolve_mode of
- * the kimi_linear model page choose between) for decoding and short inputs.
+ * the kimi_linear model page choose between) for decoding and short inputs;
+ * kda_chunk_fwd_long runs one long document as segments joined through the
+ * state hand-off; kda_chunk_bwd (and kda_chunk_bwd_noalloc) is the backward.
  * Like fused_kda_unsupported_reason on the kda_fused page, every call that
  * falls outside this scope is rejected with the first violated condition
  * (kda_last_error); there is no fallback path of any kind.
