@@ -355,19 +355,33 @@ kda_status kda_chunk_fwd_long(const uint16_t *q, const uint16_t *k, const uint16
         if ((e = cudaEventRecord(aux->fork, st)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(aux->stream, aux->fork, 0)) != cudaSuccess)
             return cuda_fail("stream fork", e);
-        if ((e = cudaMemsetAsync(vzero, 0, (size_t)Tm * row * sizeof(uint16_t), aux->stream)) != cudaSuccess)
-            return cuda_fail("zero values", e);
-        write_identity<<<148, 256, 0, aux->stream>>>(ident, (size_t)(P - 2) * H);
-        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail("identity launch", e);
-        e = kda::launch_fwd_pipe(q + o1, k + o1, vzero, g + o1, beta + (size_t)b[1] * H, cuM, P - 2, Tm, H, ident,
-                                 mst, mout, status, aux->stream);
-        if (e != cudaSuccess) return cuda_fail("transition pass launch", e);
-        if ((e = cudaEventRecord(aux->join, aux->stream)) != cudaSuccess) return cuda_fail("stream join", e);
+        const char *what = "zero values";
+        e = cudaMemsetAsync(vzero, 0, (size_t)Tm * row * sizeof(uint16_t), aux->stream);
+        if (e == cudaSuccess) {
+            what = "identity launch";
+            const size_t n_floats = (size_t)(P - 2) * H * kStateFloats;    // about 4 per thread
+            write_identity<<<(unsigned)((n_floats / 4 + 255) / 256), 256, 0, aux->stream>>>(ident,
+                                                                                          (size_t)(P - 2) * H);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) {
+            what = "transition pass launch";
+            e = kda::launch_fwd_pipe(q + o1, k + o1, vzero, g + o1, beta + (size_t)b[1] * H, cuM, P - 2, Tm, H,
+                                     ident, mst, mout, status, aux->stream);
+        }
+        const cudaError_t ej = cudaEventRecord(aux->join, aux->stream);
+        if (e != cudaSuccess || ej != cudaSuccess) {
+            // join even after a failure, so that no work of this call stays unordered with `stream`
+            if (ej == cudaSuccess) cudaStreamWaitEvent(st, aux->join, 0);
+            return e != cudaSuccess ? cuda_fail(what, e) : cuda_fail("stream join", ej);
+        }
     }
-    // stage 1a: N_p of segments 0..P-2; segment 0's outputs are final
+    // stage 1a: N_p of segments 0..P-2, at the same time as the M pass; segment 0's outputs are
+    // final.  `stream` joins the second stream after it (also when the launch failed).
     e = kda::launch_fwd_pipe(q, k, v, g, beta, cuN, P - 1, Tn, H, h0n, nst, out, status, st);
+    const cudaError_t ew = have_mid ? cudaStreamWaitEvent(st, aux->join, 0) : cudaSuccess;
     if (e != cudaSuccess) return cuda_fail("segment pass launch", e);
-    if (have_mid && (e = cudaStreamWaitEvent(st, aux->join, 0)) != cudaSuccess) return cuda_fail("stream join", e);
+    if (ew != cudaSuccess) return cuda_fail("stream join", ew);
     // stage 2: entering states of segments 1..P-1
     static bool smem_set[kMaxDevices] = {false};
     if (!smem_set[dev]) {
