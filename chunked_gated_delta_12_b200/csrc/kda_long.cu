@@ -175,6 +175,9 @@ cudaError_t aux_for(int dev, Aux **out) {
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming);
         if (e != cudaSuccess) {
+            if (a.join) cudaEventDestroy(a.join);
+            if (a.fork) cudaEventDestroy(a.fork);
+            if (a.stream) cudaStreamDestroy(a.stream);
             a = Aux{};
             return e;
         }
@@ -247,6 +250,7 @@ kda_status kda_chunk_fwd_long(const uint16_t *q, const uint16_t *k, const uint16
     if (T > 0 && segments > nch)
         return fail(KDA_ERR_INVALID_ARG, "segments (%d) exceeds the document's %lld chunks", segments,
                     (long long)nch);
+    if ((int64_t)segments * H > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "segments * H too large");
     const int P = segments;
     const size_t st_bytes = kStateFloats * sizeof(float) * (size_t)H;
     if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
