@@ -21,12 +21,12 @@
 //          O^T += U~^T_bf16 (TMEM) A_qk^T
 //          S^T += U~^T_bf16 (TMEM) Kd               (after S^T <- S^T Diag(e^{Gamma_last}))
 // The output scale is carried by Q~ and A_qk.
-// q, k, g and v tiles arrive by TMA (2-D tensor maps over [T, H*128], no
-// multicast); rows past the document end are masked with selects (and v rows
-// zeroed) because a tile may reach into the next document.  The gate exponent
-// is split at 16-row sub-block boundaries (e^{G_r - G_i} = E1_r s_RI E2_i, every factor within
-// the fp32/bf16 range).  Every
-// wait is time-limited and reports KDA_ERR_TIMEOUT.
+// q, k, g and v tiles arrive by TMA (2-D tensor maps over [T, H*128], each CTA loading its own
+// tiles).  A tile may reach into the next document, so the rows past the document end are zeroed
+// in shared memory (q, k and g when the step starts, v before the U product) and count as zero
+// in the row norms.  The gate exponent is split at 16-row sub-block boundaries
+// (e^{G_r - G_i} = E1_r s_RI E2_i, every factor within the fp32/bf16 range).  Every wait is
+// time-limited and reports KDA_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>

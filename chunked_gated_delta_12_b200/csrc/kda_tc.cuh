@@ -152,14 +152,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long 
 }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast): 2-D tiled bulk copy global -> shared, completion counted
+// TMA: 2-D tiled bulk copy global -> this CTA's shared memory, completion counted
 // in bytes on an mbarrier.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_expect_tx(uint32_t saddr, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr), "r"(bytes) : "memory");
 }
 // TMA store of one 2-D box from shared memory, tracked by the issuing thread's bulk group
-// (no multicast; x * element size must be a multiple of 16 bytes, x and y non-negative)
+// (x * element size must be a multiple of 16 bytes, x and y non-negative)
 __device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uint32_t src_saddr) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
                      reinterpret_cast<uint64_t>(tmap)),
