@@ -9,7 +9,8 @@ the workload (documents and heads are independent; no collective on the data
 path), so per-GPU work is fixed and the line reports weak scaling.
 
 `--impl reference` times the fp64 CPU oracle on this host's cores instead
-(rank 0 only), on a bounded sample of the same workload.
+(rank 0 only): the whole workload each step when the run fits a few minutes,
+else a bounded sample of it.
 """
 from __future__ import annotations
 
@@ -32,6 +33,9 @@ UNIT = "Mtokens/s"
 BYTES_PER_TOKEN_HEAD = 1540          # q,k,v bf16 768 + g fp32 512 + beta 4 + o bf16 256
 FLOPS_PER_TOKEN_HEAD = 180224        # 6 d^2 + 10 C d, d = 128, C = 64 (dense chunk tiles)
 FLOPS_PER_TOKEN_HEAD_TRI = 139264    # same, skipping the zero triangles
+# the recompute backward: reads q, k, v (768 B), g (512), beta (4) and dO (256 B); writes dq, dk, dv
+# (768 B), dg (512) and dbeta (4) -- 2824 B per (token, head), each tensor once
+BWD_BYTES_PER_TOKEN_HEAD = 2824
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -152,69 +156,89 @@ def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> floa
     return tokens_per_rank * world / (ms_per_step * 1e-3) / 1e6
 
 
-def oracle_sample_rate(w, d, tokens: int, n_threads: int):
-    """Time the fp64 oracle on the first `tokens` tokens of document 0 (all heads)."""
-    import oracle
+def oracle_rows(d, tokens: int | None):
+    """The oracle's inputs for the first `tokens` tokens of every document (all of them if None),
+    as fp32 arrays and the matching cu_seqlens."""
     from chunked_gated_delta_12_b200.inputs import bf16_bits_to_f32
-    tokens = min(tokens, int(d["cu_seqlens"][1]))
-    sl = slice(0, tokens)
-    f = lambda key: bf16_bits_to_f32(d[key][sl]).reshape(d[key][sl].shape)
-    q, k, v = f("q"), f("k"), f("v")
-    g, b = np.ascontiguousarray(d["g"][sl]), np.ascontiguousarray(d["beta"][sl])
+    cu = np.asarray(d["cu_seqlens"], dtype=np.int64)
+    if tokens is None:
+        idx = np.arange(int(cu[-1]))
+        cu_s = cu
+    else:
+        lens = np.minimum(np.diff(cu), tokens)
+        idx = np.concatenate([np.arange(cu[i], cu[i] + lens[i]) for i in range(len(lens))])
+        cu_s = np.concatenate([[0], np.cumsum(lens)])
+    f = lambda key: bf16_bits_to_f32(d[key][idx]).reshape(d[key][idx].shape)
+    return (f("q"), f("k"), f("v"), np.ascontiguousarray(d["g"][idx]), np.ascontiguousarray(d["beta"][idx]),
+            cu_s.astype(np.int32))
+
+
+def oracle_time(inputs, n_threads: int) -> float:
+    """Seconds the fp64 oracle, as it stands, takes for one pass over `inputs` (oracle_rows)."""
+    import oracle
+    q, k, v, g, b, cu = inputs
     t0 = time.perf_counter()
-    oracle.kda_fwd(q, k, v, g, b, [0, tokens], n_threads=n_threads)
-    dt = time.perf_counter() - t0
-    return tokens / dt / 1e6, dt, tokens
+    oracle.kda_fwd(q, k, v, g, b, cu, n_threads=n_threads)
+    return time.perf_counter() - t0
 
 
-def cpu_baseline(w, d, target_s: float = 12.0) -> dict:
-    """The fp64 oracle as it stands, on this host's cores, on a bounded sample of
-    the workload: the first n tokens of document 0 (all heads), n grown until one
-    run takes about `target_s` seconds or the document is exhausted, then repeated
-    until that much CPU time has been spent."""
+def oracle_plan(w, d, cores: int, budget_s: float):
+    """Inputs for one oracle step: the whole workload if one pass fits `budget_s` seconds, else the
+    first n tokens of every document (all chains kept), n sized from a calibration run."""
+    probe = oracle_rows(d, 64)
+    per_tok = oracle_time(probe, cores) / int(probe[-1][-1])
+    if per_tok * w.T <= budget_s:
+        return oracle_rows(d, None), w.T, "the whole workload"
+    n = max(64, int(budget_s / per_tok / w.n_docs))
+    inputs = oracle_rows(d, n)
+    return inputs, int(inputs[-1][-1]), f"the first {n} tokens of each of the {w.n_docs} documents"
+
+
+def cpu_baseline(w, d, target_s: float = 10.0) -> dict:
+    """The fp64 oracle as it stands, on this host's cores: the whole workload (every chain, every
+    token) when one pass takes under a minute, else a bounded sample of it, repeated until
+    `target_s` seconds of wall time have been spent."""
     cores = os.cpu_count() or 1
-    n = 256
-    _, dt, n = oracle_sample_rate(w, d, n, cores)
-    used = min(cores, w.H)            # the sample holds H independent chains
-    while dt < target_s / 4 and n < int(d["cu_seqlens"][1]):
-        n = int(min(d["cu_seqlens"][1], max(2 * n, n * (target_s / 2) / max(dt, 1e-3))))
-        _, dt, n = oracle_sample_rate(w, d, n, cores)
-    total, runs = dt, 1
-    while total < target_s:
-        _, dt, _ = oracle_sample_rate(w, d, n, cores)
-        total += dt
+    inputs, tokens, what = oracle_plan(w, d, cores, budget_s=60.0)
+    total, runs = 0.0, 0
+    while total < target_s or runs == 0:
+        total += oracle_time(inputs, cores)
         runs += 1
-    rate = runs * n / total / 1e6
+    rate = runs * tokens / total / 1e6
+    used = min(cores, w.n_docs * w.H)       # threads over independent (document, head) chains
     return {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
-            "sample": f"first {n} tokens of document 0, all {w.H} heads, {runs} run(s), {total:.1f} s"}
+            "sample": f"{what} ({tokens} tokens x {w.H} heads, {w.n_docs * w.H} chains), {runs} run(s), "
+                      f"{total:.1f} s"}
 
 
 def run_reference(args, w, d):
-    """fp64 oracle on the host cores: each step a bounded sample of the workload."""
+    """fp64 oracle on the host cores: each step one pass over the workload (the whole workload when
+    every step of the run fits about two and a half minutes, else the same sample each step)."""
     cores = os.cpu_count() or 1
-    # calibrate: seconds per token (all heads) at this core count
-    _, dt, n = oracle_sample_rate(w, d, 64, cores)
-    per_tok = dt / n
     budget = 150.0 / max(1, args.steps + args.warmup)
-    tokens = int(max(64, min(4096, budget / per_tok)))
+    inputs, tokens, what = oracle_plan(w, d, cores, budget_s=budget)
     for _ in range(args.warmup):
-        oracle_sample_rate(w, d, tokens, cores)
-    times = []
-    for _ in range(args.steps):
-        _, dt, n = oracle_sample_rate(w, d, tokens, cores)
-        times.append(dt)
+        oracle_time(inputs, cores)
+    times = [oracle_time(inputs, cores) for _ in range(args.steps)]
     total = sum(times)
-    value = args.steps * n / total / 1e6
-    sample = (f"first {n} tokens of document 0 of {w.name}, all {w.H} heads "
-              f"({w.H} independent chains, fp64 token recurrence)")
+    value = args.steps * tokens / total / 1e6
+    sample = (f"{what} of {w.name} ({tokens} tokens x {w.H} heads, {w.n_docs * w.H} independent chains, "
+              f"fp64 token recurrence)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": dict(w.describe(), sample_tokens=n),
-            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": min(cores, w.H),
-                             "sample": sample},
+            "data": "synthetic", "config": headline_config(w, 1),
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT,
+                             "cores": min(cores, w.n_docs * w.H), "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if tokens != w.T:
+        line["config"]["sample_tokens"] = tokens
     print(json.dumps(line), flush=True)
+
+
+def headline_config(w, world: int) -> dict:
+    return dict(w.describe(), l2="inputs 1.6 GB per step > 126 MB L2; no flush",
+                parallelism=f"replicas x{world}" if world > 1 else "single GPU")
 
 
 def bench_backward(kda, steps: int, dev, stream, barrier, shape=None) -> dict:
@@ -253,51 +277,72 @@ def bench_backward(kda, steps: int, dev, stream, barrier, shape=None) -> dict:
     torch.cuda.synchronize()
     kda.device_status(stream)
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+    hbm_peak, _, peak_kind = peaks()
+    alg = wb.T * wb.H * BWD_BYTES_PER_TOKEN_HEAD
+    gbs = alg / (ms * 1e-3) / 1e9
     return {"workload": wb.name, "T": wb.T, "H": wb.H, "ms_per_launch": ms, "launches": steps,
-            "Mtokens_per_s": wb.T / (ms * 1e-3) / 1e6, "workspace_bytes": ws.numel()}
+            "Mtokens_per_s": wb.T / (ms * 1e-3) / 1e6, "workspace_bytes": ws.numel(),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                         "bytes_per_token_head": BWD_BYTES_PER_TOKEN_HEAD}}
 
 
-def bench_long(kda, steps: int, dev, stream, barrier) -> dict:
-    """Device time of one document of 65536 tokens, H = 32 (32 chains), through kda_chunk_fwd and
-    through kda_chunk_fwd_long with its default segment count; inputs resident, workspace
-    allocated once; max over ranks."""
+def bench_workloads(kda, steps: int, dev, stream, barrier) -> dict:
+    """Device time of the forward on the other full-size workloads, inputs resident, max over
+    ranks: one document of 65536 tokens with H = 32 (32 chains of 1024 chunks) through
+    kda_chunk_fwd and through kda_chunk_fwd_long with its default segment count (workspace
+    allocated once), and the 16 packed documents (H = 32) through kda_chunk_fwd."""
     import torch
     from chunked_gated_delta_12_b200.inputs import generate, workload
-    wl = workload(3)
-    dl = generate(wl)
-    t = {}
-    for key in ("q", "k", "v"):
-        t[key] = torch.from_numpy(dl[key].view(np.int16)).view(torch.bfloat16).to(dev)
-    for key in ("g", "beta", "cu_seqlens"):
-        t[key] = torch.from_numpy(dl[key]).to(dev)
-    out = torch.empty_like(t["q"])
-    P = kda.long_segments(wl.T, wl.H)
-    ws = torch.empty(max(kda.long_workspace_bytes(wl.T, wl.H, P), 256), dtype=torch.uint8, device=dev)
-    runs = {
-        "kda_chunk_fwd": lambda: kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"],
-                                                   out=out, stream=stream),
-        "kda_chunk_fwd_long": lambda: kda.kda_chunk_fwd_long(t["q"], t["k"], t["v"], t["g"], t["beta"], out=out,
-                                                             segments=P, workspace=ws, stream=stream),
-    }
-    res = {"workload": wl.name, "T": wl.T, "H": wl.H, "segments": P, "workspace_bytes": ws.numel()}
     hbm_peak, _, peak_kind = peaks()
-    for name, run in runs.items():
-        for _ in range(3):
-            run()
-        kda.device_status(stream)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(steps):
-            run()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        kda.device_status(stream)
-        ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
-        gbs = wl.T * wl.H * BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
-        res[name] = {"ms_per_call": ms, "Mtokens_per_s": wl.T / (ms * 1e-3) / 1e6,
-                     "frac_of_hbm": gbs / hbm_peak, "peak_source": peak_kind}
+    res = {}
+    for idx in (3, 4):
+        wl = workload(idx)
+        dl = generate(wl, with_grad=False)
+        t = {}
+        for key in ("q", "k", "v"):
+            t[key] = torch.from_numpy(dl[key].view(np.int16)).view(torch.bfloat16).to(dev)
+        for key in ("g", "beta", "cu_seqlens"):
+            t[key] = torch.from_numpy(dl[key]).to(dev)
+        del dl
+        out = torch.empty_like(t["q"])
+        runs = {"kda_chunk_fwd": lambda: kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"],
+                                                           t["cu_seqlens"], out=out, stream=stream)}
+        entry = {"T": wl.T, "H": wl.H, "n_docs": wl.n_docs, "chains": wl.n_docs * wl.H}
+        if wl.n_docs == 1:
+            P = kda.long_segments(wl.T, wl.H)
+            ws = torch.empty(max(kda.long_workspace_bytes(wl.T, wl.H, P), 256), dtype=torch.uint8, device=dev)
+            runs["kda_chunk_fwd_long"] = lambda: kda.kda_chunk_fwd_long(t["q"], t["k"], t["v"], t["g"], t["beta"],
+                                                                        out=out, segments=P, workspace=ws,
+                                                                        stream=stream)
+            entry.update(segments=P, workspace_bytes=ws.numel())
+        best = None
+        for name, run in runs.items():
+            for _ in range(3):
+                run()
+            kda.device_status(stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(steps):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            kda.device_status(stream)
+            ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+            alg = wl.T * wl.H * BYTES_PER_TOKEN_HEAD
+            gbs = alg / (ms * 1e-3) / 1e9
+            entry[name] = {"ms_per_call": ms, "Mtokens_per_s": wl.T / (ms * 1e-3) / 1e6, "launches": steps,
+                           "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                                        "frac": gbs / hbm_peak, "peak_source": peak_kind,
+                                        "algorithmic_bytes_per_launch": alg}}
+            if best is None or ms < entry[best]["ms_per_call"]:
+                best = name
+        entry["best_public_path"] = best
+        res[wl.name] = entry
+        del t, out
+        torch.cuda.empty_cache()
     return res
 
 
@@ -364,10 +409,10 @@ def main():
     ap.add_argument("--dec-steps", type=int, default=20,
                     help="timed launches of the token-by-token kernel on one decoding step of 256 "
                          "sequences, reported under 'decode' (0 skips it)")
-    ap.add_argument("--long-steps", type=int, default=0,
-                    help="timed calls of one 65536-token document (H = 32) through kda_chunk_fwd and "
-                         "kda_chunk_fwd_long, reported under 'long_document' (0 skips it; its inputs take "
-                         "about half a minute to generate)")
+    ap.add_argument("--fwd-steps", type=int, default=10,
+                    help="timed forward calls on each of the other full-size workloads (one document of "
+                         "65536 tokens, also split by kda_chunk_fwd_long; 16 packed documents), reported "
+                         "under 'workloads' (0 skips them)")
     ap.add_argument("--bwd-shape", default=None,
                     help="DOCSxLEN:H -- run the backward on a custom dense workload instead (profiling)")
     ap.add_argument("--shape", default=None,
@@ -467,8 +512,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(w.describe(), l2="inputs 1.6 GB per step > 126 MB L2; no flush",
-                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "config": headline_config(w, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
@@ -484,8 +528,8 @@ def main():
         line["backward"] = bench_backward(kda, args.bwd_steps, dev, stream, barrier, args.bwd_shape)
     if args.dec_steps > 0:
         line["decode"] = bench_decode(kda, args.dec_steps, dev, stream, barrier)
-    if args.long_steps > 0:
-        line["long_document"] = bench_long(kda, args.long_steps, dev, stream, barrier)
+    if args.fwd_steps > 0:
+        line["workloads"] = bench_workloads(kda, args.fwd_steps, dev, stream, barrier)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, d)
     if rank == 0:

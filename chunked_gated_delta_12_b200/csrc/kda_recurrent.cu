@@ -1,8 +1,8 @@
 // kda_recurrent.cu -- the token-by-token (recurrent) KDA forward, for decode and short sequences.
 //
 // The recurrence itself, one token at a time, with no chunking (the alternative to chunk mode
-// that the pages' mode switch picks for short sequences; kda_mode / _resolve_mode on the
-// kimi_k3 model page):
+// that the pages' mode switch picks for short sequences: the kda_mode setting and
+// KimiDeltaAttention._resolve_mode on the kimi_linear model page):
 //
 //   S' = Diag(e^{g_t}) S,  p = S'^T k^,  S = S' + beta_t k^ (v_t - p)^T,  o_t = scale S^T q^
 //

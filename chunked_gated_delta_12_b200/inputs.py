@@ -19,6 +19,7 @@ seed = 20260 + workload index.
 """
 from __future__ import annotations
 
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -33,10 +34,10 @@ def _rng(seed: int, name: str) -> np.random.Generator:
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (round-to-nearest-even); returns uint16 bit patterns."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    b = x.view(np.uint32).astype(np.uint64)
-    rounded = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    """Round fp32 to bf16 (round-to-nearest-even); returns uint16 bit patterns.  Finite inputs
+    only: the 32-bit sum below cannot wrap for any finite value (largest 0xFF7FFFFF + 0x8000)."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounded = (b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return rounded.astype(np.uint16)
 
 
@@ -151,14 +152,21 @@ def generate(w: Workload, with_grad: bool | None = None) -> dict[str, np.ndarray
     """Draw the tensors of workload `w` (host numpy arrays, layouts in the module doc)."""
     T, H, d = w.T, w.H, HEAD_DIM
     n = T * H * d
-    out: dict[str, np.ndarray] = {}
-    for name in ("q", "k", "v"):
-        out[name] = f32_to_bf16_bits(_normal_f32(_rng(w.seed, name), n)).reshape(T, H, d)
-    z = _normal_f32(_rng(w.seed, "g"), n)
-    out["g"] = (-5.0 * _sigmoid(z)).astype(np.float32).reshape(T, H, d)
-    zb = _normal_f32(_rng(w.seed, "beta"), T * H)
-    out["beta"] = _sigmoid(zb).astype(np.float32).reshape(T, H)
-    out["cu_seqlens"] = w.cu_seqlens()
+
+    def draw(name: str) -> np.ndarray:
+        if name == "g":
+            return (-5.0 * _sigmoid(_normal_f32(_rng(w.seed, "g"), n))).astype(np.float32).reshape(T, H, d)
+        if name == "beta":
+            return _sigmoid(_normal_f32(_rng(w.seed, "beta"), T * H)).astype(np.float32).reshape(T, H)
+        return f32_to_bf16_bits(_normal_f32(_rng(w.seed, name), n)).reshape(T, H, d)
+
+    names = ["q", "k", "v", "g", "beta"]
     if with_grad if with_grad is not None else w.with_grad:
-        out["do"] = f32_to_bf16_bits(_normal_f32(_rng(w.seed, "do"), n)).reshape(T, H, d)
+        names.append("do")
+    # every tensor has its own random stream, so drawing them side by side (numpy releases the
+    # interpreter lock inside these loops) gives the same arrays as drawing them in turn
+    with ThreadPoolExecutor(max_workers=len(names)) as ex:
+        arrays = list(ex.map(draw, names))
+    out: dict[str, np.ndarray] = dict(zip(names, arrays))
+    out["cu_seqlens"] = w.cu_seqlens()
     return out

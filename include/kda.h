@@ -163,6 +163,10 @@ kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_
  * Streams: stage 1's M pass runs on a non-blocking stream that libkda creates, with two events,
  * once per device at the first call with P >= 3 with that device current; `stream` forks to it
  * and joins it through the events, so the call stays asynchronous and ordered on `stream`.
+ * That second stream is shared by every call with P >= 3 on the device.  While such a call is
+ * being captured into a CUDA graph, the shared stream belongs to that capture until the capture
+ * ends, so no other call with P >= 3 on the same device (from another thread or another stream)
+ * may run between the captured call and the end of its capture.
  * Ownership and errors: as kda_chunk_fwd_state; bad sizes, pointers, alignment, aliasing or a
  * small workspace return KDA_ERR_INVALID_ARG and launch nothing.
  */

@@ -5,9 +5,10 @@ another allocator (a framework's caching pool that has already reserved the free
 they must not allocate after start-up because cudaMalloc and cudaFree synchronise the device.
 kda_chunk_bwd_noalloc serves them with a fixed scratch array held in the library's device
 image instead of a caller-owned workspace.  These tests call it through the C ABI and check
-that it gives what kda_chunk_bwd gives, on two calls in a row (the second one of another size,
-so that it starts from the first call's leftover scratch), and that sizes beyond the array are
-rejected on the host.
+that it gives exactly what kda_chunk_bwd gives (the same kernel on the same inputs, so the
+gradients must be bit-identical), on two calls in a row (the second one of another size, so that
+it starts from the first call's leftover scratch), that the first call's gradients also meet the
+fp64 reverse-mode oracle, and that sizes beyond the array are rejected on the host.
 
 This file is named to be collected last: if its GPU test fails, a run that stops at the first
 failure has already run every other test.
@@ -20,9 +21,10 @@ import pytest
 from chunked_gated_delta_12_b200 import _lib
 from chunked_gated_delta_12_b200.build import build
 from chunked_gated_delta_12_b200.inputs import custom_workload, generate
-from tests.helpers import compare_grad, out_to_f64, to_device
+from tests.helpers import compare_grad, oracle_grads, out_to_f64, to_device
 
-# the bar of the other backward tests: rel-L2 <= 1e-2, max-abs <= 5e-2 of max |reference|
+# the bar of the other backward tests against the oracle: rel-L2 <= 1e-2, max-abs <= 5e-2 of
+# max |reference|
 RTOL_L2 = 1e-2
 RMAX = 5e-2
 
@@ -54,6 +56,11 @@ def _grads_host(grads):
                 dg=dg.cpu().numpy().astype(np.float64), dbeta=db.cpu().numpy().astype(np.float64))
 
 
+def _bits(grads):
+    import torch
+    return [x.view(torch.int32 if x.dtype == torch.float32 else torch.int16).cpu().numpy() for x in grads]
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_kda_chunk_bwd_on_two_calls_in_a_row():
     import torch
@@ -61,7 +68,7 @@ def test_noalloc_matches_kda_chunk_bwd_on_two_calls_in_a_row():
     torch.cuda.init()
     cases = [custom_workload("noalloc_a", [1000, 63, 65, 0, 200], 4, seed=71),
              custom_workload("noalloc_b", [130, 64, 1], 2, seed=72)]
-    for w in cases:
+    for i, w in enumerate(cases):
         d = generate(w, with_grad=True)
         assert _lib.bwd_workspace_bytes(len(d["cu_seqlens"]) - 1, int(d["cu_seqlens"][-1]), w.H) \
             <= kda.NOALLOC_SCRATCH_BYTES
@@ -74,10 +81,16 @@ def test_noalloc_matches_kda_chunk_bwd_on_two_calls_in_a_row():
         kda.kda_chunk_bwd_noalloc(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"], t["do"], *outs)
         kda.device_status()
         torch.cuda.synchronize()
-        got, exp = _grads_host(outs), _grads_host(ref)
-        cu = d["cu_seqlens"]
-        for n in ("dq", "dk", "dv", "dg"):
-            rel, mx = compare_grad(got[n], exp[n], cu, w.H)
-            assert rel <= RTOL_L2 and mx <= RMAX, (w.name, n, rel, mx)
-        rel, mx = compare_grad(got["dbeta"][..., None], exp["dbeta"][..., None], cu, w.H)
-        assert rel <= RTOL_L2 and mx <= RMAX, (w.name, "dbeta", rel, mx)
+        # the same kernel on the same inputs: every gradient bit-identical (a stale scratch value
+        # read anywhere would show here)
+        for name, a, b in zip(("dq", "dk", "dv", "dg", "dbeta"), _bits(outs), _bits(ref)):
+            assert np.array_equal(a, b), (w.name, name)
+        if i == 0:
+            # and the gradients themselves meet the fp64 reverse mode of the token recurrence
+            got, exp = _grads_host(outs), oracle_grads(d)
+            cu = d["cu_seqlens"]
+            for n in ("dq", "dk", "dv", "dg"):
+                rel, mx = compare_grad(got[n], exp[n], cu, w.H)
+                assert rel <= RTOL_L2 and mx <= RMAX, (w.name, n, rel, mx)
+            rel, mx = compare_grad(got["dbeta"][..., None], exp["dbeta"][..., None], cu, w.H)
+            assert rel <= RTOL_L2 and mx <= RMAX, (w.name, "dbeta", rel, mx)
