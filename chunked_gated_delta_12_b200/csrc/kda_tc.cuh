@@ -80,6 +80,14 @@ __device__ __forceinline__ void dealloc(uint32_t taddr, uint32_t ncols) {
 }
 
 // 32 lanes x 16 / 32 consecutive fp32 columns per warp (lane = TMEM lane)
+__device__ __forceinline__ void ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
@@ -142,8 +150,9 @@ __device__ __forceinline__ bool mbar_try(uint32_t saddr, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for phase `parity` to complete, giving up after ~`limit` clock cycles.
-__device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long long limit) {
+// Wait for phase `parity` to complete, giving up after ~`limit` clock cycles.  Kept out of line:
+// the call sites are many and the wait dwarfs the call, while inlined copies cost instruction cache.
+static __device__ __noinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long long limit) {
     if (mbar_try(saddr, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try(saddr, parity))
