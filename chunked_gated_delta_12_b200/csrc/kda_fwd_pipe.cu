@@ -1,42 +1,32 @@
 // kda_fwd_pipe.cu -- pipelined fused chunk-KDA forward (one CTA per (document, head),
 // all 128 value columns); kda_chunk_fwd launches it for every call.
 //
-// Two chunks are in flight per CTA.  In step s all 16 warps first prepare chunk s (gate factors
-// and every bf16 operand tile); then warps 0-11 finish chunk s's intra-chunk work while warps
-// 12-15 run chunk s-1's state update and output.  Every chunk product runs on the tensor cores
-// with tcgen05.mma (accumulators in tensor memory); only the UT solve's 16 x 16 block products
-// use warp-level MMA.
+// Two chunks are in flight per CTA.  In step s all 16 warps first prepare chunk
+// s; then warps 0-11 finish chunk s's intra-chunk work while warps 12-15 run
+// chunk s-1's state update on the tensor cores and the row norms of chunk s+1.
+// The state is kept transposed, S^T[v][c] in fp32 in tensor memory (lane =
+// value column v), so that both the bf16 copy of the state and the corrected
+// values U~ are tcgen05 A operands read straight from TMEM.
 //
-// Per chunk, with raw q and k, Gamma the inclusive in-chunk cumsum of g, and the row norms
-// n_r = 1/|q_r|, m_r = 1/|k_r| applied outside the products:
-//   L_qk[r,i] = sum_c q_rc k_ic e^{Gamma_rc - Gamma_ic} (i <= r),  L_kk likewise (i < r)
-//   A_kk = diag(beta m) L_kk diag(m),   T = (I + A_kk)^-1
-//   T_U  = diag(m) T diag(beta),        T_W = T_U diag(m)
-//   U' = T_U V,   W' = T_W (K e^Gamma),   U~ = U' - W' S       (U~ is diag(m) times the usual U~)
-//   O  = (Q e^Gamma) S + L_qk U~,          o = scale diag(n) O
-//   S <- Diag(e^{Gamma_63}) S + (K e^{Gamma_63 - Gamma})^T U~
-// which is the recurrence unrolled over the chunk with q^ = diag(n) q and k^ = diag(m) k.
-//
-// L_qk and L_kk come from one tcgen05 product.  The exponent is split at a reference row in the
-// middle of each 32-row half (rows 15 and 47): the row side carries e^{Gamma_r - Gamma_ref(r)},
-// the column side e^{Gamma_ref - Gamma_i}; with gates in [-5, 0] every factor lies within
-// e^{+-80}, inside the fp32 / bf16 range, and each product term keeps its true size
-// |q_rc k_ic| e^{Gamma_rc - Gamma_ic} <= |q_rc k_ic|.  The product is
-//   D[128 rows: q rows | k rows][96 cols] = X Y^T,
-//   X rows r: (q_r | k_r) e^{Gamma_r - Gamma_ref(r)},
-//   Y cols 0..63: k_i e^{Gamma_47 - Gamma_i} (the reference of rows 32..63),
-//   Y cols 64..95: k_i e^{Gamma_15 - Gamma_i}, i < 32 (the reference of rows 0..31);
-// entries of other pairs are never read.
-//
-// The state is kept transposed, S^T[v][c] in fp32 in tensor memory (lane = value column v), so
-// that both its bf16 copy and U~ are tcgen05 A operands read straight from tensor memory:
-//   state  D   = [U'^T | 0] + S^T_bf16 [-W'^T | Q~^T]   -> [U~^T | (Q~ S)^T]
-//          O^T += U~^T_bf16 L_qk^T,   S^T += U~^T_bf16 Kd     (after S^T <- S^T Diag(e^{Gamma_63}))
-// q, k and v tiles arrive by TMA (2-D tensor maps over [T, H*128]); each prep thread reads its
-// channel of g straight from global memory one step ahead (the tiles are prefetched into L2
-// two chunks ahead).  A tile may reach into the next document; rows past the document end are
-// read as zero (q, k, g, beta) or zeroed in shared memory (v), so poisoned neighbours cannot
-// leak.  Every wait is time-limited and reports KDA_ERR_TIMEOUT.
+// Per chunk (rows r, i; Gamma = in-chunk cumsum of g):
+//   A_kk[r,i] = beta_r k^_r.(k^_i e^{Gamma_r - Gamma_i}) (i < r),  A_qk (i <= r)
+//   T' = (I + A_kk)^-1 diag(beta)
+//   W  = T' K^e^Gamma,  U = T' V,  U~ = U - W S
+//   O  = Q^e^Gamma S + A_qk U~
+//   S <- Diag(e^{Gamma_last}) S + (K^ e^{Gamma_last - Gamma})^T U~
+// and on the tensor cores (M = 128 everywhere):
+//   intra  D[:, 0:64] = -(K^e^Gamma)^T T'^T = -W^T, next to Q~^T (written by the prep)
+//          -> B2 = [-W^T | Q~^T] (bf16, shared);  then D[:, 0:64] = V^T T'^T = U^T
+//   state  D   += S^T_bf16 (TMEM) B2                -> [U~^T | (Q~ S)^T]
+//          O^T += U~^T_bf16 (TMEM) A_qk^T
+//          S^T += U~^T_bf16 (TMEM) Kd               (after S^T <- S^T Diag(e^{Gamma_last}))
+// The output scale is carried by Q~ and A_qk.
+// q, k, g and v tiles arrive by TMA (2-D tensor maps over [T, H*128], each CTA loading its own
+// tiles).  A tile may reach into the next document, so the rows past the document end are zeroed
+// in shared memory (q, k and g when the step starts, v before the U product) and count as zero
+// in the row norms.  The gate exponent is split at 16-row sub-block boundaries
+// (e^{G_r - G_i} = E1_r s_RI E2_i, every factor within the fp32/bf16 range).  Every wait is
+// time-limited and reports KDA_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -54,12 +44,10 @@ namespace pipe_path {
 constexpr int kThreads = 512;
 constexpr int kStateTid0 = 384;               // first thread of warps 12-15
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSF = 0;                   // S^T fp32                   [128 lanes v][128 cols c]
-constexpr uint32_t kSB = 128;                 // S^T bf16 packed            [128][64]
-constexpr uint32_t kUB = 128;                 // U~^T bf16 packed [128][32], over S^T bf16 once the state product is done
-constexpr uint32_t kDA = 192;                 // L product [128][96]; then -W'^T [128 c][64 r]
-constexpr uint32_t kQT = 288;                 // Q~^T fp32 [128 c][64 r]
-constexpr uint32_t kDS = 352;                 // [U'^T -> U~^T | O^T]       [128 v][64 + 64]
+constexpr uint32_t kSF = 0;                   // S^T fp32          [128 lanes v][128 cols c]
+constexpr uint32_t kSB = 128;                 // S^T bf16 packed   [128][64]
+constexpr uint32_t kD0 = 192;                 // chunk accumulators, two buffers of 128 columns
+constexpr uint32_t kUB = 448;                 // U~^T bf16 packed  [128][32]
 constexpr long long kWaitLimit = 2000000000LL;
 
 // A_kk / T as ten 16x16 fp32 blocks (I <= R), rows padded to 20 floats
@@ -67,38 +55,34 @@ constexpr int kBlkPitch = 20;
 constexpr int kBlkFloats = 16 * kBlkPitch;
 
 struct Smem {
-    static constexpr int AX = 0;           // raw q, k: TMA boxes [64 rows][64 ch] at +0, +8192 (q), +16384, +24576 (k);
-                                           // then the row side X, MN-major [c][r], atoms q | k
-    static constexpr int BY = 32768;       // column side Y, MN-major [c][n], two 64-wide atoms (N = 96 used)
-    static constexpr int TU = BY;          // after the L product: T_U bf16, K-major [r][i]
-    static constexpr int TW = BY + 8192;   //                      T_W bf16, K-major [r][i]
+    static constexpr int Q = 0;            // raw q: two TMA boxes [64 rows][64 ch] (128 B rows) -> q^E1 [c][r] SW128
+    static constexpr int K = 16384;        // raw k                                                -> k^E1 [c][r] SW128
+    static constexpr int G = 32768;        // raw g: four TMA boxes [64 rows][32 ch] fp32
     static constexpr int V = 65536;        // raw v: two TMA boxes, 128B-swizzled = MN-major SW128 atoms
-    static constexpr int KGT = 81920;      // (K e^Gamma)^T, K-major [c][i]
-    static constexpr int KDT = 98304;      // two buffers: (K e^{Gamma_63 - Gamma})^T, K-major [c][r]; output staging
-    static constexpr int B2 = 131072;      // [-W'^T | Q~^T], MN-major [c][n], two 64-wide atoms
-    static constexpr int AQK = 163840;     // two buffers: L_qk [r][i], K-major (64 rows)
-    static constexpr int SMALL = 180224;
+    static constexpr int KR = 81920;       // k^E2 [c][r] SW128 -> T' (rows 0-63) and the A_qk staging tile
+    static constexpr int KGT = 98304;      // (k^ e^Gamma)^T, K-major [c][r]
+    static constexpr int KDT = 114688;     // two buffers: (k^ e^{Gamma_last-Gamma})^T, K-major [c][r]
+    static constexpr int B2 = 147456;      // [-W^T | Q'^T], MN-major [c][n], two 64-wide atoms
+    static constexpr int AQK = 180224;     // two buffers: A_qk [r][i], K-major (64 rows), read by the state side
+    static constexpr int AKK = 196608;     // A_kk blocks fp32
+    static constexpr int TM = AKK + 10 * kBlkFloats * 4;   // T blocks fp32
+    static constexpr int SMALL = TM + 10 * kBlkFloats * 4;
     static constexpr int BETA = SMALL;               // fp32 [2][64]
-    static constexpr int RQ = BETA + 512;            // fp32 [4][64]  scale / |q_r|
-    static constexpr int RK = RQ + 1024;             // fp32 [2][64]  1 / |k_r|
-    static constexpr int TOT = RK + 512;             // fp32 [4][128] per 16-row block sums of log2e g
-    static constexpr int DL = TOT + 2048;            // fp32 [2][128] e^{Gamma_63}
-    static constexpr int MBAR = DL + 1024;           // u64 [16]
+    static constexpr int RQ = BETA + 512;            // fp32 [64]
+    static constexpr int RK = RQ + 256;              // fp32 [64]
+    static constexpr int TOT = RK + 256;             // fp32 [4][128]
+    static constexpr int PS = TOT + 2048;            // bf16 [10][128] pair scales
+    static constexpr int DC = PS + 2560;             // fp32 [2][128]
+    static constexpr int MBAR = DC + 1024;           // u64 [16]
     static constexpr int TBASE = MBAR + 128;
     static constexpr int ABORT = TBASE + 16;
-    static constexpr int AKK = 186368;               // A_kk blocks fp32 (after the small arrays, 1024-aligned)
-    static constexpr int TM = AKK + 10 * kBlkFloats * 4;   // T blocks fp32
-    // raw g of the next chunk: four TMA boxes [64 rows][32 ch] fp32, landing over the A_kk / T blocks
-    // once the solve is done with them and read by the next step's prep before the next read-back
-    static constexpr int G = AKK;
-    static constexpr int BYTES = G + 32768;
+    static constexpr int BYTES = ABORT + 16;
     static constexpr int ALLOC = BYTES + 1024;
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
-static_assert(Smem::ABORT + 16 <= Smem::AKK && Smem::TM + 10 * kBlkFloats * 4 <= Smem::BYTES, "layout");
 
 // every barrier completes by tcgen05.commit or by TMA transaction bytes
-enum Mbar { kMbA = 0, kMbW, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kNumMbar };
+enum Mbar { kMbWQ = 0, kMbU, kMb2, kMb4, kMbQK, kMbG, kMbV, kNumMbar };
 
 __device__ __forceinline__ void bar_intra() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void bar_state() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
@@ -143,17 +127,14 @@ __device__ __forceinline__ uint4 pack8(const float *x, float s) {
     return make_uint4(pack_bf16(x[0] * s, x[1] * s), pack_bf16(x[2] * s, x[3] * s), pack_bf16(x[4] * s, x[5] * s),
                       pack_bf16(x[6] * s, x[7] * s));
 }
-// eight values held as four row pairs, as bf16
+// eight values held as four row pairs, as bf16 (optionally scaled by a packed multiply)
 __device__ __forceinline__ uint4 pack8x2(const float2 *x) {
     return make_uint4(pack_bf16(x[0].x, x[0].y), pack_bf16(x[1].x, x[1].y), pack_bf16(x[2].x, x[2].y),
                       pack_bf16(x[3].x, x[3].y));
 }
-// 1/x by the hardware approximation (PTX rcp.approx.ftz; x here is a product of decays in
-// [e^-80, 1], far from the denormal range)
-__device__ __forceinline__ float rcp_approx(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
+__device__ __forceinline__ uint4 pack8x2s(const float2 *x, float2 s) {
+    const float2 a = __fmul2_rn(x[0], s), b = __fmul2_rn(x[1], s), c = __fmul2_rn(x[2], s), d = __fmul2_rn(x[3], s);
+    return make_uint4(pack_bf16(a.x, a.y), pack_bf16(b.x, b.y), pack_bf16(c.x, c.y), pack_bf16(d.x, d.y));
 }
 // registers filled by tcgen05.ld are valid only after tcgen05.wait::ld: this empty asm, placed after
 // the wait, keeps the compiler from moving their first use above it
@@ -162,16 +143,20 @@ __device__ __forceinline__ void reg_fence(float (&v)[N]) {
 #pragma unroll
     for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
+__device__ __forceinline__ int pair_R(int p) { return p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0; }
 __device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
 
 // beta rows [tok0, tok0 + L) of head h, one row per calling thread (row in [0, 64); rows >= L zero-filled)
 __device__ __forceinline__ void load_beta(uint8_t *sm, const float *beta, int64_t tok0, int L, int H, int h, int buf,
                                           int row) {
-    const bool ok = row < L;
-    const float *src = ok ? beta + (tok0 + row) * H + h : beta;
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(sm + Smem::BETA + buf * 256 + row * 4)),
-                 "l"(src), "r"(ok ? 4 : 0)
-                 : "memory");
+    {
+        const bool ok = row < L;
+        const float *src = ok ? beta + (tok0 + row) * H + h : beta;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(
+                         smem_u32(sm + Smem::BETA + buf * 256 + row * 4)),
+                     "l"(src), "r"(ok ? 4 : 0)
+                     : "memory");
+    }
 }
 
 struct Maps {
@@ -182,9 +167,10 @@ struct Maps {
 // separate instance, so that the plain forward carries no trace of it
 template <bool kCkpt>
 __global__ void __launch_bounds__(kThreads, 1)
-    kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g, const float *__restrict__ beta,
-                        const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H, const float *h0,
-                        float *ht, float *ckpt, uint16_t *__restrict__ out, int *__restrict__ status) {
+    kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
+                        const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
+                        const float *h0, float *ht, float *ckpt, uint16_t *__restrict__ out,
+                        int *__restrict__ status) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     // align by offsetting the shared array itself, so every access stays in the shared window (LDS/STS)
@@ -192,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
-    // CTA -> (document, head), longest documents first; the AX area is free until the first TMA load
+    // CTA -> (document, head), longest documents first; the Q tile area is free until the first TMA load
     const int doc = doc_at_rank(cu_seqlens, n_docs, blockIdx.x / H, reinterpret_cast<int *>(sm)), h = blockIdx.x % H;
 
     if (blockIdx.x == 0 && tid == 0) {
@@ -221,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *f_rq = reinterpret_cast<float *>(sm + S::RQ);
     float *f_rk = reinterpret_cast<float *>(sm + S::RK);
     float *f_tot = reinterpret_cast<float *>(sm + S::TOT);
-    float *f_dl = reinterpret_cast<float *>(sm + S::DL);
+    __nv_bfloat16 *f_ps = reinterpret_cast<__nv_bfloat16 *>(sm + S::PS);
     float *f_akk = reinterpret_cast<float *>(sm + S::AKK);
     float *f_tm = reinterpret_cast<float *>(sm + S::TM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::ABORT);
@@ -229,8 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto mbar = [&](int i) -> uint32_t { return mb + 8u * (uint32_t)i; };
     const uint32_t sbase = smem_u32(sm);
     // UMMA shared-memory descriptors of the tile area; every operand descriptor is one of these plus the
-    // tile's constant byte offset / 16 (addresses stay below 256 KB, so the 14-bit field cannot carry)
-    const uint64_t dK = tc::sdesc(sbase, 16u, 1024u);           // K-major, 128-byte swizzled rows
+    // tile's byte offset / 16 (addresses stay below 256 KB, so the 14-bit field cannot carry).  Built
+    // once, so that issuing a product is a 64-bit add per instruction.
+    const uint64_t dK = tc::sdesc(sbase, 16u, 1024u);            // K-major, 128-byte swizzled rows
     const uint64_t dM128 = tc::sdesc(sbase, 128u * 128u, 1024u); // MN-major, 128 K rows per 64-wide atom
     const uint64_t dM64 = tc::sdesc(sbase, 64u * 128u, 1024u);   // MN-major, 64 K rows per 64-wide atom
     const int xq = h * kHeadDim;          // TMA x coordinate of this head's channel 0
@@ -238,10 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_qk = [&](int i) {          // q, k tiles of chunk i (one thread)
         const int y = (int)(doc_start + 64 * (int64_t)i);
         tc::mbar_expect_tx(mbar(kMbQK), 32768u);
-        tc::tma_load_2d(sbase + S::AX, &maps.q, xq, y, mbar(kMbQK));
-        tc::tma_load_2d(sbase + S::AX + 8192, &maps.q, xq + 64, y, mbar(kMbQK));
-        tc::tma_load_2d(sbase + S::AX + 16384, &maps.k, xq, y, mbar(kMbQK));
-        tc::tma_load_2d(sbase + S::AX + 24576, &maps.k, xq + 64, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::Q, &maps.q, xq, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::Q + 8192, &maps.q, xq + 64, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::K, &maps.k, xq, y, mbar(kMbQK));
+        tc::tma_load_2d(sbase + S::K + 8192, &maps.k, xq + 64, y, mbar(kMbQK));
     };
     auto issue_g = [&](int i) {
         const int y = (int)(doc_start + 64 * (int64_t)i);
@@ -255,29 +242,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_2d(sbase + S::V, &maps.v, xq, y, mbar(kMbV));
         tc::tma_load_2d(sbase + S::V + 8192, &maps.v, xq + 64, y, mbar(kMbV));
     };
-    // prep thread: channel pc, rows 16 pR .. 16 pR + 15 of the chunk
-    const int pc = tid & 127, pR = tid >> 7;
-    // scale/|q_r| and 1/|k_r| for rows r0..r0+15 of the raw tiles (rows >= Li count as zero), into
-    // the buffers of chunk i.  Lane = (tensor, row): lanes 0-15 sum a q row, lanes 16-31 a k row,
-    // reading its sixteen 16-byte chunks in an order rotated by the lane, so that every load
-    // instruction touches each bank group only as often as its width requires.
-    auto norms16 = [&](int r0, int Li, int i) {
-        const int r = r0 + (lane & 15);
-        const uint8_t *rowp = sm + S::AX + (lane >> 4) * 16384 + r * 128;
-        float acc0 = 0.f, acc1 = 0.f;
-        if (r < Li) {
-#pragma unroll 1
-            for (int j = 0; j < 16; ++j) {
-                const int ch = (j + lane) & 15;
-                const uint4 u = *reinterpret_cast<const uint4 *>(rowp + (ch >> 3) * 8192 + (ch & 7) * 16);
-                const float2 x0 = unpack_bf16(u.x), x1 = unpack_bf16(u.y), x2 = unpack_bf16(u.z), x3 = unpack_bf16(u.w);
-                acc0 = fmaf(x0.x, x0.x, fmaf(x0.y, x0.y, fmaf(x1.x, x1.x, fmaf(x1.y, x1.y, acc0))));
-                acc1 = fmaf(x2.x, x2.x, fmaf(x2.y, x2.y, fmaf(x3.x, x3.x, fmaf(x3.y, x3.y, acc1))));
+    // 1/|q_r| and 1/|k_r| for rows r0..r0+15 of the raw tiles (rows >= Li count as zero).
+    // Each lane sums its 4 channels for all 32 (tensor, row) pairs, then a transposed
+    // butterfly (31 shuffles) leaves lane l with the total of pair l.
+    auto norms16 = [&](int r0, int Li) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = r0 + i;
+            const uint32_t off = (lane >> 4) * 8192 + r * 128 + (lane & 15) * 8;
+            uint2 qa = *reinterpret_cast<const uint2 *>(sm + S::Q + off);
+            uint2 ka = *reinterpret_cast<const uint2 *>(sm + S::K + off);
+            if (r >= Li) qa = ka = make_uint2(0u, 0u);
+            const float2 q01 = unpack_bf16(qa.x), q23 = unpack_bf16(qa.y);
+            const float2 k01 = unpack_bf16(ka.x), k23 = unpack_bf16(ka.y);
+            v[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
+            v[16 + i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+        }
+#pragma unroll
+        for (int lv = 0; lv < 5; ++lv) {
+            const int o = 16 >> lv, half = 16 >> lv;
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int j = 0; j < half; ++j) {
+                const float send = up ? v[j] : v[j + half];
+                const float keep = up ? v[j + half] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
             }
         }
-        const float rn = rsqrtf(acc0 + acc1 + 1e-6f);
-        if (lane < 16) f_rq[(i & 3) * 64 + r] = rn * rsqrtf((float)kHeadDim);
-        else f_rk[(i & 1) * 64 + r] = rn;
+        float *dst = lane < 16 ? f_rq : f_rk;
+        dst[r0 + (lane & 15)] = rsqrtf(v[0] + 1e-6f);
     };
 
     // ---- setup ----
@@ -301,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lq = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * lq) << 16);
     if (warp >= 12) {
-        // S^T[v][c] (lane v) = h0[c][v], or zero; the O columns start at zero
+        // S^T[v][c] (lane v) = h0[c][v], or zero
         const int vcol = 32 * lq + lane;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -310,14 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) z[i] = h0 ? h0[state_off + (size_t)(c0 + i) * kHeadDim + vcol] : 0.f;
             tc::st32(lane_base + kSF + c0, z);
         }
-        float z[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = 0.f;
-        tc::st32(lane_base + kDS + 64, z);
-        tc::st32(lane_base + kDS + 96, z);
         tc::wait_st();
     }
-    // chunk 0's q, k, g (one thread polls the barriers; the CTA barrier releases the rest), then its norms
+    // chunk 0's inputs (one thread polls the barriers; the CTA barrier releases the rest), then its norms
     cp_async_wait_all();
     if (tid == 0) {
         bool ok = tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit);
@@ -325,12 +314,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) *abort_flag = 1;
     }
     __syncthreads();
-    if (warp < 4) norms16(warp * 16, chunk_len(0), 0);
+    if (warp < 4) norms16(warp * 16, chunk_len(0));
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
 
     bool aborted = *abort_flag != 0;
+    const float out_scale = rsqrtf((float)kHeadDim);
 
     for (int s = 0; s <= nchunks && !aborted; ++s) {
         const bool have_intra = s < nchunks;        // chunk s: prep + intra
@@ -341,134 +331,127 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = s & 1;
         const uint32_t par = (uint32_t)(s & 1);
 
-        // q, k, g and beta of chunk s landed before the previous step's closing barrier
+        // beta(s), q, k and g of chunk s landed before the previous step's closing barrier
 
-        // ---- prep pass 1: raw q, k (zero past the document end), per-row decays, in-block products ----
-        uint32_t qp[8], kp[8];     // rows (2j, 2j+1) of this thread's block as packed bf16 pairs
-        float a[16], sa[16];
-        if (have_intra) {
-            const uint8_t *qcol = sm + S::AX + (pc >> 6) * 8192 + (pc & 63) * 2;
-            const uint8_t *kcol = qcol + 16384;
-#pragma unroll
-            for (int j2 = 0; j2 < 8; ++j2) {
-                const int r = 16 * pR + 2 * j2;
-                const uint32_t q0 = r < L ? *reinterpret_cast<const uint16_t *>(qcol + r * 128) : 0u;
-                const uint32_t q1 = r + 1 < L ? *reinterpret_cast<const uint16_t *>(qcol + (r + 1) * 128) : 0u;
-                const uint32_t k0 = r < L ? *reinterpret_cast<const uint16_t *>(kcol + r * 128) : 0u;
-                const uint32_t k1 = r + 1 < L ? *reinterpret_cast<const uint16_t *>(kcol + (r + 1) * 128) : 0u;
-                qp[j2] = q0 | (q1 << 16);
-                kp[j2] = k0 | (k1 << 16);
+        // a partial last chunk: rows past the document end (the TMA tile reaches into the next
+        // document) are zeroed, so the prep below needs no per-element masks
+        if (have_intra && L < 64) {
+            for (int idx = tid; idx < (64 - L) * 16; idx += kThreads) {
+                const int row = L + (idx >> 4), ch = idx & 15;             // 16 chunks of 16 B per row
+                const uint32_t o = (uint32_t)row * 128u + (uint32_t)(ch & 7) * 16u;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sm + S::Q + (ch >> 3) * 8192 + o) = z;
+                *reinterpret_cast<uint4 *>(sm + S::K + (ch >> 3) * 8192 + o) = z;
+                *reinterpret_cast<uint4 *>(sm + S::G + (ch >> 3) * 16384 + o) = z;
+                *reinterpret_cast<uint4 *>(sm + S::G + (ch >> 3) * 16384 + 8192 + o) = z;
             }
-            // a_j = 2^{log2e g_j}; the block's log2 sum; then sa_j = a_{j+1} .. a_15 and, in place,
-            // a_j <- a_0 .. a_j (every such product lies in [e^-80, 1])
-            const uint8_t *gcol = sm + S::G + (pc >> 5) * 8192 + (pc & 31) * 4;
-            float tl = 0.f;
-#pragma unroll
-            for (int j2 = 0; j2 < 8; ++j2) {
-                const int r = 16 * pR + 2 * j2;
-                const float g0 = r < L ? *reinterpret_cast<const float *>(gcol + r * 128) : 0.f;
-                const float g1 = r + 1 < L ? *reinterpret_cast<const float *>(gcol + (r + 1) * 128) : 0.f;
-                const float2 t2 = __fmul2_rn(make_float2(g0, g1), make_float2(kLog2e, kLog2e));
-                tl += t2.x;
-                tl += t2.y;
-                a[2 * j2] = ex2_ftz(t2.x);
-                a[2 * j2 + 1] = ex2_ftz(t2.y);
-            }
-            sa[15] = 1.f;
-#pragma unroll
-            for (int j = 14; j >= 0; --j) sa[j] = sa[j + 1] * a[j + 1];
-#pragma unroll
-            for (int j = 1; j < 16; ++j) a[j] *= a[j - 1];
-            f_tot[pR * 128 + pc] = tl;
+            __syncthreads();
         }
-        // the previous step's U product is done: the column-side tile (T_U, T_W), KGT and V are free
+        float2 ql[8], kl[8], kr[8];      // row pairs (2j, 2j+1) of this thread's 16-row block
+        float lg0 = 0.f;
+        const int pc = tid & 127, pR = tid >> 7;
+        if (have_intra) {
+            // ---- prep pass 1: thread = (channel c, row block R) ----
+            // per-row decays a_j = 2^{log2e g_j} (one exp2 each); E1 and E2 are running products
+            // inside the 16-row block: E1_j = a_1..a_j, E2_j = a_{j+1}..a_15 (both in [e^-75, 1])
+            float2 a[8];
+            float gsum = 0.f;
+            const uint8_t *gcol = sm + S::G + (pc >> 5) * 8192 + (pc & 31) * 4;
+#pragma unroll
+            for (int j2 = 0; j2 < 8; ++j2) {
+                const int r = 16 * pR + 2 * j2;
+                const float g0 = *reinterpret_cast<const float *>(gcol + r * 128);
+                const float g1 = *reinterpret_cast<const float *>(gcol + (r + 1) * 128);
+                gsum += g0;
+                gsum += g1;
+                const float2 gl2 = __fmul2_rn(make_float2(g0, g1), make_float2(kLog2e, kLog2e));   // log2-scaled
+                if (j2 == 0) lg0 = gl2.x;
+                a[j2] = make_float2(ex2_ftz(gl2.x), ex2_ftz(gl2.y));
+            }
+            f_tot[pR * 128 + pc] = gsum * kLog2e;
+            float2 e1[8], e2[8];
+            e1[0] = make_float2(1.f, a[0].y);
+#pragma unroll
+            for (int j2 = 1; j2 < 8; ++j2) {
+                e1[j2].x = e1[j2 - 1].y * a[j2].x;
+                e1[j2].y = e1[j2].x * a[j2].y;
+            }
+            e2[7] = make_float2(a[7].y, 1.f);
+#pragma unroll
+            for (int j2 = 6; j2 >= 0; --j2) {
+                e2[j2].y = e2[j2 + 1].x * a[j2 + 1].x;
+                e2[j2].x = e2[j2].y * a[j2].y;
+            }
+            const uint8_t *qcol = sm + S::Q + (pc >> 6) * 8192 + (pc & 63) * 2;
+            const uint8_t *kcol = sm + S::K + (pc >> 6) * 8192 + (pc & 63) * 2;
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 rq4 = *reinterpret_cast<const float4 *>(f_rq + 16 * pR + 4 * j4);
+                const float4 rk4 = *reinterpret_cast<const float4 *>(f_rk + 16 * pR + 4 * j4);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int j2 = 2 * j4 + h2, r = 16 * pR + 2 * j2;
+                    const float2 qv = make_float2(bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(qcol + r * 128)),
+                                                  bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(qcol + (r + 1) * 128)));
+                    const float2 kv = make_float2(bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(kcol + r * 128)),
+                                                  bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(kcol + (r + 1) * 128)));
+                    const float2 qh = __fmul2_rn(qv, h2 ? make_float2(rq4.z, rq4.w) : make_float2(rq4.x, rq4.y));
+                    const float2 kh = __fmul2_rn(kv, h2 ? make_float2(rk4.z, rk4.w) : make_float2(rk4.x, rk4.y));
+                    ql[j2] = __fmul2_rn(qh, e1[j2]);
+                    kl[j2] = __fmul2_rn(kh, e1[j2]);
+                    kr[j2] = __fmul2_rn(kh, e2[j2]);
+                }
+            }
+        }
+        // the previous step's U product is done: V, KR and its accumulator are free
         if (tid == 0 && have_state && !tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
-        // the previous step's output store has read its staging buffer (KDT[buf], rewritten below)
+        // the previous step's output store has read its staging buffer (Kd's buffer, rewritten below)
         if (tid == kStateTid0) tc::bulk_wait_read();
         tc::fence_before();
-        // raw q, k read (the row-side tile may be written over them); block sums published.  The abort
-        // decision is taken by the barrier itself, so that every thread leaves the loop together.
+        // raw q, k, g read; block sums published.  The abort decision is taken by the barrier itself, so
+        // that every thread leaves the loop together.
         const bool stop = __syncthreads_or(*abort_flag != 0);
         tc::fence_after();
         if (stop) { aborted = true; break; }
         if (have_intra) {
-            // ---- prep pass 2: factors and operand tiles ----
-            // log2 sums of the four 16-row blocks of this channel (pR is warp-uniform: no divergence)
-            const float t0 = f_tot[pc], t1 = f_tot[128 + pc], t2 = f_tot[256 + pc], t3 = f_tot[384 + pc];
-            const float before = pR == 0 ? 0.f : pR == 1 ? t0 : pR == 2 ? t0 + t1 : (t0 + t1) + t2;
-            const float after = pR == 3 ? 0.f : pR == 2 ? t3 : pR == 1 ? t2 + t3 : (t1 + t2) + t3;
-            const float to47 = pR == 0 ? t1 + t2 : pR == 1 ? t2 : 0.f;
-            const float pre = ex2_ftz(before);   // e^{Gamma before this block}
-            const float suf = ex2_ftz(after);    // e^{Gamma_63 - Gamma at this block's end}
-            const float y1s = ex2_ftz(to47);     // e^{Gamma_47 - Gamma at this block's end} (1 for pR >= 2)
-            if (pR == 0) f_dl[buf * 128 + pc] = ex2_ftz(((t0 + t1) + t2) + t3);
-            const bool even = (pR & 1) == 0;
-            const float2 pre2 = make_float2(pre, pre), suf2 = make_float2(suf, suf), y12 = make_float2(y1s, y1s);
-            auto put = [&](int off, const float2 (&x)[4]) { *reinterpret_cast<uint4 *>(sm + off) = pack8x2(x); };
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                // rows 8 hh .. 8 hh + 7 sit in entries 0..7 (the upper half is shifted down below)
-                const int ch = 2 * pR + hh;   // 16-byte chunk of these 8 rows within a 64-row atom
-                // even blocks end at a reference row: X = 1/sa there; odd blocks start right after one:
-                // Y = 1/pa there (one reciprocal per element either way)
-                float inv[8];
+            // ---- prep pass 2 (log2-scaled Gamma) ----
+            float offs[5];
+            offs[0] = 0.f;
 #pragma unroll
-                for (int t = 0; t < 8; ++t) inv[t] = rcp_approx(even ? sa[t] : a[t]);
-                float2 qv[4], kv[4];   // rows 8 hh .. 8 hh + 7 as fp32 pairs (bf16 widens exactly)
+            for (int R = 0; R < 4; ++R) offs[R + 1] = offs[R] + f_tot[R * 128 + pc];
+            const float gm = offs[pR] + lg0;
+            const float ge = offs[pR + 1];
+            const float gl = offs[4];
+            const float P = ex2_ftz(gm);
+            const float2 Pq = make_float2(P * out_scale, P * out_scale);   // the output scale rides on Q~ and A_qk
+            // Q~ into TMEM first (lane c, columns 64+16R..), next to -W^T of the W product
+            {
+                float qtf[16];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    qv[p] = unpack_bf16(qp[p]);
-                    kv[p] = unpack_bf16(kp[p]);
+                for (int j2 = 0; j2 < 8; ++j2) {
+                    const float2 t = __fmul2_rn(ql[j2], Pq);
+                    qtf[2 * j2] = t.x;
+                    qtf[2 * j2 + 1] = t.y;
                 }
-                float2 x[4], y[4];
+                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
+                st16f(lane_base + dcol + 64 + 16 * pR, qtf);
+            }
+            const float2 P2 = make_float2(P, P);
+            const float Dkv = ex2_ftz(gl - ge);
+            const float2 Dk = make_float2(Dkv, Dkv);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {   // row side e^{Gamma_r - Gamma_ref(r)}
-                    const int j = 2 * p;
-                    const float2 fx = even ? make_float2(inv[2 * p], inv[2 * p + 1]) : make_float2(a[j], a[j + 1]);
-                    x[p] = __fmul2_rn(qv[p], fx);
-                    y[p] = __fmul2_rn(kv[p], fx);
-                }
-                put(S::AX + tc::mnmaj_chunk(ch, pc, 128), x);
-                put(S::AX + tc::mnmaj_chunk(8 + ch, pc, 128), y);
+            for (int I = 0; I < 4; ++I)
+                if (I <= pR) f_ps[pair_of(pR, I) * 128 + pc] = __float2bfloat16_rn(ex2_ftz(gm - offs[I + 1]));
+            if (pR == 0) reinterpret_cast<float *>(sm + S::DC)[buf * 128 + pc] = ex2_ftz(gl);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {   // column side e^{Gamma_47 - Gamma_i} and e^{Gamma_15 - Gamma_i}
-                    const int j = 2 * p;
-                    const float2 sa2 = make_float2(sa[j], sa[j + 1]);
-                    const float2 fy1 = pR == 3 ? make_float2(inv[2 * p], inv[2 * p + 1]) : __fmul2_rn(sa2, y12);
-                    const float2 fy0 = even ? sa2 : make_float2(inv[2 * p], inv[2 * p + 1]);
-                    x[p] = __fmul2_rn(kv[p], fy1);
-                    y[p] = __fmul2_rn(kv[p], fy0);
-                }
-                put(S::BY + tc::mnmaj_chunk(ch, pc, 128), x);
-                if (pR < 2) put(S::BY + tc::mnmaj_chunk(8 + ch, pc, 128), y);
-                float qt[8];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {   // e^{Gamma_r} (K e^Gamma, Q~) and e^{Gamma_63 - Gamma_r} (Kd)
-                    const int j = 2 * p;
-                    const float2 e = __fmul2_rn(make_float2(a[j], a[j + 1]), pre2);
-                    const float2 fd = __fmul2_rn(make_float2(sa[j], sa[j + 1]), suf2);
-                    x[p] = __fmul2_rn(kv[p], e);
-                    y[p] = __fmul2_rn(kv[p], fd);
-                    const float2 qe = __fmul2_rn(qv[p], e);
-                    qt[2 * p] = qe.x;
-                    qt[2 * p + 1] = qe.y;
-                }
-                put(S::KGT + tc::kmaj_chunk(pc, ch), x);
-                put(S::KDT + buf * 16384 + tc::kmaj_chunk(pc, ch), y);
-                uint32_t qr[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) qr[i] = __float_as_uint(qt[i]);
-                st8(lane_base + kQT + 16 * pR + 8 * hh, qr);   // lane = channel pc, columns = rows
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    a[t] = a[t + 8];
-                    sa[t] = sa[t + 8];
-                }
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    qp[p] = qp[p + 4];
-                    kp[p] = kp[p + 4];
-                }
+            for (int half = 0; half < 2; ++half) {
+                const int j0 = half * 4;
+                const uint32_t off = tc::kmaj_chunk(pc, 2 * pR + half);
+                *reinterpret_cast<uint4 *>(sm + S::Q + off) = pack8x2(ql + j0);
+                *reinterpret_cast<uint4 *>(sm + S::K + off) = pack8x2(kl + j0);
+                *reinterpret_cast<uint4 *>(sm + S::KR + off) = pack8x2(kr + j0);
+                *reinterpret_cast<uint4 *>(sm + S::KGT + off) = pack8x2s(kl + j0, P2);
+                *reinterpret_cast<uint4 *>(sm + S::KDT + buf * 16384 + off) = pack8x2s(kr + j0, Dk);
             }
             tc::wait_st();
         }
@@ -482,21 +465,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ================= intra (chunk s) =================
             if (have_intra) {
                 const float *f_beta = reinterpret_cast<const float *>(sm + S::BETA + buf * 256);
-                const float *rk = f_rk + buf * 64;
-                // ---- tcgen05: D[128 rows: q | k][96] = X Y^T ----
-                if (tid == 0) {
-                    constexpr uint32_t idA = tc::idesc_bf16(128, 96, true, true, false);
+                // ---- A_kk and A_qk, one 16x16 block pair per warp ----
+                const int aqk = S::AQK + buf * 8192;      // A_qk(s); the other buffer holds A_qk(s-1)
+                if (warp < 10) {
+                    const int p = warp;
+                    const int R = pair_R(p), I = p - R * (R + 1) / 2;
+                    const uint32_t kbase = sbase + S::K, qbase = sbase + S::Q, rbase = sbase + S::KR;
+                    const __nv_bfloat16 *ps = f_ps + p * 128;
+                    float ak[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    float aq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    const int j = lane >> 3;
+                    // the pair scale of this thread's fragment channels, as bf16x2, for all 8 k-steps
+                    __nv_bfloat162 hs[8][2];
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma(tmem + kDA, dM128 + (uint64_t)((S::AX + kk * 2048) >> 4),
-                                dM128 + (uint64_t)((S::BY + kk * 2048) >> 4), idA, kk > 0);
-                    tc::commit(mbar(kMbA));
-                }
-                if (warp >= 10) {
-                    // V is free (the previous U product is done): this chunk's v; the next chunk's beta;
-                    // warm L2 with the tiles of the next steps' loads (v of chunk s+1; q, k, g of s+2)
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int cb = kk * 16 + 2 * tq;
+                        hs[kk][0] = *reinterpret_cast<const __nv_bfloat162 *>(ps + cb);
+                        hs[kk][1] = *reinterpret_cast<const __nv_bfloat162 *>(ps + cb + 8);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = tc::kmaj_chunk(16 * kk + (lane & 7) + 8 * (j >> 1), 2 * R + (j & 1));
+                        uint32_t fk[4], fq[4], b0, b1, b2, b3;
+                        ldsm_x4_t(kbase + aoff, fk[0], fk[1], fk[2], fk[3]);
+                        ldsm_x4_t(qbase + aoff, fq[0], fq[1], fq[2], fq[3]);
+                        ldsm_x4_t(rbase + tc::kmaj_chunk(16 * kk + (lane & 7) + 8 * (j & 1), 2 * I + (j >> 1)), b0, b1,
+                                  b2, b3);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 sc = hs[kk][e >> 1];
+                            __nv_bfloat162 x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fk[e]), sc);
+                            fk[e] = *reinterpret_cast<uint32_t *>(&x);
+                            x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fq[e]), sc);
+                            fq[e] = *reinterpret_cast<uint32_t *>(&x);
+                        }
+                        mma_bf16(ak[0], fk, b0, b1);
+                        mma_bf16(ak[1], fk, b2, b3);
+                        mma_bf16(aq[0], fq, b0, b1);
+                        mma_bf16(aq[1], fq, b2, b3);
+                    }
+                    float *blk = f_akk + p * kBlkFloats;
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int i = gq + 8 * hh, jj = 8 * nt + 2 * tq;
+                            const int row = 16 * R + i, col = 16 * I + jj;
+                            const float br = f_beta[row];
+                            const float x0 = col < row ? ak[nt][2 * hh] * br : 0.f;
+                            const float x1 = col + 1 < row ? ak[nt][2 * hh + 1] * br : 0.f;
+                            *reinterpret_cast<float2 *>(blk + i * kBlkPitch + jj) = make_float2(x0, x1);
+                            const float y0 = col <= row ? aq[nt][2 * hh] * out_scale : 0.f;
+                            const float y1 = col + 1 <= row ? aq[nt][2 * hh + 1] * out_scale : 0.f;
+                            *reinterpret_cast<uint32_t *>(sm + aqk + tc::kmaj_off(row, col)) = pack_bf16(y0, y1);
+                        }
+                } else {
+                    // warps 10-11 have no A_kk block: raw g and the beta(s+1) buffer are free (prep pass 1
+                    // is done) and so is V (the previous U product is done): the next chunk's g and
+                    // beta, this chunk's v
                     if (tid == 320) {
+                        tc::fence_proxy_async();
+                        if (have_next) issue_g(s + 1);
                         issue_v(s);
+                        // warm L2 with the tiles of the next steps' loads (v of chunk s+1; q, k, g of s+2)
                         if (have_next) {
                             const int y1 = (int)(doc_start + 64 * (int64_t)(s + 1));
                             tc::tma_prefetch_2d(&maps.v, xq, y1);
@@ -514,128 +545,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (have_next) load_beta(sm, beta, doc_start + 64 * (int64_t)(s + 1), nL, H, h, buf ^ 1, tid - 320);
                     cp_async_commit();
-                }
-                if (tid == 0) {
-                    if (!tc::mbar_wait(mbar(kMbA), par, kWaitLimit)) *abort_flag = 1;
-                    tc::fence_before();
+                    // A_qk is zero above the block diagonal
+                    for (int idx = tid - 320; idx < 192; idx += 64) {
+                        const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
+                        const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
+                        const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
+                        *reinterpret_cast<uint4 *>(sm + aqk + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                            make_uint4(0, 0, 0, 0);
+                    }
                 }
                 bar_intra();
-                tc::fence_after();
-                // the row-side tile has been read: the next chunk's raw q, k
+                // the state side's tcgen05 product waits for the warp-level A_kk products to finish
+                if (have_state && warp == 0) asm volatile("bar.arrive 4, 160;" ::: "memory");
+                // q^E1 / k^E1 consumed: the next chunk's raw q, k
                 if (tid == 320 && have_next) {
                     tc::fence_proxy_async();
                     issue_qk(s + 1);
                 }
+                const uint32_t dcol = kD0 + 128 * (uint32_t)buf;
+                // warps 8-11: row norms of chunk s+1 while warps 0-7 solve for T (they rejoin at the
+                // barrier before the W readback)
                 if (warp >= 8) {
-                    // warps 8-11: row norms of chunk s+1, once warps 0-3 are through the solve (its
-                    // shared-memory chains are the critical path; the norms are needed only next step)
-                    asm volatile("bar.sync 5, %0;" ::"r"(have_state ? 384 : 256) : "memory");
                     if (have_next) {
                         if (lane == 0 && !tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit)) *abort_flag = 1;
                         __syncwarp();
-                        norms16((warp - 8) * 16, nL, s + 1);
+                        norms16((warp - 8) * 16, nL);
                     }
                 } else {
-                    // ---- read back L_qk (lanes 0-63) and L_kk (lanes 64-127) ----
-                    // lane quarter qd: q rows 0-31 | q rows 32-63 | k rows 0-31 | k rows 32-63; rows of the
-                    // first half use columns 64..95 (i < 32), rows of the second half columns 0..63.  Warp
-                    // pairs split the columns (hf = 0: the first half of them), read 8 columns at a time.
-                    {
-                        const int qd = warp & 3, hf = warp >> 2;
-                        const int row = 32 * (qd & 1) + lane;
-                        const bool second = (qd & 1) != 0;
-                        const int nI = second ? 32 : 16;
-                        const int i0 = nI * hf;
-                        const uint32_t c0 = (second ? 0u : 64u) + (uint32_t)i0;
-                        const int R = row >> 4, rr = row & 15;
-                        const float br = f_beta[row] * rk[row];
-                        uint8_t *aqk = sm + S::AQK + buf * 8192;
-#pragma unroll 1
-                        for (int g8 = 0; g8 < nI; g8 += 8) {
-                            float d[8];
-                            tc::ld8(lane_base + kDA + c0 + (uint32_t)g8, d);
-                            tc::wait_ld();
-                            reg_fence(d);
-                            const int ib = i0 + g8;   // first column i of this group
-                            if (qd < 2) {
-                                // L_qk row, bf16 K-major [r][i], i <= r (no scaling: n rides on the output,
-                                // m on U~)
-                                float x[8];
-#pragma unroll
-                                for (int t = 0; t < 8; ++t) x[t] = ib + t <= row ? d[t] : 0.f;
-                                *reinterpret_cast<uint4 *>(aqk + tc::kmaj_chunk(row, ib >> 3)) = pack8(x, 1.f);
-                            } else {
-                                // A_kk[r][i] = beta_r m_r m_i L_kk[r][i] (i < r) into the block (R, i / 16):
-                                // off-diagonal blocks row-major, the diagonal block transposed (column j at
-                                // j * 20) for the substitution's column reads
-                                const int I = ib >> 4, jb = ib & 15;
-                                float x[8];
-#pragma unroll
-                                for (int t = 0; t < 8; ++t) x[t] = d[t] * br * rk[ib + t];
-                                if (I < R) {
-                                    float *dst = f_akk + pair_of(R, I) * kBlkFloats + rr * kBlkPitch + jb;
-                                    *reinterpret_cast<float4 *>(dst) = make_float4(x[0], x[1], x[2], x[3]);
-                                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
-                                } else if (I == R) {
-                                    float *dst = f_akk + pair_of(R, R) * kBlkFloats + jb * kBlkPitch + rr;
-#pragma unroll
-                                    for (int t = 0; t < 8; ++t) dst[t * kBlkPitch] = jb + t < rr ? x[t] : 0.f;
-                                }
-                            }
-                        }
-                        // rows of the first half: L_qk is zero for i >= 32
-                        if (qd == 0)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e)
-                                *reinterpret_cast<uint4 *>(aqk + tc::kmaj_chunk(row, 4 + 2 * hf + e)) = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                    bar_solve();
-                    // ---- T = (I + A_kk)^-1, diagonal blocks: lane = column, right-looking substitution:
-                    // once x[j] is final, every later row takes its term, x[r] -= A[r][j] x[j] (r > j), with
-                    // column j of A (stored transposed) read as float4; the dependent chain is one
-                    // multiply-add per row.  T (fp32) is kept for the off-diagonal pass; T_U = diag(m) T
-                    // diag(beta) and T_W = T_U diag(m) are written as bf16.
+                    // ---- T = (I + A_kk)^-1, diagonal blocks: lane = column, left-looking substitution
+                    // x[r] = delta_rc - sum_{j<r} A[r][j] x[j] with the rows of A read as float4.
+                    // T (fp32) is kept for the off-diagonal pass, T' = T diag(beta) is written as bf16.
                     if (warp < 4) {
                         if (lane < 16) {
                             const int R = warp, col = lane;
-                            const float *blkT = f_akk + pair_of(R, R) * kBlkFloats;
+                            const float *blk = f_akk + pair_of(R, R) * kBlkFloats;
                             float x[16];
-#pragma unroll
-                            for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
-#pragma unroll
-                            for (int j = 0; j < 15; ++j) {
-                                const float xj = x[j];
-#pragma unroll
-                                for (int r4 = (j + 1) & ~3; r4 < 16; r4 += 4) {
-                                    const float4 av = *reinterpret_cast<const float4 *>(blkT + j * kBlkPitch + r4);
-                                    if (r4 > j) x[r4] -= av.x * xj;
-                                    if (r4 + 1 > j) x[r4 + 1] -= av.y * xj;
-                                    if (r4 + 2 > j) x[r4 + 2] -= av.z * xj;
-                                    if (r4 + 3 > j) x[r4 + 3] -= av.w * xj;
+    #pragma unroll
+                            for (int r = 0; r < 16; ++r) {
+                                float acc = (r == col) ? 1.f : 0.f;
+    #pragma unroll
+                                for (int j4 = 0; j4 < r; j4 += 4) {
+                                    const float4 a = *reinterpret_cast<const float4 *>(blk + r * kBlkPitch + j4);
+                                    acc -= a.x * x[j4];
+                                    if (j4 + 1 < r) acc -= a.y * x[j4 + 1];
+                                    if (j4 + 2 < r) acc -= a.z * x[j4 + 2];
+                                    if (j4 + 3 < r) acc -= a.w * x[j4 + 3];
                                 }
+                                x[r] = acc;
                             }
                             float *tb = f_tm + pair_of(R, R) * kBlkFloats;
-#pragma unroll
-                            for (int r = 0; r < 16; ++r) tb[r * kBlkPitch + col] = x[r];
-                            const float bc = f_beta[16 * R + col], mc = rk[16 * R + col];
-#pragma unroll 1
+                            const float bc = f_beta[16 * R + col];
+    #pragma unroll
                             for (int r = 0; r < 16; ++r) {
-                                const float tu = tb[r * kBlkPitch + col] * rk[16 * R + r] * bc;
-                                const uint32_t o = tc::kmaj_off(16 * R + r, 16 * R + col);
-                                *reinterpret_cast<__nv_bfloat16 *>(sm + S::TU + o) = __float2bfloat16_rn(tu);
-                                *reinterpret_cast<__nv_bfloat16 *>(sm + S::TW + o) = __float2bfloat16_rn(tu * mc);
+                                tb[r * kBlkPitch + col] = x[r];
+                                const __nv_bfloat16 t1 = __float2bfloat16_rn(x[r] * bc);
+                                *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
                             }
                         }
                     } else {
-                        // T_U and T_W are zero above the block diagonal (warps 4-7)
+                        // T' is zero above the block diagonal (warps 4-7)
                         const int t = tid - 128;
-                        for (int idx = t; idx < 384; idx += 128) {
-                            const int tile = idx >= 192 ? 1 : 0, id = idx - 192 * tile;
-                            const int b = id >> 5, row = (id & 31) >> 1, half = id & 1;
+                        for (int idx = t; idx < 192; idx += 128) {
+                            const int b = idx >> 5, row = (idx & 31) >> 1, half = idx & 1;
                             const int R = b < 3 ? 0 : b < 5 ? 1 : 2;
                             const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-                            *reinterpret_cast<uint4 *>(sm + (tile ? S::TW : S::TU) +
-                                                       tc::kmaj_chunk(16 * R + row, 2 * I + half)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                                make_uint4(0, 0, 0, 0);
                         }
                     }
                     bar_solve();
@@ -677,20 +652,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      b[2 * ks], b[2 * ks + 1]);
                         }
                     };
-                    // T_RI strip = -y: T_U = -m_row y beta_col and T_W = T_U m_col, bf16
+                    // T'_RI strip = -y diag(beta), bf16, into the B operand of the W and U products
                     auto store_tp = [&](int R, int I, int nt, const float (&y)[4]) {
                         const int cl = 8 * nt + 2 * tq;
                         const float b0 = f_beta[16 * I + cl], b1 = f_beta[16 * I + cl + 1];
-                        const float m0 = rk[16 * I + cl], m1 = rk[16 * I + cl + 1];
-#pragma unroll
-                        for (int hr = 0; hr < 2; ++hr) {
-                            const int r = 16 * R + gq + 8 * hr;
-                            const float mr = rk[r];
-                            const float u0 = -y[2 * hr] * mr * b0, u1 = -y[2 * hr + 1] * mr * b1;
-                            const uint32_t o = tc::kmaj_off(r, 16 * I + cl);
-                            *reinterpret_cast<uint32_t *>(sm + S::TU + o) = pack_bf16(u0, u1);
-                            *reinterpret_cast<uint32_t *>(sm + S::TW + o) = pack_bf16(u0 * m0, u1 * m1);
-                        }
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq, 16 * I + cl)) =
+                            pack_bf16(-y[0] * b0, -y[1] * b1);
+                        *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
+                            pack_bf16(-y[2] * b0, -y[3] * b1);
                     };
                     if (warp < 4) {
                         // level 32: T_RI = -T_RR (A_RI T_II), (R, I) = (1, 0) or (3, 2)
@@ -730,26 +699,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma16(y3, f_tm + pair_of(3, 3) * kBlkFloats, xb3);
                         store_tp(2, I, nt, y2);
                         store_tp(3, I, nt, y3);
-                        // the solve is through: release the norms (warps 8-11) and the output read-back
-                        asm volatile("bar.arrive 5, %0;" ::"r"(have_state ? 384 : 256) : "memory");
                     }
-                    tc::fence_proxy_async();   // all of T_U, T_W (diagonal, zeros, off-diagonal) to the tensor core
+                    tc::fence_proxy_async();   // all of T' (diagonal, zeros, off-diagonal) to the tensor core
                     bar_solve();
-                    // ---- tcgen05: -W'^T = -(K e^Gamma)^T T_W^T, over the read-back L product ----
-                    // the A_kk / T blocks are done with: the next chunk's g lands over them
-                    if (tid == 128 && have_next) issue_g(s + 1);
+                    // T' is complete: the W product can start now
                     if (tid == 0) {
                         tc::fence_after();
                         constexpr uint32_t id_w = tc::idesc_bf16(128, 64, false, false, true);
-#pragma unroll
+    #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc::mma(tmem + kDA, dK + (uint64_t)((S::KGT + kk * 32) >> 4),
-                                    dK + (uint64_t)((S::TW + kk * 32) >> 4), id_w, kk > 0);
-                        tc::commit(mbar(kMbW));
+                            tc::mma(tmem + dcol, dK + (uint64_t)((S::KGT + kk * 32) >> 4), dK + (uint64_t)((S::KR + kk * 32) >> 4), id_w,
+                                    kk > 0);
+                        tc::commit(mbar(kMbWQ));
                     }
                 }   // warps 0-7
                 if (tid == 0) {
-                    bool ok = tc::mbar_wait(mbar(kMbW), par, kWaitLimit);
+                    bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
                     // B2 is free once the previous chunk's state product has read it
                     if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
                     ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
@@ -759,19 +724,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bar_intra();
                 tc::fence_after();
                 if (warp < 8) {
-                    // B2 = [-W'^T | Q~^T] (bf16, MN-major [c][n]): warps 0-3 from -W'^T, warps 4-7 from Q~^T
-                    const int c = 32 * lq + lane, part = warp >> 2;
-                    const uint32_t src = part ? kQT : kDA;
-#pragma unroll 1
+                    const int c = 32 * lq + lane, cg = warp >> 2;
+#pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         float w[32];
-                        tc::ld32(lane_base + src + 32 * h2, w);
+                        tc::ld32(lane_base + dcol + 64 * cg + 32 * h2, w);
                         tc::wait_ld();
-                        reg_fence(w);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            *reinterpret_cast<uint4 *>(sm + S::B2 + tc::mnmaj_chunk(8 * part + 4 * h2 + e, c, 128)) =
+                            *reinterpret_cast<uint4 *>(sm + S::B2 + tc::mnmaj_chunk(8 * cg + 4 * h2 + e, c, 128)) =
                                 pack8(w + 8 * e, 1.f);
+                    }
+                    if (cg == 1) {
+                        // Q~ has been read: zero its columns, so that the state product can accumulate
+                        // [U~^T | (Q~ S)^T] onto [U^T | 0] with one N = 128 instruction per k-step
+                        float z[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+                        tc::st32(lane_base + dcol + 64, z);
+                        tc::st32(lane_base + dcol + 96, z);
+                        tc::wait_st();
                     }
                 } else if (L < 64) {
                     // rows of v past the document end are zero (the tile may reach the next document)
@@ -784,26 +756,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_proxy_async();
                 tc::fence_before();
                 bar_intra();
-                // ---- tcgen05: U'^T = V^T T_U^T into the state accumulator, once the state side has
-                // finished with the previous chunk's U~ and O there ----
-                if (warp == 0) {
-                    if (have_state) asm volatile("bar.sync 4, 160;" ::: "memory");
-                    if (lane == 0) {
-                        tc::fence_after();
-                        constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false, false);
+                // ---- tcgen05: D[:, 0:64] = V^T T'^T = U^T ----
+                if (tid == 0) {
+                    tc::fence_after();
+                    constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false, false);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc::mma(tmem + kDS, dM64 + (uint64_t)((S::V + kk * 2048) >> 4),
-                                    dK + (uint64_t)((S::TU + kk * 32) >> 4), id_u, kk > 0);
-                        tc::commit(mbar(kMbU));
-                    }
-                    __syncwarp();
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma(tmem + dcol, dM64 + (uint64_t)((S::V + kk * 2048) >> 4), dK + (uint64_t)((S::KR + kk * 32) >> 4), id_u,
+                                kk > 0);
+                    tc::commit(mbar(kMbU));
                 }
             }
-            // the beta rows (issued by warps 10-11) and the g tile of chunk s+1 have landed before the step ends
+            // the beta rows of chunk s+1 (issued by warps 10-11) have landed before the step ends
             cp_async_wait_all();
-            if (tid == 256 && have_next && !tc::mbar_wait(mbar(kMbG), (uint32_t)((s + 1) & 1), kWaitLimit))
-                *abort_flag = 1;
         } else {
             // ================= state warps (12-15) =================
             if (have_state) {
@@ -811,8 +776,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n = s - 1, nbuf = n & 1;
                 const int64_t ptok0 = doc_start + 64 * (int64_t)n;
                 const int pL = chunk_len(n);
-                const float *dc = f_dl + nbuf * 128;
-                // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_63})
+                const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
+                const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
+                // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_last})
                 auto sprep = [&](float (&sv)[16], int c0) {
                     uint32_t pk[8];
 #pragma unroll
@@ -827,11 +793,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     st16f(lane_base + kSF + c0, sv);
                 };
-                // two loads in flight: the next 16 columns are read while the current ones are converted;
+                // two loads in flight: the next 32 columns are read while the current ones are converted;
                 // the product's first four k-steps (key channels 0-63) start once their bf16 copy is in
                 // place, while the second half is converted
                 constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
-                auto state_mma = [&](int kk0) {   // [U~^T | (Q~ S)^T] accumulated onto [U'^T | 0]
+                auto state_mma = [&](int kk0) {   // [U~^T | (Q~ S)^T] accumulated onto [U^T | 0]
+                    if (kk0 == 0 && have_intra) asm volatile("bar.sync 4, 160;" ::: "memory");
                     tc::wait_st();
                     tc::fence_before();
                     bar_state();
@@ -839,38 +806,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::fence_after();
 #pragma unroll
                         for (int kk = kk0; kk < kk0 + 4; ++kk)
-                            mma_ts(tmem + kDS, tmem + kSB + 8 * kk, dM128 + (uint64_t)((S::B2 + kk * 2048) >> 4), id2, 1u);
+                            mma_ts(tmem + dcol, tmem + kSB + 8 * kk, dM128 + (uint64_t)((S::B2 + kk * 2048) >> 4), id2, 1u);
                     }
                 };
                 {
-                    float sa16[16], sb16[16];
-                    tc::ld16(lane_base + kSF, sa16);
+                    float sa[16], sb[16];
+                    tc::ld16(lane_base + kSF, sa);
                     tc::wait_ld();
-                    reg_fence(sa16);
-                    // the state entering chunk n, S[c][v] fp32, into its checkpoint slot
-                    auto ckpt_store = [&](const float (&cur)[16], int c0) {
+                    reg_fence(sa);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float(&cur)[16] = (ch & 1) ? sb : sa;
+                        float(&nxt)[16] = (ch & 1) ? sa : sb;
+                        if (ch < 7) tc::ld16(lane_base + kSF + 16 * (ch + 1), nxt);
                         if constexpr (kCkpt) {
+                            // the state entering chunk n, S[c][v] fp32, into its checkpoint slot
                             float *ck = ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) * (kHeadDim * kHeadDim) +
-                                        (size_t)c0 * kHeadDim + 32 * lq + lane;
+                                        (size_t)(16 * ch) * kHeadDim + 32 * lq + lane;
 #pragma unroll
                             for (int i = 0; i < 16; ++i) ck[(size_t)i * kHeadDim] = cur[i];
                         }
-                    };
-#pragma unroll 1
-                    for (int cp = 0; cp < 4; ++cp) {
-                        const int c0 = 32 * cp;
-                        tc::ld16(lane_base + kSF + c0 + 16, sb16);
-                        ckpt_store(sa16, c0);
-                        sprep(sa16, c0);
-                        tc::wait_ld();
-                        reg_fence(sb16);
-                        if (cp < 3) tc::ld16(lane_base + kSF + c0 + 32, sa16);
-                        ckpt_store(sb16, c0 + 16);
-                        sprep(sb16, c0 + 16);
-                        if (cp == 1) state_mma(0);   // key channels 0-63 converted
-                        if (cp < 3) {
+                        sprep(cur, 16 * ch);
+                        if (ch == 3) state_mma(0);
+                        if (ch < 7) {
                             tc::wait_ld();
-                            reg_fence(sa16);
+                            reg_fence(nxt);
                         }
                     }
                     state_mma(4);
@@ -882,16 +842,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 bar_state();
                 tc::fence_after();
-                // U~^T (columns 0-63) -> bf16 copy (A operand of the O and state products), over the S^T bf16
-                // copy that the state product has finished reading
+                // U~^T (columns 0-63) -> bf16 copy (A operand of the state update)
                 {
                     float u[32];
                     uint32_t pk[16];
-#pragma unroll 1
+#pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
-                        tc::ld32(lane_base + kDS + 32 * h2, u);
+                        tc::ld32(lane_base + dcol + 32 * h2, u);
                         tc::wait_ld();
-                        reg_fence(u);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(u[2 * i], u[2 * i + 1]);
                         st16(lane_base + kUB + 16 * h2, pk);
@@ -902,12 +860,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bar_state();
                 if (tid == kStateTid0) {
                     tc::fence_after();
-                    // O^T += U~^T L_qk^T (L_qk [r][i] is the K-major B operand), then the state update
+                    // O^T += U~^T A_qk^T (A_qk [r][i] is the K-major B operand), then the state update
                     constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + kDS + 64, tmem + kUB + 8 * kk,
-                               dK + (uint64_t)((S::AQK + kk * 32) >> 4) + (uint64_t)(nbuf * (8192 >> 4)), id_o, 1u);
+                        mma_ts(tmem + dcol + 64, tmem + kUB + 8 * kk,
+                               dK + (uint64_t)((S::AQK + kk * 32) >> 4) + (uint64_t)(nbuf * (8192 >> 4)), id_o,
+                               1u);
                     constexpr uint32_t id4 = tc::idesc_bf16(128, 128, false, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -920,36 +879,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 bar_state();
                 tc::fence_after();
-                // wait until the intra warps are through the UT solve (its latency-bound chains are the
-                // step's critical path; the output has slack until the next U product)
-                if (have_intra) asm volatile("bar.sync 5, 384;" ::: "memory");
-                // O^T (columns 64-127): lane v holds O[r][v]; o = (scale / |q_r|) O, taken eight rows at a
-                // time.  Each thread writes its column v of every row (lanes = consecutive v, so one store
-                // instruction covers a contiguous run of a row).
+                // O^T (columns 64-127; the output scale is already applied): lane v holds o[r][v].
+                // Lane pairs swap values so that each thread writes the pair (v, v+1) of one row.
                 {
                     const int vcol = 32 * lq + lane;
-                    const float *rq = f_rq + (n & 3) * 64;
+                    const bool odd = lane & 1;
                     if (pL == 64) {
                         // whole chunk: stage o[r][v] as bf16 in Kd's buffer (free now, rewritten only by the
                         // next step's prep; two 64-channel boxes, 128-B swizzled rows) and write it with one
-                        // TMA store per box
-                        const uint32_t vb = (uint32_t)(vcol & 63) * 2;          // byte of v in its row
+                        // TMA store per box.  Even lanes take rows with
+                        // (r & 4) == 0, odd lanes the row 4 below, so one store instruction covers 32 banks.
+                        const uint32_t vb = (uint32_t)(vcol & 62) * 2;          // byte of the pair in its row
                         const uint32_t stage_off = S::KDT + (uint32_t)nbuf * 16384u;
                         uint8_t *stage = sm + stage_off + (vcol >> 6) * 8192;
-#pragma unroll 1
-                        for (int r0 = 0; r0 < 64; r0 += 8) {
-                            float o[8];
-                            tc::ld8(lane_base + kDS + 64 + (uint32_t)r0, o);
-                            tc::wait_ld();
-                            reg_fence(o);
-                            const float4 ra = *reinterpret_cast<const float4 *>(rq + r0);
-                            const float4 rb = *reinterpret_cast<const float4 *>(rq + r0 + 4);
-                            const float sc[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int r = r0 + i;
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float o[32];
+                            tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
+                            tc::wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int ja = (i & 3) + 8 * (i >> 2), jb = ja + 4;
+                                const float send = odd ? o[ja] : o[jb];
+                                const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                                const float lo = odd ? recv : o[ja];
+                                const float hi = odd ? o[jb] : recv;
+                                const int r = 32 * h2 + (odd ? jb : ja);
                                 const uint32_t off = (uint32_t)r * 128u + ((((vb >> 4) ^ (uint32_t)(r & 7)) << 4) | (vb & 15u));
-                                *reinterpret_cast<__nv_bfloat16 *>(stage + off) = __float2bfloat16_rn(o[i] * sc[i]);
+                                *reinterpret_cast<uint32_t *>(stage + off) = pack_bf16(lo, hi);
                             }
                         }
                         tc::fence_proxy_async();
@@ -962,32 +919,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         // partial chunk: rows past the document end belong to the next document, so
                         // store the valid rows directly
-#pragma unroll 1
-                        for (int r0 = 0; r0 < 64; r0 += 8) {
-                            float o[8];
-                            tc::ld8(lane_base + kDS + 64 + (uint32_t)r0, o);
-                            tc::wait_ld();
-                            reg_fence(o);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int r = r0 + i;
-                                if (r < pL)
-                                    reinterpret_cast<__nv_bfloat16 *>(out)[((ptok0 + r) * H + h) * kHeadDim + vcol] =
-                                        __float2bfloat16_rn(o[i] * rq[r]);
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float o[32];
+                            tc::ld32(lane_base + dcol + 64 + 32 * h2, o);
+                            tc::wait_ld();
+                            // even lanes store rows 32h2 + [0,16), odd lanes rows 32h2 + [16,32)
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float mine_for_partner = odd ? o[i] : o[16 + i];
+                                const float from_partner = __shfl_xor_sync(0xffffffffu, mine_for_partner, 1);
+                                const int r = 32 * h2 + (odd ? 16 + i : i);
+                                const float lo = odd ? from_partner : o[i];
+                                const float hi = odd ? o[16 + i] : from_partner;
+                                if (r < pL) {
+                                    uint32_t *dst = reinterpret_cast<uint32_t *>(
+                                        out + ((ptok0 + r) * H + h) * kHeadDim + (vcol & ~1));
+                                    *dst = pack_bf16(lo, hi);
+                                }
                             }
                         }
                     }
-                    // the O columns start the next chunk's state product from zero
-                    float z[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) z[i] = 0.f;
-                    tc::st32(lane_base + kDS + 64, z);
-                    tc::st32(lane_base + kDS + 96, z);
-                    tc::wait_st();
                 }
-                // U~ and O have been read: the state accumulator is free for the next U product
-                tc::fence_before();
-                if (have_intra) asm volatile("bar.arrive 4, 160;" ::: "memory");
+            }
+            // the raw q, k and g of chunk s+1 have landed before the step ends
+            if (tid == kStateTid0 && have_next) {
+                bool ok = tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit);
+                ok = tc::mbar_wait(mbar(kMbG), (uint32_t)((s + 1) & 1), kWaitLimit) && ok;
+                if (!ok) *abort_flag = 1;
             }
         }
         tc::fence_before();
@@ -1072,7 +1031,7 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (int64_t)n_docs * H;
-    kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, g, beta, cu, n_docs, T, H, h0, ht, ckpt, out, status);
+    kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt, out, status);
     return cudaGetLastError();
 }
 
