@@ -306,9 +306,18 @@ def bench_workloads(kda, steps: int, dev, stream, barrier) -> dict:
             t[key] = torch.from_numpy(dl[key]).to(dev)
         del dl
         out = torch.empty_like(t["q"])
+        split = kda.use_split(wl.n_docs, wl.T, wl.H)
+        ws_split = torch.empty(max(kda.split_workspace_bytes(wl.n_docs, wl.T, wl.H), 256), dtype=torch.uint8,
+                               device=dev) if split else None
+        # kda_chunk_fwd as a user calls it (few chains: routed to kda_chunk_fwd_split), and unsplit
         runs = {"kda_chunk_fwd": lambda: kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"],
-                                                           t["cu_seqlens"], out=out, stream=stream)}
-        entry = {"T": wl.T, "H": wl.H, "n_docs": wl.n_docs, "chains": wl.n_docs * wl.H}
+                                                           t["cu_seqlens"], out=out, stream=stream,
+                                                           workspace=ws_split)}
+        if split:
+            runs["kda_chunk_fwd_unsplit"] = lambda: kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"],
+                                                                      t["cu_seqlens"], out=out, stream=stream,
+                                                                      split=False)
+        entry = {"T": wl.T, "H": wl.H, "n_docs": wl.n_docs, "chains": wl.n_docs * wl.H, "split": split}
         if wl.n_docs == 1:
             P = kda.long_segments(wl.T, wl.H)
             ws = torch.empty(max(kda.long_workspace_bytes(wl.T, wl.H, P), 256), dtype=torch.uint8, device=dev)

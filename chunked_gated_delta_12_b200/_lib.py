@@ -53,6 +53,10 @@ def lib() -> ctypes.CDLL:
                                     ctypes.c_size_t, vp]
         L.kda_chunk_bwd_noalloc.restype = i32
         L.kda_chunk_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.kda_chunk_fwd_split.restype = i32
+        L.kda_chunk_fwd_split.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.kda_chunk_fwd_split_workspace_size.restype = ctypes.c_size_t
+        L.kda_chunk_fwd_split_workspace_size.argtypes = [i32, i64, i32]
         L.kda_chunk_fwd_long.restype = i32
         L.kda_chunk_fwd_long.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.kda_chunk_fwd_long_workspace_size.restype = ctypes.c_size_t
@@ -109,21 +113,57 @@ def _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state, output_final_
     return q, k, v, g, beta, out, n_docs, T, H, final_state
 
 
+# Documents shorter than this many tokens are never cut (three segments of at least 8 chunks).
+SPLIT_MIN_TOKENS = 3 * 8 * 64
+
+
+def use_split(n_docs: int, T: int, H: int, num_sms: int | None = None) -> bool:
+    """Whether ``kda_chunk_fwd`` routes a call through kda_chunk_fwd_split: when its (document, head)
+    chains fill less than half of the GPU's SMs and it has enough tokens for a cut to exist.  The
+    device-side planner then decides which documents (if any) are cut."""
+    if num_sms is None:
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return T >= SPLIT_MIN_TOKENS and 2 * n_docs * H < num_sms
+
+
+def split_workspace_bytes(n_docs: int, T: int, H: int) -> int:
+    """Device workspace bytes kda_chunk_fwd_split needs on the current device
+    (kda_chunk_fwd_split_workspace_size)."""
+    return int(lib().kda_chunk_fwd_split_workspace_size(n_docs, T, H))
+
+
 def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                   beta: torch.Tensor, cu_seqlens: torch.Tensor, out: torch.Tensor | None = None,
                   stream: torch.cuda.Stream | None = None, initial_state: torch.Tensor | None = None,
-                  output_final_state: bool = False, final_state: torch.Tensor | None = None):
-    """Chunked KDA forward through libkda's kda_chunk_fwd (kda_chunk_fwd_state with states).
+                  output_final_state: bool = False, final_state: torch.Tensor | None = None,
+                  split: bool | None = None, workspace: torch.Tensor | None = None):
+    """Chunked KDA forward through libkda: kda_chunk_fwd (kda_chunk_fwd_state with states), or
+    kda_chunk_fwd_split when the call has few (document, head) chains.
 
     q, k, v: [T, H, 128] bf16 (a leading batch dim of 1 is accepted); g: [T, H, 128] fp32;
     beta: [T, H] fp32; cu_seqlens: [n_docs + 1] int32, all on the same CUDA device.
     initial_state: optional [n_docs, H, 128, 128] fp32 starting states (zero if None).
+    split: None chooses by ``use_split``; True / False force kda_chunk_fwd_split / the plain call.
+    workspace: a CUDA uint8 tensor of at least ``split_workspace_bytes`` bytes for the split call,
+    allocated by torch when not given.
     Returns out [T, H, 128] bf16 (allocated by torch if not given), or (out, final_state
     [n_docs, H, 128, 128] fp32) when output_final_state (or a final_state buffer) is given.
     """
     want_state = initial_state is not None or final_state is not None or output_final_state
     q, k, v, g, beta, out, n_docs, T, H, final_state = _fwd_checked(q, k, v, g, beta, cu_seqlens, out, initial_state,
                                                                      output_final_state, final_state)
+    if split is None:
+        split = use_split(n_docs, T, H)
+    if split:
+        need = split_workspace_bytes(n_docs, T, H)
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        rc = lib().kda_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
+                                       _ptr(initial_state), _ptr(final_state), _ptr(out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       ctypes.c_void_p(_stream_handle(stream)))
+        _check(rc)
+        return (out, final_state) if final_state is not None else out
     if not want_state:
         rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
                                  n_docs, T, H, _ptr(out), ctypes.c_void_p(_stream_handle(stream)))

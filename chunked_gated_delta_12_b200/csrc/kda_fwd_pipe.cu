@@ -49,6 +49,9 @@ constexpr uint32_t kSB = 128;                 // S^T bf16 packed   [128][64]
 constexpr uint32_t kD0 = 192;                 // chunk accumulators, two buffers of 128 columns
 constexpr uint32_t kUB = 448;                 // U~^T bf16 packed  [128][32]
 constexpr long long kWaitLimit = 2000000000LL;
+// kernel modes (what a CTA's token range is) and the segment-table state slot encoding
+constexpr int kDocs = 0, kSegs = 1, kTransition = 2;
+constexpr int kSlotCaller = kSplitSlotCaller;
 
 // A_kk / T as ten 16x16 fp32 blocks (I <= R), rows padded to 20 floats
 constexpr int kBlkPitch = 20;
@@ -76,7 +79,8 @@ struct Smem {
     static constexpr int MBAR = DC + 1024;           // u64 [16]
     static constexpr int TBASE = MBAR + 128;
     static constexpr int ABORT = TBASE + 16;
-    static constexpr int BYTES = ABORT + 16;
+    static constexpr int HTP = ABORT + 16;           // this chain's final-state pointer (read after the loop)
+    static constexpr int BYTES = HTP + 16;
     static constexpr int ALLOC = BYTES + 1024;
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
@@ -164,13 +168,18 @@ struct Maps {
 };
 
 // kCkpt: also store the state entering every chunk into `ckpt` (the backward's checkpoints); a
-// separate instance, so that the plain forward carries no trace of it
-template <bool kCkpt>
+// separate instance, so that the plain forward carries no trace of it.
+// kMode: what a CTA's token range is -- kDocs: document blockIdx.x / H of cu_seqlens (every plain
+// forward); kSegs: entry blockIdx.x / H of a segment table built on the device (a document cut into
+// pieces, see kda_split.cu), outputs written; kTransition: the same with v taken as zero, the
+// identity as the entering state and no outputs (a segment's transition map M, its final state).
+template <bool kCkpt, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
                         const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
                         const float *h0, float *ht, float *ckpt, uint16_t *__restrict__ out,
-                        int *__restrict__ status) {
+                        int *__restrict__ status, const int4 *__restrict__ seg, const int *__restrict__ seg_count,
+                        float *ws_states) {
     using S = Smem;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     // align by offsetting the shared array itself, so every access stays in the shared window (LDS/STS)
@@ -178,24 +187,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
-    // CTA -> (document, head), longest documents first; the Q tile area is free until the first TMA load
-    const int doc = doc_at_rank(cu_seqlens, n_docs, blockIdx.x / H, reinterpret_cast<int *>(sm)), h = blockIdx.x % H;
-
-    if (blockIdx.x == 0 && tid == 0) {
-        if (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[n_docs] != T) atomicExch(status, kStatusBadSeqlens);
+    const int h = blockIdx.x % H;
+    int doc = 0;
+    int64_t doc_start, doc_end;
+    // initial / final state of this chain, [128 key channels][128 value columns] fp32, or NULL
+    const float *h0p = nullptr;
+    float *htp = nullptr;
+    if constexpr (kMode == kDocs) {
+        // CTA -> (document, head), longest documents first; the Q tile area is free until the first TMA load
+        doc = doc_at_rank(cu_seqlens, n_docs, blockIdx.x / H, reinterpret_cast<int *>(sm));
+        if (blockIdx.x == 0 && tid == 0) {
+            if (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[n_docs] != T) atomicExch(status, kStatusBadSeqlens);
+        }
+        doc_start = cu_seqlens[doc];
+        doc_end = cu_seqlens[doc + 1];
+        const size_t state_off = ((size_t)doc * H + h) * kHeadDim * kHeadDim;   // [n_docs * H] states
+        if (h0) h0p = h0 + state_off;
+        if (ht) htp = ht + state_off;
+    } else {
+        // CTA -> (table entry, head); entries past the count written by the planner have no work
+        const int rank = blockIdx.x / H;
+        if (rank >= *seg_count) return;
+        const int4 e = seg[rank];
+        doc_start = e.x;
+        doc_end = e.y;
+        auto slot = [&](int sl, const float *caller) -> const float * {
+            if (sl < 0) return nullptr;
+            if (sl < kSlotCaller) return ws_states + ((size_t)sl * H + h) * kHeadDim * kHeadDim;
+            return caller ? caller + ((size_t)(sl - kSlotCaller) * H + h) * kHeadDim * kHeadDim : nullptr;
+        };
+        if constexpr (kMode == kSegs) h0p = slot(e.z, h0);
+        htp = const_cast<float *>(slot(e.w, ht));
     }
-    const int64_t doc_start = cu_seqlens[doc], doc_end = cu_seqlens[doc + 1];
     if (doc_start < 0 || doc_end < doc_start || doc_end > T) {
         if (tid == 0) atomicExch(status, kStatusBadSeqlens);
         return;
     }
-    // initial / final state of this chain: [n_docs * H][128 key channels][128 value columns] fp32
-    const size_t state_off = ((size_t)doc * H + h) * kHeadDim * kHeadDim;
     if (doc_end == doc_start) {
         // nothing to process: the final state is the initial one
-        if (ht)
+        if (htp)
             for (int idx = tid; idx < kHeadDim * kHeadDim; idx += kThreads)
-                ht[state_off + idx] = h0 ? h0[state_off + idx] : 0.f;
+                htp[idx] = h0p ? h0p[idx] : (kMode == kTransition && idx / kHeadDim == idx % kHeadDim ? 1.f : 0.f);
         return;
     }
     const int nchunks = (int)((doc_end - doc_start + 63) / 64);
@@ -275,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // ---- setup ----
+    // the final-state pointer waits in shared memory until after the loop (one register pair less there)
+    if (tid == 0) *reinterpret_cast<float **>(sm + S::HTP) = htp;
     if (warp == 0) tc::alloc(smem_u32(sm + S::TBASE), kTmemCols);
     if (tid == 0) {
         for (int i = 0; i < kNumMbar; ++i) tc::mbar_init(mbar(i), 1);
@@ -295,13 +329,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lq = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * lq) << 16);
     if (warp >= 12) {
-        // S^T[v][c] (lane v) = h0[c][v], or zero
+        // S^T[v][c] (lane v) = h0[c][v], or zero (the identity for a transition pass)
         const int vcol = 32 * lq + lane;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
             float z[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = h0 ? h0[state_off + (size_t)(c0 + i) * kHeadDim + vcol] : 0.f;
+            for (int i = 0; i < 32; ++i)
+                z[i] = kMode == kTransition ? (c0 + i == vcol ? 1.f : 0.f)
+                                            : (h0p ? h0p[(size_t)(c0 + i) * kHeadDim + vcol] : 0.f);
             tc::st32(lane_base + kSF + c0, z);
         }
         tc::wait_st();
@@ -526,9 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (tid == 320) {
                         tc::fence_proxy_async();
                         if (have_next) issue_g(s + 1);
-                        issue_v(s);
+                        if constexpr (kMode != kTransition) issue_v(s);
                         // warm L2 with the tiles of the next steps' loads (v of chunk s+1; q, k, g of s+2)
-                        if (have_next) {
+                        if (kMode != kTransition && have_next) {
                             const int y1 = (int)(doc_start + 64 * (int64_t)(s + 1));
                             tc::tma_prefetch_2d(&maps.v, xq, y1);
                             tc::tma_prefetch_2d(&maps.v, xq + 64, y1);
@@ -717,7 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
                     // B2 is free once the previous chunk's state product has read it
                     if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
-                    ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;    // v(s) landed
+                    if constexpr (kMode != kTransition) ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;   // v(s) landed
                     if (!ok) *abort_flag = 1;
                     tc::fence_before();
                 }
@@ -735,17 +771,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4 *>(sm + S::B2 + tc::mnmaj_chunk(8 * cg + 4 * h2 + e, c, 128)) =
                                 pack8(w + 8 * e, 1.f);
                     }
-                    if (cg == 1) {
+                    if (cg == 1 || kMode == kTransition) {
                         // Q~ has been read: zero its columns, so that the state product can accumulate
-                        // [U~^T | (Q~ S)^T] onto [U^T | 0] with one N = 128 instruction per k-step
+                        // [U~^T | (Q~ S)^T] onto [U^T | 0] with one N = 128 instruction per k-step.  With
+                        // v = 0 (a transition pass) U = 0 too, and -W^T's columns are zeroed instead of
+                        // running the U product.
                         float z[32];
 #pragma unroll
                         for (int i = 0; i < 32; ++i) z[i] = 0.f;
-                        tc::st32(lane_base + dcol + 64, z);
-                        tc::st32(lane_base + dcol + 96, z);
+                        tc::st32(lane_base + dcol + 64 * cg, z);
+                        tc::st32(lane_base + dcol + 64 * cg + 32, z);
                         tc::wait_st();
                     }
-                } else if (L < 64) {
+                } else if (kMode != kTransition && L < 64) {
                     // rows of v past the document end are zero (the tile may reach the next document)
                     for (int idx = tid - 256; idx < (64 - L) * 16; idx += 128) {
                         const int row = L + (idx >> 4), ch = idx & 15;
@@ -759,11 +797,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- tcgen05: D[:, 0:64] = V^T T'^T = U^T ----
                 if (tid == 0) {
                     tc::fence_after();
-                    constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false, false);
+                    if constexpr (kMode != kTransition) {
+                        constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false, false);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma(tmem + dcol, dM64 + (uint64_t)((S::V + kk * 2048) >> 4), dK + (uint64_t)((S::KR + kk * 32) >> 4), id_u,
-                                kk > 0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma(tmem + dcol, dM64 + (uint64_t)((S::V + kk * 2048) >> 4),
+                                    dK + (uint64_t)((S::KR + kk * 32) >> 4), id_u, kk > 0);
+                    }
+                    // (with no product issued the commit tracks the W product alone: the step's tensor
+                    // work is done when it arrives)
                     tc::commit(mbar(kMbU));
                 }
             }
@@ -880,8 +922,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bar_state();
                 tc::fence_after();
                 // O^T (columns 64-127; the output scale is already applied): lane v holds o[r][v].
-                // Lane pairs swap values so that each thread writes the pair (v, v+1) of one row.
-                {
+                // Lane pairs swap values so that each thread writes the pair (v, v+1) of one row.  (A
+                // transition pass has no output.)
+                if constexpr (kMode != kTransition) {
                     const int vcol = 32 * lq + lane;
                     const bool odd = lane & 1;
                     if (pL == 64) {
@@ -956,7 +999,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- final state: ht[c][v] = S^T[v][c] (the last state update has completed) ----
-    if (!aborted && ht && warp >= 12) {
+    htp = *reinterpret_cast<float *volatile *>(sm + S::HTP);
+    if (!aborted && htp && warp >= 12) {
         const int vcol = 32 * lq + lane;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -964,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::ld32(lane_base + kSF + c0, z);
             tc::wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ht[state_off + (size_t)(c0 + i) * kHeadDim + vcol] = z[i];
+            for (int i = 0; i < 32; ++i) htp[(size_t)(c0 + i) * kHeadDim + vcol] = z[i];
         }
     }
 
@@ -1014,25 +1058,66 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
 
 }  // namespace pipe_path
 
+namespace {
+
+// TMA maps of one launch; `v` and `out` may be NULL for a transition pass (never loaded or stored:
+// their maps are then built over q, only to have a valid descriptor)
+bool make_maps(pipe_path::Maps &maps, const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+               uint16_t *out, int64_t T, int H) {
+    using namespace pipe_path;
+    const uint64_t cols = (uint64_t)H * kHeadDim;
+    const void *vb = v ? static_cast<const void *>(v) : q;
+    const void *ob = out ? static_cast<const void *>(out) : q;
+    return make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           make_map(&maps.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)T, cols, 64, 32, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           make_map(&maps.v, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+           make_map(&maps.o, ob, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <bool kCkpt, int kMode>
+cudaError_t launch_mode(const pipe_path::Maps &maps, const float *beta, const int32_t *cu, int n_docs, int64_t T,
+                        int H, const float *h0, float *ht, float *ckpt, uint16_t *out, int *status, const int4 *seg,
+                        const int *seg_count, float *ws_states, int64_t ctas, cudaStream_t stream) {
+    using namespace pipe_path;
+    constexpr int bytes = Smem::ALLOC;
+    auto kernel = kda_fwd_pipe_kernel<kCkpt, kMode>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    kernel<<<(unsigned)ctas, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt, out, status, seg,
+                                                          seg_count, ws_states);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, const float *h0,
                             float *ht, uint16_t *out, int *status, cudaStream_t stream, float *ckpt) {
     using namespace pipe_path;
     Maps maps;
-    const uint64_t cols = (uint64_t)H * kHeadDim;
-    if (!make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)T, cols, 64, 32, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps.o, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_maps(maps, q, k, v, g, out, T, H)) return cudaErrorInvalidValue;
+    const int64_t ctas = (int64_t)n_docs * H;
+    return ckpt ? launch_mode<true, kDocs>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt, out, status, nullptr, nullptr,
+                                           nullptr, ctas, stream)
+                : launch_mode<false, kDocs>(maps, beta, cu, n_docs, T, H, h0, ht, nullptr, out, status, nullptr,
+                                            nullptr, nullptr, ctas, stream);
+}
+
+cudaError_t launch_fwd_segments(bool transition, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                const float *g, const float *beta, int64_t T, int H, const int4 *seg,
+                                const int *seg_count, int max_segs, const float *h0, float *ht, float *ws_states,
+                                uint16_t *out, int *status, cudaStream_t stream) {
+    using namespace pipe_path;
+    if (max_segs <= 0) return cudaSuccess;
+    Maps maps;
+    if (!make_maps(maps, q, k, transition ? nullptr : v, g, transition ? nullptr : out, T, H))
         return cudaErrorInvalidValue;
-    constexpr int bytes = Smem::ALLOC;
-    auto kernel = ckpt ? kda_fwd_pipe_kernel<true> : kda_fwd_pipe_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    const int64_t blocks = (int64_t)n_docs * H;
-    kernel<<<(unsigned)blocks, kThreads, bytes, stream>>>(maps, beta, cu, n_docs, T, H, h0, ht, ckpt, out, status);
-    return cudaGetLastError();
+    const int64_t ctas = (int64_t)max_segs * H;
+    return transition ? launch_mode<false, kTransition>(maps, beta, nullptr, 0, T, H, nullptr, ht, nullptr, nullptr,
+                                                        status, seg, seg_count, ws_states, ctas, stream)
+                      : launch_mode<false, kSegs>(maps, beta, nullptr, 0, T, H, h0, ht, nullptr, out, status, seg,
+                                                  seg_count, ws_states, ctas, stream);
 }
 
 }  // namespace kda

@@ -21,6 +21,19 @@ cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t
                             const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream,
                             float *ckpt = nullptr);
 
+// Segment-table forward (kda_split.cu builds the tables on the device): CTA (entry, head) runs
+// entry blockIdx.x / H of `seg`, {first token, end token, entering-state slot, final-state slot},
+// for entries below *seg_count; max_segs bounds the count (the grid is max_segs * H CTAs).  A slot
+// is -1 (zero entering state / no final state), a workspace slot s < kSplitSlotCaller (the state at
+// ws_states + (s * H + head) * 128 * 128), or kSplitSlotCaller + d (document d of h0 / ht).
+// transition: v taken as zero, the identity as every entering state, no outputs (the transition
+// map M of each segment lands in its final-state slot).
+constexpr int kSplitSlotCaller = 1 << 24;
+cudaError_t launch_fwd_segments(bool transition, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                const float *g, const float *beta, int64_t T, int H, const int4 *seg,
+                                const int *seg_count, int max_segs, const float *h0, float *ht, float *ws_states,
+                                uint16_t *out, int *status, cudaStream_t stream);
+
 // Token-by-token forward (the recurrence itself, no chunking): one CTA of 128 threads per
 // (document, head), the state in registers.  Same arguments and contract as launch_fwd_pipe.
 cudaError_t launch_fwd_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,

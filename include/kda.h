@@ -20,8 +20,8 @@
  * kda_recurrent_fwd is the token-by-token mode (the "recurrent" alternative to
  * "chunk" that the kda_mode setting and KimiDeltaAttention._resolve_mode of
  * the kimi_linear model page choose between) for decoding and short inputs;
- * kda_chunk_fwd_long runs one long document as segments joined through the
- * state hand-off; kda_chunk_bwd (and kda_chunk_bwd_noalloc) is the backward.
+ * kda_chunk_fwd_split (and kda_chunk_fwd_long, its one-document form) cuts long
+ * documents into segments joined through the state hand-off; kda_chunk_bwd (and kda_chunk_bwd_noalloc) is the backward.
  * Like fused_kda_unsupported_reason on the kda_fused page, every call that
  * falls outside this scope is rejected with the first violated condition
  * (kda_last_error); there is no fallback path of any kind.
@@ -129,6 +129,59 @@ kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_
                              const float *initial_state, float *final_state, uint16_t *out, void *stream);
 
 /*
+ * kda_chunk_fwd_split -- kda_chunk_fwd_state with long documents cut into segments that run side
+ * by side (for calls with few (document, head) chains: one long document, or a few long documents
+ * packed with short ones).
+ *
+ * Why: the chunked kernel runs one CTA per (document, head) chain, so a call with few chains keeps
+ * few SMs busy and takes as long as its longest serial chain of chunk steps.
+ *
+ * Operation: the same result as kda_chunk_fwd_state, up to rounding.  The recurrence in the header
+ * comment is affine in the state: a segment of tokens maps its entering state to
+ * S_out = M S_in + N, where N is the segment run from the zero state and M the product of its
+ * per-token maps (I - beta k k^T) Diag(exp(g)) (the same run with v = 0 from the identity state).
+ * A planner kernel reads cu_seqlens on the device and cuts the documents with the longest chains
+ * into P segments at chunk boundaries (at least 8 chunks each, P <= 16), as many as keep the first
+ * stage within one wave of the GPU's SMs (a cut document holds 2 P - 3 chains per head there);
+ * documents that are not cut run whole in the first stage.  A cut document runs as
+ *   1. N_p of segments 0..P-2 (segment 0 from its initial state; its outputs are final), while a
+ *      second, library-owned stream computes M_p of the middle segments 1..P-2;
+ *   2. the hand-off, in fp32: S_in(1) = N_0, S_in(p + 1) = M_p S_in(p) + N_p;
+ *   3. segments 1..P-1 from their entering states: their outputs and the final state.
+ * The state hand-off between pieces of one sequence is how the kimi_k3 model page runs KDA under
+ * context parallelism (KimiDeltaAttention._forward_with_cp passes the recurrent state from one shard
+ * to the next); the transition map M lets the pieces run at the same time on one GPU.  Outputs of
+ * documents that are not cut, and of every first segment, are bit-identical to kda_chunk_fwd_state's.
+ *
+ * Arguments: as kda_chunk_fwd_state, plus
+ *   workspace       DEVICE memory, 256-byte aligned, at least
+ *                   kda_chunk_fwd_split_workspace_size(n_docs, T, H) bytes for the current device,
+ *                   overlapping no other argument; its contents on entry do not matter.  Calls that
+ *                   share a workspace must be ordered (one stream).
+ * Streams: the M pass runs on a non-blocking stream that libkda creates, with two events, once per
+ * device at the first call that needs it, with that device current; `stream` forks to it and joins
+ * it through the events, so the call stays asynchronous and ordered on `stream`.  That second stream
+ * is shared by every call on the device: while a call is being captured into a CUDA graph, the shared
+ * stream belongs to that capture until the capture ends, so no other split call on the same device
+ * (from another thread or another stream) may run between the captured call and the end of its
+ * capture.
+ * Ownership and errors: as kda_chunk_fwd_state (a malformed cu_seqlens table is found by the planner
+ * on the device, nothing runs, and kda_device_status() reports KDA_ERR_BAD_SEQLENS); bad sizes,
+ * pointers, alignment, aliasing or a small workspace return KDA_ERR_INVALID_ARG and launch nothing.
+ */
+kda_status kda_chunk_fwd_split(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                               const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                               const float *initial_state, float *final_state, uint16_t *out, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
+ * kda_chunk_fwd_split_workspace_size -- bytes of workspace kda_chunk_fwd_split needs for these sizes
+ * on the current device (it depends on the device's SM count, not on the document lengths); 0 for
+ * invalid sizes.  About 3 (SMs / H) states of 64 KB per head plus the segment tables.
+ */
+size_t kda_chunk_fwd_split_workspace_size(int n_docs, int64_t T, int H);
+
+/*
  * kda_chunk_fwd_long -- kda_chunk_fwd_state for ONE document, its chunk chain split into
  * `segments` pieces that run side by side.
  *
@@ -160,13 +213,7 @@ kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_
  *                   kda_chunk_fwd_long_workspace_size(T, H, segments) bytes, overlapping no
  *                   other argument; its contents on entry do not matter.  Calls that share a
  *                   workspace must be ordered (one stream).
- * Streams: stage 1's M pass runs on a non-blocking stream that libkda creates, with two events,
- * once per device at the first call with P >= 3 with that device current; `stream` forks to it
- * and joins it through the events, so the call stays asynchronous and ordered on `stream`.
- * That second stream is shared by every call with P >= 3 on the device.  While such a call is
- * being captured into a CUDA graph, the shared stream belongs to that capture until the capture
- * ends, so no other call with P >= 3 on the same device (from another thread or another stream)
- * may run between the captured call and the end of its capture.
+ * Streams: as kda_chunk_fwd_split (this is that call with one document and a fixed segment count).
  * Ownership and errors: as kda_chunk_fwd_state; bad sizes, pointers, alignment, aliasing or a
  * small workspace return KDA_ERR_INVALID_ARG and launch nothing.
  */
@@ -177,9 +224,8 @@ kda_status kda_chunk_fwd_long(const uint16_t *q, const uint16_t *k, const uint16
 
 /*
  * kda_chunk_fwd_long_workspace_size -- bytes of workspace kda_chunk_fwd_long needs for these
- * sizes (0 for invalid sizes): 256 bytes of cu_seqlens tables; for P >= 2, per head
- * 3 (P - 1) states of 64 KB; for P >= 3, per head 2 (P - 2) more states and two bf16
- * [tokens of segments 1..P-2, H, 128] buffers (zero values and the M pass's unused outputs).
+ * sizes (0 for invalid sizes): the segment tables and, for P >= 2, per head 3 P - 4 states of
+ * 64 KB (N and entering states of P - 1 segments, M of P - 2).
  */
 size_t kda_chunk_fwd_long_workspace_size(int64_t T, int H, int segments);
 

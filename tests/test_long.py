@@ -39,13 +39,13 @@ def test_segment_choice(L):
 def test_workspace_size(L):
     size = L.kda_chunk_fwd_long_workspace_size
     assert size(65536, 32, 0) == 0 and size(65536, 32, 17) == 0 and size(65536, 0, 3) == 0
-    assert size(100, 2, 1) == 256            # only the cu_seqlens tables
-    for T, H, P in ((65536, 32, 3), (1937, 2, 5), (4096, 8, 2)):
-        b = bounds(T, P)
-        mid_tokens = b[P - 1] - b[1] if P >= 3 else 0
-        up = lambda x: (x + 255) // 256 * 256
-        want = 256 + 3 * up((P - 1) * H * STATE) + 2 * up(max(P - 2, 0) * H * STATE) \
-            + 2 * up(mid_tokens * H * 128 * 2)
+    up = lambda x: (x + 255) // 256 * 256
+    assert size(100, 2, 1) == 256 + up(16)   # the table counts and one table entry
+    for T, H, P in ((65536, 32, 3), (1937, 2, 5), (4096, 8, 2), (100, 3, 1)):
+        # counts; N, M and final tables and the hand-off record (16 bytes per entry); per head
+        # 3 P - 4 states (N and entering states of P - 1 segments, M of P - 2)
+        want = 256 + up(P * 16) + up(max(P - 2, 0) * 16) + up(max(P - 1, 0) * 16) + up((P >= 2) * 16) \
+            + up(max(3 * P - 4, 0) * H * STATE)
         assert size(T, H, P) == want, (T, H, P)
 
 

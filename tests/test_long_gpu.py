@@ -54,9 +54,10 @@ def run_long(kda, d, P, h0=None, final=False, workspace=None, in_place=False):
 
 
 def run_plain(kda, d):
+    """The unsplit forward (kda_chunk_fwd itself, whatever the chain count)."""
     import torch
     t = to_device(d)
-    o = kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"])
+    o = kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"], split=False)
     kda.device_status()
     torch.cuda.synchronize()
     return out_to_f64(o)
