@@ -7,14 +7,16 @@
 //   S' = Diag(e^{g_t}) S,  p = S'^T k^,  S = S' + beta_t k^ (v_t - p)^T,  o_t = scale S^T q^
 //
 // A chain's 128 value columns are split over 4 CTAs of 128 threads (the columns of S evolve
-// independently given q, k, g and beta, so the split needs no exchange).  Four adjacent lanes
-// share value column v and keep 32 rows each of the fp32 state column S[:, v] in registers, so a
-// token costs 4 x 32 multiply-adds per thread, with the token's q, k and decays broadcast from
-// shared memory, one barrier, and the next token's inputs loaded while this one computes.  The norms are applied
-// to the dot products rather than to the vectors: S'^T k^ = rk S'^T k and likewise for q.
-// The state may start from an initial state and be written out at the end, as in
-// kda_chunk_fwd_state.  Meant for few tokens per document (decode after a prefill); the chunked
-// kernel is far faster per token on long documents.
+// independently given q, k, g and beta, so the split needs no exchange).  Thread (quad, group)
+// keeps 4 adjacent columns of 8 rows of the fp32 state in registers, so that the state moves as
+// 16-byte vectors and every warp instruction covers four whole 128-byte row pieces.  Per token the
+// CTA stages q, k and the decays in shared memory with the norm partial sums, each thread forms
+// its rows' share of S'^T k and S'^T q for its 4 columns, the 16 row groups meet by two shuffle
+// levels and one exchange between the 4 warps, and every thread applies the rank-one update to
+// its rows.  The norms are applied to the dot products rather than to the vectors:
+// S'^T k^ = rk S'^T k and likewise for q.  The state may start from an initial state and be
+// written out at the end, as in kda_chunk_fwd_state.  Meant for few tokens per document (decode
+// after a prefill); the chunked kernel is far faster per token on long documents.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -30,16 +32,22 @@ constexpr int kThreads = 128;
 
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-// One token's inputs as this thread loads them: channel c of q, k and g, column `col` of v, beta.
+// One token's inputs as this thread loads them: channel c of q, k and g, its 4 columns of v, beta.
 struct Tok {
-    float q, k, g, v, beta;
+    float q, k, g, beta;
+    uint2 v;   // four bf16
 };
 
-// kSplit threads share one value column, each holding kRows = 128 / kSplit rows of it; a CTA of
-// 128 threads covers kCols = 128 / kSplit columns, so a chain takes kSplit CTAs (the columns of
-// S evolve independently given q, k, g and beta, so splitting them needs no exchange).
-template <int kSplit, int kAhead>
-__global__ void __launch_bounds__(kThreads) kda_recurrent_kernel(const uint16_t *__restrict__ q,
+constexpr int kSplit = 4;                // CTAs per chain, 32 columns each
+constexpr int kCols = D / kSplit;        // columns of a CTA
+constexpr int kQuads = kCols / 4;        // 8 column quads
+constexpr int kGroups = kThreads / kQuads;   // 16 row groups
+constexpr int kRows = D / kGroups;       // 8 rows per group
+constexpr int kAhead = 1;                // tokens of inputs in flight
+
+// 6 CTAs per SM (80 registers): enough state bytes in flight for the decoding step to run at ~0.9 of
+// the HBM copy rate (4 CTAs at the natural 108-128 registers reached ~0.79)
+__global__ void __launch_bounds__(kThreads, 6) kda_recurrent_kernel(const uint16_t *__restrict__ q,
                                                                  const uint16_t *__restrict__ k,
                                                                  const uint16_t *__restrict__ v,
                                                                  const float *__restrict__ g,
@@ -48,9 +56,6 @@ __global__ void __launch_bounds__(kThreads) kda_recurrent_kernel(const uint16_t 
                                                                  int64_t T, int H, const float *h0, float *ht,
                                                                  uint16_t *__restrict__ out,
                                                                  int *__restrict__ status) {
-    static_assert(kAhead % 2 == 0, "the smem double buffer alternates by token parity");
-    constexpr int kRows = D / kSplit, kCols = D / kSplit;
-    constexpr int kVec = D + 4 * kSplit;    // smem vector: each row block shifted by 4 floats (other banks)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int chain = blockIdx.x, doc = chain / H, h = chain % H;
     if (chain == 0 && blockIdx.y == 0 && tid == 0 && (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[n_docs] != T))
@@ -60,37 +65,38 @@ __global__ void __launch_bounds__(kThreads) kda_recurrent_kernel(const uint16_t 
         if (tid == 0) atomicExch(status, kStatusBadSeqlens);
         return;
     }
-    // thread (col, part): S[part*kRows + r][col], r < kRows, as kRows/2 packed pairs; the kSplit
-    // threads of a column are adjacent lanes and meet with shuffles
-    const int part = tid % kSplit, col = blockIdx.y * kCols + tid / kSplit, r0 = part * kRows;
+    // thread (quad, group): columns col..col+3, rows r0..r0+7; the 4 groups of a warp hold the same
+    // quads (lanes 8 apart)
+    const int quad = tid & (kQuads - 1), grp = tid / kQuads;
+    const int col = blockIdx.y * kCols + 4 * quad, r0 = kRows * grp;
     const size_t soff = (size_t)chain * D * D;
-    float2 S[kRows / 2];
+    float4 S[kRows];
 #pragma unroll
-    for (int j = 0; j < kRows / 2; ++j)
-        S[j] = h0 ? make_float2(h0[soff + (size_t)(r0 + 2 * j) * D + col], h0[soff + (size_t)(r0 + 2 * j + 1) * D + col])
-                  : make_float2(0.f, 0.f);
+    for (int j = 0; j < kRows; ++j)
+        S[j] = h0 ? *reinterpret_cast<const float4 *>(h0 + soff + (size_t)(r0 + j) * D + col)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
 
-    // Per-token broadcast vectors (raw q, raw k, e^g) and the norm partial sums, double-buffered
-    // by token parity: a thread writing token t+2's buffers has passed token t+1's barrier,
-    // which every reader of token t's buffers reached only after its last read of them.
-    __shared__ __align__(16) float sq[2][kVec], sk[2][kVec], sa[2][kVec];
+    // Per-token broadcast vectors (raw q, raw k, e^g), the norm partial sums and the warps' column
+    // sums, double-buffered by token parity: a thread writing token t+2's buffers has passed both
+    // barriers of token t+1, which every reader of token t's buffers reached only after its last
+    // read of them.
+    __shared__ __align__(16) float sq[2][D], sk[2][D], sa[2][D];
     __shared__ float sred[2][3][4];
+    __shared__ __align__(16) float4 spw[2][4][kQuads][2];   // [parity][warp][quad]{S'^T k, S'^T q}
     const float scale = rsqrtf((float)D);
     const int c = tid;                       // key channel of the load phase
-    const int cs = c + (c / kRows) * 4;      // its smem slot
     auto load = [&](int64_t t) {
         const size_t row = ((size_t)t * H + h) * D;
         Tok x;
         x.q = bf2f(q[row + c]);
         x.k = bf2f(k[row + c]);
         x.g = g[row + c];
-        x.v = bf2f(v[row + col]);
+        x.v = *reinterpret_cast<const uint2 *>(v + row + col);
         x.beta = beta[(size_t)t * H + h];
         return x;
     };
     // Inputs run kAhead tokens ahead of the arithmetic: token t's registers are refilled with
-    // token t + kAhead right after they are staged, and the loop is unrolled kAhead times so
-    // that no register copy waits for a load issued less than kAhead tokens earlier.
+    // token t + kAhead right after they are staged.
     Tok x[kAhead];
 #pragma unroll
     for (int i = 0; i < kAhead; ++i)
@@ -100,10 +106,10 @@ __global__ void __launch_bounds__(kThreads) kda_recurrent_kernel(const uint16_t 
         for (int i = 0; i < kAhead; ++i) {
             const int64_t t = tb + i;
             if (t >= t1) break;
-            const int b = i & 1;             // (t - t0) & 1, kAhead being even
-            sq[b][cs] = x[i].q;
-            sk[b][cs] = x[i].k;
-            sa[b][cs] = ex2_ftz(x[i].g * kLog2e);
+            const int b = (int)((t - t0) & 1);   // buffer parity of this token
+            sq[b][c] = x[i].q;
+            sk[b][c] = x[i].k;
+            sa[b][c] = ex2_ftz(x[i].g * kLog2e);
             float pq = x[i].q * x[i].q, pk = x[i].k * x[i].k, pqk = x[i].q * x[i].k;
 #pragma unroll
             for (int o = 16; o; o >>= 1) {
@@ -116,73 +122,85 @@ __global__ void __launch_bounds__(kThreads) kda_recurrent_kernel(const uint16_t 
                 sred[b][1][warp] = pk;
                 sred[b][2][warp] = pqk;
             }
-            const float v_t = x[i].v, b_t = x[i].beta;
+            const uint2 v_t = x[i].v;
+            const float b_t = x[i].beta;
             if (t + kAhead < t1) x[i] = load(t + kAhead);
             __syncthreads();
             const float rq = rsqrtf(sred[b][0][0] + sred[b][0][1] + sred[b][0][2] + sred[b][0][3] + 1e-6f);
             const float rk = rsqrtf(sred[b][1][0] + sred[b][1][1] + sred[b][1][2] + sred[b][1][3] + 1e-6f);
             const float qk = (sred[b][2][0] + sred[b][2][1] + sred[b][2][2] + sred[b][2][3]) * rq * rk;
-            // S' = Diag(e^g) S, p = S'^T k (raw k), w = S'^T q (raw q), over this thread's rows
-            float2 pa = make_float2(0.f, 0.f), pb = pa, wa = pa, wb = pa;
-            const int base = r0 + part * 4;
-            const float4 *a4 = reinterpret_cast<const float4 *>(sa[b] + base);
-            const float4 *k4 = reinterpret_cast<const float4 *>(sk[b] + base);
-            const float4 *q4 = reinterpret_cast<const float4 *>(sq[b] + base);
+            // S' = Diag(e^g) S; this thread's rows' share of p = S'^T k and w = S'^T q (raw k, q)
+            float kr[kRows];
+            float4 p = make_float4(0.f, 0.f, 0.f, 0.f), w = p;
 #pragma unroll
-            for (int j4 = 0; j4 < kRows / 4; ++j4) {
-                const float4 a = a4[j4], kk = k4[j4], qq = q4[j4];
-                S[2 * j4] = __fmul2_rn(S[2 * j4], make_float2(a.x, a.y));
-                S[2 * j4 + 1] = __fmul2_rn(S[2 * j4 + 1], make_float2(a.z, a.w));
-                pa = __ffma2_rn(S[2 * j4], make_float2(kk.x, kk.y), pa);
-                pb = __ffma2_rn(S[2 * j4 + 1], make_float2(kk.z, kk.w), pb);
-                wa = __ffma2_rn(S[2 * j4], make_float2(qq.x, qq.y), wa);
-                wb = __ffma2_rn(S[2 * j4 + 1], make_float2(qq.z, qq.w), wb);
+            for (int j4 = 0; j4 < kRows; j4 += 4) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(sa[b] + r0 + j4);
+                const float4 k4 = *reinterpret_cast<const float4 *>(sk[b] + r0 + j4);
+                const float4 q4 = *reinterpret_cast<const float4 *>(sq[b] + r0 + j4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float4 &sj = S[j4 + u];
+                    sj.x *= av[u]; sj.y *= av[u]; sj.z *= av[u]; sj.w *= av[u];
+                    p.x = fmaf(sj.x, kv[u], p.x); p.y = fmaf(sj.y, kv[u], p.y);
+                    p.z = fmaf(sj.z, kv[u], p.z); p.w = fmaf(sj.w, kv[u], p.w);
+                    w.x = fmaf(sj.x, qv[u], w.x); w.y = fmaf(sj.y, qv[u], w.y);
+                    w.z = fmaf(sj.z, qv[u], w.z); w.w = fmaf(sj.w, qv[u], w.w);
+                    kr[j4 + u] = kv[u];
+                }
             }
-            float p = (pa.x + pb.x) + (pa.y + pb.y), w = (wa.x + wb.x) + (wa.y + wb.y);
+            // the 4 row groups of the warp (lanes 8 apart) meet by shuffles, the 4 warps in shared memory
 #pragma unroll
-            for (int o = 1; o < kSplit; o <<= 1) {
-                p += __shfl_xor_sync(0xffffffffu, p, o);
-                w += __shfl_xor_sync(0xffffffffu, w, o);
+            for (int o = 8; o < 32; o <<= 1) {
+                p.x += __shfl_xor_sync(0xffffffffu, p.x, o); p.y += __shfl_xor_sync(0xffffffffu, p.y, o);
+                p.z += __shfl_xor_sync(0xffffffffu, p.z, o); p.w += __shfl_xor_sync(0xffffffffu, p.w, o);
+                w.x += __shfl_xor_sync(0xffffffffu, w.x, o); w.y += __shfl_xor_sync(0xffffffffu, w.y, o);
+                w.z += __shfl_xor_sync(0xffffffffu, w.z, o); w.w += __shfl_xor_sync(0xffffffffu, w.w, o);
+            }
+            if (lane < kQuads) {
+                spw[b][warp][quad][0] = p;
+                spw[b][warp][quad][1] = w;
+            }
+            __syncthreads();
+            p = w = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int ww = 0; ww < 4; ++ww) {
+                const float4 pp = spw[b][ww][quad][0], qq = spw[b][ww][quad][1];
+                p.x += pp.x; p.y += pp.y; p.z += pp.z; p.w += pp.w;
+                w.x += qq.x; w.y += qq.y; w.z += qq.z; w.w += qq.w;
             }
             // e = beta (v - S'^T k^); S = S' + k^ e^T; o = scale S^T q^ = scale (S'^T q^ + (q^.k^) e)
-            const float e = b_t * (v_t - p * rk);
-            if (part == 0)
-                out[((size_t)t * H + h) * D + col] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(scale * (w * rq + qk * e)));
-            const float2 e2 = make_float2(e * rk, e * rk);
+            const float2 v01 = unpack_bf16(v_t.x), v23 = unpack_bf16(v_t.y);
+            const float4 e = make_float4(b_t * (v01.x - p.x * rk), b_t * (v01.y - p.y * rk),
+                                         b_t * (v23.x - p.z * rk), b_t * (v23.y - p.w * rk));
+            if (grp == 0) {
+                const uint2 o2 = make_uint2(pack_bf16(scale * (w.x * rq + qk * e.x), scale * (w.y * rq + qk * e.y)),
+                                            pack_bf16(scale * (w.z * rq + qk * e.z), scale * (w.w * rq + qk * e.w)));
+                *reinterpret_cast<uint2 *>(out + ((size_t)t * H + h) * D + col) = o2;
+            }
+            const float4 er = make_float4(e.x * rk, e.y * rk, e.z * rk, e.w * rk);
 #pragma unroll
-            for (int j4 = 0; j4 < kRows / 4; ++j4) {
-                const float4 kk = k4[j4];
-                S[2 * j4] = __ffma2_rn(make_float2(kk.x, kk.y), e2, S[2 * j4]);
-                S[2 * j4 + 1] = __ffma2_rn(make_float2(kk.z, kk.w), e2, S[2 * j4 + 1]);
+            for (int j = 0; j < kRows; ++j) {
+                S[j].x = fmaf(kr[j], er.x, S[j].x); S[j].y = fmaf(kr[j], er.y, S[j].y);
+                S[j].z = fmaf(kr[j], er.z, S[j].z); S[j].w = fmaf(kr[j], er.w, S[j].w);
             }
         }
     }
     if (ht) {
 #pragma unroll
-        for (int j = 0; j < kRows / 2; ++j) {
-            ht[soff + (size_t)(r0 + 2 * j) * D + col] = S[j].x;
-            ht[soff + (size_t)(r0 + 2 * j + 1) * D + col] = S[j].y;
-        }
+        for (int j = 0; j < kRows; ++j) *reinterpret_cast<float4 *>(ht + soff + (size_t)(r0 + j) * D + col) = S[j];
     }
 }
 
 }  // namespace recurrent
 
-#ifndef KDA_RECURRENT_SPLIT
-#define KDA_RECURRENT_SPLIT 4
-#endif
-#ifndef KDA_RECURRENT_AHEAD
-#define KDA_RECURRENT_AHEAD 2
-#endif
-
 cudaError_t launch_fwd_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                                  const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, const float *h0,
                                  float *ht, uint16_t *out, int *status, cudaStream_t stream) {
-    constexpr int kSplit = KDA_RECURRENT_SPLIT;
-    const dim3 grid((unsigned)(n_docs * H), kSplit);
-    recurrent::kda_recurrent_kernel<kSplit, KDA_RECURRENT_AHEAD><<<grid, recurrent::kThreads, 0, stream>>>(q, k, v, g, beta, cu, n_docs,
-                                                                                           T, H, h0, ht, out, status);
+    const dim3 grid((unsigned)(n_docs * H), recurrent::kSplit);
+    recurrent::kda_recurrent_kernel<<<grid, recurrent::kThreads, 0, stream>>>(q, k, v, g, beta, cu, n_docs, T, H, h0,
+                                                                             ht, out, status);
     return cudaGetLastError();
 }
 
