@@ -237,8 +237,10 @@ def run_reference(args, w, d):
 
 
 def headline_config(w, world: int) -> dict:
-    return dict(w.describe(), l2="inputs 1.6 GB per step > 126 MB L2; no flush",
-                parallelism=f"replicas x{world}" if world > 1 else "single GPU")
+    gb = w.T * w.H * BYTES_PER_TOKEN_HEAD / 1e9
+    l2 = (f"inputs and output {gb:.2f} GB per step > 126 MB L2; no flush" if gb * 1e3 > 126
+          else f"inputs and output {gb * 1e3:.1f} MB per step fit the 126 MB L2; not flushed (small case)")
+    return dict(w.describe(), l2=l2, parallelism=f"replicas x{world}" if world > 1 else "single GPU")
 
 
 def bench_backward(kda, steps: int, dev, stream, barrier, shape=None) -> dict:
