@@ -1,389 +1,713 @@
 // kda_bwd.cu -- recompute-from-inputs backward of the chunk-KDA forward.
 //
-// Given the forward's inputs and the upstream gradient dO, computes dq, dk (of the
-// raw, un-normalised q and k), dv, dg and dbeta; the pages' fused backward is a
-// recompute backward with these outputs (kda_fused page of
-// nemo_automodel.components.models.kimi_k3, the backward of fused_chunk_kda).
+// Given the forward's inputs and the upstream gradient dO, computes dq, dk (of the raw,
+// un-normalised q and k), dv, dg and dbeta; the pages' fused backward is a recompute backward
+// with these outputs (kda_fused page of nemo_automodel.components.models.kimi_k3, the backward
+// of fused_chunk_kda).
 //
-// First the pipelined forward kernel (kda_fwd_pipe.cu) runs over the same inputs and writes the
-// state entering every chunk into the workspace's checkpoint slots (its output o goes to dq, which is
-// overwritten here).  Then one CTA per (document, head) chain walks the chain's 64-token chunks in
-// reverse, carrying dS (the gradient of the state leaving the chunk):
+// Per 64-token chunk, with G the in-chunk inclusive cumsum of g, QG = q^ e^G, Kd = k^ e^{G_last - G},
+// D = e^{G_last}, T = (I + A_kk)^-1, W = T diag(beta) K^e^G, U~ = U - W S and dS the gradient of the
+// state leaving the chunk, the reverse mode is
 //
-//  reverse sweep   per chunk: recompute A_kk, T = (I + A_kk)^-1, W = T diag(beta) K^e^G,
-//                  U = T diag(beta) V, then
-//                  dU~ = A_qk^T dO + Kd dS,  dS_in = (Q^e^G)^T dO + Diag(e^{G_last}) dS - W^T dU~,
-//                  dQG = dO S^T, dA_qk = lower(dO U~^T), dKd = U~ dS^T, dW = -dU~ S^T,
-//                  dT = dW (beta KG)^T + dU~ (beta V)^T, dA_kk = strict_lower(-T^T dT T^T),
-//                  and the chain rule through beta, the pairwise decays, e^G, the in-chunk
-//                  cumsum (dg = reverse cumsum of dG) and the l2 norms.
+//   dU~ = A_qk^T dO + Kd dS                     dS_in = D dS + QG^T dO - W^T dU~
+//   dQG = dO S^T    dA_qk = lower(dO U~^T)      dKd = U~ dS^T     dW = -dU~ S^T
+//   dT = dW (beta KG)^T + dU~ (beta V)^T        dA_kk = strict_lower(-T^T dT T^T)
 //
-// G is the in-chunk inclusive cumsum of g.  Pairwise decays e^{G_r - G_i} (r >= i) are
-// split at 16-row blocks, e^{G_r - G_16R} s_RI e^{G_16I+15 - G_i} with
-// s_RI = e^{G_16R - G_16I+15}, so no factor leaves the fp32 range.  The chunk products run
-// on bf16 warp MMA with a hi/lo split of both operands (gemm), the pairwise-decay products on
-// tf32 warp MMA with a hi/lo split (three products per tile in both, about 2^-17 and 2^-21
-// relative error per product); the triangular inverse and all elementwise work are fp32.
-// Per-chain scratch lives in the caller's workspace; libkda allocates nothing.
+// and then the chain rule through beta, the pairwise decays e^{G_r - G_i}, the factors e^G, the
+// in-chunk cumsum (dg = reverse cumsum of dG) and the l2 norms.  Only dS crosses chunks, so the
+// work splits into four launches:
+//
+//   1. the pipelined forward kernel (kda_fwd_pipe.cu) in its checkpoint instance: the state
+//      entering every chunk, S^T in bf16;
+//   2. intra (one CTA per chunk and head, all chunks at once): norms, G, A_kk and A_qk, T and W,
+//      written as the bf16 tensor-core operands the sweep below reads (-W, A_qk, Kd, QG), plus
+//      T, A_hat and D;
+//   3. dstate (one CTA per document and head, chunks in reverse): the dS recurrence on tcgen05
+//      with dS^T in tensor memory (fp32), writing dS^T and dU~^T of every chunk;
+//   4. grad (one CTA per chunk and head, all chunks at once): every gradient, from the chunk's
+//      inputs, S, dS and dU~, with warp-level bf16 MMAs.
+//
+// Precision: every product takes bf16 operands with fp32 accumulation; T = (I + A_kk)^-1 and all
+// elementwise work are fp32.  The pairwise-decay sums of dg cancel between their row and column
+// sides; both sides multiply by the same bf16-rounded operands (k^ E1, q^ E1, k^ E2), so the
+// cancellation stays exact and the rounding does not reach dg amplified.
+//
+// Tiles: every bf16 tile, in shared memory and in the workspace alike, is stored in 128-byte
+// swizzled atoms: 64-column halves of rows x 128 bytes, the 16-byte chunk index XORed with
+// (row & 7).  That is the tensor core's SWIZZLE_128B layout (K-major with rows = M or N, or
+// MN-major with rows = K), and ldmatrix reads it without bank conflicts, so workspace tiles are
+// copied to shared memory as flat byte images.  The library allocates nothing.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_tc.cuh"
 
 namespace kda {
 namespace bwd {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
 constexpr int C = 64;     // chunk
 constexpr int D = 128;    // head dim (K = V)
-constexpr int CD = C * D, CC = C * C, DD = D * D;
+constexpr float kScale = 0.08838834764831845f;   // 1 / sqrt(128)
+constexpr long long kWaitLimit = 2000000000LL;
 
-// per-chain scratch, in floats
+// ---------------------------------------------------------------------------------------------
+// Workspace: three regions, each [n_slots * H] blocks; the slot of chunk j of document d is
+// cu[d] / 64 + d + j (unique, below T / 64 + n_docs, found without reading the lengths).
+// ---------------------------------------------------------------------------------------------
 struct Ws {
-    static constexpr size_t DS = 0, DSN = DS + DD;
-    static constexpr size_t QN = DSN + DD, KN = QN + CD, VV = KN + CD, DO = VV + CD, G = DO + CD, EG = G + CD,
-                            KG = EG + CD, QG = KG + CD, KD = QG + CD, BK = KD + CD, BV = BK + CD, W = BV + CD,
-                            U = W + CD, UT = U + CD, DUT = UT + CD, DQG = DUT + CD, DKD = DQG + CD, DW = DKD + CD,
-                            DBK = DW + CD, DBV = DBK + CD, DKN = DBV + CD, DQN = DKN + CD, DG = DQN + CD,
-                            X1 = DG + CD, Y1 = X1 + CD, Q1 = Y1 + CD, E1 = Q1 + CD, E2 = E1 + CD,
-                            A24 = E2 + CD;
-    static constexpr size_t TM = A24 + CD, AH = TM + CC, AQ = AH + CC, DT = AQ + CC, XM = DT + CC, DAH = XM + CC,
-                            DAQ = DAH + CC;
-    static constexpr size_t SP = DAQ + CC;    // pair scales [10][128]
-    static constexpr size_t RQ = SP + 10 * D, RK = RQ + C, BB = RK + C, DB = BB + C, DL = DB + C, DGL = DL + D;
-    static constexpr size_t TOTAL = DGL + D;
+    static constexpr size_t CK = 32768;   // forward checkpoint: S^T bf16 [128 v][128 c]
+    // intra outputs
+    static constexpr size_t AQ = 0;                   // scale * A_qk bf16 [64 t][64 s]
+    static constexpr size_t KD = AQ + 8192;           // Kd bf16 [64 s][128 c]
+    static constexpr size_t QG = KD + 16384;          // scale * QG bf16 [64 t][128 c]
+    static constexpr size_t WN = QG + 16384;          // -W bf16 [64 s][128 c]
+    static constexpr size_t TB = WN + 16384;          // T bf16 [64 r][64 i]
+    static constexpr size_t AH = TB + 8192;           // A_hat bf16 [64 r][64 i] (strictly lower, no beta)
+    static constexpr size_t DL = AH + 8192;           // D = e^{G_last} fp32 [128]
+    static constexpr size_t INTRA = DL + 1024;
+    // dstate outputs
+    static constexpr size_t DS = 0;                   // dS^T bf16 [128 v][128 c] (dS leaving the chunk)
+    static constexpr size_t DU = DS + 32768;          // dU~^T bf16 [128 v][64 s]
+    static constexpr size_t DST = DU + 16384;
+    static constexpr size_t PER_SLOT = CK + INTRA + DST;
 };
 
-__device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
-
-// tf32 split x = hi + lo: hi keeps the top 19 bits of x (exactly representable in tf32), lo = x - hi
-// is exact in fp32; the tensor core reads lo's top 19 bits.  hi*hi + hi*lo + lo*hi then carries
-// about 2^-21 relative error per product.
-__device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
-__device__ __forceinline__ uint32_t tf32_lo(float x, uint32_t hi) { return __float_as_uint(x - __uint_as_float(hi)); }
-
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// byte offset of bf16 element (row, col) in a tile of `rows` rows (128-byte swizzled atoms)
+__device__ __forceinline__ uint32_t at(int row, int col, int rows) {
+    return (uint32_t)((col >> 6) * rows * 128 + row * 128 + ((((col >> 3) & 7) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
 
-// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for two values packed as bf16x2 (the lower
-// k index in the low half); hi*hi + hi*lo + lo*hi then carries about 2^-17 relative error per
-// product, with twice the k-depth of a tf32 instruction per bf16 one
-__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-    const float2 hf = __bfloat1622float2(h);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-    hi = *reinterpret_cast<const uint32_t *>(&h);
-    lo = *reinterpret_cast<const uint32_t *>(&l);
-}
-
-// acc(16x8) += op(A)(16 x 8k) op(B)(8k x 8) with tf32 hi/lo splits; a[e], b[e] fp32
-__device__ __forceinline__ void mma3(float (&acc)[4], const float (&av)[4], float bv0, float bv1) {
-    uint32_t ah[4], al[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        ah[e] = tf32_hi(av[e]);
-        al[e] = tf32_lo(av[e], ah[e]);
-    }
-    const uint32_t bh0 = tf32_hi(bv0), bh1 = tf32_hi(bv1);
-    const uint32_t bl0 = tf32_lo(bv0, bh0), bl1 = tf32_lo(bv1, bh1);
-    mma_tf32(acc, al, bh0, bh1);
-    mma_tf32(acc, ah, bl0, bl1);
-    mma_tf32(acc, ah, bh0, bh1);
-}
-
-// shared-memory operand buffers of gemm: two matrices of up to 128 rows, rows padded by 8 floats
-// (with that pitch the fragment reads of both layouts hit 32 distinct banks)
-constexpr int kPad = 8;
-constexpr int kOpFloats = 128 * (128 + kPad);
-
-// copy a contiguous [ROWS][COLS] fp32 matrix to shared memory with row pitch PITCH (no barrier):
-// every load of the thread is issued before its first store, so they are in flight together
-template <int ROWS, int COLS, int PITCH>
-__device__ __forceinline__ void stage(float *dst, const float *src) {
-    constexpr int n4 = ROWS * COLS / 4, it = (n4 + kThreads - 1) / kThreads;
-    float4 r[it];
-#pragma unroll
-    for (int i = 0; i < it; ++i) {
-        const int idx = threadIdx.x + i * kThreads;
-        if (n4 % kThreads == 0 || idx < n4) r[i] = reinterpret_cast<const float4 *>(src)[idx];
-    }
-#pragma unroll
-    for (int i = 0; i < it; ++i) {
-        const int idx = threadIdx.x + i * kThreads;
-        if (n4 % kThreads == 0 || idx < n4) {
-            const int row = (idx * 4) / COLS, c = (idx * 4) % COLS;
-            *reinterpret_cast<float4 *>(dst + row * PITCH + c) = r[i];
-        }
+// ---- warp-level bf16 MMA (m16n8k16) fragments from atom tiles --------------------------------
+// A fragment (16 x 16 at m0, k0) of a tile stored [m][k] (rows = m) or, kT, [k][m] (rows = k)
+template <bool kT>
+__device__ __forceinline__ void frag_a(uint32_t base, int rows, int m0, int k0, uint32_t (&a)[4]) {
+    const int lane = threadIdx.x & 31, j = lane >> 3, r = lane & 7;
+    if constexpr (!kT) {
+        ldsm_x4(base + at(m0 + (j & 1) * 8 + r, k0 + (j >> 1) * 8, rows), a[0], a[1], a[2], a[3]);
+    } else {
+        ldsm_x4_t(base + at(k0 + (j >> 1) * 8 + r, m0 + (j & 1) * 8, rows), a[0], a[1], a[2], a[3]);
     }
 }
-
-// C(M x N) = alpha * op(A) op(B) + (accumulate ? C : 0), CTA-wide.  A is stored row-major as
-// [M][K] (or [K][M] when transA), B as [K][N] (or [N][K] when transB), both contiguous; C(i, j)
-// = Cm[i*ldc + j].  M % 16 == N % 8 == 0.  Both operands are first copied to shared
-// memory (float4, padded rows); each warp then owns a strip of 16x8 output tiles of one 16-row
-// block, splitting both operands into bf16 hi + lo parts (split_bf16) and accumulating
-// hi*hi + hi*lo + lo*hi with m16n8k16 warp MMAs.  K % 16 == 0.  Ends with a CTA barrier.
-template <int M, int N, int K, bool transA, bool transB>
-__device__ void gemm(float alpha, const float *A, const float *B, bool accumulate, float *Cm, int ldc, float *sa,
-                     float *sb) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    constexpr int acols = transA ? M : K, arows = transA ? K : M;
-    constexpr int bcols = transB ? K : N, brows = transB ? N : K;
-    // row pads: an operand read along its rows (k pairs contiguous) is read as float2 and padded by 8
-    // floats; one read across its rows is padded by 4; both patterns are then free of bank conflicts
-    constexpr int ald = acols + (transA ? 4 : kPad), bld = bcols + (transB ? kPad : 4);
-    stage<arows, acols, ald>(sa, A);
-    stage<brows, bcols, bld>(sb, B);
-    __syncthreads();
-    // each warp owns a 16-row strip of kTpw consecutive 16x8 tiles, taken kSub at a time, so that
-    // one split A fragment serves kSub tiles
-    constexpr int nt = N / 8, tiles = (M / 16) * nt, kTpw = tiles / kWarps, kSub = kTpw < 4 ? kTpw : 4;
-    static_assert(tiles % kWarps == 0 && nt % kTpw == 0 && kTpw % kSub == 0, "tile split");
-    static_assert(K % 16 == 0, "k-steps of 16");
-    const int t0 = warp * kTpw, i0 = (t0 / nt) * 16;
-#pragma unroll 1
-    for (int sub = 0; sub < kTpw; sub += kSub) {
-        const int jb = (t0 % nt + sub) * 8;
-        float *c0 = Cm + (i0 + gq) * ldc + jb + 2 * tq, *c1 = c0 + 8 * ldc;
-        // the values accumulated onto are fetched before the products, so their latency overlaps them
-        float2 p0[kSub], p1[kSub];
-#pragma unroll
-        for (int j = 0; j < kSub; ++j) {
-            p0[j] = accumulate ? *reinterpret_cast<const float2 *>(c0 + 8 * j) : make_float2(0.f, 0.f);
-            p1[j] = accumulate ? *reinterpret_cast<const float2 *>(c1 + 8 * j) : make_float2(0.f, 0.f);
-        }
-        float acc[kSub][4];
-#pragma unroll
-        for (int j = 0; j < kSub; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+// B fragments of two n-tiles (k0..k0+15, n0..n0+15) of a tile stored [n][k] (rows = n) or, kT, [k][n]
+// (rows = k): b[0], b[1] for columns n0..n0+7, b[2], b[3] for n0+8..n0+15
+template <bool kT>
+__device__ __forceinline__ void frag_b2(uint32_t base, int rows, int k0, int n0, uint32_t (&b)[4]) {
+    const int lane = threadIdx.x & 31, j = lane >> 3, r = lane & 7;
+    if constexpr (!kT) {
+        ldsm_x4(base + at(n0 + (j >> 1) * 8 + r, k0 + (j & 1) * 8, rows), b[0], b[1], b[2], b[3]);
+    } else {
+        ldsm_x4_t(base + at(k0 + (j & 1) * 8 + r, n0 + (j >> 1) * 8, rows), b[0], b[1], b[2], b[3]);
+    }
+}
+// acc[NT][4] += A(16 rows from m0, k in [k0, k1)) * B(k, NT * 8 columns from n0); NT even
+template <int NT, bool kAT, bool kBT>
+__device__ __forceinline__ void mma_rows(float (&acc)[NT][4], uint32_t a_base, int a_rows, int m0, uint32_t b_base,
+                                         int b_rows, int n0, int k0, int k1) {
 #pragma unroll 2
-        for (int k0 = 0; k0 < K; k0 += 16) {
-            // A fragment of m16n8k16: rows gq, gq+8; k pairs (2tq, 2tq+1) and (2tq+8, 2tq+9)
-            const int ka = k0 + 2 * tq;
-            uint32_t ah[4], al[4];
-            if constexpr (!transA) {
-                const float2 x0 = *reinterpret_cast<const float2 *>(sa + (i0 + gq) * ald + ka);
-                const float2 x1 = *reinterpret_cast<const float2 *>(sa + (i0 + gq + 8) * ald + ka);
-                const float2 x2 = *reinterpret_cast<const float2 *>(sa + (i0 + gq) * ald + ka + 8);
-                const float2 x3 = *reinterpret_cast<const float2 *>(sa + (i0 + gq + 8) * ald + ka + 8);
-                split_bf16(x0.x, x0.y, ah[0], al[0]);
-                split_bf16(x1.x, x1.y, ah[1], al[1]);
-                split_bf16(x2.x, x2.y, ah[2], al[2]);
-                split_bf16(x3.x, x3.y, ah[3], al[3]);
-            } else {
-                split_bf16(sa[ka * ald + i0 + gq], sa[(ka + 1) * ald + i0 + gq], ah[0], al[0]);
-                split_bf16(sa[ka * ald + i0 + gq + 8], sa[(ka + 1) * ald + i0 + gq + 8], ah[1], al[1]);
-                split_bf16(sa[(ka + 8) * ald + i0 + gq], sa[(ka + 9) * ald + i0 + gq], ah[2], al[2]);
-                split_bf16(sa[(ka + 8) * ald + i0 + gq + 8], sa[(ka + 9) * ald + i0 + gq + 8], ah[3], al[3]);
-            }
+    for (int k = k0; k < k1; k += 16) {
+        uint32_t a[4];
+        frag_a<kAT>(a_base, a_rows, m0, k, a);
 #pragma unroll
-            for (int j = 0; j < kSub; ++j) {
-                const int col = jb + 8 * j + gq;
-                uint32_t bh0, bl0, bh1, bl1;
-                if constexpr (transB) {
-                    const float2 y0 = *reinterpret_cast<const float2 *>(sb + col * bld + ka);
-                    const float2 y1 = *reinterpret_cast<const float2 *>(sb + col * bld + ka + 8);
-                    split_bf16(y0.x, y0.y, bh0, bl0);
-                    split_bf16(y1.x, y1.y, bh1, bl1);
-                } else {
-                    split_bf16(sb[ka * bld + col], sb[(ka + 1) * bld + col], bh0, bl0);
-                    split_bf16(sb[(ka + 8) * bld + col], sb[(ka + 9) * bld + col], bh1, bl1);
-                }
-                mma_bf16(acc[j], al, bh0, bh1);
-                mma_bf16(acc[j], ah, bl0, bl1);
-                mma_bf16(acc[j], ah, bh0, bh1);
-            }
+        for (int t = 0; t < NT; t += 2) {
+            uint32_t b[4];
+            frag_b2<kBT>(b_base, b_rows, k, n0 + 8 * t, b);
+            mma_bf16(acc[t], a, b[0], b[1]);
+            mma_bf16(acc[t + 1], a, b[2], b[3]);
+        }
+    }
+}
+template <int NT>
+__device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+}
+
+__device__ __forceinline__ float bfl(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f2b(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ float2 bf2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// chunk slot -> (document, first token, length); false when the slot holds no chunk or the
+// document's bounds are invalid (the forward pass records KDA_ERR_BAD_SEQLENS for those)
+__device__ __forceinline__ bool slot_chunk(const int32_t *cu, int n_docs, int64_t T, int slot, int &doc,
+                                           int64_t &tok0, int &L) {
+    int lo = 0, hi = n_docs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const int base = (int)((unsigned)cu[mid] / C) + mid;
+        if (cu[mid] >= 0 && base <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    const int64_t d0 = cu[lo], d1 = cu[lo + 1];
+    if (d0 < 0 || d1 < d0 || d1 > T) return false;
+    const int64_t j = (int64_t)slot - (d0 / C + lo);
+    if (j < 0) return false;
+    tok0 = d0 + j * C;
+    if (tok0 >= d1) return false;
+    doc = lo;
+    L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
+    return true;
+}
+
+// pair index p of block pair (R, I), I <= R, and back
+__device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
+__device__ __forceinline__ int pair_R(int p) { return p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0; }
+
+// l2 norms of rows [0, 64) of q and k (rows >= L zero): rq[r] = 1/sqrt(|q_r|^2 + 1e-6), rk likewise;
+// one warp per row, nwarps warps
+__device__ __forceinline__ void row_norms(const uint16_t *q, const uint16_t *k, int64_t tok0, int L, int H, int h,
+                                          float *rq, float *rk, int nwarps) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < C; r += nwarps) {
+        float sq = 0.f, sk = 0.f;
+        if (r < L) {
+            const int64_t off = ((tok0 + r) * H + h) * D + 4 * lane;
+            const uint2 q4 = *reinterpret_cast<const uint2 *>(q + off), k4 = *reinterpret_cast<const uint2 *>(k + off);
+            const float2 a = bf2(q4.x), b = bf2(q4.y), c = bf2(k4.x), d = bf2(k4.y);
+            sq = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+            sk = c.x * c.x + c.y * c.y + d.x * d.x + d.y * d.y;
         }
 #pragma unroll
-        for (int j = 0; j < kSub; ++j) {
-            *reinterpret_cast<float2 *>(c0 + 8 * j) =
-                make_float2(fmaf(alpha, acc[j][0], p0[j].x), fmaf(alpha, acc[j][1], p0[j].y));
-            *reinterpret_cast<float2 *>(c1 + 8 * j) =
-                make_float2(fmaf(alpha, acc[j][2], p1[j].x), fmaf(alpha, acc[j][3], p1[j].y));
+        for (int o = 16; o; o >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        }
+        if (lane == 0) {
+            rq[r] = rsqrtf(sq + 1e-6f);
+            rk[r] = rsqrtf(sk + 1e-6f);
+        }
+    }
+}
+
+// flat copy of `bytes` (a multiple of 16) between 16-byte aligned buffers, all threads of the CTA
+__device__ __forceinline__ void copy_out(uint8_t *dst, const uint8_t *src, int bytes, int nthreads) {
+    for (int i = threadIdx.x; i < bytes / 16; i += nthreads)
+        reinterpret_cast<uint4 *>(dst)[i] = reinterpret_cast<const uint4 *>(src)[i];
+}
+
+// =============================================================================================
+// 2. intra: one CTA per (chunk slot, head)
+// =============================================================================================
+namespace intra {
+constexpr int kThreads = 256;
+struct Sm {
+    static constexpr int X = 0;          // k^ E1 bf16 [64][128]; then beta k^ e^G (Bk)
+    static constexpr int Q = 16384;      // q^ E1; then T bf16 [64][64] (+0) and solve scratch (+8192)
+    static constexpr int Y = 32768;      // k^ E2; then -W bf16 [64][128]
+    static constexpr int AF = 49152;     // A_kk fp32 [64][64]
+    static constexpr int TF = 65536;     // T fp32 [64][64]
+    static constexpr int AQO = 81920;    // scale * A_qk bf16 [64][64]
+    static constexpr int AHO = 90112;    // A_hat bf16 [64][64]
+    static constexpr int PS = 98304;     // pair scales fp32 [10][128]
+    static constexpr int GB = PS + 5120; // G (log2 units) at block rows 16R and 16R+15, fp32 [4][2][128]
+    static constexpr int RQ = GB + 4096, RK = RQ + 256, BETA = RK + 256;
+    static constexpr int TOTAL = BETA + 256;
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const float *beta, const int32_t *cu,
+                     int n_docs, int64_t T, int H, uint8_t *ws_intra) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const int slot = blockIdx.x / H, h = blockIdx.x % H;
+    int doc, L;
+    int64_t tok0;
+    if (!slot_chunk(cu, n_docs, T, slot, doc, tok0, L)) return;
+    uint8_t *out = ws_intra + ((size_t)slot * H + h) * Ws::INTRA;
+    const uint32_t sbase = smem_u32(sm);
+    float *rq = reinterpret_cast<float *>(sm + Sm::RQ), *rk = reinterpret_cast<float *>(sm + Sm::RK);
+    float *sbeta = reinterpret_cast<float *>(sm + Sm::BETA), *gb = reinterpret_cast<float *>(sm + Sm::GB);
+    float *ps = reinterpret_cast<float *>(sm + Sm::PS);
+    float *af = reinterpret_cast<float *>(sm + Sm::AF), *tf = reinterpret_cast<float *>(sm + Sm::TF);
+
+    if (tid < C) sbeta[tid] = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
+    row_norms(q, k, tok0, L, H, h, rq, rk, kThreads / 32);
+
+    // ---- G (log2 units) per channel: thread (c, half) keeps its 32 rows in registers ----
+    const int c = tid & (D - 1), hf = tid >> 7;
+    float g2[32];
+    {
+        float run = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int r = 32 * hf + i;
+            run += (r < L ? g[((tok0 + r) * H + h) * D + c] : 0.f) * kLog2e;
+            g2[i] = run;
+        }
+        // the second half adds the first half's total (passed through the pair-scale buffer)
+        if (hf == 0) ps[c] = run;
+        __syncthreads();
+        const float off = hf ? ps[c] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) g2[i] += off;
+        gb[(2 * hf) * 256 + c] = g2[0];
+        gb[(2 * hf) * 256 + 128 + c] = g2[15];
+        gb[(2 * hf + 1) * 256 + c] = g2[16];
+        gb[(2 * hf + 1) * 256 + 128 + c] = g2[31];
+        __syncthreads();
+    }
+    const float gl = gb[3 * 256 + 128 + c];   // G at row 63 (= row L - 1: rows past L add zero)
+    // pair scales s_RI = e^{G_16R - G_16I+15}
+    for (int p = 5 * hf; p < 5 * hf + 5; ++p) {
+        const int R = pair_R(p), I = p - R * (R + 1) / 2;
+        ps[p * D + c] = ex2_ftz(gb[R * 256 + c] - gb[I * 256 + 128 + c]);
+    }
+    if (hf == 1) reinterpret_cast<float *>(out + Ws::DL)[c] = ex2_ftz(gl);
+    // operand tiles, one (row, channel) element per step
+    {
+        uint8_t *okd = out + Ws::KD, *oqg = out + Ws::QG;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int r = 32 * hf + i, R = r >> 4;
+            float qv = 0.f, kv = 0.f;
+            if (r < L) {
+                const int64_t off = ((tok0 + r) * H + h) * D + c;
+                qv = bfl(q[off]) * rq[r];
+                kv = bfl(k[off]) * rk[r];
+            }
+            const float e1 = ex2_ftz(g2[i] - gb[R * 256 + c]), e2 = ex2_ftz(gb[R * 256 + 128 + c] - g2[i]);
+            const uint32_t o = at(r, c, C);
+            *reinterpret_cast<uint16_t *>(sm + Sm::X + o) = f2b(kv * e1);
+            *reinterpret_cast<uint16_t *>(sm + Sm::Q + o) = f2b(qv * e1);
+            *reinterpret_cast<uint16_t *>(sm + Sm::Y + o) = f2b(kv * e2);
+            *reinterpret_cast<uint16_t *>(okd + o) = f2b(kv * ex2_ftz(gl - g2[i]));
+            *reinterpret_cast<uint16_t *>(oqg + o) = f2b(kScale * qv * ex2_ftz(g2[i]));
         }
     }
     __syncthreads();
-}
 
-// A_hat (strictly lower) and, if full, A_qk (lower incl.), block pair by block pair:
-// block (R, I) = (X_R diag(s_RI)) Y_I^T with X = k^ e^{G-G_16R} (or q^ ...), Y = k^ e^{G_16I+15-G}.
-__device__ void pair_products(float *w, bool full, float *sm) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    constexpr int P = D + 4;                    // pitch: row-wise fragment reads hit 32 banks
-    float *sx = sm, *sq = sm + C * P, *sy = sm + 2 * C * P, *ss = sm + 3 * C * P;
-    stage<C, D, P>(sx, w + Ws::X1);
-    if (full) stage<C, D, P>(sq, w + Ws::Q1);
-    stage<C, D, P>(sy, w + Ws::Y1);
-    stage<10, D, D>(ss, w + Ws::SP);
-    __syncthreads();
-    const int items = full ? 40 : 20;          // (pair, 8-column half, which)
-    for (int t = warp; t < items; t += kWarps) {
-        const int which = t / 20, p = (t % 20) >> 1, nh = t & 1;
-        const int R = p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0, I = p - R * (R + 1) / 2;
-        const float *X = (which ? sq : sx) + (16 * R) * P, *Y = sy + (16 * I + 8 * nh) * P;
-        const float *sp = ss + p * D;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int k0 = 0; k0 < D; k0 += 8) {
-            const float s0 = sp[k0 + tq], s1 = sp[k0 + tq + 4];
-            const float av[4] = {X[gq * P + k0 + tq] * s0, X[(gq + 8) * P + k0 + tq] * s0,
-                                 X[gq * P + k0 + tq + 4] * s1, X[(gq + 8) * P + k0 + tq + 4] * s1};
-            mma3(acc, av, Y[gq * P + k0 + tq], Y[gq * P + k0 + tq + 4]);
-        }
-        float *out = w + (which ? Ws::AQ : Ws::AH);
+    // ---- A_hat (strictly lower) and A_qk (lower), block pair by block pair (warp MMA) ----
+    // block (R, I) = (X_R diag(s_RI)) Y_I^T; the pair scale rides on the A fragment
+    for (int p = warp; p < 10; p += kThreads / 32) {
+        const int R = pair_R(p), I = p - R * (R + 1) / 2;
+        float ak[2][4], aq[2][4];
+        zero_acc(ak);
+        zero_acc(aq);
+#pragma unroll 2
+        for (int kk = 0; kk < D; kk += 16) {
+            uint32_t fx[4], fq[4], b[4];
+            frag_a<false>(sbase + Sm::X, C, 16 * R, kk, fx);
+            frag_a<false>(sbase + Sm::Q, C, 16 * R, kk, fq);
+            frag_b2<false>(sbase + Sm::Y, C, kk, 16 * I, b);
+            const float2 s0 = *reinterpret_cast<const float2 *>(ps + p * D + kk + 2 * tq);
+            const float2 s1 = *reinterpret_cast<const float2 *>(ps + p * D + kk + 8 + 2 * tq);
+            const __nv_bfloat162 h0 = __floats2bfloat162_rn(s0.x, s0.y), h1 = __floats2bfloat162_rn(s1.x, s1.y);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int row = 16 * R + gq + 8 * (e >> 1), col = 16 * I + 8 * nh + 2 * tq + (e & 1);
-            out[row * C + col] = (which ? col <= row : col < row) ? acc[e] : 0.f;
+            for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 sc = (e >> 1) ? h1 : h0;
+                __nv_bfloat162 x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fx[e]), sc);
+                fx[e] = *reinterpret_cast<uint32_t *>(&x);
+                x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fq[e]), sc);
+                fq[e] = *reinterpret_cast<uint32_t *>(&x);
+            }
+            mma_bf16(ak[0], fx, b[0], b[1]);
+            mma_bf16(ak[1], fx, b[2], b[3]);
+            mma_bf16(aq[0], fq, b[0], b[1]);
+            mma_bf16(aq[1], fq, b[2], b[3]);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = 16 * R + gq + 8 * hh, col = 16 * I + 8 * nt + 2 * tq;
+                const float x0 = col < row ? ak[nt][2 * hh] : 0.f, x1 = col + 1 < row ? ak[nt][2 * hh + 1] : 0.f;
+                const float y0 = col <= row ? kScale * aq[nt][2 * hh] : 0.f;
+                const float y1 = col + 1 <= row ? kScale * aq[nt][2 * hh + 1] : 0.f;
+                const float br = sbeta[row];
+                *reinterpret_cast<float2 *>(af + row * C + col) = make_float2(br * x0, br * x1);
+                *reinterpret_cast<uint32_t *>(sm + Sm::AHO + at(row, col, C)) = pack_bf16(x0, x1);
+                *reinterpret_cast<uint32_t *>(sm + Sm::AQO + at(row, col, C)) = pack_bf16(y0, y1);
+            }
     }
     // blocks above the diagonal are zero
-    for (int idx = threadIdx.x; idx < 6 * 256; idx += kThreads) {
+    for (int idx = tid; idx < 6 * 256; idx += kThreads) {
         const int b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
         const int R = b < 3 ? 0 : b < 5 ? 1 : 2, I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-        w[Ws::AH + (16 * R + rr) * C + 16 * I + cc] = 0.f;
-        if (full) w[Ws::AQ + (16 * R + rr) * C + 16 * I + cc] = 0.f;
-    }
-    __syncthreads();   // also frees the staging buffers
-}
-
-// Pairwise-decay sums of the reverse sweep, block pair by block pair (dA = dA_hat*beta, dA_qk):
-//   row side    (r in block R):  a1 = E1 sum_{I<=R} s_RI (dA_RI Y_I),   a3 = same with dA_qk
-//   column side (i in block I):  a24 = E2 sum_{R>=I} s_RI (dA_RI^T X_R + dA_qk,RI^T Q_R)
-// a1 -> DKN, a3 -> DQN, a24 -> A24.
-__device__ void pair_grads(float *w, float *sm) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    constexpr int PA = C + 4, PB = D + 8;       // pitches for the fragment read patterns below
-    float *dah = sm, *daq = sm + C * PA, *sx = sm + 2 * C * PA, *sy = sx + C * PB, *sq = sy + C * PB;
-    stage<C, C, PA>(dah, w + Ws::DAH);
-    stage<C, C, PA>(daq, w + Ws::DAQ);
-    stage<C, D, PB>(sx, w + Ws::X1);
-    stage<C, D, PB>(sy, w + Ws::Y1);
-    stage<C, D, PB>(sq, w + Ws::Q1);
-    __syncthreads();
-    for (int t = warp; t < 128; t += kWarps) {
-        const bool col_side = t >= 64;
-        const int B = (t & 63) >> 4, c0 = (t & 15) * 8;      // block (R or I) and 8-channel tile
-        float acc1[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-        const int lo = col_side ? B : 0, hi = col_side ? 3 : B;
-        for (int o = lo; o <= hi; ++o) {
-            const int R = col_side ? o : B, I = col_side ? B : o, p = pair_of(R, I);
-            float t1[4] = {0.f, 0.f, 0.f, 0.f}, t2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < 16; k0 += 8) {
-                if (!col_side) {
-                    // A(row, k) = dA[16R + row][16I + k], B(k, j) = Y[16I + k][c0 + j]
-                    const float *a1p = dah + (16 * R) * PA + 16 * I, *a3p = daq + (16 * R) * PA + 16 * I;
-                    const float *Y = sy + (16 * I) * PB + c0;
-                    const float b0 = Y[(k0 + tq) * PB + gq], b1 = Y[(k0 + tq + 4) * PB + gq];
-                    const float av1[4] = {a1p[gq * PA + k0 + tq], a1p[(gq + 8) * PA + k0 + tq], a1p[gq * PA + k0 + tq + 4],
-                                          a1p[(gq + 8) * PA + k0 + tq + 4]};
-                    const float av3[4] = {a3p[gq * PA + k0 + tq], a3p[(gq + 8) * PA + k0 + tq], a3p[gq * PA + k0 + tq + 4],
-                                          a3p[(gq + 8) * PA + k0 + tq + 4]};
-                    mma3(t1, av1, b0, b1);
-                    mma3(t2, av3, b0, b1);
-                } else {
-                    // A(row, k) = dA[16R + k][16I + row], B(k, j) = X[16R + k][c0 + j]
-                    const float *a1p = dah + (16 * R) * PA + 16 * I, *a3p = daq + (16 * R) * PA + 16 * I;
-                    const float *X = sx + (16 * R) * PB + c0, *Q = sq + (16 * R) * PB + c0;
-                    const float av1[4] = {a1p[(k0 + tq) * PA + gq], a1p[(k0 + tq) * PA + gq + 8], a1p[(k0 + tq + 4) * PA + gq],
-                                          a1p[(k0 + tq + 4) * PA + gq + 8]};
-                    const float av3[4] = {a3p[(k0 + tq) * PA + gq], a3p[(k0 + tq) * PA + gq + 8], a3p[(k0 + tq + 4) * PA + gq],
-                                          a3p[(k0 + tq + 4) * PA + gq + 8]};
-                    mma3(t1, av1, X[(k0 + tq) * PB + gq], X[(k0 + tq + 4) * PB + gq]);
-                    mma3(t2, av3, Q[(k0 + tq) * PB + gq], Q[(k0 + tq + 4) * PB + gq]);
-                }
-            }
-            const float s0 = w[Ws::SP + p * D + c0 + 2 * tq], s1 = w[Ws::SP + p * D + c0 + 2 * tq + 1];
-            acc1[0] += s0 * t1[0]; acc1[1] += s1 * t1[1]; acc1[2] += s0 * t1[2]; acc1[3] += s1 * t1[3];
-            acc2[0] += s0 * t2[0]; acc2[1] += s1 * t2[1]; acc2[2] += s0 * t2[2]; acc2[3] += s1 * t2[3];
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int row = 16 * B + gq + 8 * (e >> 1), c = c0 + 2 * tq + (e & 1);
-            const int idx = row * D + c;
-            if (!col_side) {
-                const float e1 = w[Ws::E1 + idx];
-                w[Ws::DKN + idx] = e1 * acc1[e];
-                w[Ws::DQN + idx] = e1 * acc2[e];
-            } else {
-                w[Ws::A24 + idx] = w[Ws::E2 + idx] * (acc1[e] + acc2[e]);
-            }
-        }
+        const int row = 16 * R + rr, col = 16 * I + cc;
+        af[row * C + col] = 0.f;
+        *reinterpret_cast<uint16_t *>(sm + Sm::AHO + at(row, col, C)) = 0;
+        *reinterpret_cast<uint16_t *>(sm + Sm::AQO + at(row, col, C)) = 0;
     }
     __syncthreads();
-}
+    copy_out(out + Ws::AQ, sm + Sm::AQO, 8192, kThreads);
+    copy_out(out + Ws::AH, sm + Sm::AHO, 8192, kThreads);
 
-// T = (I + B)^-1 with B = diag(beta) A_hat strictly lower (T unit lower), by 16 x 16 blocks:
-//   diagonal blocks  T_RR = (I + B_RR)^-1, lane = column, row-by-row substitution (warps 0-3);
-//   off-diagonal     T_RI = -T_RR sum_{J=I..R-1} B_RJ T_JI, by block distance R - I = 1, 2, 3,
-//                    each level as X = sum B T into `sx`, then -T_RR X (one element per thread).
-// fp32 throughout; seven CTA barriers.  `sx` is 3 * 256 floats of free shared memory.
-__device__ void tri_inverse(float *w, float *sA, float *sT, float *sx) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr int P = C + 1;
-    for (int idx = tid; idx < CC; idx += kThreads) {
-        const int r = idx / C, i = idx % C;
-        sA[r * P + i] = w[Ws::BB + r] * w[Ws::AH + idx];
-        sT[r * P + i] = 0.f;
+    // ---- Bk = beta k^ e^G over the k^ E1 tile (free now) ----
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        const float kv = r < L ? bfl(k[((tok0 + r) * H + h) * D + c]) * rk[r] : 0.f;
+        *reinterpret_cast<uint16_t *>(sm + Sm::X + at(r, c, C)) = f2b(sbeta[r] * kv * ex2_ftz(g2[i]));
     }
+
+    // ---- T = (I + A_kk)^-1 by 16 x 16 blocks (fp32) ----
+    //   diagonal blocks T_RR = (I + A_RR)^-1, lane = column, row-by-row substitution (warps 0-3);
+    //   off-diagonal T_RI = -T_RR sum_{J=I..R-1} A_RJ T_JI by block distance 1, 2, 3
+    float *sx = reinterpret_cast<float *>(sm + Sm::Q + 8192);
+    for (int idx = tid; idx < C * C; idx += kThreads) tf[idx] = 0.f;
     __syncthreads();
     if (warp < 4 && lane < 16) {
-        const int R = warp, c = lane;
-        const float *b = sA + (16 * R) * P + 16 * R;
+        const int R = warp, cc = lane;
+        const float *b = af + (16 * R) * C + 16 * R;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc = (r == c) ? 1.f : 0.f;
+            float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < r; ++i) acc = fmaf(-b[r * P + i], x[i], acc);
+            for (int i = 0; i < r; ++i) acc = fmaf(-b[r * C + i], x[i], acc);
             x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(16 * R + r) * P + 16 * R + c] = x[r];
+        for (int r = 0; r < 16; ++r) tf[(16 * R + r) * C + 16 * R + cc] = x[r];
     }
     __syncthreads();
 #pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        const int nblk = 4 - d;   // blocks (R, I) = (I + d, I), I = 0 .. 3 - d
+    for (int dd = 1; dd < 4; ++dd) {
+        const int nblk = 4 - dd;
         for (int e = tid; e < nblk * 256; e += kThreads) {
-            const int I = e >> 8, R = I + d, r = (e >> 4) & 15, c = e & 15;
+            const int I = e >> 8, R = I + dd, r = (e >> 4) & 15, cc = e & 15;
             float acc = 0.f;
             for (int J = I; J < R; ++J) {
-                const float *brow = sA + (16 * R + r) * P + 16 * J;
-                const float *tcol = sT + (16 * J) * P + 16 * I + c;
+                const float *arow = af + (16 * R + r) * C + 16 * J;
+                const float *tcol = tf + (16 * J) * C + 16 * I + cc;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc = fmaf(brow[i], tcol[i * P], acc);
+                for (int i = 0; i < 16; ++i) acc = fmaf(arow[i], tcol[i * C], acc);
             }
             sx[e] = acc;
         }
         __syncthreads();
         for (int e = tid; e < nblk * 256; e += kThreads) {
-            const int I = e >> 8, R = I + d, r = (e >> 4) & 15, c = e & 15;
-            const float *trow = sT + (16 * R + r) * P + 16 * R;
-            const float *xc = sx + (I << 8) + c;
+            const int I = e >> 8, R = I + dd, r = (e >> 4) & 15, cc = e & 15;
+            const float *trow = tf + (16 * R + r) * C + 16 * R;
+            const float *xc = sx + (I << 8) + cc;
             float acc = 0.f;
 #pragma unroll
             for (int m = 0; m < 16; ++m) acc = fmaf(trow[m], xc[m * 16], acc);
-            sT[(16 * R + r) * P + 16 * I + c] = -acc;
+            tf[(16 * R + r) * C + 16 * I + cc] = -acc;
         }
         __syncthreads();
     }
-    for (int idx = tid; idx < CC; idx += kThreads) w[Ws::TM + idx] = sT[(idx / C) * P + idx % C];
+    // T in bf16 (the operand of W here and of the gradient products)
+    for (int idx = tid; idx < C * C / 2; idx += kThreads) {
+        const int r = idx >> 5, col = 2 * (idx & 31);
+        const float2 t2 = *reinterpret_cast<const float2 *>(tf + r * C + col);
+        *reinterpret_cast<uint32_t *>(sm + Sm::Q + at(r, col, C)) = pack_bf16(t2.x, t2.y);
+    }
     __syncthreads();
+    copy_out(out + Ws::TB, sm + Sm::Q, 8192, kThreads);
+
+    // ---- -W = -T Bk: warp w owns rows 16 (w & 3), columns 64 (w >> 2) ----
+    {
+        const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
+        float acc[8][4];
+        zero_acc(acc);
+        mma_rows<8, false, true>(acc, sbase + Sm::Q, C, m0, sbase + Sm::X, C, n0, 0, C);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int col = n0 + 8 * t + 2 * tq;
+            *reinterpret_cast<uint32_t *>(sm + Sm::Y + at(m0 + gq, col, C)) = pack_bf16(-acc[t][0], -acc[t][1]);
+            *reinterpret_cast<uint32_t *>(sm + Sm::Y + at(m0 + gq + 8, col, C)) = pack_bf16(-acc[t][2], -acc[t][3]);
+        }
+    }
+    __syncthreads();
+    copy_out(out + Ws::WN, sm + Sm::Y, 16384, kThreads);
+}
+}  // namespace intra
+
+// =============================================================================================
+// 3. dstate: one CTA per (document, head), chunks in reverse, dS^T [v][c] fp32 in tensor memory
+//    (lane = value column v).  Per chunk, with the operands in shared memory:
+//      dU~^T  = dS^T_bf16 Kd^T + dO^T (scale A_qk)          (N = 64)
+//      dS^T  <- dS^T Diag(D) + dO^T (scale QG) + dU~^T_bf16 (-W)   (N = 128)
+//    dS^T (bf16, before the update) and dU~^T (bf16) go to the chunk's workspace block.
+// =============================================================================================
+namespace dstate {
+constexpr int kThreads = 128;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kFS = 0;     // dS^T fp32 [128 v][128 c]
+constexpr uint32_t kSB = 128;   // dS^T bf16, packed [128][64]
+constexpr uint32_t kUB = 128;   // dU~^T bf16, packed [128][32] (over kSB once the dU~ product has read it)
+constexpr uint32_t kDU = 192;   // dU~^T fp32 [128 v][64 s]
+struct Sm {
+    static constexpr int KD = 0;          // Kd [64 s][128 c]      K-major B (N = s, K = c)
+    static constexpr int AQ = 16384;      // scale A_qk [64 t][64 s]   MN-major B (K = t, N = s)
+    static constexpr int QG = 24576;      // scale QG [64 t][128 c]    MN-major B (K = t, N = c)
+    static constexpr int WN = 40960;      // -W [64 s][128 c]          MN-major B (K = s, N = c)
+    static constexpr int DO = 57344;      // dout [64 t][128 v]        MN-major A (K = t, M = v)
+    static constexpr int DL = 73728;      // D fp32 [128]
+    static constexpr int MBAR = DL + 512; // mbarriers: inputs, dU~ product, state product
+    static constexpr int TBASE = MBAR + 32, FLAG = TBASE + 8;
+    static constexpr int TOTAL = FLAG + 8;
+    static constexpr uint32_t kInBytes = 57344 + 512;   // bulk bytes per chunk (KD..WN, DL)
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
 
-__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
-__device__ __forceinline__ uint16_t f2bf(float x) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+__global__ void __launch_bounds__(kThreads, 2)
+kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64_t T, int H, const uint8_t *ws_intra,
+                      uint8_t *ws_dst, int *status) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x % H;
+    const int doc = doc_at_rank(cu, n_docs, blockIdx.x / H, reinterpret_cast<int *>(sm));
+    const int64_t d0 = cu[doc], d1 = cu[doc + 1];
+    if (d0 < 0 || d1 < d0 || d1 > T || d1 == d0) return;
+    const int nch = (int)((d1 - d0 + C - 1) / C);
+    const int64_t slot0 = d0 / C + doc;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t mb_in = sbase + Sm::MBAR, mb_u = mb_in + 8, mb_s = mb_in + 16;
+    volatile int *flag = reinterpret_cast<volatile int *>(sm + Sm::FLAG);
+    const float *dl = reinterpret_cast<const float *>(sm + Sm::DL);
+    if (warp == 0) tc::alloc(sbase + Sm::TBASE, kTmemCols);
+    if (tid == 0) {
+        tc::mbar_init(mb_in, 1);
+        tc::mbar_init(mb_u, 1);
+        tc::mbar_init(mb_s, 1);
+        *flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + Sm::TBASE);
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    const int v = 32 * warp + lane;   // this thread's TMEM lane = value column
+
+    // descriptors: K-major (Kd) and MN-major with 64 K rows per 64-wide atom (the rest)
+    const uint64_t dK = tc::sdesc(sbase, 16u, 1024u), dM = tc::sdesc(sbase, 64u * 128u, 1024u);
+    constexpr uint32_t id_u1 = tc::idesc_bf16(128, 64, false, false, false);   // dS^T_bf16 (TMEM) x Kd^T
+    constexpr uint32_t id_u2 = tc::idesc_bf16(128, 64, true, true, false);     // dO^T x A_qk
+    constexpr uint32_t id_s1 = tc::idesc_bf16(128, 128, true, true, false);    // dO^T x QG
+    constexpr uint32_t id_s2 = tc::idesc_bf16(128, 128, false, true, false);   // dU~^T_bf16 (TMEM) x (-W)
+
+    auto issue_loads = [&](int j) {
+        const int64_t tok = d0 + (int64_t)j * C;
+        const int Lj = (int)((d1 - tok) < C ? (d1 - tok) : C);
+        if (tid == 0) {
+            const uint8_t *src = ws_intra + ((size_t)(slot0 + j) * H + h) * Ws::INTRA;
+            tc::mbar_expect_tx(mb_in, Sm::kInBytes);
+            bulk_load(sbase + Sm::KD, src + Ws::KD, 16384, mb_in);
+            bulk_load(sbase + Sm::AQ, src + Ws::AQ, 8192, mb_in);
+            bulk_load(sbase + Sm::QG, src + Ws::QG, 16384, mb_in);
+            bulk_load(sbase + Sm::WN, src + Ws::WN, 16384, mb_in);
+            bulk_load(sbase + Sm::DL, src + Ws::DL, 512, mb_in);
+        }
+        // dout rows (zero past the document end) into the swizzled MN-major tile
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int idx = tid + i * kThreads, t = idx >> 4, m = idx & 15;
+            const bool ok = t < Lj;
+            const uint16_t *src = ok ? dout + ((tok + t) * H + h) * D + 8 * m : dout;
+            cp_async16(sbase + Sm::DO + at(t, 8 * m, C), src, ok ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    // dS^T row v as bf16 into the workspace block of chunk j (and, optionally, into TMEM)
+    auto store_ds = [&](int j, bool to_tmem) {
+        uint8_t *dst = ws_dst + ((size_t)(slot0 + j) * H + h) * Ws::DST + Ws::DS + (size_t)v * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float x[32];
+            tc::ld32(lane_base + kFS + 32 * q4, x);
+            tc::wait_ld();
+            reg_fence(x);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+            if (to_tmem) st16(lane_base + kSB + 16 * q4, pk);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int m = 4 * (q4 & 1) + e;   // 16-byte piece of channels 32 q4 + 8 e within the half
+                *reinterpret_cast<uint4 *>(dst + (size_t)(q4 >> 1) * (128 * 128) + ((m ^ (v & 7)) << 4)) =
+                    make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+        }
+    };
+
+    // dS leaving the last chunk is zero
+    {
+        float z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tc::st32(lane_base + kFS + 32 * q4, z);
+        tc::st32(lane_base + kSB, z);
+        tc::st32(lane_base + kSB + 32, z);
+        tc::wait_st();
+    }
+    store_ds(nch - 1, false);
+    issue_loads(nch - 1);
+    int last_j = nch - 1;   // the chunk whose inputs were issued last
+
+    bool aborted = false;
+    int n_commit_s = 0;   // completions of the state-product barrier so far (the next has parity n & 1)
+    for (int j = nch - 1; j >= 0; --j) {
+        const uint32_t par = (uint32_t)((nch - 1 - j) & 1);
+        cp_async_wait_all();
+        tc::fence_proxy_async();
+        bool ok = tc::mbar_wait(mb_in, par, kWaitLimit);
+        tc::wait_st();
+        tc::fence_before();
+        if (__syncthreads_or(!ok)) {
+            aborted = true;
+            break;
+        }
+        if (tid == 0) {
+            tc::fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ts(tmem + kDU, tmem + kSB + 8 * kk,
+                       dK + (uint64_t)((Sm::KD + (kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_u1, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma(tmem + kDU, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dM + (uint64_t)((Sm::AQ + kk * 2048) >> 4),
+                        id_u2, 1u);
+            tc::commit(mb_u);
+        }
+        // dS^T <- dS^T Diag(D) (the fp32 columns; the product above reads the bf16 copy)
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float x[32];
+            tc::ld32(lane_base + kFS + 32 * q4, x);
+            tc::wait_ld();
+            reg_fence(x);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] *= dl[32 * q4 + i];
+            tc::st32(lane_base + kFS + 32 * q4, x);
+        }
+        ok = tc::mbar_wait(mb_u, par, kWaitLimit);
+        tc::fence_after();
+        if (ok) {
+            // dU~^T -> workspace (bf16 row v) and -> TMEM as the A operand of the update
+            uint8_t *dst = ws_dst + ((size_t)(slot0 + j) * H + h) * Ws::DST + Ws::DU + (size_t)v * 128;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                float x[32];
+                tc::ld32(lane_base + kDU + 32 * h2, x);
+                tc::wait_ld();
+                reg_fence(x);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+                st16(lane_base + kUB + 16 * h2, pk);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int m = 4 * h2 + e;
+                    *reinterpret_cast<uint4 *>(dst + ((m ^ (v & 7)) << 4)) =
+                        make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+        }
+        tc::wait_st();
+        tc::fence_before();
+        if (__syncthreads_or(!ok)) {
+            aborted = true;
+            break;
+        }
+        if (tid == 0) {
+            tc::fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma(tmem + kFS, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dM + (uint64_t)((Sm::QG + kk * 2048) >> 4),
+                        id_s1, 1u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts(tmem + kFS, tmem + kUB + 8 * kk, dM + (uint64_t)((Sm::WN + kk * 2048) >> 4), id_s2, 1u);
+            tc::commit(mb_s);
+        }
+        ++n_commit_s;
+        ok = tc::mbar_wait(mb_s, par, kWaitLimit);
+        tc::fence_after();
+        if (__syncthreads_or(!ok)) {
+            aborted = true;
+            break;
+        }
+        if (j > 0) {
+            issue_loads(j - 1);
+            last_j = j - 1;
+            store_ds(j - 1, true);
+            tc::wait_st();
+        }
+    }
+    if (aborted) {
+        // a wait ran out of time: record it, then wait (bounded) for the copies and tensor-core
+        // operations still in flight before the CTA's shared memory and columns are released
+        if (tid == 0) {
+            atomicExch(status, kStatusTimeout);
+            tc::mbar_wait(mb_in, (uint32_t)((nch - 1 - last_j) & 1), kWaitLimit);
+            tc::commit(mb_s);
+            tc::mbar_wait(mb_s, (uint32_t)(n_commit_s & 1), kWaitLimit);
+        }
+        cp_async_wait_all();
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (warp == 0) tc::dealloc(tmem, kTmemCols);
 }
+}  // namespace dstate
+
+// =============================================================================================
+// 4. grad: one CTA per (chunk slot, head), 16 warps.  For 64 x 128 results warp w owns rows
+//    16 (w & 3) .. +15 and columns 32 (w >> 2) .. +31 (four 16 x 8 tiles); the gradients of k^,
+//    q^ and G at those positions stay in its registers from the first product to the last.
+// =============================================================================================
+namespace grad {
+constexpr int kThreads = 512;
+struct Sm {
+    static constexpr int ST = 0;          // S^T [128 v][128 c]; then dW [64 s][128 c]
+    static constexpr int DST = 32768;     // dS^T [128 v][128 c]; then dA_qk, dT, Xm, dA_hat (8 KB each)
+    static constexpr int DAQ = DST, DT = DST + 8192, XM = DST + 16384, DAH = DST + 24576;
+    static constexpr int DUT = 65536;     // dU~^T [128 v][64 s]; then pair scales fp32 [10][128]
+    static constexpr int PS = DUT;
+    static constexpr int WN = 81920;      // -W [64 s][128 c]; then k^ E1
+    static constexpr int XT = WN;
+    static constexpr int TB = 98304;      // T [64 r][64 i]
+    static constexpr int AH = 106496;     // A_hat [64 r][64 i]
+    static constexpr int DO = 114688;     // dout [64 t][128 v]
+    static constexpr int BV = 131072;     // beta v [64][128]; then q^ E1
+    static constexpr int QT = BV;
+    static constexpr int BK = 147456;     // beta k^ e^G [64][128]; then k^ E2
+    static constexpr int YT = BK;
+    static constexpr int UT = 163840;     // U~ [64 s][128 v]
+    static constexpr int GF = 180224;     // G (log2 units) fp32 [64][128], swizzled; then dG
+    // partial sums are kept per producing warp and added in a fixed order (bit-reproducible results):
+    // DGLP [6][128] dG_last (2 halves of S.dS, 4 row blocks of dKd Kd); DBP [12][64] dbeta (4 column
+    // warps each of dBk.KG, dBv.v, dA_kk.A_hat); RED [2][64][4] the row dots of dq and dk
+    static constexpr int RQ = 212992, RK = RQ + 256, BETA = RK + 256, DGLP = BETA + 256, DLS = DGLP + 3072,
+                         GLS = DLS + 512, DBP = GLS + 512, RED = DBP + 3072, TOT = RED + 2048;
+    static constexpr int TOTAL = TOT + 2048;
+};
+// fp32 [64][128] tile with the 8-float group index XORed with (row & 7): float2 reads of fragment
+// positions (8 rows x 8 columns per warp) touch all 32 banks
+__device__ __forceinline__ int gfi(int row, int col) { return row * D + (col ^ ((row & 7) << 3)); }
 
 struct Args {
     const uint16_t *q, *k, *v, *dout;
@@ -392,386 +716,557 @@ struct Args {
     int n_docs;
     int64_t T;
     int H;
+    const uint8_t *ws_ck, *ws_intra, *ws_dst;
     uint16_t *dq, *dk, *dv;
     float *dg, *dbeta;
-    float *ckpt;      // [(T/64 + n_docs) * H][128][128]
-    float *scratch;   // [n_docs * H][Ws::TOTAL]
-    int *status;
 };
 
-// Loads and recomputes everything a chunk needs.  full: also A_qk and Q^e^G (reverse sweep).
-__device__ void recompute_chunk(const Args &a, float *w, float *sA, float *sT, float *ga, float *gb, float *sred,
-                                int64_t tok0, int L, int h, bool full) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float *qn = w + Ws::QN, *kn = w + Ws::KN, *vv = w + Ws::VV, *G = w + Ws::G;
-    float *rq = w + Ws::RQ, *rk = w + Ws::RK, *bb = w + Ws::BB;
-    const int H = a.H;
-    // raw rows, four channels per access (rows >= L are zero: they then add nothing to any product)
+__global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const int H = a.H, slot = blockIdx.x / H, h = blockIdx.x % H;
+    int doc, L;
+    int64_t tok0;
+    if (!slot_chunk(a.cu, a.n_docs, a.T, slot, doc, tok0, L)) return;
+    const size_t blk = (size_t)slot * H + h;
+    const uint8_t *ck = a.ws_ck + blk * Ws::CK, *in = a.ws_intra + blk * Ws::INTRA, *dsb = a.ws_dst + blk * Ws::DST;
+    const uint32_t sbase = smem_u32(sm);
+    float *rq = reinterpret_cast<float *>(sm + Sm::RQ), *rk = reinterpret_cast<float *>(sm + Sm::RK);
+    float *sbeta = reinterpret_cast<float *>(sm + Sm::BETA), *dglp = reinterpret_cast<float *>(sm + Sm::DGLP);
+    float *dls = reinterpret_cast<float *>(sm + Sm::DLS), *gls = reinterpret_cast<float *>(sm + Sm::GLS);
+    float *dbp = reinterpret_cast<float *>(sm + Sm::DBP), *red = reinterpret_cast<float *>(sm + Sm::RED);
+    float *tot = reinterpret_cast<float *>(sm + Sm::TOT), *gf = reinterpret_cast<float *>(sm + Sm::GF);
+    float *ps = reinterpret_cast<float *>(sm + Sm::PS);
+
+    // ---- loads: workspace tiles as flat images, dout rows (zero past the document end) ----
     {
-        constexpr int it = CD / 4 / kThreads;
-        uint2 rq4[it], rk4[it], rv4[it], rd4[it];
-        float4 rg4[it];
+        const uint8_t *src[6] = {ck, dsb + Ws::DS, dsb + Ws::DU, in + Ws::WN, in + Ws::TB, in + Ws::AH};
+        const int dst[6] = {Sm::ST, Sm::DST, Sm::DUT, Sm::WN, Sm::TB, Sm::AH};
+        const int bytes[6] = {32768, 32768, 16384, 16384, 8192, 8192};
 #pragma unroll
-        for (int i = 0; i < it; ++i) {
-            const int idx = 4 * (tid + i * kThreads), r = idx / D, c = idx % D;
-            const int64_t off = ((tok0 + r) * H + h) * D + c;
-            const uint2 z2 = make_uint2(0u, 0u);
-            const bool ok = r < L;
-            rq4[i] = ok ? *reinterpret_cast<const uint2 *>(a.q + off) : z2;
-            rk4[i] = ok ? *reinterpret_cast<const uint2 *>(a.k + off) : z2;
-            rv4[i] = ok ? *reinterpret_cast<const uint2 *>(a.v + off) : z2;
-            rg4[i] = ok ? *reinterpret_cast<const float4 *>(a.g + off) : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (full) rd4[i] = ok ? *reinterpret_cast<const uint2 *>(a.dout + off) : z2;
-        }
-        auto f4 = [](uint2 u, float sc) {
-            return make_float4(bf2f((uint16_t)(u.x & 0xffffu)) * sc, bf2f((uint16_t)(u.x >> 16)) * sc,
-                               bf2f((uint16_t)(u.y & 0xffffu)) * sc, bf2f((uint16_t)(u.y >> 16)) * sc);
-        };
+        for (int t = 0; t < 6; ++t)
+            for (int i = tid; i < bytes[t] / 16; i += kThreads) cp_async16(sbase + dst[t] + 16 * i, src[t] + 16 * i, 16);
 #pragma unroll
-        for (int i = 0; i < it; ++i) {
-            const int idx = 4 * (tid + i * kThreads);
-            *reinterpret_cast<float4 *>(qn + idx) = f4(rq4[i], 1.f);
-            *reinterpret_cast<float4 *>(kn + idx) = f4(rk4[i], 1.f);
-            *reinterpret_cast<float4 *>(vv + idx) = f4(rv4[i], 1.f);
-            *reinterpret_cast<float4 *>(G + idx) = rg4[i];
-            if (full) *reinterpret_cast<float4 *>(w + Ws::DO + idx) = f4(rd4[i], rsqrtf((float)D));   // dO = scale dout
+        for (int i = 0; i < 2; ++i) {
+            const int idx = tid + i * kThreads, t = idx >> 4, m = idx & 15;
+            const bool ok = t < L;
+            const uint16_t *s = ok ? a.dout + ((tok0 + t) * H + h) * D + 8 * m : a.dout;
+            cp_async16(sbase + Sm::DO + at(t, 8 * m, C), s, ok ? 16 : 0);
         }
+        cp_async_commit();
     }
-    if (tid < C) bb[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
+    if (tid < C) sbeta[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
+    if (tid < D) dls[tid] = reinterpret_cast<const float *>(in + Ws::DL)[tid];
+    row_norms(a.q, a.k, tok0, L, H, h, rq, rk, kThreads / 32);
     __syncthreads();
-    // l2 norms: one warp per row
-    for (int r = warp; r < C; r += kWarps) {
-        const float4 q4 = *reinterpret_cast<const float4 *>(qn + r * D + 4 * lane);
-        const float4 k4 = *reinterpret_cast<const float4 *>(kn + r * D + 4 * lane);
-        float sq = q4.x * q4.x + q4.y * q4.y + q4.z * q4.z + q4.w * q4.w;
-        float sk = k4.x * k4.x + k4.y * k4.y + k4.z * k4.z + k4.w * k4.w;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            sk += __shfl_xor_sync(0xffffffffu, sk, o);
-        }
-        const float iq = rsqrtf(sq + 1e-6f), ik = rsqrtf(sk + 1e-6f);
-        *reinterpret_cast<float4 *>(qn + r * D + 4 * lane) = make_float4(q4.x * iq, q4.y * iq, q4.z * iq, q4.w * iq);
-        *reinterpret_cast<float4 *>(kn + r * D + 4 * lane) = make_float4(k4.x * ik, k4.y * ik, k4.z * ik, k4.w * ik);
-        if (lane == 0) {
-            rq[r] = iq;
-            rk[r] = ik;
-        }
-    }
-    // in-chunk cumsum per channel: thread (c, quarter) scans 16 rows in registers, then adds the
-    // totals of the quarters above it
+
+    // ---- G (log2 units) per channel, Bk = beta k^ e^G, Bv = beta v: thread (c, block qd) ----
     {
-        const int c = tid & (D - 1), qr = tid >> 7;
+        const int c = tid & (D - 1), qd = tid >> 7;
         float x[16];
+        float run = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) x[j] = G[(16 * qr + j) * D + c];
-#pragma unroll
-        for (int j = 1; j < 16; ++j) x[j] += x[j - 1];
-        sred[qr * D + c] = x[15];
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * qd + i;
+            run += (r < L ? a.g[((tok0 + r) * H + h) * D + c] : 0.f) * kLog2e;
+            x[i] = run;
+        }
+        tot[qd * D + c] = run;
         __syncthreads();
         float off = 0.f;
-        for (int q2 = 0; q2 < qr; ++q2) off += sred[q2 * D + c];
+        for (int q2 = 0; q2 < qd; ++q2) off += tot[q2 * D + c];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) G[(16 * qr + j) * D + c] = x[j] + off;
-        if (qr == 3) w[Ws::DL + c] = expf(x[15] + off);          // e^{G_last}
-        __syncthreads();
-    }
-    // decay factors: E1 = e^{G_r - G_16R}, E2 = e^{G_16R+15 - G_r}, pair scales s_RI = e^{G_16R - G_16I+15}
-    // (four channels per thread and step, every operand read and written as float4)
-    for (int idx = 4 * tid; idx < CD; idx += 4 * kThreads) {
-        const int r = idx / D, c = idx % D, R = r >> 4;
-        const float4 gr4 = *reinterpret_cast<const float4 *>(G + idx);
-        const float4 gl4 = *reinterpret_cast<const float4 *>(G + (C - 1) * D + c);
-        const float4 g04 = *reinterpret_cast<const float4 *>(G + (16 * R) * D + c);
-        const float4 g14 = *reinterpret_cast<const float4 *>(G + (16 * R + 15) * D + c);
-        const float4 k4 = *reinterpret_cast<const float4 *>(kn + idx);
-        const float4 q4 = *reinterpret_cast<const float4 *>(qn + idx);
-        const float4 v4 = *reinterpret_cast<const float4 *>(vv + idx);
-        const float br = bb[r];
-        const float grv[4] = {gr4.x, gr4.y, gr4.z, gr4.w}, glv[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
-        const float g0v[4] = {g04.x, g04.y, g04.z, g04.w}, g1v[4] = {g14.x, g14.y, g14.z, g14.w};
-        const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
-        const float vvv[4] = {v4.x, v4.y, v4.z, v4.w};
-        float e1[4], e2[4], x1[4], y1[4], q1[4], ev[4], kg[4], bk[4], bv[4], kd[4], qg[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            e1[j] = expf(grv[j] - g0v[j]);
-            e2[j] = expf(g1v[j] - grv[j]);
-            x1[j] = kv[j] * e1[j];
-            y1[j] = kv[j] * e2[j];
-            q1[j] = qv[j] * e1[j];
-            ev[j] = expf(grv[j]);
-            kg[j] = kv[j] * ev[j];
-            bk[j] = br * kv[j] * ev[j];
-            bv[j] = br * vvv[j];
-            kd[j] = kv[j] * expf(glv[j] - grv[j]);
-            qg[j] = qv[j] * ev[j];
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * qd + i;
+            x[i] += off;
+            gf[gfi(r, c)] = x[i];
+            float kv = 0.f, vv = 0.f;
+            if (r < L) {
+                const int64_t o = ((tok0 + r) * H + h) * D + c;
+                kv = bfl(a.k[o]) * rk[r];
+                vv = bfl(a.v[o]);
+            }
+            const uint32_t o2 = at(r, c, C);
+            *reinterpret_cast<uint16_t *>(sm + Sm::BK + o2) = f2b(sbeta[r] * kv * ex2_ftz(x[i]));
+            *reinterpret_cast<uint16_t *>(sm + Sm::BV + o2) = f2b(sbeta[r] * vv);
         }
-        auto st4 = [&](size_t off, const float (&x)[4]) {
-            *reinterpret_cast<float4 *>(w + off + idx) = make_float4(x[0], x[1], x[2], x[3]);
-        };
-        st4(Ws::E1, e1);
-        st4(Ws::E2, e2);
-        st4(Ws::X1, x1);
-        st4(Ws::Y1, y1);
-        if (full) st4(Ws::Q1, q1);
-        st4(Ws::EG, ev);
-        st4(Ws::KG, kg);
-        st4(Ws::BK, bk);
-        st4(Ws::BV, bv);
-        st4(Ws::KD, kd);
-        if (full) st4(Ws::QG, qg);
+        if (qd == 3) gls[c] = x[15];
     }
-    for (int idx = tid; idx < 10 * D; idx += kThreads) {
-        const int p = idx / D, c = idx % D;
-        const int R = p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0, I = p - R * (R + 1) / 2;
-        w[Ws::SP + idx] = expf(G[(16 * R) * D + c] - G[(16 * I + 15) * D + c]);
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- dG_last part 1: D[c] sum_v S[c][v] dS[c][v], from matching B fragments of S^T and dS^T ----
+    {
+        const int c0 = 16 * (warp & 7), kb = 64 * (warp >> 3);
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 64; kk += 16) {
+            uint32_t bs[4], bd[4];
+            frag_b2<true>(sbase + Sm::ST, D, kb + kk, c0, bs);
+            frag_b2<true>(sbase + Sm::DST, D, kb + kk, c0, bd);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = bf2(bs[e]), y = bf2(bd[e]);
+                const float p = x.x * y.x + x.y * y.y;
+                if (e < 2) s0 += p;
+                else s1 += p;
+            }
+        }
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        if (tq == 0) {
+            dglp[(warp >> 3) * D + c0 + gq] = dls[c0 + gq] * s0;
+            dglp[(warp >> 3) * D + c0 + 8 + gq] = dls[c0 + 8 + gq] * s1;
+        }
+    }
+
+    const int rb = warp & 3, cb = warp >> 2, m0 = 16 * rb, n0 = 32 * cb;
+    float dkn[4][4], dqn[4][4], dG[4][4];
+    zero_acc(dkn);
+    zero_acc(dqn);
+    zero_acc(dG);
+    // element (t, e) of a 64 x 128 result: row m0 + gq + 8 (e >> 1), column n0 + 8 t + 2 tq + (e & 1)
+    // raw bf16 pair (row, col..col+1) of q / k / v, zero past the document end
+    auto ld_pair = [&](const uint16_t *p, int row, int col) {
+        return row < L ? bf2(*reinterpret_cast<const uint32_t *>(p + ((tok0 + row) * H + h) * D + col))
+                       : make_float2(0.f, 0.f);
+    };
+
+    // ---- U~ = T (beta V) + (-W) S ----
+    {
+        float acc[4][4];
+        zero_acc(acc);
+        mma_rows<4, false, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::BV, C, n0, 0, C);
+        mma_rows<4, false, false>(acc, sbase + Sm::WN, C, m0, sbase + Sm::ST, D, n0, 0, D);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint32_t *>(sm + Sm::UT + at(m0 + gq + 8 * hh, n0 + 8 * t + 2 * tq, C)) =
+                    pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
     }
     __syncthreads();
-    // A_hat[r][i] = sum_c k^_rc k^_ic e^{G_rc - G_ic} (i < r); A_qk the same with q^ (i <= r)
-    pair_products(w, full, ga);
-    // T = (I + diag(beta) A_hat)^-1
-    tri_inverse(w, sA, sT, ga);
-    // W = T (beta K^e^G), U = T (beta V)
-    gemm<C, D, C, false, false>(1.f, w + Ws::TM, w + Ws::BK, false, w + Ws::W, D, ga, gb);
-    gemm<C, D, C, false, false>(1.f, w + Ws::TM, w + Ws::BV, false, w + Ws::U, D, ga, gb);
-}
 
-__global__ void __launch_bounds__(kThreads, 1) kda_bwd_kernel(const Args a) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    extern __shared__ __align__(16) float smem[];
-    // CTA -> (document, head), longest documents first (the shared memory is not in use yet);
-    // `chain` indexes this CTA's scratch
-    const int H = a.H, chain = blockIdx.x, h = chain % H;
-    const int doc = doc_at_rank(a.cu, a.n_docs, chain / H, reinterpret_cast<int *>(smem));
-    if (blockIdx.x == 0 && tid == 0 && (a.cu[0] != 0 || (int64_t)a.cu[a.n_docs] != a.T))
-        atomicExch(a.status, kStatusBadSeqlens);
-    const int64_t d0 = a.cu[doc], d1 = a.cu[doc + 1];
-    if (d0 < 0 || d1 < d0 || d1 > a.T) {
-        if (tid == 0) atomicExch(a.status, kStatusBadSeqlens);
-        return;
+    // ---- dKd = U~ dS^T: dk^ += dKd e^{G_last - G}, dG -= dKd Kd, dG_last += sum_r dKd Kd ----
+    {
+        float acc[4][4];
+        zero_acc(acc);
+        mma_rows<4, false, true>(acc, sbase + Sm::UT, C, m0, sbase + Sm::DST, D, n0, 0, D);
+        float cs[4][2];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            cs[t][0] = cs[t][1] = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
+                const float2 kr = ld_pair(a.k, row, col);
+                const float ed0 = ex2_ftz(gls[col] - g2.x), ed1 = ex2_ftz(gls[col + 1] - g2.y);
+                const float kd0 = kr.x * rk[row] * ed0, kd1 = kr.y * rk[row] * ed1;
+                const float x0 = acc[t][2 * hh], x1 = acc[t][2 * hh + 1];
+                dkn[t][2 * hh] += x0 * ed0;
+                dkn[t][2 * hh + 1] += x1 * ed1;
+                dG[t][2 * hh] -= x0 * kd0;
+                dG[t][2 * hh + 1] -= x1 * kd1;
+                cs[t][0] += x0 * kd0;
+                cs[t][1] += x1 * kd1;
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float x = cs[t][e];
+                x += __shfl_xor_sync(0xffffffffu, x, 4);
+                x += __shfl_xor_sync(0xffffffffu, x, 8);
+                x += __shfl_xor_sync(0xffffffffu, x, 16);
+                if (gq == 0) dglp[(2 + rb) * D + n0 + 8 * t + 2 * tq + e] = x;
+            }
     }
-    if (d1 == d0) return;
-    const int nch = (int)((d1 - d0 + C - 1) / C);
-    const int64_t slot0 = d0 / C + doc;                     // checkpoint slots of this document
-    float *w = a.scratch + (size_t)chain * Ws::TOTAL;
-    float *ga = smem, *gb = smem + kOpFloats;                 // gemm operand buffers
-    float *sA = gb + kOpFloats, *sT = sA + C * (C + 1);       // triangular inverse
-    float *sred = sT + C * (C + 1);                           // [4][128] partial sums
+    // ---- dQG = scale dO S^T: dq^ += dQG e^G, dG += dQG QG ----
+    {
+        float acc[4][4];
+        zero_acc(acc);
+        mma_rows<4, false, true>(acc, sbase + Sm::DO, C, m0, sbase + Sm::ST, D, n0, 0, D);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
+                const float2 qr = ld_pair(a.q, row, col);
+                const float e0 = ex2_ftz(g2.x), e1 = ex2_ftz(g2.y);
+                const float x0 = kScale * acc[t][2 * hh], x1 = kScale * acc[t][2 * hh + 1];
+                dqn[t][2 * hh] += x0 * e0;
+                dqn[t][2 * hh + 1] += x1 * e1;
+                dG[t][2 * hh] += x0 * qr.x * rq[row] * e0;
+                dG[t][2 * hh + 1] += x1 * qr.y * rq[row] * e1;
+            }
+    }
+    // ---- dW = -dU~ S^T (kept in registers until every warp is done with S) ----
+    float dw[4][4];
+    zero_acc(dw);
+    mma_rows<4, true, true>(dw, sbase + Sm::DUT, D, m0, sbase + Sm::ST, D, n0, 0, D);
+    __syncthreads();   // S^T and dS^T are read: their space takes dW and the 64 x 64 tiles
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+            *reinterpret_cast<uint32_t *>(sm + Sm::ST + at(m0 + gq + 8 * hh, n0 + 8 * t + 2 * tq, C)) =
+                pack_bf16(-dw[t][2 * hh], -dw[t][2 * hh + 1]);
 
-    // The state entering every chunk is in the checkpoint slots: the pipelined forward kernel wrote
-    // them (launch_bwd runs it first).
+    // 64 x 64 results: warp w owns rows 16 (w & 3) and columns 16 (w >> 2) (two 16 x 8 tiles)
+    const int n64 = 16 * cb;
+    // ---- dA_qk = scale lower(dO U~^T) ----
+    {
+        float acc[2][4];
+        zero_acc(acc);
+        mma_rows<2, false, false>(acc, sbase + Sm::DO, C, m0, sbase + Sm::UT, C, n64, 0, D);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n64 + 8 * t + 2 * tq;
+                const float x0 = col <= row ? kScale * acc[t][2 * hh] : 0.f;
+                const float x1 = col + 1 <= row ? kScale * acc[t][2 * hh + 1] : 0.f;
+                *reinterpret_cast<uint32_t *>(sm + Sm::DAQ + at(row, col, C)) = pack_bf16(x0, x1);
+            }
+    }
+    __syncthreads();   // dW in place
+    // ---- dT = dW (beta KG)^T + dU~ (beta V)^T ----
+    {
+        float acc[2][4];
+        zero_acc(acc);
+        mma_rows<2, false, false>(acc, sbase + Sm::ST, C, m0, sbase + Sm::BK, C, n64, 0, D);
+        mma_rows<2, true, false>(acc, sbase + Sm::DUT, D, m0, sbase + Sm::BV, C, n64, 0, D);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint32_t *>(sm + Sm::DT + at(m0 + gq + 8 * hh, n64 + 8 * t + 2 * tq, C)) =
+                    pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
+    }
+    // ---- dBk = T^T dW: dKG = beta dBk; dk^ += dKG e^G, dG += dKG KG, dbeta += dBk . KG ----
+    {
+        float acc[4][4];
+        zero_acc(acc);
+        mma_rows<4, true, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::ST, C, n0, 0, C);
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
+                const float2 kr = ld_pair(a.k, row, col);
+                const float e0 = ex2_ftz(g2.x), e1 = ex2_ftz(g2.y);
+                const float kg0 = kr.x * rk[row] * e0, kg1 = kr.y * rk[row] * e1;
+                const float b = sbeta[row];
+                const float x0 = acc[t][2 * hh], x1 = acc[t][2 * hh + 1];
+                dkn[t][2 * hh] += b * x0 * e0;
+                dkn[t][2 * hh + 1] += b * x1 * e1;
+                dG[t][2 * hh] += b * x0 * kg0;
+                dG[t][2 * hh + 1] += b * x1 * kg1;
+                rs[hh] += x0 * kg0 + x1 * kg1;
+            }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float x = rs[hh];
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            if (tq == 0) dbp[(0 + cb) * C + m0 + gq + 8 * hh] = x;
+        }
+    }
+    // ---- dBv = T^T dU~: dv = beta dBv, dbeta += dBv . v ----
+    {
+        float acc[4][4];
+        zero_acc(acc);
+        mma_rows<4, true, false>(acc, sbase + Sm::TB, C, m0, sbase + Sm::DUT, D, n0, 0, C);
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float x0 = acc[t][2 * hh], x1 = acc[t][2 * hh + 1];
+                if (row < L) {
+                    const float2 vr = ld_pair(a.v, row, col);
+                    rs[hh] += x0 * vr.x + x1 * vr.y;
+                    const float b = sbeta[row];
+                    *reinterpret_cast<uint32_t *>(a.dv + ((tok0 + row) * H + h) * D + col) = pack_bf16(b * x0, b * x1);
+                }
+            }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float x = rs[hh];
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            if (tq == 0) dbp[(4 + cb) * C + m0 + gq + 8 * hh] = x;
+        }
+    }
+    __syncthreads();   // dT in place; dW, dU~^T, beta V, beta KG are read
+    // ---- Xm = T^T dT ----
+    {
+        float acc[2][4];
+        zero_acc(acc);
+        mma_rows<2, true, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::DT, C, n64, 0, C);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint32_t *>(sm + Sm::XM + at(m0 + gq + 8 * hh, n64 + 8 * t + 2 * tq, C)) =
+                    pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
+    }
+    // ---- k^ E1, q^ E1, k^ E2 (the pairwise-decay operands, bf16) and the pair scales ----
+    {
+        const int c = tid & (D - 1), qd = tid >> 7;
+        const float gs = gf[gfi(16 * qd, c)], ge = gf[gfi(16 * qd + 15, c)];
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * qd + i;
+            float kv = 0.f, qv = 0.f;
+            if (r < L) {
+                const int64_t o = ((tok0 + r) * H + h) * D + c;
+                kv = bfl(a.k[o]) * rk[r];
+                qv = bfl(a.q[o]) * rq[r];
+            }
+            const float g2 = gf[gfi(r, c)];
+            const float e1 = ex2_ftz(g2 - gs), e2 = ex2_ftz(ge - g2);
+            const uint32_t o2 = at(r, c, C);
+            *reinterpret_cast<uint16_t *>(sm + Sm::XT + o2) = f2b(kv * e1);
+            *reinterpret_cast<uint16_t *>(sm + Sm::QT + o2) = f2b(qv * e1);
+            *reinterpret_cast<uint16_t *>(sm + Sm::YT + o2) = f2b(kv * e2);
+        }
+        for (int p = qd; p < 10; p += 4) {
+            const int R = pair_R(p), I = p - R * (R + 1) / 2;
+            ps[p * D + c] = ex2_ftz(gf[gfi(16 * R, c)] - gf[gfi(16 * I + 15, c)]);
+        }
+    }
+    __syncthreads();   // Xm in place
+    // ---- dA_kk = strict_lower(-Xm T^T): dbeta += dA_kk . A_hat, dA_hat = beta dA_kk ----
+    {
+        float acc[2][4];
+        zero_acc(acc);
+        mma_rows<2, false, false>(acc, sbase + Sm::XM, C, m0, sbase + Sm::TB, C, n64, 0, C);
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n64 + 8 * t + 2 * tq;
+                const float x0 = col < row ? -acc[t][2 * hh] : 0.f, x1 = col + 1 < row ? -acc[t][2 * hh + 1] : 0.f;
+                const float2 ah = bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::AH + at(row, col, C)));
+                rs[hh] += x0 * ah.x + x1 * ah.y;
+                const float b = sbeta[row];
+                *reinterpret_cast<uint32_t *>(sm + Sm::DAH + at(row, col, C)) = pack_bf16(b * x0, b * x1);
+            }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float x = rs[hh];
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            if (tq == 0) dbp[(8 + cb) * C + m0 + gq + 8 * hh] = x;
+        }
+    }
+    __syncthreads();   // dA_hat, dA_qk, the pairwise operands and scales in place
+    // ---- pairwise-decay sums, block pair by block pair (pair scale per column) ----
+    //   row side    (rows r in block rb): P1 = sum_{I<=rb} s (dA_hat[rb,I] Y~_I),  P3 likewise with dA_qk
+    //   column side (rows i in block rb): P24 = sum_{R>=rb} s (dA_hat[R,rb]^T X~_R + dA_qk[R,rb]^T Q~_R)
+    //   dk^ += E1 P1 + E2 P24,  dq^ += E1 P3,  dG += X~ P1 + Q~ P3 - Y~ P24
+    {
+        float p1[4][4], p3[4][4];
+        zero_acc(p1);
+        zero_acc(p3);
+        for (int I = 0; I <= rb; ++I) {
+            const int p = pair_of(rb, I);
+            float t1[4][4], t3[4][4];
+            zero_acc(t1);
+            zero_acc(t3);
+            mma_rows<4, false, true>(t1, sbase + Sm::DAH, C, m0, sbase + Sm::YT, C, n0, 16 * I, 16 * I + 16);
+            mma_rows<4, false, true>(t3, sbase + Sm::DAQ, C, m0, sbase + Sm::YT, C, n0, 16 * I, 16 * I + 16);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 s = *reinterpret_cast<const float2 *>(ps + p * D + n0 + 8 * t + 2 * tq);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float se = (e & 1) ? s.y : s.x;
+                    p1[t][e] += se * t1[t][e];
+                    p3[t][e] += se * t3[t][e];
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
+                const float2 gs = *reinterpret_cast<const float2 *>(gf + gfi(m0, col));
+                const float e0 = ex2_ftz(g2.x - gs.x), e1 = ex2_ftz(g2.y - gs.y);
+                const float2 xt = bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::XT + at(row, col, C)));
+                const float2 qt = bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::QT + at(row, col, C)));
+                dkn[t][2 * hh] += e0 * p1[t][2 * hh];
+                dkn[t][2 * hh + 1] += e1 * p1[t][2 * hh + 1];
+                dqn[t][2 * hh] += e0 * p3[t][2 * hh];
+                dqn[t][2 * hh + 1] += e1 * p3[t][2 * hh + 1];
+                dG[t][2 * hh] += xt.x * p1[t][2 * hh] + qt.x * p3[t][2 * hh];
+                dG[t][2 * hh + 1] += xt.y * p1[t][2 * hh + 1] + qt.y * p3[t][2 * hh + 1];
+            }
+    }
+    {
+        float p24[4][4];
+        zero_acc(p24);
+        for (int R = rb; R < 4; ++R) {
+            const int p = pair_of(R, rb);
+            float t2[4][4];
+            zero_acc(t2);
+            mma_rows<4, true, true>(t2, sbase + Sm::DAH, C, m0, sbase + Sm::XT, C, n0, 16 * R, 16 * R + 16);
+            mma_rows<4, true, true>(t2, sbase + Sm::DAQ, C, m0, sbase + Sm::QT, C, n0, 16 * R, 16 * R + 16);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 s = *reinterpret_cast<const float2 *>(ps + p * D + n0 + 8 * t + 2 * tq);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p24[t][e] += ((e & 1) ? s.y : s.x) * t2[t][e];
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
+                const float2 ge = *reinterpret_cast<const float2 *>(gf + gfi(m0 + 15, col));
+                const float e0 = ex2_ftz(ge.x - g2.x), e1 = ex2_ftz(ge.y - g2.y);
+                const float2 yt = bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::YT + at(row, col, C)));
+                dkn[t][2 * hh] += e0 * p24[t][2 * hh];
+                dkn[t][2 * hh + 1] += e1 * p24[t][2 * hh + 1];
+                dG[t][2 * hh] -= yt.x * p24[t][2 * hh];
+                dG[t][2 * hh + 1] -= yt.y * p24[t][2 * hh + 1];
+            }
+    }
 
-    // ---------------- reverse sweep ----------------
-    float *dS = w + Ws::DS, *dSn = w + Ws::DSN;
-    for (int idx = tid; idx < DD; idx += kThreads) dS[idx] = 0.f;
-    __syncthreads();
-    for (int n = nch - 1; n >= 0; --n) {
-        const int64_t tok0 = d0 + (int64_t)n * C;
-        const int L = (int)((d1 - tok0) < C ? (d1 - tok0) : C);
-        recompute_chunk(a, w, sA, sT, ga, gb, sred, tok0, L, h, true);
-        const float *Sin = a.ckpt + ((size_t)(slot0 + n) * H + h) * DD;
-        float *Ut = w + Ws::UT, *dUt = w + Ws::DUT, *dO = w + Ws::DO;
-        for (int idx = tid; idx < CD; idx += kThreads) Ut[idx] = w[Ws::U + idx];
-        __syncthreads();
-        gemm<C, D, D, false, false>(-1.f, w + Ws::W, Sin, true, Ut, D, ga, gb);
-        // dU~ = A_qk^T dO + Kd dS
-        gemm<C, D, C, true, false>(1.f, w + Ws::AQ, dO, false, dUt, D, ga, gb);
-        gemm<C, D, D, false, false>(1.f, w + Ws::KD, dS, true, dUt, D, ga, gb);
-        // dS_in = QG^T dO + Diag(e^{G_last}) dS - W^T dU~
-        gemm<D, D, C, true, false>(1.f, w + Ws::QG, dO, false, dSn, D, ga, gb);
-        for (int idx = tid; idx < DD; idx += kThreads) dSn[idx] += w[Ws::DL + idx / D] * dS[idx];
-        __syncthreads();
-        gemm<D, D, C, true, false>(-1.f, w + Ws::W, dUt, true, dSn, D, ga, gb);
-        // dQG = dO S^T, dA_qk = lower(dO U~^T), dKd = U~ dS^T, dW = -dU~ S^T
-        gemm<C, D, D, false, true>(1.f, dO, Sin, false, w + Ws::DQG, D, ga, gb);
-        gemm<C, C, D, false, true>(1.f, dO, Ut, false, w + Ws::DAQ, C, ga, gb);
-        gemm<C, D, D, false, true>(1.f, Ut, dS, false, w + Ws::DKD, D, ga, gb);
-        gemm<C, D, D, false, true>(-1.f, dUt, Sin, false, w + Ws::DW, D, ga, gb);
-        // dG_last (from Diag(e^{G_last}) S) and the lower mask of dA_qk
-        {
-            const int c = tid >> 2, part = tid & 3;
-            float acc = 0.f;
+    // ---- dq, dk through the l2 norms (row dots across the four column warps), dG to shared ----
+    {
+        float sq[2] = {0.f, 0.f}, sk[2] = {0.f, 0.f};
 #pragma unroll
-            for (int x = 32 * part; x < 32 * part + 32; x += 4) {
-                const float4 s4 = *reinterpret_cast<const float4 *>(Sin + c * D + x);
-                const float4 d4 = *reinterpret_cast<const float4 *>(dS + c * D + x);
-                acc += s4.x * d4.x + s4.y * d4.y + s4.z * d4.z + s4.w * d4.w;
-            }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (part == 0) w[Ws::DGL + c] = w[Ws::DL + c] * acc;
-        }
-        for (int idx = tid; idx < CC; idx += kThreads)
-            if (idx % C > idx / C) w[Ws::DAQ + idx] = 0.f;
-        __syncthreads();
-        // dT = dW (beta KG)^T + dU~ (beta V)^T;  dBk = T^T dW, dBv = T^T dU~
-        gemm<C, C, D, false, true>(1.f, w + Ws::DW, w + Ws::BK, false, w + Ws::DT, C, ga, gb);
-        gemm<C, C, D, false, true>(1.f, dUt, w + Ws::BV, true, w + Ws::DT, C, ga, gb);
-        gemm<C, D, C, true, false>(1.f, w + Ws::TM, w + Ws::DW, false, w + Ws::DBK, D, ga, gb);
-        gemm<C, D, C, true, false>(1.f, w + Ws::TM, dUt, false, w + Ws::DBV, D, ga, gb);
-        // dA_kk = strict_lower(-T^T dT T^T)
-        gemm<C, C, C, true, false>(1.f, w + Ws::TM, w + Ws::DT, false, w + Ws::XM, C, ga, gb);
-        gemm<C, C, C, false, true>(-1.f, w + Ws::XM, w + Ws::TM, false, w + Ws::DAH, C, ga, gb);
-        // dbeta (rows), dv, dKG = beta dBk, dA_hat = beta dA_kk
-        for (int r = warp; r < C; r += kWarps) {
-            const int c4 = r * D + 4 * lane;
-            const float4 dbv = *reinterpret_cast<const float4 *>(w + Ws::DBV + c4);
-            const float4 vv4 = *reinterpret_cast<const float4 *>(w + Ws::VV + c4);
-            const float4 dbk = *reinterpret_cast<const float4 *>(w + Ws::DBK + c4);
-            const float4 kg4 = *reinterpret_cast<const float4 *>(w + Ws::KG + c4);
-            float acc = dbv.x * vv4.x + dbv.y * vv4.y + dbv.z * vv4.z + dbv.w * vv4.w + dbk.x * kg4.x + dbk.y * kg4.y +
-                        dbk.z * kg4.z + dbk.w * kg4.w;
-            const float2 dah = *reinterpret_cast<const float2 *>(w + Ws::DAH + r * C + 2 * lane);
-            const float2 ah = *reinterpret_cast<const float2 *>(w + Ws::AH + r * C + 2 * lane);
-            if (2 * lane < r) acc += dah.x * ah.x;
-            if (2 * lane + 1 < r) acc += dah.y * ah.y;
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) w[Ws::DB + r] = acc;
-        }
-        __syncthreads();
-        for (int idx = 4 * tid; idx < CC; idx += 4 * kThreads) {
-            const int r = idx / C, i = idx % C;
-            const float b = w[Ws::BB + r];
-            const float4 x = *reinterpret_cast<const float4 *>(w + Ws::DAH + idx);
-            *reinterpret_cast<float4 *>(w + Ws::DAH + idx) =
-                make_float4(i < r ? b * x.x : 0.f, i + 1 < r ? b * x.y : 0.f, i + 2 < r ? b * x.z : 0.f,
-                            i + 3 < r ? b * x.w : 0.f);
-        }
-        for (int idx = 4 * tid; idx < CD; idx += 4 * kThreads) {
-            const int r = idx / D;
-            const float b = w[Ws::BB + r];
-            const float4 dbv = *reinterpret_cast<const float4 *>(w + Ws::DBV + idx);
-            if (r < L)
-                *reinterpret_cast<uint2 *>(a.dv + ((tok0 + r) * H + h) * D + idx % D) =
-                    make_uint2((uint32_t)f2bf(b * dbv.x) | ((uint32_t)f2bf(b * dbv.y) << 16),
-                               (uint32_t)f2bf(b * dbv.z) | ((uint32_t)f2bf(b * dbv.w) << 16));
-            const float4 dbk = *reinterpret_cast<const float4 *>(w + Ws::DBK + idx);
-            *reinterpret_cast<float4 *>(w + Ws::DBK + idx) = make_float4(b * dbk.x, b * dbk.y, b * dbk.z, b * dbk.w);   // now dKG
-        }
-        __syncthreads();
-        // pairwise-decay sums (block MMA), then the elementwise chain rule per (row r, channel c)
-        pair_grads(w, ga);
-        for (int idx = 4 * tid; idx < CD; idx += 4 * kThreads) {
-            const int c = idx % D;
-            auto ld4 = [&](size_t off) {
-                const float4 x = *reinterpret_cast<const float4 *>(w + off + idx);
-                return x;
-            };
-            const float4 a1 = ld4(Ws::DKN), a3 = ld4(Ws::DQN), a24 = ld4(Ws::A24), knv = ld4(Ws::KN), qnv = ld4(Ws::QN);
-            const float4 eg = ld4(Ws::EG), dKG = ld4(Ws::DBK), dQG = ld4(Ws::DQG), dKd = ld4(Ws::DKD), kg = ld4(Ws::KG);
-            const float4 qg = ld4(Ws::QG), kd = ld4(Ws::KD), gr = ld4(Ws::G);
-            const float4 gl = *reinterpret_cast<const float4 *>(w + Ws::G + (C - 1) * D + c);
-            const float a1v[4] = {a1.x, a1.y, a1.z, a1.w}, a3v[4] = {a3.x, a3.y, a3.z, a3.w};
-            const float a24v[4] = {a24.x, a24.y, a24.z, a24.w}, knvv[4] = {knv.x, knv.y, knv.z, knv.w};
-            const float qnvv[4] = {qnv.x, qnv.y, qnv.z, qnv.w}, egv[4] = {eg.x, eg.y, eg.z, eg.w};
-            const float dkgv[4] = {dKG.x, dKG.y, dKG.z, dKG.w}, dqgv[4] = {dQG.x, dQG.y, dQG.z, dQG.w};
-            const float dkdv[4] = {dKd.x, dKd.y, dKd.z, dKd.w}, kgv[4] = {kg.x, kg.y, kg.z, kg.w};
-            const float qgv[4] = {qg.x, qg.y, qg.z, qg.w}, kdv[4] = {kd.x, kd.y, kd.z, kd.w};
-            const float grv[4] = {gr.x, gr.y, gr.z, gr.w}, glv[4] = {gl.x, gl.y, gl.z, gl.w};
-            float dkn[4], dqn[4], dg[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float e3 = expf(glv[j] - grv[j]);
-                dkn[j] = a1v[j] + a24v[j] + dkgv[j] * egv[j] + dkdv[j] * e3;
-                dqn[j] = a3v[j] + dqgv[j] * egv[j];
-                dg[j] = knvv[j] * (a1v[j] - a24v[j]) + qnvv[j] * a3v[j] + dkgv[j] * kgv[j] + dqgv[j] * qgv[j] -
-                        dkdv[j] * kdv[j];
-            }
-            *reinterpret_cast<float4 *>(w + Ws::DKN + idx) = make_float4(dkn[0], dkn[1], dkn[2], dkn[3]);
-            *reinterpret_cast<float4 *>(w + Ws::DQN + idx) = make_float4(dqn[0], dqn[1], dqn[2], dqn[3]);
-            *reinterpret_cast<float4 *>(w + Ws::DG + idx) = make_float4(dg[0], dg[1], dg[2], dg[3]);
-        }
-        __syncthreads();
-        // dg: reverse cumsum of dG per channel, plus the G_last terms (which reach every row):
-        // thread (c, quarter) holds 16 rows in registers; quarter sums go through shared memory
-        {
-            const int c = tid & (D - 1), qr = tid >> 7;
-            float x[16];
-            float gl = 0.f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int idx = (16 * qr + j) * D + c;
-                x[j] = w[Ws::DG + idx];
-                gl += w[Ws::DKD + idx] * w[Ws::KD + idx];
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                const float2 qr = ld_pair(a.q, row, col), kr = ld_pair(a.k, row, col);
+                sq[hh] += rq[row] * (qr.x * dqn[t][2 * hh] + qr.y * dqn[t][2 * hh + 1]);
+                sk[hh] += rk[row] * (kr.x * dkn[t][2 * hh] + kr.y * dkn[t][2 * hh + 1]);
             }
 #pragma unroll
-            for (int j = 14; j >= 0; --j) x[j] += x[j + 1];
-            sred[qr * D + c] = x[0];
-            __syncthreads();
-            float off = w[Ws::DGL + c];
-            for (int q2 = 0; q2 < 4; ++q2) {
-                if (q2 > qr) off += sred[q2 * D + c];
-            }
-            __syncthreads();
-            sred[qr * D + c] = gl;
-            __syncthreads();
-            for (int q2 = 0; q2 < 4; ++q2) off += sred[q2 * D + c];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int r = 16 * qr + j;
-                if (r < L) a.dg[((tok0 + r) * H + h) * D + c] = x[j] + off;
+        for (int hh = 0; hh < 2; ++hh) {
+            float x = sq[hh], y = sk[hh];
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            y += __shfl_xor_sync(0xffffffffu, y, 1);
+            y += __shfl_xor_sync(0xffffffffu, y, 2);
+            if (tq == 0) {
+                red[(m0 + gq + 8 * hh) * 4 + cb] = x;
+                red[256 + (m0 + gq + 8 * hh) * 4 + cb] = y;
             }
         }
-        // dq, dk through the l2 norms; dbeta
-        for (int r = warp; r < C; r += kWarps) {
-            if (r >= L) continue;
-            const int c4 = r * D + 4 * lane;
-            const float4 qn4 = *reinterpret_cast<const float4 *>(w + Ws::QN + c4);
-            const float4 dqn4 = *reinterpret_cast<const float4 *>(w + Ws::DQN + c4);
-            const float4 kn4 = *reinterpret_cast<const float4 *>(w + Ws::KN + c4);
-            const float4 dkn4 = *reinterpret_cast<const float4 *>(w + Ws::DKN + c4);
-            float sq = qn4.x * dqn4.x + qn4.y * dqn4.y + qn4.z * dqn4.z + qn4.w * dqn4.w;
-            float sk = kn4.x * dkn4.x + kn4.y * dkn4.y + kn4.z * dkn4.z + kn4.w * dkn4.w;
+    }
+    __syncthreads();   // row dots in place; every read of G is done
 #pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                sq += __shfl_xor_sync(0xffffffffu, sq, o);
-                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+            *reinterpret_cast<float2 *>(gf + gfi(row, col)) = make_float2(dG[t][2 * hh], dG[t][2 * hh + 1]);
+            if (row < L) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(red + row * 4);
+                const float4 k4 = *reinterpret_cast<const float4 *>(red + 256 + row * 4);
+                const float sq = s4.x + s4.y + s4.z + s4.w, sk = k4.x + k4.y + k4.z + k4.w;
+                const float2 qr = ld_pair(a.q, row, col), kr = ld_pair(a.k, row, col);
+                const float iq = rq[row], ik = rk[row];
+                const int64_t o = ((tok0 + row) * H + h) * D + col;
+                *reinterpret_cast<uint32_t *>(a.dq + o) =
+                    pack_bf16(iq * (dqn[t][2 * hh] - qr.x * iq * sq), iq * (dqn[t][2 * hh + 1] - qr.y * iq * sq));
+                *reinterpret_cast<uint32_t *>(a.dk + o) =
+                    pack_bf16(ik * (dkn[t][2 * hh] - kr.x * ik * sk), ik * (dkn[t][2 * hh + 1] - kr.y * ik * sk));
             }
-            const float iq = w[Ws::RQ + r], ik = w[Ws::RK + r];
-            const int64_t row = ((tok0 + r) * H + h) * D;
-            auto pk = [](float x0, float x1) { return (uint32_t)f2bf(x0) | ((uint32_t)f2bf(x1) << 16); };
-            *reinterpret_cast<uint2 *>(a.dq + row + 4 * lane) =
-                make_uint2(pk(iq * (dqn4.x - qn4.x * sq), iq * (dqn4.y - qn4.y * sq)),
-                           pk(iq * (dqn4.z - qn4.z * sq), iq * (dqn4.w - qn4.w * sq)));
-            *reinterpret_cast<uint2 *>(a.dk + row + 4 * lane) =
-                make_uint2(pk(ik * (dkn4.x - kn4.x * sk), ik * (dkn4.y - kn4.y * sk)),
-                           pk(ik * (dkn4.z - kn4.z * sk), ik * (dkn4.w - kn4.w * sk)));
-            if (lane == 0) a.dbeta[(tok0 + r) * H + h] = w[Ws::DB + r];
         }
+    __syncthreads();   // dG in place
+    // ---- dg = reverse cumsum of dG over the chunk + dG_last (which reaches every row); dbeta ----
+    {
+        const int c = tid & (D - 1), qd = tid >> 7;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = gf[gfi(16 * qd + i, c)];
+#pragma unroll
+        for (int i = 14; i >= 0; --i) x[i] += x[i + 1];
+        tot[qd * D + c] = x[0];
         __syncthreads();
-        float *t = dS;
-        dS = dSn;
-        dSn = t;
+        float off = 0.f;
+#pragma unroll
+        for (int i = 0; i < 6; ++i) off += dglp[i * D + c];
+        for (int q2 = qd + 1; q2 < 4; ++q2) off += tot[q2 * D + c];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * qd + i;
+            if (r < L) a.dg[((tok0 + r) * H + h) * D + c] = x[i] + off;
+        }
+        if (tid < L) {
+            float x = 0.f;
+#pragma unroll
+            for (int i = 0; i < 12; ++i) x += dbp[i * C + tid];
+            a.dbeta[(tok0 + tid) * H + h] = x;
+        }
     }
 }
+}  // namespace grad
 
 }  // namespace bwd
 
+// workspace bytes of the backward: per chunk slot and head, the forward checkpoint, the intra
+// outputs and the dstate outputs
 size_t bwd_workspace_floats(int n_docs, int64_t T, int H) {
-    return ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * bwd::DD + (size_t)n_docs * H * bwd::Ws::TOTAL;
+    return ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * (bwd::Ws::PER_SLOT / sizeof(float));
 }
 
 cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g, const float *beta,
                        const int32_t *cu, int n_docs, int64_t T, int H, const uint16_t *dout, uint16_t *dq,
                        uint16_t *dk, uint16_t *dv, float *dg, float *dbeta, float *workspace, int *status,
                        cudaStream_t stream) {
-    bwd::Args a;
+    using namespace bwd;
+    const size_t blocks = ((size_t)(T / C) + (size_t)n_docs) * (size_t)H;
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    uint8_t *ws_ck = ws, *ws_intra = ws + blocks * Ws::CK, *ws_dst = ws_intra + blocks * Ws::INTRA;
+    // 1. forward with checkpoints (its output o goes to dq, which is overwritten below)
+    cudaError_t e = launch_fwd_pipe(q, k, v, g, beta, cu, n_docs, T, H, nullptr, nullptr, dq, status, stream,
+                                    reinterpret_cast<uint16_t *>(ws_ck));
+    if (e != cudaSuccess) return e;
+    // 2. intra
+    e = cudaFuncSetAttribute(intra::kda_bwd_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             intra::Sm::TOTAL);
+    if (e != cudaSuccess) return e;
+    intra::kda_bwd_intra_kernel<<<(unsigned)blocks, intra::kThreads, intra::Sm::TOTAL, stream>>>(
+        q, k, g, beta, cu, n_docs, T, H, ws_intra);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // 3. dstate
+    e = cudaFuncSetAttribute(dstate::kda_bwd_dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dstate::Sm::TOTAL);
+    if (e != cudaSuccess) return e;
+    dstate::kda_bwd_dstate_kernel<<<(unsigned)(n_docs * H), dstate::kThreads, dstate::Sm::TOTAL, stream>>>(
+        dout, cu, n_docs, T, H, ws_intra, ws_dst, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // 4. grad
+    grad::Args a;
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.g = g; a.beta = beta; a.cu = cu;
     a.n_docs = n_docs; a.T = T; a.H = H;
+    a.ws_ck = ws_ck; a.ws_intra = ws_intra; a.ws_dst = ws_dst;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
-    a.ckpt = workspace;
-    a.scratch = workspace + ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * bwd::DD;
-    a.status = status;
-    // forward pass first: the pipelined forward kernel writes the state entering every chunk into the
-    // checkpoint slots; its output o goes to dq, which the backward overwrites
-    cudaError_t e0 = launch_fwd_pipe(q, k, v, g, beta, cu, n_docs, T, H, nullptr, nullptr, dq, status, stream, a.ckpt);
-    if (e0 != cudaSuccess) return e0;
-    constexpr int smem = (2 * bwd::kOpFloats + 2 * bwd::C * (bwd::C + 1) + 4 * bwd::D) * (int)sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(bwd::kda_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(grad::kda_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad::Sm::TOTAL);
     if (e != cudaSuccess) return e;
-    bwd::kda_bwd_kernel<<<n_docs * H, bwd::kThreads, smem, stream>>>(a);
+    grad::kda_bwd_grad_kernel<<<(unsigned)blocks, grad::kThreads, grad::Sm::TOTAL, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -167,8 +167,9 @@ struct Maps {
     CUtensorMap q, k, g, v, o;
 };
 
-// kCkpt: also store the state entering every chunk into `ckpt` (the backward's checkpoints); a
-// separate instance, so that the plain forward carries no trace of it.
+// kCkpt: also store the state entering every chunk into `ckpt` (the backward's checkpoints: S^T[v][c]
+// as bf16, 128-byte-swizzled atoms of 128 rows v, 32 KB per chunk and head); a separate instance, so
+// that the plain forward carries no trace of it.
 // kMode: what a CTA's token range is -- kDocs: document blockIdx.x / H of cu_seqlens (every plain
 // forward); kSegs: entry blockIdx.x / H of a segment table built on the device (a document cut into
 // pieces, see kda_split.cu), outputs written; kTransition: the same with v taken as zero, the
@@ -177,7 +178,7 @@ template <bool kCkpt, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_pipe_kernel(const __grid_constant__ Maps maps, const float *__restrict__ beta,
                         const int32_t *__restrict__ cu_seqlens, int n_docs, int64_t T, int H,
-                        const float *h0, float *ht, float *ckpt, uint16_t *__restrict__ out,
+                        const float *h0, float *ht, uint16_t *ckpt, uint16_t *__restrict__ out,
                         int *__restrict__ status, const int4 *__restrict__ seg, const int *__restrict__ seg_count,
                         float *ws_states) {
     using S = Smem;
@@ -862,11 +863,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float(&nxt)[16] = (ch & 1) ? sa : sb;
                         if (ch < 7) tc::ld16(lane_base + kSF + 16 * (ch + 1), nxt);
                         if constexpr (kCkpt) {
-                            // the state entering chunk n, S[c][v] fp32, into its checkpoint slot
-                            float *ck = ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) * (kHeadDim * kHeadDim) +
-                                        (size_t)(16 * ch) * kHeadDim + 32 * lq + lane;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) ck[(size_t)i * kHeadDim] = cur[i];
+                            // the state entering chunk n into its checkpoint slot: row v of S^T, channels
+                            // 16ch..16ch+15 as bf16, two 16-byte pieces of the row's 128-byte atom
+                            const int vrow = 32 * lq + lane, m0 = (2 * ch) & 7;
+                            uint8_t *ck = reinterpret_cast<uint8_t *>(ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) *
+                                                                                 (kHeadDim * kHeadDim)) +
+                                          (size_t)(ch >> 2) * (128 * 128) + (size_t)vrow * 128;
+                            *reinterpret_cast<uint4 *>(ck + ((m0 ^ (vrow & 7)) << 4)) = pack8(cur, 1.f);
+                            *reinterpret_cast<uint4 *>(ck + (((m0 + 1) ^ (vrow & 7)) << 4)) = pack8(cur + 8, 1.f);
                         }
                         sprep(cur, 16 * ch);
                         if (ch == 3) state_mma(0);
@@ -1077,7 +1081,7 @@ bool make_maps(pipe_path::Maps &maps, const uint16_t *q, const uint16_t *k, cons
 
 template <bool kCkpt, int kMode>
 cudaError_t launch_mode(const pipe_path::Maps &maps, const float *beta, const int32_t *cu, int n_docs, int64_t T,
-                        int H, const float *h0, float *ht, float *ckpt, uint16_t *out, int *status, const int4 *seg,
+                        int H, const float *h0, float *ht, uint16_t *ckpt, uint16_t *out, int *status, const int4 *seg,
                         const int *seg_count, float *ws_states, int64_t ctas, cudaStream_t stream) {
     using namespace pipe_path;
     constexpr int bytes = Smem::ALLOC;
@@ -1093,7 +1097,7 @@ cudaError_t launch_mode(const pipe_path::Maps &maps, const float *beta, const in
 
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H, const float *h0,
-                            float *ht, uint16_t *out, int *status, cudaStream_t stream, float *ckpt) {
+                            float *ht, uint16_t *out, int *status, cudaStream_t stream, uint16_t *ckpt) {
     using namespace pipe_path;
     Maps maps;
     if (!make_maps(maps, q, k, v, g, out, T, H)) return cudaErrorInvalidValue;

@@ -14,12 +14,13 @@ constexpr int kStatusTimeout = 5;
 // columns, two chunks in flight (intra-chunk work of chunk s overlapped with the
 // state update of chunk s-1).
 // h0 / ht: optional initial / final states, [n_docs * H][128][128] fp32 (NULL: zero / not written).
-// ckpt: optional, receives the state entering every chunk, S[c][v] fp32, in slot
-// (cu[d] / 64 + d + j) * H + h for chunk j of document d (the backward's checkpoint layout).
+// ckpt: optional, receives the state entering every chunk as S^T[v][c] in bf16 (128-byte-swizzled
+// atoms of 128 rows, 16384 values), in slot (cu[d] / 64 + d + j) * H + h for chunk j of document d
+// (the backward's checkpoint layout).
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
                             const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream,
-                            float *ckpt = nullptr);
+                            uint16_t *ckpt = nullptr);
 
 // Segment-table forward (kda_split.cu builds the tables on the device): CTA (entry, head) runs
 // entry blockIdx.x / H of `seg`, {first token, end token, entering-state slot, final-state slot},
