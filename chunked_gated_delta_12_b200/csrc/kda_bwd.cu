@@ -18,14 +18,14 @@
 // work splits into four launches:
 //
 //   1. the pipelined forward kernel (kda_fwd_pipe.cu) in its checkpoint instance: the state
-//      entering every chunk, S^T in bf16;
+//      entering every chunk and the chunk's U~, both transposed, in bf16;
 //   2. intra (one CTA per chunk and head, all chunks at once): norms, G, A_kk and A_qk, T and W,
 //      written as the bf16 tensor-core operands the sweep below reads (-W, A_qk, Kd, QG), plus
 //      T, A_hat and D;
 //   3. dstate (one CTA per document and head, chunks in reverse): the dS recurrence on tcgen05
 //      with dS^T in tensor memory (fp32), writing dS^T and dU~^T of every chunk;
 //   4. grad (one CTA per chunk and head, all chunks at once): every gradient, from the chunk's
-//      inputs, S, dS and dU~, with warp-level bf16 MMAs.
+//      inputs, S, U~, dS and dU~, with warp-level bf16 MMAs.
 //
 // Precision: every product takes bf16 operands with fp32 accumulation; T = (I + A_kk)^-1 and all
 // elementwise work are fp32.  The pairwise-decay sums of dg cancel between their row and column
@@ -58,7 +58,8 @@ constexpr long long kWaitLimit = 2000000000LL;
 // cu[d] / 64 + d + j (unique, below T / 64 + n_docs, found without reading the lengths).
 // ---------------------------------------------------------------------------------------------
 struct Ws {
-    static constexpr size_t CK = 32768;   // forward checkpoint: S^T bf16 [128 v][128 c]
+    static constexpr size_t CK = 49152;   // forward checkpoint: S^T bf16 [128 v][128 c], then U~^T [128 v][64 s]
+    static constexpr size_t CK_UT = 32768;
     // intra outputs
     static constexpr size_t AQ = 0;                   // scale * A_qk bf16 [64 t][64 s]
     static constexpr size_t KD = AQ + 8192;           // Kd bf16 [64 s][128 c]
@@ -190,7 +191,9 @@ __device__ __forceinline__ void copy_out(uint8_t *dst, const uint8_t *src, int b
 }
 
 // =============================================================================================
-// 2. intra: one CTA per (chunk slot, head)
+// 2. intra: one CTA per (chunk slot, head).  Elementwise work maps warp w to rows 8w .. 8w + 7 and
+//    lane l to channels 4l .. 4l + 3, so every global access moves 8 or 16 bytes per lane and all of
+//    a thread's loads are issued before the first use.
 // =============================================================================================
 namespace intra {
 constexpr int kThreads = 256;
@@ -203,10 +206,21 @@ struct Sm {
     static constexpr int AQO = 81920;    // scale * A_qk bf16 [64][64]
     static constexpr int AHO = 90112;    // A_hat bf16 [64][64]
     static constexpr int PS = 98304;     // pair scales fp32 [10][128]
-    static constexpr int GB = PS + 5120; // G (log2 units) at block rows 16R and 16R+15, fp32 [4][2][128]
-    static constexpr int RQ = GB + 4096, RK = RQ + 256, BETA = RK + 256;
+    static constexpr int GT = PS + 5120; // per-row-group totals of G, then block-boundary G: fp32 [8][128]
+    static constexpr int GB = GT + 4096; // G (log2 units) at block rows 16R and 16R+15, fp32 [4][2][128]
+    static constexpr int BETA = GB + 4096;
     static constexpr int TOTAL = BETA + 256;
 };
+
+__device__ __forceinline__ float4 ld4g(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ uint2 ld2g(const uint16_t *p) { return __ldg(reinterpret_cast<const uint2 *>(p)); }
+__device__ __forceinline__ void unpack4(uint2 u, float (&x)[4]) {
+    const float2 a = bf2(u.x), b = bf2(u.y);
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
+    return make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+}
 
 __global__ void __launch_bounds__(kThreads, 2)
 kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const float *beta, const int32_t *cu,
@@ -219,90 +233,150 @@ kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const
     if (!slot_chunk(cu, n_docs, T, slot, doc, tok0, L)) return;
     uint8_t *out = ws_intra + ((size_t)slot * H + h) * Ws::INTRA;
     const uint32_t sbase = smem_u32(sm);
-    float *rq = reinterpret_cast<float *>(sm + Sm::RQ), *rk = reinterpret_cast<float *>(sm + Sm::RK);
     float *sbeta = reinterpret_cast<float *>(sm + Sm::BETA), *gb = reinterpret_cast<float *>(sm + Sm::GB);
-    float *ps = reinterpret_cast<float *>(sm + Sm::PS);
+    float *gt = reinterpret_cast<float *>(sm + Sm::GT), *ps = reinterpret_cast<float *>(sm + Sm::PS);
     float *af = reinterpret_cast<float *>(sm + Sm::AF), *tf = reinterpret_cast<float *>(sm + Sm::TF);
 
-    if (tid < C) sbeta[tid] = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
-    row_norms(q, k, tok0, L, H, h, rq, rk, kThreads / 32);
-
-    // ---- G (log2 units) per channel: thread (c, half) keeps its 32 rows in registers ----
-    const int c = tid & (D - 1), hf = tid >> 7;
-    float g2[32];
-    {
-        float run = 0.f;
+    // ---- this thread's 8 rows x 4 channels of q, k, g (zero past the document end) ----
+    const int c0 = 4 * lane, r0 = 8 * warp;
+    uint2 qr[8], kr[8];
+    float4 gr[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hf + i;
-            run += (r < L ? g[((tok0 + r) * H + h) * D + c] : 0.f) * kLog2e;
-            g2[i] = run;
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + i;
+        if (r < L) {
+            const int64_t o = ((tok0 + r) * H + h) * D + c0;
+            qr[i] = ld2g(q + o);
+            kr[i] = ld2g(k + o);
+            gr[i] = ld4g(g + o);
+        } else {
+            qr[i] = kr[i] = make_uint2(0u, 0u);
+            gr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        // the second half adds the first half's total (passed through the pair-scale buffer)
-        if (hf == 0) ps[c] = run;
-        __syncthreads();
-        const float off = hf ? ps[c] : 0.f;
+    }
+    if (tid < C) sbeta[tid] = tid < L ? __ldg(beta + (tok0 + tid) * H + h) : 0.f;
+    // row norms: the warp holds whole rows
+    float rq[8], rk[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) g2[i] += off;
-        gb[(2 * hf) * 256 + c] = g2[0];
-        gb[(2 * hf) * 256 + 128 + c] = g2[15];
-        gb[(2 * hf + 1) * 256 + c] = g2[16];
-        gb[(2 * hf + 1) * 256 + 128 + c] = g2[31];
-        __syncthreads();
+    for (int i = 0; i < 8; ++i) {
+        float a[4], b[4];
+        unpack4(qr[i], a);
+        unpack4(kr[i], b);
+        float sq = a[0] * a[0] + a[1] * a[1] + a[2] * a[2] + a[3] * a[3];
+        float sk = b[0] * b[0] + b[1] * b[1] + b[2] * b[2] + b[3] * b[3];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        }
+        rq[i] = rsqrtf(sq + 1e-6f);
+        rk[i] = rsqrtf(sk + 1e-6f);
     }
-    const float gl = gb[3 * 256 + 128 + c];   // G at row 63 (= row L - 1: rows past L add zero)
-    // pair scales s_RI = e^{G_16R - G_16I+15}
-    for (int p = 5 * hf; p < 5 * hf + 5; ++p) {
-        const int R = pair_R(p), I = p - R * (R + 1) / 2;
-        ps[p * D + c] = ex2_ftz(gb[R * 256 + c] - gb[I * 256 + 128 + c]);
-    }
-    if (hf == 1) reinterpret_cast<float *>(out + Ws::DL)[c] = ex2_ftz(gl);
-    // operand tiles, one (row, channel) element per step
+    // ---- G (log2 units): running sums over the 8 rows, then the totals of the row groups above ----
+    float g2[8][4];
     {
-        uint8_t *okd = out + Ws::KD, *oqg = out + Ws::QG;
+        float run[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hf + i, R = r >> 4;
-            float qv = 0.f, kv = 0.f;
-            if (r < L) {
-                const int64_t off = ((tok0 + r) * H + h) * D + c;
-                qv = bfl(q[off]) * rq[r];
-                kv = bfl(k[off]) * rk[r];
+        for (int i = 0; i < 8; ++i) {
+            const float x[4] = {gr[i].x, gr[i].y, gr[i].z, gr[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                run[e] += x[e] * kLog2e;
+                g2[i][e] = run[e];
             }
-            const float e1 = ex2_ftz(g2[i] - gb[R * 256 + c]), e2 = ex2_ftz(gb[R * 256 + 128 + c] - g2[i]);
-            const uint32_t o = at(r, c, C);
-            *reinterpret_cast<uint16_t *>(sm + Sm::X + o) = f2b(kv * e1);
-            *reinterpret_cast<uint16_t *>(sm + Sm::Q + o) = f2b(qv * e1);
-            *reinterpret_cast<uint16_t *>(sm + Sm::Y + o) = f2b(kv * e2);
-            *reinterpret_cast<uint16_t *>(okd + o) = f2b(kv * ex2_ftz(gl - g2[i]));
-            *reinterpret_cast<uint16_t *>(oqg + o) = f2b(kScale * qv * ex2_ftz(g2[i]));
         }
+        *reinterpret_cast<float4 *>(gt + warp * D + c0) = make_float4(run[0], run[1], run[2], run[3]);
+        __syncthreads();
+        float off[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int w2 = 0; w2 < warp; ++w2) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(gt + w2 * D + c0);
+            off[0] += t4.x; off[1] += t4.y; off[2] += t4.z; off[3] += t4.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) g2[i][e] += off[e];
+        // block R = warp >> 1 starts in the even warp's first row and ends in the odd warp's last
+        const int R = warp >> 1;
+        const int i_edge = (warp & 1) ? 7 : 0;
+        *reinterpret_cast<float4 *>(gb + R * 256 + (warp & 1) * 128 + c0) =
+            make_float4(g2[i_edge][0], g2[i_edge][1], g2[i_edge][2], g2[i_edge][3]);
+        __syncthreads();
+    }
+    const int R = warp >> 1;
+    float gs[4], ge[4], gl[4];
+    {
+        const float4 a4 = *reinterpret_cast<const float4 *>(gb + R * 256 + c0);
+        const float4 b4 = *reinterpret_cast<const float4 *>(gb + R * 256 + 128 + c0);
+        const float4 l4 = *reinterpret_cast<const float4 *>(gb + 3 * 256 + 128 + c0);   // row 63 (= L - 1 onward)
+        gs[0] = a4.x; gs[1] = a4.y; gs[2] = a4.z; gs[3] = a4.w;
+        ge[0] = b4.x; ge[1] = b4.y; ge[2] = b4.z; ge[3] = b4.w;
+        gl[0] = l4.x; gl[1] = l4.y; gl[2] = l4.z; gl[3] = l4.w;
+    }
+    // pair scales s_RI = e^{G_16R - G_16I+15}: warp w computes pairs w and w + 8
+    for (int p = warp; p < 10; p += 8) {
+        const int PR = pair_R(p), PI = p - PR * (PR + 1) / 2;
+        const float4 a4 = *reinterpret_cast<const float4 *>(gb + PR * 256 + c0);
+        const float4 b4 = *reinterpret_cast<const float4 *>(gb + PI * 256 + 128 + c0);
+        *reinterpret_cast<float4 *>(ps + p * D + c0) =
+            make_float4(ex2_ftz(a4.x - b4.x), ex2_ftz(a4.y - b4.y), ex2_ftz(a4.z - b4.z), ex2_ftz(a4.w - b4.w));
+    }
+    if (warp == 7)
+        *reinterpret_cast<float4 *>(out + Ws::DL + 4 * c0) =
+            make_float4(ex2_ftz(gl[0]), ex2_ftz(gl[1]), ex2_ftz(gl[2]), ex2_ftz(gl[3]));
+    // ---- operand tiles; beta k^ e^G is kept packed until the pair products release its tile ----
+    uint2 bk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + i;
+        float qv[4], kv[4], x[4], y[4], z[4], kd[4], qg[4], b[4];
+        unpack4(qr[i], qv);
+        unpack4(kr[i], kv);
+        const float br = sbeta[r];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float kh = kv[e] * rk[i], qh = qv[e] * rq[i], eg = ex2_ftz(g2[i][e]);
+            const float e1 = ex2_ftz(g2[i][e] - gs[e]);
+            x[e] = kh * e1;
+            y[e] = qh * e1;
+            z[e] = kh * ex2_ftz(ge[e] - g2[i][e]);
+            kd[e] = kh * ex2_ftz(gl[e] - g2[i][e]);
+            qg[e] = kScale * qh * eg;
+            b[e] = br * kh * eg;
+        }
+        const uint32_t o = at(r, c0, C);
+        *reinterpret_cast<uint2 *>(sm + Sm::X + o) = pack4(x);
+        *reinterpret_cast<uint2 *>(sm + Sm::Q + o) = pack4(y);
+        *reinterpret_cast<uint2 *>(sm + Sm::Y + o) = pack4(z);
+        *reinterpret_cast<uint2 *>(out + Ws::KD + o) = pack4(kd);
+        *reinterpret_cast<uint2 *>(out + Ws::QG + o) = pack4(qg);
+        bk[i] = pack4(b);
     }
     __syncthreads();
 
     // ---- A_hat (strictly lower) and A_qk (lower), block pair by block pair (warp MMA) ----
     // block (R, I) = (X_R diag(s_RI)) Y_I^T; the pair scale rides on the A fragment
     for (int p = warp; p < 10; p += kThreads / 32) {
-        const int R = pair_R(p), I = p - R * (R + 1) / 2;
+        const int PR = pair_R(p), PI = p - PR * (PR + 1) / 2;
         float ak[2][4], aq[2][4];
         zero_acc(ak);
         zero_acc(aq);
 #pragma unroll 2
         for (int kk = 0; kk < D; kk += 16) {
             uint32_t fx[4], fq[4], b[4];
-            frag_a<false>(sbase + Sm::X, C, 16 * R, kk, fx);
-            frag_a<false>(sbase + Sm::Q, C, 16 * R, kk, fq);
-            frag_b2<false>(sbase + Sm::Y, C, kk, 16 * I, b);
+            frag_a<false>(sbase + Sm::X, C, 16 * PR, kk, fx);
+            frag_a<false>(sbase + Sm::Q, C, 16 * PR, kk, fq);
+            frag_b2<false>(sbase + Sm::Y, C, kk, 16 * PI, b);
             const float2 s0 = *reinterpret_cast<const float2 *>(ps + p * D + kk + 2 * tq);
             const float2 s1 = *reinterpret_cast<const float2 *>(ps + p * D + kk + 8 + 2 * tq);
             const __nv_bfloat162 h0 = __floats2bfloat162_rn(s0.x, s0.y), h1 = __floats2bfloat162_rn(s1.x, s1.y);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const __nv_bfloat162 sc = (e >> 1) ? h1 : h0;
-                __nv_bfloat162 x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fx[e]), sc);
-                fx[e] = *reinterpret_cast<uint32_t *>(&x);
-                x = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fq[e]), sc);
-                fq[e] = *reinterpret_cast<uint32_t *>(&x);
+                __nv_bfloat162 xx = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fx[e]), sc);
+                fx[e] = *reinterpret_cast<uint32_t *>(&xx);
+                xx = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fq[e]), sc);
+                fq[e] = *reinterpret_cast<uint32_t *>(&xx);
             }
             mma_bf16(ak[0], fx, b[0], b[1]);
             mma_bf16(ak[1], fx, b[2], b[3]);
@@ -313,7 +387,7 @@ kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int row = 16 * R + gq + 8 * hh, col = 16 * I + 8 * nt + 2 * tq;
+                const int row = 16 * PR + gq + 8 * hh, col = 16 * PI + 8 * nt + 2 * tq;
                 const float x0 = col < row ? ak[nt][2 * hh] : 0.f, x1 = col + 1 < row ? ak[nt][2 * hh + 1] : 0.f;
                 const float y0 = col <= row ? kScale * aq[nt][2 * hh] : 0.f;
                 const float y1 = col + 1 <= row ? kScale * aq[nt][2 * hh + 1] : 0.f;
@@ -326,33 +400,27 @@ kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const
     // blocks above the diagonal are zero
     for (int idx = tid; idx < 6 * 256; idx += kThreads) {
         const int b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
-        const int R = b < 3 ? 0 : b < 5 ? 1 : 2, I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-        const int row = 16 * R + rr, col = 16 * I + cc;
+        const int BR = b < 3 ? 0 : b < 5 ? 1 : 2, BI = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
+        const int row = 16 * BR + rr, col = 16 * BI + cc;
         af[row * C + col] = 0.f;
         *reinterpret_cast<uint16_t *>(sm + Sm::AHO + at(row, col, C)) = 0;
         *reinterpret_cast<uint16_t *>(sm + Sm::AQO + at(row, col, C)) = 0;
     }
+    for (int idx = tid; idx < C * C; idx += kThreads) tf[idx] = 0.f;
     __syncthreads();
     copy_out(out + Ws::AQ, sm + Sm::AQO, 8192, kThreads);
     copy_out(out + Ws::AH, sm + Sm::AHO, 8192, kThreads);
-
-    // ---- Bk = beta k^ e^G over the k^ E1 tile (free now) ----
+    // beta k^ e^G over the k^ E1 tile (free now)
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        const float kv = r < L ? bfl(k[((tok0 + r) * H + h) * D + c]) * rk[r] : 0.f;
-        *reinterpret_cast<uint16_t *>(sm + Sm::X + at(r, c, C)) = f2b(sbeta[r] * kv * ex2_ftz(g2[i]));
-    }
+    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint2 *>(sm + Sm::X + at(r0 + i, c0, C)) = bk[i];
 
     // ---- T = (I + A_kk)^-1 by 16 x 16 blocks (fp32) ----
     //   diagonal blocks T_RR = (I + A_RR)^-1, lane = column, row-by-row substitution (warps 0-3);
     //   off-diagonal T_RI = -T_RR sum_{J=I..R-1} A_RJ T_JI by block distance 1, 2, 3
     float *sx = reinterpret_cast<float *>(sm + Sm::Q + 8192);
-    for (int idx = tid; idx < C * C; idx += kThreads) tf[idx] = 0.f;
-    __syncthreads();
     if (warp < 4 && lane < 16) {
-        const int R = warp, cc = lane;
-        const float *b = af + (16 * R) * C + 16 * R;
+        const int BR = warp, cc = lane;
+        const float *b = af + (16 * BR) * C + 16 * BR;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
@@ -362,18 +430,18 @@ kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const
             x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) tf[(16 * R + r) * C + 16 * R + cc] = x[r];
+        for (int r = 0; r < 16; ++r) tf[(16 * BR + r) * C + 16 * BR + cc] = x[r];
     }
     __syncthreads();
 #pragma unroll 1
     for (int dd = 1; dd < 4; ++dd) {
         const int nblk = 4 - dd;
         for (int e = tid; e < nblk * 256; e += kThreads) {
-            const int I = e >> 8, R = I + dd, r = (e >> 4) & 15, cc = e & 15;
+            const int BI = e >> 8, BR = BI + dd, r = (e >> 4) & 15, cc = e & 15;
             float acc = 0.f;
-            for (int J = I; J < R; ++J) {
-                const float *arow = af + (16 * R + r) * C + 16 * J;
-                const float *tcol = tf + (16 * J) * C + 16 * I + cc;
+            for (int J = BI; J < BR; ++J) {
+                const float *arow = af + (16 * BR + r) * C + 16 * J;
+                const float *tcol = tf + (16 * J) * C + 16 * BI + cc;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc = fmaf(arow[i], tcol[i * C], acc);
             }
@@ -381,13 +449,13 @@ kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const
         }
         __syncthreads();
         for (int e = tid; e < nblk * 256; e += kThreads) {
-            const int I = e >> 8, R = I + dd, r = (e >> 4) & 15, cc = e & 15;
-            const float *trow = tf + (16 * R + r) * C + 16 * R;
-            const float *xc = sx + (I << 8) + cc;
+            const int BI = e >> 8, BR = BI + dd, r = (e >> 4) & 15, cc = e & 15;
+            const float *trow = tf + (16 * BR + r) * C + 16 * BR;
+            const float *xc = sx + (BI << 8) + cc;
             float acc = 0.f;
 #pragma unroll
             for (int m = 0; m < 16; ++m) acc = fmaf(trow[m], xc[m * 16], acc);
-            tf[(16 * R + r) * C + 16 * I + cc] = -acc;
+            tf[(16 * BR + r) * C + 16 * BI + cc] = -acc;
         }
         __syncthreads();
     }
@@ -687,8 +755,7 @@ struct Sm {
     static constexpr int DAQ = DST, DT = DST + 8192, XM = DST + 16384, DAH = DST + 24576;
     static constexpr int DUT = 65536;     // dU~^T [128 v][64 s]; then pair scales fp32 [10][128]
     static constexpr int PS = DUT;
-    static constexpr int WN = 81920;      // -W [64 s][128 c]; then k^ E1
-    static constexpr int XT = WN;
+    static constexpr int XT = 81920;      // row-group totals of G (prep); then k^ E1 [64][128]
     static constexpr int TB = 98304;      // T [64 r][64 i]
     static constexpr int AH = 106496;     // A_hat [64 r][64 i]
     static constexpr int DO = 114688;     // dout [64 t][128 v]
@@ -696,7 +763,7 @@ struct Sm {
     static constexpr int QT = BV;
     static constexpr int BK = 147456;     // beta k^ e^G [64][128]; then k^ E2
     static constexpr int YT = BK;
-    static constexpr int UT = 163840;     // U~ [64 s][128 v]
+    static constexpr int UT = 163840;     // U~^T [128 v][64 s]
     static constexpr int GF = 180224;     // G (log2 units) fp32 [64][128], swizzled; then dG
     // partial sums are kept per producing warp and added in a fixed order (bit-reproducible results):
     // DGLP [6][128] dG_last (2 halves of S.dS, 4 row blocks of dKd Kd); DBP [12][64] dbeta (4 column
@@ -740,9 +807,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
 
     // ---- loads: workspace tiles as flat images, dout rows (zero past the document end) ----
     {
-        const uint8_t *src[6] = {ck, dsb + Ws::DS, dsb + Ws::DU, in + Ws::WN, in + Ws::TB, in + Ws::AH};
-        const int dst[6] = {Sm::ST, Sm::DST, Sm::DUT, Sm::WN, Sm::TB, Sm::AH};
-        const int bytes[6] = {32768, 32768, 16384, 16384, 8192, 8192};
+        const uint8_t *src[6] = {ck, ck + Ws::CK_UT, dsb + Ws::DS, dsb + Ws::DU, in + Ws::TB, in + Ws::AH};
+        const int dst[6] = {Sm::ST, Sm::UT, Sm::DST, Sm::DUT, Sm::TB, Sm::AH};
+        const int bytes[6] = {32768, 16384, 32768, 16384, 8192, 8192};
 #pragma unroll
         for (int t = 0; t < 6; ++t)
             for (int i = tid; i < bytes[t] / 16; i += kThreads) cp_async16(sbase + dst[t] + 16 * i, src[t] + 16 * i, 16);
@@ -755,42 +822,85 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         }
         cp_async_commit();
     }
-    if (tid < C) sbeta[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
+    if (tid < C) sbeta[tid] = tid < L ? __ldg(a.beta + (tok0 + tid) * H + h) : 0.f;
     if (tid < D) dls[tid] = reinterpret_cast<const float *>(in + Ws::DL)[tid];
-    row_norms(a.q, a.k, tok0, L, H, h, rq, rk, kThreads / 32);
-    __syncthreads();
 
-    // ---- G (log2 units) per channel, Bk = beta k^ e^G, Bv = beta v: thread (c, block qd) ----
+    // ---- prep: warp w holds rows 4w .. 4w + 3, lane l channels 4l .. 4l + 3: row norms, G (log2
+    //      units), beta k^ e^G and beta v ----
     {
-        const int c = tid & (D - 1), qd = tid >> 7;
-        float x[16];
-        float run = 0.f;
+        const int c0 = 4 * lane, r0 = 4 * warp;
+        uint2 qr[4], kr[4], vr[4];
+        float4 gr[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = 16 * qd + i;
-            run += (r < L ? a.g[((tok0 + r) * H + h) * D + c] : 0.f) * kLog2e;
-            x[i] = run;
-        }
-        tot[qd * D + c] = run;
-        __syncthreads();
-        float off = 0.f;
-        for (int q2 = 0; q2 < qd; ++q2) off += tot[q2 * D + c];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = 16 * qd + i;
-            x[i] += off;
-            gf[gfi(r, c)] = x[i];
-            float kv = 0.f, vv = 0.f;
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
             if (r < L) {
-                const int64_t o = ((tok0 + r) * H + h) * D + c;
-                kv = bfl(a.k[o]) * rk[r];
-                vv = bfl(a.v[o]);
+                const int64_t o = ((tok0 + r) * H + h) * D + c0;
+                qr[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + o));
+                kr[i] = __ldg(reinterpret_cast<const uint2 *>(a.k + o));
+                vr[i] = __ldg(reinterpret_cast<const uint2 *>(a.v + o));
+                gr[i] = __ldg(reinterpret_cast<const float4 *>(a.g + o));
+            } else {
+                qr[i] = kr[i] = vr[i] = make_uint2(0u, 0u);
+                gr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            const uint32_t o2 = at(r, c, C);
-            *reinterpret_cast<uint16_t *>(sm + Sm::BK + o2) = f2b(sbeta[r] * kv * ex2_ftz(x[i]));
-            *reinterpret_cast<uint16_t *>(sm + Sm::BV + o2) = f2b(sbeta[r] * vv);
         }
-        if (qd == 3) gls[c] = x[15];
+        float rkr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 qa = bf2(qr[i].x), qb = bf2(qr[i].y), ka = bf2(kr[i].x), kb = bf2(kr[i].y);
+            float sq = qa.x * qa.x + qa.y * qa.y + qb.x * qb.x + qb.y * qb.y;
+            float sk = ka.x * ka.x + ka.y * ka.y + kb.x * kb.x + kb.y * kb.y;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+            }
+            rkr[i] = rsqrtf(sk + 1e-6f);
+            if (lane == 0) {
+                rq[r0 + i] = rsqrtf(sq + 1e-6f);
+                rk[r0 + i] = rkr[i];
+            }
+        }
+        float g2[4][4], run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float x[4] = {gr[i].x, gr[i].y, gr[i].z, gr[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                run[e] += x[e] * kLog2e;
+                g2[i][e] = run[e];
+            }
+        }
+        float *gt = reinterpret_cast<float *>(sm + Sm::XT);   // [16][128] row-group totals
+        *reinterpret_cast<float4 *>(gt + warp * D + c0) = make_float4(run[0], run[1], run[2], run[3]);
+        __syncthreads();
+        float off[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int w2 = 0; w2 < warp; ++w2) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(gt + w2 * D + c0);
+            off[0] += t4.x; off[1] += t4.y; off[2] += t4.z; off[3] += t4.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
+            float bk[4], bv[4];
+            const float2 ka = bf2(kr[i].x), kb = bf2(kr[i].y), va = bf2(vr[i].x), vb = bf2(vr[i].y);
+            const float kv[4] = {ka.x, ka.y, kb.x, kb.y}, vv[4] = {va.x, va.y, vb.x, vb.y};
+            const float br = sbeta[r];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                g2[i][e] += off[e];
+                bk[e] = br * kv[e] * rkr[i] * ex2_ftz(g2[i][e]);
+                bv[e] = br * vv[e];
+            }
+            *reinterpret_cast<float4 *>(gf + gfi(r, c0)) = make_float4(g2[i][0], g2[i][1], g2[i][2], g2[i][3]);
+            const uint32_t o2 = at(r, c0, C);
+            *reinterpret_cast<uint2 *>(sm + Sm::BK + o2) =
+                make_uint2(pack_bf16(bk[0], bk[1]), pack_bf16(bk[2], bk[3]));
+            *reinterpret_cast<uint2 *>(sm + Sm::BV + o2) =
+                make_uint2(pack_bf16(bv[0], bv[1]), pack_bf16(bv[2], bv[3]));
+        }
+        if (warp == 15) *reinterpret_cast<float4 *>(gls + c0) = make_float4(g2[3][0], g2[3][1], g2[3][2], g2[3][3]);
     }
     cp_async_wait_all();
     __syncthreads();
@@ -828,32 +938,26 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     zero_acc(dqn);
     zero_acc(dG);
     // element (t, e) of a 64 x 128 result: row m0 + gq + 8 (e >> 1), column n0 + 8 t + 2 tq + (e & 1)
-    // raw bf16 pair (row, col..col+1) of q / k / v, zero past the document end
-    auto ld_pair = [&](const uint16_t *p, int row, int col) {
-        return row < L ? bf2(*reinterpret_cast<const uint32_t *>(p + ((tok0 + row) * H + h) * D + col))
-                       : make_float2(0.f, 0.f);
-    };
-
-    // ---- U~ = T (beta V) + (-W) S ----
-    {
-        float acc[4][4];
-        zero_acc(acc);
-        mma_rows<4, false, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::BV, C, n0, 0, C);
-        mma_rows<4, false, false>(acc, sbase + Sm::WN, C, m0, sbase + Sm::ST, D, n0, 0, D);
+    // raw bf16 pairs (row, col..col+1) of q / k / v at this thread's result positions (zero past the
+    // document end), read through the non-coherent path and issued before the product they serve
+    auto ld_pairs = [&](const uint16_t *p, uint32_t (&u)[4][2]) {
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint32_t *>(sm + Sm::UT + at(m0 + gq + 8 * hh, n0 + 8 * t + 2 * tq, C)) =
-                    pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
-    }
-    __syncthreads();
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
+                u[t][hh] = row < L ? __ldg(reinterpret_cast<const unsigned int *>(p + ((tok0 + row) * H + h) * D + col))
+                                   : 0u;
+            }
+    };
 
     // ---- dKd = U~ dS^T: dk^ += dKd e^{G_last - G}, dG -= dKd Kd, dG_last += sum_r dKd Kd ----
     {
+        uint32_t kp[4][2];
+        ld_pairs(a.k, kp);
         float acc[4][4];
         zero_acc(acc);
-        mma_rows<4, false, true>(acc, sbase + Sm::UT, C, m0, sbase + Sm::DST, D, n0, 0, D);
+        mma_rows<4, true, true>(acc, sbase + Sm::UT, D, m0, sbase + Sm::DST, D, n0, 0, D);
         float cs[4][2];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -862,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
             for (int hh = 0; hh < 2; ++hh) {
                 const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
                 const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
-                const float2 kr = ld_pair(a.k, row, col);
+                const float2 kr = bf2(kp[t][hh]);
                 const float ed0 = ex2_ftz(gls[col] - g2.x), ed1 = ex2_ftz(gls[col + 1] - g2.y);
                 const float kd0 = kr.x * rk[row] * ed0, kd1 = kr.y * rk[row] * ed1;
                 const float x0 = acc[t][2 * hh], x1 = acc[t][2 * hh + 1];
@@ -887,6 +991,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     }
     // ---- dQG = scale dO S^T: dq^ += dQG e^G, dG += dQG QG ----
     {
+        uint32_t qp[4][2];
+        ld_pairs(a.q, qp);
         float acc[4][4];
         zero_acc(acc);
         mma_rows<4, false, true>(acc, sbase + Sm::DO, C, m0, sbase + Sm::ST, D, n0, 0, D);
@@ -896,7 +1002,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
             for (int hh = 0; hh < 2; ++hh) {
                 const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
                 const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
-                const float2 qr = ld_pair(a.q, row, col);
+                const float2 qr = bf2(qp[t][hh]);
                 const float e0 = ex2_ftz(g2.x), e1 = ex2_ftz(g2.y);
                 const float x0 = kScale * acc[t][2 * hh], x1 = kScale * acc[t][2 * hh + 1];
                 dqn[t][2 * hh] += x0 * e0;
@@ -923,7 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     {
         float acc[2][4];
         zero_acc(acc);
-        mma_rows<2, false, false>(acc, sbase + Sm::DO, C, m0, sbase + Sm::UT, C, n64, 0, D);
+        mma_rows<2, false, true>(acc, sbase + Sm::DO, C, m0, sbase + Sm::UT, D, n64, 0, D);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -950,6 +1056,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     }
     // ---- dBk = T^T dW: dKG = beta dBk; dk^ += dKG e^G, dG += dKG KG, dbeta += dBk . KG ----
     {
+        uint32_t kp[4][2];
+        ld_pairs(a.k, kp);
         float acc[4][4];
         zero_acc(acc);
         mma_rows<4, true, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::ST, C, n0, 0, C);
@@ -960,7 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
             for (int hh = 0; hh < 2; ++hh) {
                 const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
                 const float2 g2 = *reinterpret_cast<const float2 *>(gf + gfi(row, col));
-                const float2 kr = ld_pair(a.k, row, col);
+                const float2 kr = bf2(kp[t][hh]);
                 const float e0 = ex2_ftz(g2.x), e1 = ex2_ftz(g2.y);
                 const float kg0 = kr.x * rk[row] * e0, kg1 = kr.y * rk[row] * e1;
                 const float b = sbeta[row];
@@ -981,6 +1089,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     }
     // ---- dBv = T^T dU~: dv = beta dBv, dbeta += dBv . v ----
     {
+        uint32_t vp[4][2];
+        ld_pairs(a.v, vp);
         float acc[4][4];
         zero_acc(acc);
         mma_rows<4, true, false>(acc, sbase + Sm::TB, C, m0, sbase + Sm::DUT, D, n0, 0, C);
@@ -992,7 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
                 const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
                 const float x0 = acc[t][2 * hh], x1 = acc[t][2 * hh + 1];
                 if (row < L) {
-                    const float2 vr = ld_pair(a.v, row, col);
+                    const float2 vr = bf2(vp[t][hh]);
                     rs[hh] += x0 * vr.x + x1 * vr.y;
                     const float b = sbeta[row];
                     *reinterpret_cast<uint32_t *>(a.dv + ((tok0 + row) * H + h) * D + col) = pack_bf16(b * x0, b * x1);
@@ -1019,29 +1129,52 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
                 *reinterpret_cast<uint32_t *>(sm + Sm::XM + at(m0 + gq + 8 * hh, n64 + 8 * t + 2 * tq, C)) =
                     pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
     }
-    // ---- k^ E1, q^ E1, k^ E2 (the pairwise-decay operands, bf16) and the pair scales ----
+    // ---- k^ E1, q^ E1, k^ E2 (the pairwise-decay operands, bf16) and the pair scales: warp w holds
+    //      rows 4w .. 4w + 3, lane l channels 4l .. 4l + 3 ----
     {
-        const int c = tid & (D - 1), qd = tid >> 7;
-        const float gs = gf[gfi(16 * qd, c)], ge = gf[gfi(16 * qd + 15, c)];
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const int r = 16 * qd + i;
-            float kv = 0.f, qv = 0.f;
+        const int c0 = 4 * lane, r0 = 4 * warp, BR = warp >> 2;
+        uint2 qr[4], kr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
             if (r < L) {
-                const int64_t o = ((tok0 + r) * H + h) * D + c;
-                kv = bfl(a.k[o]) * rk[r];
-                qv = bfl(a.q[o]) * rq[r];
+                const int64_t o = ((tok0 + r) * H + h) * D + c0;
+                qr[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + o));
+                kr[i] = __ldg(reinterpret_cast<const uint2 *>(a.k + o));
+            } else {
+                qr[i] = kr[i] = make_uint2(0u, 0u);
             }
-            const float g2 = gf[gfi(r, c)];
-            const float e1 = ex2_ftz(g2 - gs), e2 = ex2_ftz(ge - g2);
-            const uint32_t o2 = at(r, c, C);
-            *reinterpret_cast<uint16_t *>(sm + Sm::XT + o2) = f2b(kv * e1);
-            *reinterpret_cast<uint16_t *>(sm + Sm::QT + o2) = f2b(qv * e1);
-            *reinterpret_cast<uint16_t *>(sm + Sm::YT + o2) = f2b(kv * e2);
         }
-        for (int p = qd; p < 10; p += 4) {
-            const int R = pair_R(p), I = p - R * (R + 1) / 2;
-            ps[p * D + c] = ex2_ftz(gf[gfi(16 * R, c)] - gf[gfi(16 * I + 15, c)]);
+        const float4 gs4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * BR, c0));
+        const float4 ge4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * BR + 15, c0));
+        const float gs[4] = {gs4.x, gs4.y, gs4.z, gs4.w}, ge[4] = {ge4.x, ge4.y, ge4.z, ge4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
+            const float4 g4 = *reinterpret_cast<const float4 *>(gf + gfi(r, c0));
+            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+            const float2 qa = bf2(qr[i].x), qb = bf2(qr[i].y), ka = bf2(kr[i].x), kb = bf2(kr[i].y);
+            const float qv[4] = {qa.x, qa.y, qb.x, qb.y}, kv[4] = {ka.x, ka.y, kb.x, kb.y};
+            const float iq = rq[r], ik = rk[r];
+            float x[4], y[4], z[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float e1 = ex2_ftz(gv[e] - gs[e]);
+                x[e] = kv[e] * ik * e1;
+                y[e] = qv[e] * iq * e1;
+                z[e] = kv[e] * ik * ex2_ftz(ge[e] - gv[e]);
+            }
+            const uint32_t o2 = at(r, c0, C);
+            *reinterpret_cast<uint2 *>(sm + Sm::XT + o2) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+            *reinterpret_cast<uint2 *>(sm + Sm::QT + o2) = make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
+            *reinterpret_cast<uint2 *>(sm + Sm::YT + o2) = make_uint2(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]));
+        }
+        if (warp < 10) {
+            const int PR = pair_R(warp), PI = warp - PR * (PR + 1) / 2;
+            const float4 a4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * PR, c0));
+            const float4 b4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * PI + 15, c0));
+            *reinterpret_cast<float4 *>(ps + warp * D + c0) =
+                make_float4(ex2_ftz(a4.x - b4.x), ex2_ftz(a4.y - b4.y), ex2_ftz(a4.z - b4.z), ex2_ftz(a4.w - b4.w));
         }
     }
     __syncthreads();   // Xm in place
@@ -1115,6 +1248,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
                 dG[t][2 * hh + 1] += xt.y * p1[t][2 * hh + 1] + qt.y * p3[t][2 * hh + 1];
             }
     }
+    uint32_t qf[4][2], kf[4][2];   // q and k at the result positions, for the final phase
+    ld_pairs(a.q, qf);
+    ld_pairs(a.k, kf);
     {
         float p24[4][4];
         zero_acc(p24);
@@ -1154,8 +1290,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         for (int t = 0; t < 4; ++t)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int row = m0 + gq + 8 * hh, col = n0 + 8 * t + 2 * tq;
-                const float2 qr = ld_pair(a.q, row, col), kr = ld_pair(a.k, row, col);
+                const int row = m0 + gq + 8 * hh;
+                const float2 qr = bf2(qf[t][hh]), kr = bf2(kf[t][hh]);
                 sq[hh] += rq[row] * (qr.x * dqn[t][2 * hh] + qr.y * dqn[t][2 * hh + 1]);
                 sk[hh] += rk[row] * (kr.x * dkn[t][2 * hh] + kr.y * dkn[t][2 * hh + 1]);
             }
@@ -1183,7 +1319,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
                 const float4 s4 = *reinterpret_cast<const float4 *>(red + row * 4);
                 const float4 k4 = *reinterpret_cast<const float4 *>(red + 256 + row * 4);
                 const float sq = s4.x + s4.y + s4.z + s4.w, sk = k4.x + k4.y + k4.z + k4.w;
-                const float2 qr = ld_pair(a.q, row, col), kr = ld_pair(a.k, row, col);
+                const float2 qr = bf2(qf[t][hh]), kr = bf2(kf[t][hh]);
                 const float iq = rq[row], ik = rk[row];
                 const int64_t o = ((tok0 + row) * H + h) * D + col;
                 *reinterpret_cast<uint32_t *>(a.dq + o) =

@@ -42,6 +42,7 @@ namespace kda {
 namespace pipe_path {
 
 constexpr int kThreads = 512;
+constexpr size_t kCkptElems = 128 * 128 + 128 * 64;   // bf16 values per checkpoint slot: S^T, then U~^T
 constexpr int kStateTid0 = 384;               // first thread of warps 12-15
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSF = 0;                   // S^T fp32          [128 lanes v][128 cols c]
@@ -167,9 +168,9 @@ struct Maps {
     CUtensorMap q, k, g, v, o;
 };
 
-// kCkpt: also store the state entering every chunk into `ckpt` (the backward's checkpoints: S^T[v][c]
-// as bf16, 128-byte-swizzled atoms of 128 rows v, 32 KB per chunk and head); a separate instance, so
-// that the plain forward carries no trace of it.
+// kCkpt: also store, per chunk and head, the state entering the chunk and the chunk's U~ into `ckpt`
+// (the backward's checkpoints: S^T[v][c] and U~^T[v][s] as bf16 in 128-byte-swizzled atoms of 128
+// rows v, 32 KB + 16 KB); a separate instance, so that the plain forward carries no trace of it.
 // kMode: what a CTA's token range is -- kDocs: document blockIdx.x / H of cu_seqlens (every plain
 // forward); kSegs: entry blockIdx.x / H of a segment table built on the device (a document cut into
 // pieces, see kda_split.cu), outputs written; kTransition: the same with v taken as zero, the
@@ -867,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // 16ch..16ch+15 as bf16, two 16-byte pieces of the row's 128-byte atom
                             const int vrow = 32 * lq + lane, m0 = (2 * ch) & 7;
                             uint8_t *ck = reinterpret_cast<uint8_t *>(ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) *
-                                                                                 (kHeadDim * kHeadDim)) +
+                                                                                 kCkptElems) +
                                           (size_t)(ch >> 2) * (128 * 128) + (size_t)vrow * 128;
                             *reinterpret_cast<uint4 *>(ck + ((m0 ^ (vrow & 7)) << 4)) = pack8(cur, 1.f);
                             *reinterpret_cast<uint4 *>(ck + (((m0 + 1) ^ (vrow & 7)) << 4)) = pack8(cur + 8, 1.f);
@@ -899,6 +900,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(u[2 * i], u[2 * i + 1]);
                         st16(lane_base + kUB + 16 * h2, pk);
+                        if constexpr (kCkpt) {
+                            // U~^T row v, s = 32 h2 .. 32 h2 + 31, after the chunk's S^T in its checkpoint slot
+                            const int vrow = 32 * lq + lane;
+                            uint8_t *cu8 = reinterpret_cast<uint8_t *>(ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) *
+                                                                                  kCkptElems + kHeadDim * kHeadDim) +
+                                           (size_t)vrow * 128;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                *reinterpret_cast<uint4 *>(cu8 + (((4 * h2 + e) ^ (vrow & 7)) << 4)) =
+                                    make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        }
                     }
                     tc::wait_st();
                 }
