@@ -15,17 +15,16 @@
 //
 // and then the chain rule through beta, the pairwise decays e^{G_r - G_i}, the factors e^G, the
 // in-chunk cumsum (dg = reverse cumsum of dG) and the l2 norms.  Only dS crosses chunks, so the
-// work splits into four launches:
+// work splits into three launches:
 //
-//   1. the pipelined forward kernel (kda_fwd_pipe.cu) in its checkpoint instance: the state
-//      entering every chunk and the chunk's U~, both transposed, in bf16;
-//   2. intra (one CTA per chunk and head, all chunks at once): norms, G, A_kk and A_qk, T and W,
-//      written as the bf16 tensor-core operands the sweep below reads (-W, A_qk, Kd, QG), plus
-//      T, A_hat and D;
-//   3. dstate (one CTA per document and head, chunks in reverse): the dS recurrence on tcgen05
-//      with dS^T in tensor memory (fp32), writing dS^T and dU~^T of every chunk;
-//   4. grad (one CTA per chunk and head, all chunks at once): every gradient, from the chunk's
-//      inputs, S, U~, dS and dU~, with warp-level bf16 MMAs.
+//   1. the pipelined forward kernel (kda_fwd_pipe.cu) in its checkpoint instance: per chunk, the
+//      state entering it and its U~ (transposed, bf16), the tensor-core operand tiles it built
+//      anyway ([-W^T | scale QG^T], Kd^T, scale A_qk, bf16), T and A_hat (bf16) and D (fp32);
+//   2. dstate (one CTA per document and head, chunks in reverse): the dS recurrence on tcgen05
+//      with dS^T in tensor memory (fp32), its operands copied from the checkpoint block as flat
+//      images, writing dS^T and dU~^T of every chunk;
+//   3. grad (one CTA per chunk and head, all chunks at once): every gradient, from the chunk's
+//      inputs, S, U~, T, A_hat, dS and dU~, with warp-level bf16 MMAs.
 //
 // Precision: every product takes bf16 operands with fp32 accumulation; T = (I + A_kk)^-1 and all
 // elementwise work are fp32.  The pairwise-decay sums of dg cancel between their row and column
@@ -58,22 +57,21 @@ constexpr long long kWaitLimit = 2000000000LL;
 // cu[d] / 64 + d + j (unique, below T / 64 + n_docs, found without reading the lengths).
 // ---------------------------------------------------------------------------------------------
 struct Ws {
-    static constexpr size_t CK = 49152;   // forward checkpoint: S^T bf16 [128 v][128 c], then U~^T [128 v][64 s]
-    static constexpr size_t CK_UT = 32768;
-    // intra outputs
-    static constexpr size_t AQ = 0;                   // scale * A_qk bf16 [64 t][64 s]
-    static constexpr size_t KD = AQ + 8192;           // Kd bf16 [64 s][128 c]
-    static constexpr size_t QG = KD + 16384;          // scale * QG bf16 [64 t][128 c]
-    static constexpr size_t WN = QG + 16384;          // -W bf16 [64 s][128 c]
-    static constexpr size_t TB = WN + 16384;          // T bf16 [64 r][64 i]
-    static constexpr size_t AH = TB + 8192;           // A_hat bf16 [64 r][64 i] (strictly lower, no beta)
-    static constexpr size_t DL = AH + 8192;           // D = e^{G_last} fp32 [128]
-    static constexpr size_t INTRA = DL + 1024;
+    // forward checkpoint block (written by the forward kernel's checkpoint instance)
+    static constexpr size_t S = 0;                    // S^T bf16 [128 v][128 c]
+    static constexpr size_t UT = 32768;               // U~^T bf16 [128 v][64 s]
+    static constexpr size_t B2 = 49152;               // [-W^T | scale QG^T] bf16 [128 c][64 s | 64 t]
+    static constexpr size_t KD = 81920;               // Kd^T bf16 [128 c][64 s]
+    static constexpr size_t AQ = 98304;               // scale A_qk bf16 [64 t][64 s]
+    static constexpr size_t TB = 106496;              // T bf16 [64 r][64 i]
+    static constexpr size_t AH = 114688;              // A_hat bf16 [64 r][64 i], valid below the diagonal
+    static constexpr size_t DL = 122880;              // D = e^{G_last} fp32 [128]
+    static constexpr size_t CK = 123904;
     // dstate outputs
     static constexpr size_t DS = 0;                   // dS^T bf16 [128 v][128 c] (dS leaving the chunk)
     static constexpr size_t DU = DS + 32768;          // dU~^T bf16 [128 v][64 s]
     static constexpr size_t DST = DU + 16384;
-    static constexpr size_t PER_SLOT = CK + INTRA + DST;
+    static constexpr size_t PER_SLOT = CK + DST;
 };
 
 // byte offset of bf16 element (row, col) in a tile of `rows` rows (128-byte swizzled atoms)
@@ -117,6 +115,48 @@ __device__ __forceinline__ void mma_rows(float (&acc)[NT][4], uint32_t a_base, i
             frag_b2<kBT>(b_base, b_rows, k, n0 + 8 * t, b);
             mma_bf16(acc[t], a, b[0], b[1]);
             mma_bf16(acc[t + 1], a, b[2], b[3]);
+        }
+    }
+}
+// The same product with compile-time tile heights (AR, BR rows) and k range [K0, K1): addresses are
+// per-thread constants plus compile-time offsets.  For a 16-aligned k the swizzled chunk of a lane's
+// 16-byte row piece is ((k >> 3) & 7) ^ key with a per-thread key, and moving along the row index
+// of a tile is a plain multiple of 128 bytes.
+template <int NT, bool kAT, bool kBT, int AR, int BR, int K0, int K1>
+__device__ __forceinline__ void mma_fix(float (&acc)[NT][4], uint32_t a_base, int m0, uint32_t b_base, int n0) {
+    const int lane = threadIdx.x & 31, r = lane & 7, jlo = (lane >> 3) & 1, jhi = lane >> 4;
+    uint32_t a_p, a_key4 = 0;
+    if constexpr (!kAT) {
+        a_p = a_base + (uint32_t)((m0 + jlo * 8 + r) * 128);
+        a_key4 = (uint32_t)((jhi ^ r) << 4);
+    } else {
+        a_p = a_base + (uint32_t)((m0 >> 6) * AR * 128 + (jhi * 8 + r) * 128 + ((((m0 >> 3) & 7) ^ jlo ^ r) << 4));
+    }
+    uint32_t b_p[NT / 2];
+    const uint32_t b_key4 = (uint32_t)((jlo ^ r) << 4);
+#pragma unroll
+    for (int tt = 0; tt < NT / 2; ++tt) {
+        const int n = n0 + 16 * tt;
+        if constexpr (!kBT) b_p[tt] = b_base + (uint32_t)((n + jhi * 8 + r) * 128);
+        else b_p[tt] = b_base + (uint32_t)((n >> 6) * BR * 128 + (jlo * 8 + r) * 128 + ((((n >> 3) & 7) ^ jhi ^ r) << 4));
+    }
+#pragma unroll
+    for (int k = K0; k < K1; k += 16) {
+        uint32_t a[4];
+        if constexpr (!kAT)
+            ldsm_x4(a_p + (uint32_t)((k >> 6) * AR * 128) + ((uint32_t)(((k >> 3) & 7) << 4) ^ a_key4), a[0], a[1], a[2], a[3]);
+        else
+            ldsm_x4_t(a_p + (uint32_t)(k * 128), a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int tt = 0; tt < NT / 2; ++tt) {
+            uint32_t b[4];
+            if constexpr (!kBT)
+                ldsm_x4(b_p[tt] + (uint32_t)((k >> 6) * BR * 128) + ((uint32_t)(((k >> 3) & 7) << 4) ^ b_key4), b[0], b[1],
+                        b[2], b[3]);
+            else
+                ldsm_x4_t(b_p[tt] + (uint32_t)(k * 128), b[0], b[1], b[2], b[3]);
+            mma_bf16(acc[2 * tt], a, b[0], b[1]);
+            mma_bf16(acc[2 * tt + 1], a, b[2], b[3]);
         }
     }
 }
@@ -191,303 +231,7 @@ __device__ __forceinline__ void copy_out(uint8_t *dst, const uint8_t *src, int b
 }
 
 // =============================================================================================
-// 2. intra: one CTA per (chunk slot, head).  Elementwise work maps warp w to rows 8w .. 8w + 7 and
-//    lane l to channels 4l .. 4l + 3, so every global access moves 8 or 16 bytes per lane and all of
-//    a thread's loads are issued before the first use.
-// =============================================================================================
-namespace intra {
-constexpr int kThreads = 256;
-struct Sm {
-    static constexpr int X = 0;          // k^ E1 bf16 [64][128]; then beta k^ e^G (Bk)
-    static constexpr int Q = 16384;      // q^ E1; then T bf16 [64][64] (+0) and solve scratch (+8192)
-    static constexpr int Y = 32768;      // k^ E2; then -W bf16 [64][128]
-    static constexpr int AF = 49152;     // A_kk fp32 [64][64]
-    static constexpr int TF = 65536;     // T fp32 [64][64]
-    static constexpr int AQO = 81920;    // scale * A_qk bf16 [64][64]
-    static constexpr int AHO = 90112;    // A_hat bf16 [64][64]
-    static constexpr int PS = 98304;     // pair scales fp32 [10][128]
-    static constexpr int GT = PS + 5120; // per-row-group totals of G, then block-boundary G: fp32 [8][128]
-    static constexpr int GB = GT + 4096; // G (log2 units) at block rows 16R and 16R+15, fp32 [4][2][128]
-    static constexpr int BETA = GB + 4096;
-    static constexpr int TOTAL = BETA + 256;
-};
-
-__device__ __forceinline__ float4 ld4g(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
-__device__ __forceinline__ uint2 ld2g(const uint16_t *p) { return __ldg(reinterpret_cast<const uint2 *>(p)); }
-__device__ __forceinline__ void unpack4(uint2 u, float (&x)[4]) {
-    const float2 a = bf2(u.x), b = bf2(u.y);
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
-__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
-    return make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
-}
-
-__global__ void __launch_bounds__(kThreads, 2)
-kda_bwd_intra_kernel(const uint16_t *q, const uint16_t *k, const float *g, const float *beta, const int32_t *cu,
-                     int n_docs, int64_t T, int H, uint8_t *ws_intra) {
-    extern __shared__ __align__(1024) uint8_t sm[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const int slot = blockIdx.x / H, h = blockIdx.x % H;
-    int doc, L;
-    int64_t tok0;
-    if (!slot_chunk(cu, n_docs, T, slot, doc, tok0, L)) return;
-    uint8_t *out = ws_intra + ((size_t)slot * H + h) * Ws::INTRA;
-    const uint32_t sbase = smem_u32(sm);
-    float *sbeta = reinterpret_cast<float *>(sm + Sm::BETA), *gb = reinterpret_cast<float *>(sm + Sm::GB);
-    float *gt = reinterpret_cast<float *>(sm + Sm::GT), *ps = reinterpret_cast<float *>(sm + Sm::PS);
-    float *af = reinterpret_cast<float *>(sm + Sm::AF), *tf = reinterpret_cast<float *>(sm + Sm::TF);
-
-    // ---- this thread's 8 rows x 4 channels of q, k, g (zero past the document end) ----
-    const int c0 = 4 * lane, r0 = 8 * warp;
-    uint2 qr[8], kr[8];
-    float4 gr[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = r0 + i;
-        if (r < L) {
-            const int64_t o = ((tok0 + r) * H + h) * D + c0;
-            qr[i] = ld2g(q + o);
-            kr[i] = ld2g(k + o);
-            gr[i] = ld4g(g + o);
-        } else {
-            qr[i] = kr[i] = make_uint2(0u, 0u);
-            gr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
-    if (tid < C) sbeta[tid] = tid < L ? __ldg(beta + (tok0 + tid) * H + h) : 0.f;
-    // row norms: the warp holds whole rows
-    float rq[8], rk[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float a[4], b[4];
-        unpack4(qr[i], a);
-        unpack4(kr[i], b);
-        float sq = a[0] * a[0] + a[1] * a[1] + a[2] * a[2] + a[3] * a[3];
-        float sk = b[0] * b[0] + b[1] * b[1] + b[2] * b[2] + b[3] * b[3];
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            sk += __shfl_xor_sync(0xffffffffu, sk, o);
-        }
-        rq[i] = rsqrtf(sq + 1e-6f);
-        rk[i] = rsqrtf(sk + 1e-6f);
-    }
-    // ---- G (log2 units): running sums over the 8 rows, then the totals of the row groups above ----
-    float g2[8][4];
-    {
-        float run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float x[4] = {gr[i].x, gr[i].y, gr[i].z, gr[i].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                run[e] += x[e] * kLog2e;
-                g2[i][e] = run[e];
-            }
-        }
-        *reinterpret_cast<float4 *>(gt + warp * D + c0) = make_float4(run[0], run[1], run[2], run[3]);
-        __syncthreads();
-        float off[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int w2 = 0; w2 < warp; ++w2) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(gt + w2 * D + c0);
-            off[0] += t4.x; off[1] += t4.y; off[2] += t4.z; off[3] += t4.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) g2[i][e] += off[e];
-        // block R = warp >> 1 starts in the even warp's first row and ends in the odd warp's last
-        const int R = warp >> 1;
-        const int i_edge = (warp & 1) ? 7 : 0;
-        *reinterpret_cast<float4 *>(gb + R * 256 + (warp & 1) * 128 + c0) =
-            make_float4(g2[i_edge][0], g2[i_edge][1], g2[i_edge][2], g2[i_edge][3]);
-        __syncthreads();
-    }
-    const int R = warp >> 1;
-    float gs[4], ge[4], gl[4];
-    {
-        const float4 a4 = *reinterpret_cast<const float4 *>(gb + R * 256 + c0);
-        const float4 b4 = *reinterpret_cast<const float4 *>(gb + R * 256 + 128 + c0);
-        const float4 l4 = *reinterpret_cast<const float4 *>(gb + 3 * 256 + 128 + c0);   // row 63 (= L - 1 onward)
-        gs[0] = a4.x; gs[1] = a4.y; gs[2] = a4.z; gs[3] = a4.w;
-        ge[0] = b4.x; ge[1] = b4.y; ge[2] = b4.z; ge[3] = b4.w;
-        gl[0] = l4.x; gl[1] = l4.y; gl[2] = l4.z; gl[3] = l4.w;
-    }
-    // pair scales s_RI = e^{G_16R - G_16I+15}: warp w computes pairs w and w + 8
-    for (int p = warp; p < 10; p += 8) {
-        const int PR = pair_R(p), PI = p - PR * (PR + 1) / 2;
-        const float4 a4 = *reinterpret_cast<const float4 *>(gb + PR * 256 + c0);
-        const float4 b4 = *reinterpret_cast<const float4 *>(gb + PI * 256 + 128 + c0);
-        *reinterpret_cast<float4 *>(ps + p * D + c0) =
-            make_float4(ex2_ftz(a4.x - b4.x), ex2_ftz(a4.y - b4.y), ex2_ftz(a4.z - b4.z), ex2_ftz(a4.w - b4.w));
-    }
-    if (warp == 7)
-        *reinterpret_cast<float4 *>(out + Ws::DL + 4 * c0) =
-            make_float4(ex2_ftz(gl[0]), ex2_ftz(gl[1]), ex2_ftz(gl[2]), ex2_ftz(gl[3]));
-    // ---- operand tiles; beta k^ e^G is kept packed until the pair products release its tile ----
-    uint2 bk[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = r0 + i;
-        float qv[4], kv[4], x[4], y[4], z[4], kd[4], qg[4], b[4];
-        unpack4(qr[i], qv);
-        unpack4(kr[i], kv);
-        const float br = sbeta[r];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float kh = kv[e] * rk[i], qh = qv[e] * rq[i], eg = ex2_ftz(g2[i][e]);
-            const float e1 = ex2_ftz(g2[i][e] - gs[e]);
-            x[e] = kh * e1;
-            y[e] = qh * e1;
-            z[e] = kh * ex2_ftz(ge[e] - g2[i][e]);
-            kd[e] = kh * ex2_ftz(gl[e] - g2[i][e]);
-            qg[e] = kScale * qh * eg;
-            b[e] = br * kh * eg;
-        }
-        const uint32_t o = at(r, c0, C);
-        *reinterpret_cast<uint2 *>(sm + Sm::X + o) = pack4(x);
-        *reinterpret_cast<uint2 *>(sm + Sm::Q + o) = pack4(y);
-        *reinterpret_cast<uint2 *>(sm + Sm::Y + o) = pack4(z);
-        *reinterpret_cast<uint2 *>(out + Ws::KD + o) = pack4(kd);
-        *reinterpret_cast<uint2 *>(out + Ws::QG + o) = pack4(qg);
-        bk[i] = pack4(b);
-    }
-    __syncthreads();
-
-    // ---- A_hat (strictly lower) and A_qk (lower), block pair by block pair (warp MMA) ----
-    // block (R, I) = (X_R diag(s_RI)) Y_I^T; the pair scale rides on the A fragment
-    for (int p = warp; p < 10; p += kThreads / 32) {
-        const int PR = pair_R(p), PI = p - PR * (PR + 1) / 2;
-        float ak[2][4], aq[2][4];
-        zero_acc(ak);
-        zero_acc(aq);
-#pragma unroll 2
-        for (int kk = 0; kk < D; kk += 16) {
-            uint32_t fx[4], fq[4], b[4];
-            frag_a<false>(sbase + Sm::X, C, 16 * PR, kk, fx);
-            frag_a<false>(sbase + Sm::Q, C, 16 * PR, kk, fq);
-            frag_b2<false>(sbase + Sm::Y, C, kk, 16 * PI, b);
-            const float2 s0 = *reinterpret_cast<const float2 *>(ps + p * D + kk + 2 * tq);
-            const float2 s1 = *reinterpret_cast<const float2 *>(ps + p * D + kk + 8 + 2 * tq);
-            const __nv_bfloat162 h0 = __floats2bfloat162_rn(s0.x, s0.y), h1 = __floats2bfloat162_rn(s1.x, s1.y);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 sc = (e >> 1) ? h1 : h0;
-                __nv_bfloat162 xx = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fx[e]), sc);
-                fx[e] = *reinterpret_cast<uint32_t *>(&xx);
-                xx = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&fq[e]), sc);
-                fq[e] = *reinterpret_cast<uint32_t *>(&xx);
-            }
-            mma_bf16(ak[0], fx, b[0], b[1]);
-            mma_bf16(ak[1], fx, b[2], b[3]);
-            mma_bf16(aq[0], fq, b[0], b[1]);
-            mma_bf16(aq[1], fq, b[2], b[3]);
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int row = 16 * PR + gq + 8 * hh, col = 16 * PI + 8 * nt + 2 * tq;
-                const float x0 = col < row ? ak[nt][2 * hh] : 0.f, x1 = col + 1 < row ? ak[nt][2 * hh + 1] : 0.f;
-                const float y0 = col <= row ? kScale * aq[nt][2 * hh] : 0.f;
-                const float y1 = col + 1 <= row ? kScale * aq[nt][2 * hh + 1] : 0.f;
-                const float br = sbeta[row];
-                *reinterpret_cast<float2 *>(af + row * C + col) = make_float2(br * x0, br * x1);
-                *reinterpret_cast<uint32_t *>(sm + Sm::AHO + at(row, col, C)) = pack_bf16(x0, x1);
-                *reinterpret_cast<uint32_t *>(sm + Sm::AQO + at(row, col, C)) = pack_bf16(y0, y1);
-            }
-    }
-    // blocks above the diagonal are zero
-    for (int idx = tid; idx < 6 * 256; idx += kThreads) {
-        const int b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
-        const int BR = b < 3 ? 0 : b < 5 ? 1 : 2, BI = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
-        const int row = 16 * BR + rr, col = 16 * BI + cc;
-        af[row * C + col] = 0.f;
-        *reinterpret_cast<uint16_t *>(sm + Sm::AHO + at(row, col, C)) = 0;
-        *reinterpret_cast<uint16_t *>(sm + Sm::AQO + at(row, col, C)) = 0;
-    }
-    for (int idx = tid; idx < C * C; idx += kThreads) tf[idx] = 0.f;
-    __syncthreads();
-    copy_out(out + Ws::AQ, sm + Sm::AQO, 8192, kThreads);
-    copy_out(out + Ws::AH, sm + Sm::AHO, 8192, kThreads);
-    // beta k^ e^G over the k^ E1 tile (free now)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint2 *>(sm + Sm::X + at(r0 + i, c0, C)) = bk[i];
-
-    // ---- T = (I + A_kk)^-1 by 16 x 16 blocks (fp32) ----
-    //   diagonal blocks T_RR = (I + A_RR)^-1, lane = column, row-by-row substitution (warps 0-3);
-    //   off-diagonal T_RI = -T_RR sum_{J=I..R-1} A_RJ T_JI by block distance 1, 2, 3
-    float *sx = reinterpret_cast<float *>(sm + Sm::Q + 8192);
-    if (warp < 4 && lane < 16) {
-        const int BR = warp, cc = lane;
-        const float *b = af + (16 * BR) * C + 16 * BR;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-            for (int i = 0; i < r; ++i) acc = fmaf(-b[r * C + i], x[i], acc);
-            x[r] = acc;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) tf[(16 * BR + r) * C + 16 * BR + cc] = x[r];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int dd = 1; dd < 4; ++dd) {
-        const int nblk = 4 - dd;
-        for (int e = tid; e < nblk * 256; e += kThreads) {
-            const int BI = e >> 8, BR = BI + dd, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
-            for (int J = BI; J < BR; ++J) {
-                const float *arow = af + (16 * BR + r) * C + 16 * J;
-                const float *tcol = tf + (16 * J) * C + 16 * BI + cc;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc = fmaf(arow[i], tcol[i * C], acc);
-            }
-            sx[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nblk * 256; e += kThreads) {
-            const int BI = e >> 8, BR = BI + dd, r = (e >> 4) & 15, cc = e & 15;
-            const float *trow = tf + (16 * BR + r) * C + 16 * BR;
-            const float *xc = sx + (BI << 8) + cc;
-            float acc = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) acc = fmaf(trow[m], xc[m * 16], acc);
-            tf[(16 * BR + r) * C + 16 * BI + cc] = -acc;
-        }
-        __syncthreads();
-    }
-    // T in bf16 (the operand of W here and of the gradient products)
-    for (int idx = tid; idx < C * C / 2; idx += kThreads) {
-        const int r = idx >> 5, col = 2 * (idx & 31);
-        const float2 t2 = *reinterpret_cast<const float2 *>(tf + r * C + col);
-        *reinterpret_cast<uint32_t *>(sm + Sm::Q + at(r, col, C)) = pack_bf16(t2.x, t2.y);
-    }
-    __syncthreads();
-    copy_out(out + Ws::TB, sm + Sm::Q, 8192, kThreads);
-
-    // ---- -W = -T Bk: warp w owns rows 16 (w & 3), columns 64 (w >> 2) ----
-    {
-        const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
-        float acc[8][4];
-        zero_acc(acc);
-        mma_rows<8, false, true>(acc, sbase + Sm::Q, C, m0, sbase + Sm::X, C, n0, 0, C);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const int col = n0 + 8 * t + 2 * tq;
-            *reinterpret_cast<uint32_t *>(sm + Sm::Y + at(m0 + gq, col, C)) = pack_bf16(-acc[t][0], -acc[t][1]);
-            *reinterpret_cast<uint32_t *>(sm + Sm::Y + at(m0 + gq + 8, col, C)) = pack_bf16(-acc[t][2], -acc[t][3]);
-        }
-    }
-    __syncthreads();
-    copy_out(out + Ws::WN, sm + Sm::Y, 16384, kThreads);
-}
-}  // namespace intra
-
-// =============================================================================================
-// 3. dstate: one CTA per (document, head), chunks in reverse, dS^T [v][c] fp32 in tensor memory
+// 2. dstate: one CTA per (document, head), chunks in reverse, dS^T [v][c] fp32 in tensor memory
 //    (lane = value column v).  Per chunk, with the operands in shared memory:
 //      dU~^T  = dS^T_bf16 Kd^T + dO^T (scale A_qk)          (N = 64)
 //      dS^T  <- dS^T Diag(D) + dO^T (scale QG) + dU~^T_bf16 (-W)   (N = 128)
@@ -501,11 +245,11 @@ constexpr uint32_t kSB = 128;   // dS^T bf16, packed [128][64]
 constexpr uint32_t kUB = 128;   // dU~^T bf16, packed [128][32] (over kSB once the dU~ product has read it)
 constexpr uint32_t kDU = 192;   // dU~^T fp32 [128 v][64 s]
 struct Sm {
-    static constexpr int KD = 0;          // Kd [64 s][128 c]      K-major B (N = s, K = c)
-    static constexpr int AQ = 16384;      // scale A_qk [64 t][64 s]   MN-major B (K = t, N = s)
-    static constexpr int QG = 24576;      // scale QG [64 t][128 c]    MN-major B (K = t, N = c)
-    static constexpr int WN = 40960;      // -W [64 s][128 c]          MN-major B (K = s, N = c)
-    static constexpr int DO = 57344;      // dout [64 t][128 v]        MN-major A (K = t, M = v)
+    static constexpr int KD = 0;          // Kd^T [128 c][64 s]          MN-major B (K = c, N = s)
+    static constexpr int AQ = 16384;      // scale A_qk [64 t][64 s]     MN-major B (K = t, N = s)
+    static constexpr int WN = 24576;      // -W^T [128 c][64 s]          K-major B (N = c, K = s)
+    static constexpr int QG = 40960;      // scale QG^T [128 c][64 t]    K-major B (N = c, K = t)
+    static constexpr int DO = 57344;      // dout [64 t][128 v]          MN-major A (K = t, M = v)
     static constexpr int DL = 73728;      // D fp32 [128]
     static constexpr int MBAR = DL + 512; // mbarriers: inputs, dU~ product, state product
     static constexpr int TBASE = MBAR + 32, FLAG = TBASE + 8;
@@ -539,7 +283,7 @@ __device__ __forceinline__ void reg_fence(float (&v)[N]) {
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
-kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64_t T, int H, const uint8_t *ws_intra,
+kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64_t T, int H, const uint8_t *ws_ck,
                       uint8_t *ws_dst, int *status) {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -568,23 +312,22 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     const int v = 32 * warp + lane;   // this thread's TMEM lane = value column
 
-    // descriptors: K-major (Kd) and MN-major with 64 K rows per 64-wide atom (the rest)
+    // descriptors: K-major (-W^T, QG^T) and MN-major (dout, A_qk, Kd^T; 64-wide atoms 8 KB apart)
     const uint64_t dK = tc::sdesc(sbase, 16u, 1024u), dM = tc::sdesc(sbase, 64u * 128u, 1024u);
-    constexpr uint32_t id_u1 = tc::idesc_bf16(128, 64, false, false, false);   // dS^T_bf16 (TMEM) x Kd^T
+    constexpr uint32_t id_u1 = tc::idesc_bf16(128, 64, false, true, false);    // dS^T_bf16 (TMEM) x Kd^T
     constexpr uint32_t id_u2 = tc::idesc_bf16(128, 64, true, true, false);     // dO^T x A_qk
-    constexpr uint32_t id_s1 = tc::idesc_bf16(128, 128, true, true, false);    // dO^T x QG
-    constexpr uint32_t id_s2 = tc::idesc_bf16(128, 128, false, true, false);   // dU~^T_bf16 (TMEM) x (-W)
+    constexpr uint32_t id_s1 = tc::idesc_bf16(128, 128, true, false, false);   // dO^T x QG
+    constexpr uint32_t id_s2 = tc::idesc_bf16(128, 128, false, false, false);  // dU~^T_bf16 (TMEM) x (-W)
 
     auto issue_loads = [&](int j) {
         const int64_t tok = d0 + (int64_t)j * C;
         const int Lj = (int)((d1 - tok) < C ? (d1 - tok) : C);
         if (tid == 0) {
-            const uint8_t *src = ws_intra + ((size_t)(slot0 + j) * H + h) * Ws::INTRA;
+            const uint8_t *src = ws_ck + ((size_t)(slot0 + j) * H + h) * Ws::CK;
             tc::mbar_expect_tx(mb_in, Sm::kInBytes);
             bulk_load(sbase + Sm::KD, src + Ws::KD, 16384, mb_in);
             bulk_load(sbase + Sm::AQ, src + Ws::AQ, 8192, mb_in);
-            bulk_load(sbase + Sm::QG, src + Ws::QG, 16384, mb_in);
-            bulk_load(sbase + Sm::WN, src + Ws::WN, 16384, mb_in);
+            bulk_load(sbase + Sm::WN, src + Ws::B2, 32768, mb_in);   // [-W^T | scale QG^T]
             bulk_load(sbase + Sm::DL, src + Ws::DL, 512, mb_in);
         }
         // dout rows (zero past the document end) into the swizzled MN-major tile
@@ -651,8 +394,7 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
             tc::fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tmem + kDU, tmem + kSB + 8 * kk,
-                       dK + (uint64_t)((Sm::KD + (kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_u1, kk > 0);
+                mma_ts(tmem + kDU, tmem + kSB + 8 * kk, dM + (uint64_t)((Sm::KD + kk * 2048) >> 4), id_u1, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma(tmem + kDU, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dM + (uint64_t)((Sm::AQ + kk * 2048) >> 4),
@@ -703,11 +445,11 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
             tc::fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                tc::mma(tmem + kFS, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dM + (uint64_t)((Sm::QG + kk * 2048) >> 4),
+                tc::mma(tmem + kFS, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dK + (uint64_t)((Sm::QG + kk * 32) >> 4),
                         id_s1, 1u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_ts(tmem + kFS, tmem + kUB + 8 * kk, dM + (uint64_t)((Sm::WN + kk * 2048) >> 4), id_s2, 1u);
+                mma_ts(tmem + kFS, tmem + kUB + 8 * kk, dK + (uint64_t)((Sm::WN + kk * 32) >> 4), id_s2, 1u);
             tc::commit(mb_s);
         }
         ++n_commit_s;
@@ -743,7 +485,7 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
 }  // namespace dstate
 
 // =============================================================================================
-// 4. grad: one CTA per (chunk slot, head), 16 warps.  For 64 x 128 results warp w owns rows
+// 3. grad: one CTA per (chunk slot, head), 16 warps.  For 64 x 128 results warp w owns rows
 //    16 (w & 3) .. +15 and columns 32 (w >> 2) .. +31 (four 16 x 8 tiles); the gradients of k^,
 //    q^ and G at those positions stay in its registers from the first product to the last.
 // =============================================================================================
@@ -783,7 +525,7 @@ struct Args {
     int n_docs;
     int64_t T;
     int H;
-    const uint8_t *ws_ck, *ws_intra, *ws_dst;
+    const uint8_t *ws_ck, *ws_dst;
     uint16_t *dq, *dk, *dv;
     float *dg, *dbeta;
 };
@@ -796,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     int64_t tok0;
     if (!slot_chunk(a.cu, a.n_docs, a.T, slot, doc, tok0, L)) return;
     const size_t blk = (size_t)slot * H + h;
-    const uint8_t *ck = a.ws_ck + blk * Ws::CK, *in = a.ws_intra + blk * Ws::INTRA, *dsb = a.ws_dst + blk * Ws::DST;
+    const uint8_t *ck = a.ws_ck + blk * Ws::CK, *dsb = a.ws_dst + blk * Ws::DST;
     const uint32_t sbase = smem_u32(sm);
     float *rq = reinterpret_cast<float *>(sm + Sm::RQ), *rk = reinterpret_cast<float *>(sm + Sm::RK);
     float *sbeta = reinterpret_cast<float *>(sm + Sm::BETA), *dglp = reinterpret_cast<float *>(sm + Sm::DGLP);
@@ -807,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
 
     // ---- loads: workspace tiles as flat images, dout rows (zero past the document end) ----
     {
-        const uint8_t *src[6] = {ck, ck + Ws::CK_UT, dsb + Ws::DS, dsb + Ws::DU, in + Ws::TB, in + Ws::AH};
+        const uint8_t *src[6] = {ck + Ws::S, ck + Ws::UT, dsb + Ws::DS, dsb + Ws::DU, ck + Ws::TB, ck + Ws::AH};
         const int dst[6] = {Sm::ST, Sm::UT, Sm::DST, Sm::DUT, Sm::TB, Sm::AH};
         const int bytes[6] = {32768, 16384, 32768, 16384, 8192, 8192};
 #pragma unroll
@@ -823,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         cp_async_commit();
     }
     if (tid < C) sbeta[tid] = tid < L ? __ldg(a.beta + (tok0 + tid) * H + h) : 0.f;
-    if (tid < D) dls[tid] = reinterpret_cast<const float *>(in + Ws::DL)[tid];
+    if (tid < D) dls[tid] = reinterpret_cast<const float *>(ck + Ws::DL)[tid];
 
     // ---- prep: warp w holds rows 4w .. 4w + 3, lane l channels 4l .. 4l + 3: row norms, G (log2
     //      units), beta k^ e^G and beta v ----
@@ -957,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         ld_pairs(a.k, kp);
         float acc[4][4];
         zero_acc(acc);
-        mma_rows<4, true, true>(acc, sbase + Sm::UT, D, m0, sbase + Sm::DST, D, n0, 0, D);
+        mma_fix<4, true, true, D, D, 0, D>(acc, sbase + Sm::UT, m0, sbase + Sm::DST, n0);
         float cs[4][2];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -995,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         ld_pairs(a.q, qp);
         float acc[4][4];
         zero_acc(acc);
-        mma_rows<4, false, true>(acc, sbase + Sm::DO, C, m0, sbase + Sm::ST, D, n0, 0, D);
+        mma_fix<4, false, true, C, D, 0, D>(acc, sbase + Sm::DO, m0, sbase + Sm::ST, n0);
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
@@ -1014,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     // ---- dW = -dU~ S^T (kept in registers until every warp is done with S) ----
     float dw[4][4];
     zero_acc(dw);
-    mma_rows<4, true, true>(dw, sbase + Sm::DUT, D, m0, sbase + Sm::ST, D, n0, 0, D);
+    mma_fix<4, true, true, D, D, 0, D>(dw, sbase + Sm::DUT, m0, sbase + Sm::ST, n0);
     __syncthreads();   // S^T and dS^T are read: their space takes dW and the 64 x 64 tiles
 #pragma unroll
     for (int t = 0; t < 4; ++t)
@@ -1029,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     {
         float acc[2][4];
         zero_acc(acc);
-        mma_rows<2, false, true>(acc, sbase + Sm::DO, C, m0, sbase + Sm::UT, D, n64, 0, D);
+        mma_fix<2, false, true, C, D, 0, D>(acc, sbase + Sm::DO, m0, sbase + Sm::UT, n64);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -1045,8 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     {
         float acc[2][4];
         zero_acc(acc);
-        mma_rows<2, false, false>(acc, sbase + Sm::ST, C, m0, sbase + Sm::BK, C, n64, 0, D);
-        mma_rows<2, true, false>(acc, sbase + Sm::DUT, D, m0, sbase + Sm::BV, C, n64, 0, D);
+        mma_fix<2, false, false, C, C, 0, D>(acc, sbase + Sm::ST, m0, sbase + Sm::BK, n64);
+        mma_fix<2, true, false, D, C, 0, D>(acc, sbase + Sm::DUT, m0, sbase + Sm::BV, n64);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -1060,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         ld_pairs(a.k, kp);
         float acc[4][4];
         zero_acc(acc);
-        mma_rows<4, true, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::ST, C, n0, 0, C);
+        mma_fix<4, true, true, C, C, 0, C>(acc, sbase + Sm::TB, m0, sbase + Sm::ST, n0);
         float rs[2] = {0.f, 0.f};
 #pragma unroll
         for (int t = 0; t < 4; ++t)
@@ -1093,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         ld_pairs(a.v, vp);
         float acc[4][4];
         zero_acc(acc);
-        mma_rows<4, true, false>(acc, sbase + Sm::TB, C, m0, sbase + Sm::DUT, D, n0, 0, C);
+        mma_fix<4, true, false, C, D, 0, C>(acc, sbase + Sm::TB, m0, sbase + Sm::DUT, n0);
         float rs[2] = {0.f, 0.f};
 #pragma unroll
         for (int t = 0; t < 4; ++t)
@@ -1121,7 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     {
         float acc[2][4];
         zero_acc(acc);
-        mma_rows<2, true, true>(acc, sbase + Sm::TB, C, m0, sbase + Sm::DT, C, n64, 0, C);
+        mma_fix<2, true, true, C, C, 0, C>(acc, sbase + Sm::TB, m0, sbase + Sm::DT, n64);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -1182,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     {
         float acc[2][4];
         zero_acc(acc);
-        mma_rows<2, false, false>(acc, sbase + Sm::XM, C, m0, sbase + Sm::TB, C, n64, 0, C);
+        mma_fix<2, false, false, C, C, 0, C>(acc, sbase + Sm::XM, m0, sbase + Sm::TB, n64);
         float rs[2] = {0.f, 0.f};
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -1190,8 +932,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
             for (int hh = 0; hh < 2; ++hh) {
                 const int row = m0 + gq + 8 * hh, col = n64 + 8 * t + 2 * tq;
                 const float x0 = col < row ? -acc[t][2 * hh] : 0.f, x1 = col + 1 < row ? -acc[t][2 * hh + 1] : 0.f;
-                const float2 ah = bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::AH + at(row, col, C)));
-                rs[hh] += x0 * ah.x + x1 * ah.y;
+                // A_hat is defined below the diagonal only: the rest of its tile is never read
+                const float2 ah = col < row ? bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::AH + at(row, col, C)))
+                                            : make_float2(0.f, 0.f);
+                rs[hh] += x0 * ah.x + (col + 1 < row ? x1 * ah.y : 0.f);
                 const float b = sbeta[row];
                 *reinterpret_cast<uint32_t *>(sm + Sm::DAH + at(row, col, C)) = pack_bf16(b * x0, b * x1);
             }
@@ -1360,8 +1104,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
 
 }  // namespace bwd
 
-// workspace bytes of the backward: per chunk slot and head, the forward checkpoint, the intra
-// outputs and the dstate outputs
+// workspace bytes of the backward: per chunk slot and head, the forward checkpoint block and the
+// dstate outputs
 size_t bwd_workspace_floats(int n_docs, int64_t T, int H) {
     return ((size_t)(T / bwd::C) + (size_t)n_docs) * (size_t)H * (bwd::Ws::PER_SLOT / sizeof(float));
 }
@@ -1373,32 +1117,24 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     using namespace bwd;
     const size_t blocks = ((size_t)(T / C) + (size_t)n_docs) * (size_t)H;
     uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
-    uint8_t *ws_ck = ws, *ws_intra = ws + blocks * Ws::CK, *ws_dst = ws_intra + blocks * Ws::INTRA;
+    uint8_t *ws_ck = ws, *ws_dst = ws + blocks * Ws::CK;
     // 1. forward with checkpoints (its output o goes to dq, which is overwritten below)
     cudaError_t e = launch_fwd_pipe(q, k, v, g, beta, cu, n_docs, T, H, nullptr, nullptr, dq, status, stream,
                                     reinterpret_cast<uint16_t *>(ws_ck));
     if (e != cudaSuccess) return e;
-    // 2. intra
-    e = cudaFuncSetAttribute(intra::kda_bwd_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             intra::Sm::TOTAL);
-    if (e != cudaSuccess) return e;
-    intra::kda_bwd_intra_kernel<<<(unsigned)blocks, intra::kThreads, intra::Sm::TOTAL, stream>>>(
-        q, k, g, beta, cu, n_docs, T, H, ws_intra);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // 3. dstate
+    // 2. dstate
     e = cudaFuncSetAttribute(dstate::kda_bwd_dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dstate::Sm::TOTAL);
     if (e != cudaSuccess) return e;
     dstate::kda_bwd_dstate_kernel<<<(unsigned)(n_docs * H), dstate::kThreads, dstate::Sm::TOTAL, stream>>>(
-        dout, cu, n_docs, T, H, ws_intra, ws_dst, status);
+        dout, cu, n_docs, T, H, ws_ck, ws_dst, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // 4. grad
+    // 3. grad
     grad::Args a;
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.g = g; a.beta = beta; a.cu = cu;
     a.n_docs = n_docs; a.T = T; a.H = H;
-    a.ws_ck = ws_ck; a.ws_intra = ws_intra; a.ws_dst = ws_dst;
+    a.ws_ck = ws_ck; a.ws_dst = ws_dst;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
     e = cudaFuncSetAttribute(grad::kda_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad::Sm::TOTAL);
     if (e != cudaSuccess) return e;

@@ -42,7 +42,11 @@ namespace kda {
 namespace pipe_path {
 
 constexpr int kThreads = 512;
-constexpr size_t kCkptElems = 128 * 128 + 128 * 64;   // bf16 values per checkpoint slot: S^T, then U~^T
+// The backward's checkpoint block per chunk and head (bytes): S^T and U~^T (bf16 [128 v] rows), the
+// chunk's tensor-core operands [-W^T | Q~^T] (B2) and Kd^T, A_qk, T = (I + A_kk)^-1 and A_hat (bf16,
+// A_hat without beta and valid below the diagonal only), and e^{Gamma_last} (fp32)
+constexpr size_t kCkS = 0, kCkU = 32768, kCkB2 = 49152, kCkKD = 81920, kCkAQ = 98304, kCkT = 106496,
+                 kCkAH = 114688, kCkDL = 122880, kCkptBytes = 123904;
 constexpr int kStateTid0 = 384;               // first thread of warps 12-15
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSF = 0;                   // S^T fp32          [128 lanes v][128 cols c]
@@ -149,6 +153,11 @@ __device__ __forceinline__ void reg_fence(float (&v)[N]) {
     for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
 __device__ __forceinline__ int pair_R(int p) { return p >= 6 ? 3 : p >= 3 ? 2 : p >= 1 ? 1 : 0; }
+// bulk copy shared -> global (16-byte aligned, size a multiple of 16), tracked by the issuing thread's bulk group
+__device__ __forceinline__ void bulk_store(void *gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ int pair_of(int R, int I) { return R * (R + 1) / 2 + I; }
 
 // beta rows [tok0, tok0 + L) of head h, one row per calling thread (row in [0, 64); rows >= L zero-filled)
@@ -233,6 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     const int nchunks = (int)((doc_end - doc_start + 63) / 64);
+    // the checkpoint block of chunk i of this chain (kCkpt)
+    auto ck_block = [&](int i) -> uint8_t * {
+        return reinterpret_cast<uint8_t *>(ckpt) + ((size_t)(doc_start / 64 + doc + i) * H + h) * kCkptBytes;
+    };
     auto chunk_len = [&](int i) -> int {
         const int64_t rem = doc_end - (doc_start + 64 * (int64_t)i);
         return rem <= 0 ? 0 : (rem < 64 ? (int)rem : 64);
@@ -553,6 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float x0 = col < row ? ak[nt][2 * hh] * br : 0.f;
                             const float x1 = col + 1 < row ? ak[nt][2 * hh + 1] * br : 0.f;
                             *reinterpret_cast<float2 *>(blk + i * kBlkPitch + jj) = make_float2(x0, x1);
+                            if constexpr (kCkpt)
+                                *reinterpret_cast<uint32_t *>(ck_block(s) + kCkAH + tc::kmaj_off(row, col)) =
+                                    pack_bf16(col < row ? ak[nt][2 * hh] : 0.f, col + 1 < row ? ak[nt][2 * hh + 1] : 0.f);
                             const float y0 = col <= row ? aq[nt][2 * hh] * out_scale : 0.f;
                             const float y1 = col + 1 <= row ? aq[nt][2 * hh + 1] * out_scale : 0.f;
                             *reinterpret_cast<uint32_t *>(sm + aqk + tc::kmaj_off(row, col)) = pack_bf16(y0, y1);
@@ -636,6 +652,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     #pragma unroll
                             for (int r = 0; r < 16; ++r) {
                                 tb[r * kBlkPitch + col] = x[r];
+                                if constexpr (kCkpt)
+                                    *reinterpret_cast<__nv_bfloat16 *>(ck_block(s) + kCkT + tc::kmaj_off(16 * R + r, 16 * R + col)) =
+                                        __float2bfloat16_rn(x[r]);
                                 const __nv_bfloat16 t1 = __float2bfloat16_rn(x[r] * bc);
                                 *reinterpret_cast<__nv_bfloat16 *>(sm + S::KR + tc::kmaj_off(16 * R + r, 16 * R + col)) = t1;
                             }
@@ -649,6 +668,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int I = b < 3 ? b + 1 : b < 5 ? b - 1 : 3;
                             *reinterpret_cast<uint4 *>(sm + S::KR + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
                                 make_uint4(0, 0, 0, 0);
+                            if constexpr (kCkpt)
+                                *reinterpret_cast<uint4 *>(ck_block(s) + kCkT + tc::kmaj_chunk(16 * R + row, 2 * I + half)) =
+                                    make_uint4(0, 0, 0, 0);
                         }
                     }
                     bar_solve();
@@ -698,6 +720,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pack_bf16(-y[0] * b0, -y[1] * b1);
                         *reinterpret_cast<uint32_t *>(sm + S::KR + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
                             pack_bf16(-y[2] * b0, -y[3] * b1);
+                        if constexpr (kCkpt) {
+                            uint8_t *tt = ck_block(s) + kCkT;
+                            *reinterpret_cast<uint32_t *>(tt + tc::kmaj_off(16 * R + gq, 16 * I + cl)) = pack_bf16(-y[0], -y[1]);
+                            *reinterpret_cast<uint32_t *>(tt + tc::kmaj_off(16 * R + gq + 8, 16 * I + cl)) =
+                                pack_bf16(-y[2], -y[3]);
+                        }
                     };
                     if (warp < 4) {
                         // level 32: T_RI = -T_RR (A_RI T_II), (R, I) = (1, 0) or (3, 2)
@@ -822,6 +850,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int pL = chunk_len(n);
                 const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
                 const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
+                if constexpr (kCkpt) {
+                    // chunk n's operand tiles, complete since the previous step, to its checkpoint block by
+                    // bulk copies; their reads of shared memory are awaited before this step's state product,
+                    // whose completion releases B2 to the next readback
+                    if (tid == kStateTid0) {
+                        uint8_t *cb = ck_block(n);
+                        bulk_store(cb + kCkB2, sbase + S::B2, 32768);
+                        bulk_store(cb + kCkKD, sbase + S::KDT + nbuf * 16384, 16384);
+                        bulk_store(cb + kCkAQ, sbase + S::AQK + nbuf * 8192, 8192);
+                        bulk_store(cb + kCkDL, sbase + S::DC + nbuf * 512, 512);
+                        tc::bulk_commit();
+                    }
+                }
                 // S^T -> bf16 copy (A operand), then S^T <- S^T Diag(e^{Gamma_last})
                 auto sprep = [&](float (&sv)[16], int c0) {
                     uint32_t pk[8];
@@ -843,6 +884,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
                 auto state_mma = [&](int kk0) {   // [U~^T | (Q~ S)^T] accumulated onto [U^T | 0]
                     if (kk0 == 0 && have_intra) asm volatile("bar.sync 4, 160;" ::: "memory");
+                    if constexpr (kCkpt)
+                        if (kk0 == 0 && tid == kStateTid0) tc::bulk_wait_read();
                     tc::wait_st();
                     tc::fence_before();
                     bar_state();
@@ -867,9 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // the state entering chunk n into its checkpoint slot: row v of S^T, channels
                             // 16ch..16ch+15 as bf16, two 16-byte pieces of the row's 128-byte atom
                             const int vrow = 32 * lq + lane, m0 = (2 * ch) & 7;
-                            uint8_t *ck = reinterpret_cast<uint8_t *>(ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) *
-                                                                                 kCkptElems) +
-                                          (size_t)(ch >> 2) * (128 * 128) + (size_t)vrow * 128;
+                            uint8_t *ck = ck_block(n) + kCkS + (size_t)(ch >> 2) * (128 * 128) + (size_t)vrow * 128;
                             *reinterpret_cast<uint4 *>(ck + ((m0 ^ (vrow & 7)) << 4)) = pack8(cur, 1.f);
                             *reinterpret_cast<uint4 *>(ck + (((m0 + 1) ^ (vrow & 7)) << 4)) = pack8(cur + 8, 1.f);
                         }
@@ -903,9 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if constexpr (kCkpt) {
                             // U~^T row v, s = 32 h2 .. 32 h2 + 31, after the chunk's S^T in its checkpoint slot
                             const int vrow = 32 * lq + lane;
-                            uint8_t *cu8 = reinterpret_cast<uint8_t *>(ckpt + ((size_t)(doc_start / 64 + doc + n) * H + h) *
-                                                                                  kCkptElems + kHeadDim * kHeadDim) +
-                                           (size_t)vrow * 128;
+                            uint8_t *cu8 = ck_block(n) + kCkU + (size_t)vrow * 128;
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
                                 *reinterpret_cast<uint4 *>(cu8 + (((4 * h2 + e) ^ (vrow & 7)) << 4)) =
