@@ -780,6 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }   // warps 0-7
                 if (tid == 0) {
+                    if constexpr (kCkpt) tc::bulk_wait_read();   // the previous chunk's B2 copy has read it
                     bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
                     // B2 is free once the previous chunk's state product has read it
                     if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
@@ -827,6 +828,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- tcgen05: D[:, 0:64] = V^T T'^T = U^T ----
                 if (tid == 0) {
                     tc::fence_after();
+                    if constexpr (kCkpt) {
+                        // [-W^T | Q~^T] and A_qk of chunk s, complete now, to its checkpoint block
+                        bulk_store(ck_block(s) + kCkB2, sbase + S::B2, 32768);
+                        bulk_store(ck_block(s) + kCkAQ, sbase + S::AQK + buf * 8192, 8192);
+                        tc::bulk_commit();
+                    }
                     if constexpr (kMode != kTransition) {
                         constexpr uint32_t id_u = tc::idesc_bf16(128, 64, true, false, false);
 #pragma unroll
@@ -851,15 +858,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dcol = kD0 + 128 * (uint32_t)nbuf;
                 const float *dc = reinterpret_cast<const float *>(sm + S::DC) + nbuf * 128;
                 if constexpr (kCkpt) {
-                    // chunk n's operand tiles, complete since the previous step, to its checkpoint block by
-                    // bulk copies; their reads of shared memory are awaited before this step's state product,
-                    // whose completion releases B2 to the next readback
+                    // Kd^T and e^{Gamma_last} of chunk n to its checkpoint block (bulk copies, read-awaited
+                    // before this step's output is staged in Kd's buffer)
                     if (tid == kStateTid0) {
-                        uint8_t *cb = ck_block(n);
-                        bulk_store(cb + kCkB2, sbase + S::B2, 32768);
-                        bulk_store(cb + kCkKD, sbase + S::KDT + nbuf * 16384, 16384);
-                        bulk_store(cb + kCkAQ, sbase + S::AQK + nbuf * 8192, 8192);
-                        bulk_store(cb + kCkDL, sbase + S::DC + nbuf * 512, 512);
+                        bulk_store(ck_block(n) + kCkKD, sbase + S::KDT + nbuf * 16384, 16384);
+                        bulk_store(ck_block(n) + kCkDL, sbase + S::DC + nbuf * 512, 512);
                         tc::bulk_commit();
                     }
                 }
@@ -884,8 +887,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
                 auto state_mma = [&](int kk0) {   // [U~^T | (Q~ S)^T] accumulated onto [U^T | 0]
                     if (kk0 == 0 && have_intra) asm volatile("bar.sync 4, 160;" ::: "memory");
-                    if constexpr (kCkpt)
-                        if (kk0 == 0 && tid == kStateTid0) tc::bulk_wait_read();
                     tc::wait_st();
                     tc::fence_before();
                     bar_state();
@@ -972,6 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::commit(mbar(kMb4));
                     // the output tile is staged in Kd's buffer, which the state update reads
                     if (!tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                    if constexpr (kCkpt) tc::bulk_wait_read();   // and the checkpoint copy of Kd^T
                     tc::fence_before();
                 }
                 bar_state();
@@ -1070,6 +1072,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- teardown ----
     cp_async_wait_all();
     if (tid == kStateTid0) tc::bulk_wait();   // output tiles written before shared memory goes away
+    if constexpr (kCkpt)
+        if (tid == 0) tc::bulk_wait();       // and the checkpoint copies
     if (aborted) {
         if (tid == 0) atomicExch(status, kStatusTimeout);
         // let any tensor-core work or copy still in flight land before TMEM and shared memory go away
