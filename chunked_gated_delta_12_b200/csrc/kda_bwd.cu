@@ -58,8 +58,8 @@ constexpr long long kWaitLimit = 2000000000LL;
 // ---------------------------------------------------------------------------------------------
 struct Ws {
     // forward checkpoint block (written by the forward kernel's checkpoint instance)
-    static constexpr size_t S = 0;                    // S^T bf16 [128 v][128 c]
-    static constexpr size_t UT = 32768;               // U~^T bf16 [128 v][64 s]
+    static constexpr size_t S = 0;                    // S^T bf16 [128 v][128 c], column groups of 16
+    static constexpr size_t UT = 32768;               // U~^T bf16 [128 v][64 s], column groups of 32
     static constexpr size_t B2 = 49152;               // [-W^T | scale QG^T] bf16 [128 c][64 s | 64 t]
     static constexpr size_t KD = 81920;               // Kd^T bf16 [128 c][64 s]
     static constexpr size_t AQ = 98304;               // scale A_qk bf16 [64 t][64 s]
@@ -68,11 +68,19 @@ struct Ws {
     static constexpr size_t DL = 122880;              // D = e^{G_last} fp32 [128]
     static constexpr size_t CK = 123904;
     // dstate outputs
-    static constexpr size_t DS = 0;                   // dS^T bf16 [128 v][128 c] (dS leaving the chunk)
-    static constexpr size_t DU = DS + 32768;          // dU~^T bf16 [128 v][64 s]
+    static constexpr size_t DS = 0;                   // dS^T bf16 [128 v][128 c] (dS leaving the chunk), groups of 32
+    static constexpr size_t DU = DS + 32768;          // dU~^T bf16 [128 v][64 s], column groups of 32
     static constexpr size_t DST = DU + 16384;
     static constexpr size_t PER_SLOT = CK + DST;
 };
+
+// Row-major tiles written by one thread per row (S^T, U~^T, dS^T, dU~^T in the workspace) are stored
+// as column groups: the group's values of row 0, then of row 1, ..., so that the 32 rows of a warp
+// land in one contiguous piece.  Byte offset of the 16 bytes holding columns 8m .. 8m + 7 of row r,
+// with G columns per group and 128 rows:
+__device__ __forceinline__ uint32_t grp_off(int r, int m, int G) {
+    return (uint32_t)((8 * m / G) * 128 * G * 2 + r * G * 2 + (8 * m % G) * 2);
+}
 
 // byte offset of bf16 element (row, col) in a tile of `rows` rows (128-byte swizzled atoms)
 __device__ __forceinline__ uint32_t at(int row, int col, int rows) {
@@ -342,7 +350,7 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
     };
     // dS^T row v as bf16 into the workspace block of chunk j (and, optionally, into TMEM)
     auto store_ds = [&](int j, bool to_tmem) {
-        uint8_t *dst = ws_dst + ((size_t)(slot0 + j) * H + h) * Ws::DST + Ws::DS + (size_t)v * 128;
+        uint8_t *dst = ws_dst + ((size_t)(slot0 + j) * H + h) * Ws::DST + Ws::DS + (size_t)v * 64;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
             float x[32];
@@ -354,11 +362,9 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
             for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
             if (to_tmem) st16(lane_base + kSB + 16 * q4, pk);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int m = 4 * (q4 & 1) + e;   // 16-byte piece of channels 32 q4 + 8 e within the half
-                *reinterpret_cast<uint4 *>(dst + (size_t)(q4 >> 1) * (128 * 128) + ((m ^ (v & 7)) << 4)) =
+            for (int e = 0; e < 4; ++e)   // channels 32 q4 + 8 e .. (column group q4)
+                *reinterpret_cast<uint4 *>(dst + (size_t)q4 * (128 * 64) + 16 * e) =
                     make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-            }
         }
     };
 
@@ -416,7 +422,7 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
         tc::fence_after();
         if (ok) {
             // dU~^T -> workspace (bf16 row v) and -> TMEM as the A operand of the update
-            uint8_t *dst = ws_dst + ((size_t)(slot0 + j) * H + h) * Ws::DST + Ws::DU + (size_t)v * 128;
+            uint8_t *dst = ws_dst + ((size_t)(slot0 + j) * H + h) * Ws::DST + Ws::DU + (size_t)v * 64;
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 float x[32];
@@ -428,11 +434,9 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
                 for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
                 st16(lane_base + kUB + 16 * h2, pk);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = 4 * h2 + e;
-                    *reinterpret_cast<uint4 *>(dst + ((m ^ (v & 7)) << 4)) =
+                for (int e = 0; e < 4; ++e)   // s = 32 h2 + 8 e .. (column group h2)
+                    *reinterpret_cast<uint4 *>(dst + (size_t)h2 * (128 * 64) + 16 * e) =
                         make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                }
             }
         }
         tc::wait_st();
@@ -549,12 +553,21 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
 
     // ---- loads: workspace tiles as flat images, dout rows (zero past the document end) ----
     {
-        const uint8_t *src[6] = {ck + Ws::S, ck + Ws::UT, dsb + Ws::DS, dsb + Ws::DU, ck + Ws::TB, ck + Ws::AH};
-        const int dst[6] = {Sm::ST, Sm::UT, Sm::DST, Sm::DUT, Sm::TB, Sm::AH};
-        const int bytes[6] = {32768, 16384, 32768, 16384, 8192, 8192};
+        // S^T, U~^T, dS^T, dU~^T: column groups -> swizzled atoms; T, A_hat: flat images
+        const uint8_t *gsrc[4] = {ck + Ws::S, ck + Ws::UT, dsb + Ws::DS, dsb + Ws::DU};
+        const int gdst[4] = {Sm::ST, Sm::UT, Sm::DST, Sm::DUT}, gcols[4] = {128, 64, 128, 64}, ggrp[4] = {16, 32, 32, 32};
 #pragma unroll
-        for (int t = 0; t < 6; ++t)
-            for (int i = tid; i < bytes[t] / 16; i += kThreads) cp_async16(sbase + dst[t] + 16 * i, src[t] + 16 * i, 16);
+        for (int t = 0; t < 4; ++t) {
+            const int per_row = gcols[t] / 8;
+            for (int i = tid; i < 128 * per_row; i += kThreads) {
+                const int r = i / per_row, m = i % per_row;
+                cp_async16(sbase + gdst[t] + at(r, 8 * m, D), gsrc[t] + grp_off(r, m, ggrp[t]), 16);
+            }
+        }
+        for (int i = tid; i < 8192 / 16; i += kThreads) {
+            cp_async16(sbase + Sm::TB + 16 * i, ck + Ws::TB + 16 * i, 16);
+            cp_async16(sbase + Sm::AH + 16 * i, ck + Ws::AH + 16 * i, 16);
+        }
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int idx = tid + i * kThreads, t = idx >> 4, m = idx & 15;

@@ -42,9 +42,11 @@ namespace kda {
 namespace pipe_path {
 
 constexpr int kThreads = 512;
-// The backward's checkpoint block per chunk and head (bytes): S^T and U~^T (bf16 [128 v] rows), the
-// chunk's tensor-core operands [-W^T | Q~^T] (B2) and Kd^T, A_qk, T = (I + A_kk)^-1 and A_hat (bf16,
-// A_hat without beta and valid below the diagonal only), and e^{Gamma_last} (fp32)
+// The backward's checkpoint block per chunk and head (bytes): S^T and U~^T (bf16, stored as column
+// groups of 16 (S^T) or 32 (U~^T) values per row v, rows v consecutive inside a group, so that a
+// warp's stores cover whole contiguous pieces), the chunk's tensor-core operands [-W^T | Q~^T] (B2)
+// and Kd^T, A_qk, T = (I + A_kk)^-1 and A_hat (bf16, A_hat without beta and valid below the diagonal
+// only), and e^{Gamma_last} (fp32)
 constexpr size_t kCkS = 0, kCkU = 32768, kCkB2 = 49152, kCkKD = 81920, kCkAQ = 98304, kCkT = 106496,
                  kCkAH = 114688, kCkDL = 122880, kCkptBytes = 123904;
 constexpr int kStateTid0 = 384;               // first thread of warps 12-15
@@ -909,11 +911,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (ch < 7) tc::ld16(lane_base + kSF + 16 * (ch + 1), nxt);
                         if constexpr (kCkpt) {
                             // the state entering chunk n into its checkpoint slot: row v of S^T, channels
-                            // 16ch..16ch+15 as bf16, two 16-byte pieces of the row's 128-byte atom
-                            const int vrow = 32 * lq + lane, m0 = (2 * ch) & 7;
-                            uint8_t *ck = ck_block(n) + kCkS + (size_t)(ch >> 2) * (128 * 128) + (size_t)vrow * 128;
-                            *reinterpret_cast<uint4 *>(ck + ((m0 ^ (vrow & 7)) << 4)) = pack8(cur, 1.f);
-                            *reinterpret_cast<uint4 *>(ck + (((m0 + 1) ^ (vrow & 7)) << 4)) = pack8(cur + 8, 1.f);
+                            // 16ch..16ch+15 as bf16, in column group ch
+                            const int vrow = 32 * lq + lane;
+                            uint8_t *ck = ck_block(n) + kCkS + (size_t)ch * (128 * 32) + (size_t)vrow * 32;
+                            *reinterpret_cast<uint4 *>(ck) = pack8(cur, 1.f);
+                            *reinterpret_cast<uint4 *>(ck + 16) = pack8(cur + 8, 1.f);
                         }
                         sprep(cur, 16 * ch);
                         if (ch == 3) state_mma(0);
@@ -943,12 +945,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(u[2 * i], u[2 * i + 1]);
                         st16(lane_base + kUB + 16 * h2, pk);
                         if constexpr (kCkpt) {
-                            // U~^T row v, s = 32 h2 .. 32 h2 + 31, after the chunk's S^T in its checkpoint slot
+                            // U~^T row v, s = 32 h2 .. 32 h2 + 31 (column group h2), after the chunk's S^T
                             const int vrow = 32 * lq + lane;
-                            uint8_t *cu8 = ck_block(n) + kCkU + (size_t)vrow * 128;
+                            uint8_t *cu8 = ck_block(n) + kCkU + (size_t)h2 * (128 * 64) + (size_t)vrow * 64;
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
-                                *reinterpret_cast<uint4 *>(cu8 + (((4 * h2 + e) ^ (vrow & 7)) << 4)) =
+                                *reinterpret_cast<uint4 *>(cu8 + 16 * e) =
                                     make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                         }
                     }
