@@ -260,8 +260,15 @@ size_t kda_chunk_bwd_workspace_size(int n_docs, int64_t T, int H);
  *              [0, T) is written.  Outputs must not alias an input or each other.
  *   workspace  device buffer of at least kda_chunk_bwd_workspace_size(n_docs, T, H) bytes,
  *              16-byte aligned, owned by the caller; its content on entry is ignored and on
- *              return is unspecified (it holds the state entering every chunk and per-chain
- *              scratch).  libkda allocates no memory of its own.
+ *              return is unspecified.  It holds, per chunk and head (about 169 KB), what the
+ *              forward pass saves (the state entering the chunk, U~, the chunk's operand tiles,
+ *              T and A_hat) and what the reverse dS sweep writes (dS and dU~).  libkda allocates
+ *              no memory of its own.
+ *
+ * Work: three launches on `stream` -- the forward kernel in its checkpoint instance, the reverse
+ * sweep over dS (one CTA per document and head, tcgen05 with dS^T in tensor memory), and the
+ * gradient kernel (one CTA per chunk and head).  Results are bit-reproducible: no atomics, fixed
+ * summation orders.
  *   stream     cudaStream_t (NULL = legacy default stream); the call is asynchronous
  *
  * Errors: as kda_chunk_fwd; a workspace smaller than required is KDA_ERR_INVALID_ARG.
@@ -293,7 +300,8 @@ kda_status kda_chunk_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
  * Limit: calls whose kda_chunk_bwd_workspace_size(n_docs, T, H) exceeds
  * KDA_BWD_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_INVALID_ARG and a message naming
  * the sizes (for example 1 document of 2048 tokens with 8 heads fits; 4096 tokens with 32
- * heads does not); those callers need kda_chunk_bwd.
+ * heads does not); those callers need kda_chunk_bwd.  The results are bit-identical to
+ * kda_chunk_bwd's.
  *
  * Memory held: every GPU that loads libkda's device code keeps the array until the process
  * exits.  Its device address is looked up on the first call made on each device (with that
