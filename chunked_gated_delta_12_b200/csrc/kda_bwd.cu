@@ -532,7 +532,6 @@ struct Args {
     const uint8_t *ws_ck, *ws_dst;
     uint16_t *dq, *dk, *dv;
     float *dg, *dbeta;
-    int *status;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a) {
@@ -1116,605 +1115,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
 }
 }  // namespace grad
 
-// =============================================================================================
-// 3'. grad on tcgen05: the 64 x 128 products transposed so that the channel (or value) index is the
-//     tensor-core M = 128 and the chunk row is N; their results and the gradients of k^, q^ and G
-//     (transposed, [128 c][64 r] fp32) live in tensor memory.  Lane c of warp w (quadrant w & 3)
-//     handles TMEM columns 16 (w >> 2) .. +15 of every 64-column result.  The 64 x 64 products stay
-//     on warp MMA.
-// =============================================================================================
-namespace grad2 {
-constexpr int kThreads = 512;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAK = 0, kAQ = 64, kAG = 128;          // dk^T, dq^T, dG^T accumulators [c][r]
-constexpr uint32_t kPA = 192, kPB = 256, kPC = 320;       // product results [c or v][64]
-constexpr uint32_t kPD = 384;                             // dW^T bf16 (32 packed columns); then a 64-column result
-struct Sm {
-    static constexpr int ST = 0;          // S^T [128 v][128 c]; then dW [128 c][64 s]
-    static constexpr int DWS = 0;
-    static constexpr int DST = 32768;     // dS^T [128 v][128 c]; then dA_qk [t][s], dA_qk^T [s][t], dT, Xm
-    static constexpr int DAQ = DST, DAQ2 = DST + 8192, DT = DST + 16384, XM = DST + 24576;
-    static constexpr int UT = 65536;      // U~^T [128 v][64 s]; then k^ E2 [64][128]
-    static constexpr int YT = UT;
-    static constexpr int DUT = 81920;     // dU~^T [128 v][64 s]; then pair scales fp32 [10][128]
-    static constexpr int PS = DUT;
-    static constexpr int DO = 98304;      // dout [64 t][128 v]; then dA_hat [r][i], dA_hat^T [i][r]
-    static constexpr int DAH = DO, DAH2 = DO + 8192;
-    static constexpr int TB = 114688;     // T [64 r][64 i]
-    static constexpr int AH = 122880;     // A_hat [64 r][64 i]
-    static constexpr int BK = 131072;     // beta k^ e^G [64][128]; then k^ E1
-    static constexpr int XT = BK;
-    static constexpr int BV = 147456;     // beta v [64][128]; then q^ E1
-    static constexpr int QT = BV;
-    static constexpr int GF = 163840;     // G (log2 units) fp32 [64][128], swizzled
-    static constexpr int RQ = 196608, RK = RQ + 256, BETA = RK + 256, GLS = BETA + 256, DLS = GLS + 512,
-                         DGLP = DLS + 512, DBP = DGLP + 4096, RED = DBP + 3072, TOT = RED + 2048, MBAR = TOT + 2048,
-                         TBASE = MBAR + 32;
-    static constexpr int TOTAL = TBASE + 16;
-};
-using grad::Args;
-using grad::gfi;
-
-__device__ __forceinline__ void ld16f(uint32_t taddr, float (&v)[16]) { tc::ld16(taddr, v); }
-__device__ __forceinline__ void st16f(uint32_t taddr, const float (&v)[16]) {
-    uint32_t r[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(v[i]);
-    dstate::st16(taddr, r);
-}
-// sum over the 32 lanes of each of 16 per-lane values: afterwards lane l holds the total of value
-// col(l) = 8 b4 + 4 b3 + 2 b2 + b1 (b_k = bit k of l), lanes 2j and 2j+1 alike
-__device__ __forceinline__ float lane_sum16(float (&x)[16], int lane) {
-#pragma unroll
-    for (int o = 16, n = 8; o >= 2; o >>= 1, n >>= 1) {
-#pragma unroll
-        for (int i = 0; i < n; ++i) {
-            const bool up = lane & o;
-            const float keep = up ? x[i + n] : x[i], send = up ? x[i] : x[i + n];
-            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-    }
-    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
-}
-__device__ __forceinline__ int lane_sum16_col(int lane) {
-    return 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
-}
-
-__global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad2_kernel(const Args a) {
-    extern __shared__ __align__(1024) uint8_t sm[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const int H = a.H, slot = blockIdx.x / H, h = blockIdx.x % H;
-    int doc, L;
-    int64_t tok0;
-    if (!slot_chunk(a.cu, a.n_docs, a.T, slot, doc, tok0, L)) return;
-    const size_t blk = (size_t)slot * H + h;
-    const uint8_t *ck = a.ws_ck + blk * Ws::CK, *dsb = a.ws_dst + blk * Ws::DST;
-    const uint32_t sbase = smem_u32(sm);
-    float *rq = reinterpret_cast<float *>(sm + Sm::RQ), *rk = reinterpret_cast<float *>(sm + Sm::RK);
-    float *sbeta = reinterpret_cast<float *>(sm + Sm::BETA), *dglp = reinterpret_cast<float *>(sm + Sm::DGLP);
-    float *dls = reinterpret_cast<float *>(sm + Sm::DLS), *gls = reinterpret_cast<float *>(sm + Sm::GLS);
-    float *dbp = reinterpret_cast<float *>(sm + Sm::DBP), *red = reinterpret_cast<float *>(sm + Sm::RED);
-    float *tot = reinterpret_cast<float *>(sm + Sm::TOT), *gf = reinterpret_cast<float *>(sm + Sm::GF);
-    float *ps = reinterpret_cast<float *>(sm + Sm::PS);
-    const uint32_t mb = sbase + Sm::MBAR;
-    int mb_phase = 0;   // completions of the tensor-core barrier so far
-
-    // ---- loads (as the warp-MMA version): column-group tiles -> swizzled atoms, flat T / A_hat, dout ----
-    {
-        const uint8_t *gsrc[4] = {ck + Ws::S, ck + Ws::UT, dsb + Ws::DS, dsb + Ws::DU};
-        const int gdst[4] = {Sm::ST, Sm::UT, Sm::DST, Sm::DUT}, gcols[4] = {128, 64, 128, 64}, ggrp[4] = {16, 32, 32, 32};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int per_row = gcols[t] / 8;
-            for (int i = tid; i < 128 * per_row; i += kThreads) {
-                const int r = i / per_row, m = i % per_row;
-                cp_async16(sbase + gdst[t] + at(r, 8 * m, D), gsrc[t] + grp_off(r, m, ggrp[t]), 16);
-            }
-        }
-        for (int i = tid; i < 8192 / 16; i += kThreads) {
-            cp_async16(sbase + Sm::TB + 16 * i, ck + Ws::TB + 16 * i, 16);
-            cp_async16(sbase + Sm::AH + 16 * i, ck + Ws::AH + 16 * i, 16);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int idx = tid + i * kThreads, t = idx >> 4, m = idx & 15;
-            const bool ok = t < L;
-            const uint16_t *s2 = ok ? a.dout + ((tok0 + t) * H + h) * D + 8 * m : a.dout;
-            cp_async16(sbase + Sm::DO + at(t, 8 * m, C), s2, ok ? 16 : 0);
-        }
-        cp_async_commit();
-    }
-    if (tid < C) sbeta[tid] = tid < L ? __ldg(a.beta + (tok0 + tid) * H + h) : 0.f;
-    if (tid < D) dls[tid] = reinterpret_cast<const float *>(ck + Ws::DL)[tid];
-    if (warp == 0) tc::alloc(sbase + Sm::TBASE, kTmemCols);
-    if (tid == 0) {
-        tc::mbar_init(mb, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    // ---- prep: warp w holds rows 4w .. 4w + 3, lane l channels 4l .. 4l + 3 ----
-    {
-        const int c0 = 4 * lane, r0 = 4 * warp;
-        uint2 qr[4], kr[4], vr[4];
-        float4 gr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = r0 + i;
-            if (r < L) {
-                const int64_t o = ((tok0 + r) * H + h) * D + c0;
-                qr[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + o));
-                kr[i] = __ldg(reinterpret_cast<const uint2 *>(a.k + o));
-                vr[i] = __ldg(reinterpret_cast<const uint2 *>(a.v + o));
-                gr[i] = __ldg(reinterpret_cast<const float4 *>(a.g + o));
-            } else {
-                qr[i] = kr[i] = vr[i] = make_uint2(0u, 0u);
-                gr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-        float rkr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 qa = bf2(qr[i].x), qb = bf2(qr[i].y), ka = bf2(kr[i].x), kb = bf2(kr[i].y);
-            float sq = qa.x * qa.x + qa.y * qa.y + qb.x * qb.x + qb.y * qb.y;
-            float sk = ka.x * ka.x + ka.y * ka.y + kb.x * kb.x + kb.y * kb.y;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                sq += __shfl_xor_sync(0xffffffffu, sq, o);
-                sk += __shfl_xor_sync(0xffffffffu, sk, o);
-            }
-            rkr[i] = rsqrtf(sk + 1e-6f);
-            if (lane == 0) {
-                rq[r0 + i] = rsqrtf(sq + 1e-6f);
-                rk[r0 + i] = rkr[i];
-            }
-        }
-        float g2[4][4], run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float x[4] = {gr[i].x, gr[i].y, gr[i].z, gr[i].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                run[e] += x[e] * kLog2e;
-                g2[i][e] = run[e];
-            }
-        }
-        float *gt = reinterpret_cast<float *>(sm + Sm::BK);   // [16][128] row-group totals (before Bk)
-        *reinterpret_cast<float4 *>(gt + warp * D + c0) = make_float4(run[0], run[1], run[2], run[3]);
-        __syncthreads();
-        float off[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int w2 = 0; w2 < warp; ++w2) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(gt + w2 * D + c0);
-            off[0] += t4.x; off[1] += t4.y; off[2] += t4.z; off[3] += t4.w;
-        }
-        __syncthreads();   // the totals are read before Bk overwrites them
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = r0 + i;
-            float bk[4], bv[4];
-            const float2 ka = bf2(kr[i].x), kb = bf2(kr[i].y), va = bf2(vr[i].x), vb = bf2(vr[i].y);
-            const float kv[4] = {ka.x, ka.y, kb.x, kb.y}, vv[4] = {va.x, va.y, vb.x, vb.y};
-            const float br = sbeta[r];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                g2[i][e] += off[e];
-                bk[e] = br * kv[e] * rkr[i] * ex2_ftz(g2[i][e]);
-                bv[e] = br * vv[e];
-            }
-            *reinterpret_cast<float4 *>(gf + gfi(r, c0)) = make_float4(g2[i][0], g2[i][1], g2[i][2], g2[i][3]);
-            const uint32_t o2 = at(r, c0, C);
-            *reinterpret_cast<uint2 *>(sm + Sm::BK + o2) = make_uint2(pack_bf16(bk[0], bk[1]), pack_bf16(bk[2], bk[3]));
-            *reinterpret_cast<uint2 *>(sm + Sm::BV + o2) = make_uint2(pack_bf16(bv[0], bv[1]), pack_bf16(bv[2], bv[3]));
-        }
-        if (warp == 15) *reinterpret_cast<float4 *>(gls + c0) = make_float4(g2[3][0], g2[3][1], g2[3][2], g2[3][3]);
-    }
-    cp_async_wait_all();
-    tc::fence_proxy_async();
-    tc::fence_before();
-    __syncthreads();
-    tc::fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + Sm::TBASE);
-    const int qd = warp & 3, cg = warp >> 2, c = 32 * qd + lane, r0 = 16 * cg;
-    const uint32_t lb = tmem + ((uint32_t)(32 * qd) << 16);   // this warp's lane quadrant
-    const uint64_t dK = tc::sdesc(sbase, 16u, 1024u);
-    const uint64_t dM128 = tc::sdesc(sbase, 128u * 128u, 1024u), dM64 = tc::sdesc(sbase, 64u * 128u, 1024u);
-    auto desc = [](uint64_t d, int off) { return d + (uint64_t)(off >> 4); };
-    auto wait_mb = [&]() {
-        const bool ok = tc::mbar_wait(mb, (uint32_t)(mb_phase & 1), kWaitLimit);
-        ++mb_phase;
-        tc::fence_after();
-        return ok;
-    };
-
-    // ---- products 1: dKd^T = dS U~^T, dQG^T = S dout^T, dW^T = -S dU~^T  ([128 c][64]) ----
-    if (tid == 0) {
-        constexpr uint32_t id_kd = tc::idesc_bf16(128, 64, true, true, false);
-        constexpr uint32_t id_qg = tc::idesc_bf16(128, 64, true, false, false);
-        constexpr uint32_t id_w = tc::idesc_bf16(128, 64, true, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            tc::mma(tmem + kPA, desc(dM128, Sm::DST + kk * 2048), desc(dM128, Sm::UT + kk * 2048), id_kd, kk > 0);
-            tc::mma(tmem + kPB, desc(dM128, Sm::ST + kk * 2048), desc(dK, Sm::DO + (kk >> 2) * 8192 + (kk & 3) * 32), id_qg,
-                    kk > 0);
-            tc::mma(tmem + kPC, desc(dM128, Sm::ST + kk * 2048), desc(dM128, Sm::DUT + kk * 2048), id_w, kk > 0);
-        }
-        tc::commit(mb);
-    }
-    // meanwhile: dG_last part 1, D[c] sum_v S[c][v] dS[c][v] (this warp's 32 rows v of column c)
-    {
-        float sacc = 0.f;
-#pragma unroll 8
-        for (int v = 32 * cg; v < 32 * cg + 32; ++v) {
-            const uint32_t o = at(v, c, D);
-            sacc += bfl(*reinterpret_cast<const uint16_t *>(sm + Sm::ST + o)) *
-                    bfl(*reinterpret_cast<const uint16_t *>(sm + Sm::DST + o));
-        }
-        dglp[cg * D + c] = dls[c] * sacc;
-    }
-    // this warp's 16 columns r of k and q at channel c (zero past the document end)
-    float kh[16], qh[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int r = r0 + i;
-        const int64_t o = ((tok0 + r) * H + h) * D + c;
-        kh[i] = r < L ? bfl(__ldg(a.k + o)) * rk[r] : 0.f;
-        qh[i] = r < L ? bfl(__ldg(a.q + o)) * rq[r] : 0.f;
-    }
-    bool ok = wait_mb();
-    {
-        // dKd: dk^ += dKd e^{G_last - G}, dG -= dKd Kd, dG_last += sum_s dKd Kd
-        float x[16], ak[16], ag[16], aq[16];
-        ld16f(lb + kPA + r0, x);
-        tc::wait_ld();
-        dstate::reg_fence(x);
-        float cs = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float g2 = gf[gfi(r0 + i, c)];
-            const float ed = ex2_ftz(gls[c] - g2), kd = kh[i] * ed;
-            ak[i] = x[i] * ed;
-            ag[i] = -x[i] * kd;
-            cs += x[i] * kd;
-        }
-        dglp[(4 + cg) * D + c] = cs;
-        // dQG (scale dout S^T): dq^ += dQG e^G, dG += dQG QG
-        ld16f(lb + kPB + r0, x);
-        tc::wait_ld();
-        dstate::reg_fence(x);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float eg = ex2_ftz(gf[gfi(r0 + i, c)]);
-            const float y = kScale * x[i] * eg;
-            aq[i] = y;
-            ag[i] += y * qh[i];
-        }
-        st16f(lb + kAK + r0, ak);
-        st16f(lb + kAQ + r0, aq);
-        st16f(lb + kAG + r0, ag);
-        // dW^T (negated by the product) -> bf16: TMEM (A of dBk^T) and shared [c][s] (A of dT)
-        ld16f(lb + kPC + r0, x);
-        tc::wait_ld();
-        dstate::reg_fence(x);
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(lb + kPD + r0 / 2),
-                     "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]), "r"(pk[7])
-                     : "memory");
-        *reinterpret_cast<uint4 *>(sm + Sm::DWS + at(c, r0, D)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4 *>(sm + Sm::DWS + at(c, r0 + 8, D)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
-    tc::wait_st();
-    tc::fence_proxy_async();
-    tc::fence_before();
-    if (__syncthreads_or(!ok)) ok = false;
-    tc::fence_after();
-    // ---- products 2: dBk^T = dW^T T (A in TMEM), dBv^T = dU~^T T ----
-    if (tid == 0) {
-        constexpr uint32_t id_bk = tc::idesc_bf16(128, 64, false, true, false);
-        constexpr uint32_t id_bv = tc::idesc_bf16(128, 64, false, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            dstate::mma_ts(tmem + kPA, tmem + kPD + 8 * kk, desc(dM64, Sm::TB + kk * 2048), id_bk, kk > 0);
-            tc::mma(tmem + kPB, desc(dK, Sm::DUT + kk * 32), desc(dM64, Sm::TB + kk * 2048), id_bv, kk > 0);
-        }
-        tc::commit(mb);
-    }
-    // meanwhile (warp MMA): dA_qk = scale lower(dout U~^T) and dT = dW (beta KG)^T + dU~ (beta V)^T;
-    // warp w owns rows 16 (w & 3) and columns 16 (w >> 2) of each 64 x 64 result
-    {
-        const int m0 = 16 * qd, n64 = 16 * cg;
-        float acc[2][4];
-        zero_acc(acc);
-        mma_fix<2, false, true, C, D, 0, D>(acc, sbase + Sm::DO, m0, sbase + Sm::UT, n64);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int row = m0 + gq + 8 * hh, col = n64 + 8 * t + 2 * tq;
-                const float x0 = col <= row ? kScale * acc[t][2 * hh] : 0.f;
-                const float x1 = col + 1 <= row ? kScale * acc[t][2 * hh + 1] : 0.f;
-                const uint32_t pkv = pack_bf16(x0, x1);
-                *reinterpret_cast<uint32_t *>(sm + Sm::DAQ + at(row, col, C)) = pkv;
-                *reinterpret_cast<uint16_t *>(sm + Sm::DAQ2 + at(col, row, C)) = (uint16_t)(pkv & 0xffffu);
-                *reinterpret_cast<uint16_t *>(sm + Sm::DAQ2 + at(col + 1, row, C)) = (uint16_t)(pkv >> 16);
-            }
-        zero_acc(acc);
-        mma_fix<2, true, false, D, C, 0, D>(acc, sbase + Sm::DWS, m0, sbase + Sm::BK, n64);
-        mma_fix<2, true, false, D, C, 0, D>(acc, sbase + Sm::DUT, m0, sbase + Sm::BV, n64);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint32_t *>(sm + Sm::DT + at(m0 + gq + 8 * hh, n64 + 8 * t + 2 * tq, C)) =
-                    pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
-    }
-    ok = wait_mb() && ok;
-    {
-        // dBk^T [c][i]: dKG = beta dBk; dk^ += dKG e^G, dG += dKG KG, dbeta_i += sum_c dBk KG
-        float x[16], ak[16], ag[16], db[16];
-        ld16f(lb + kPA + r0, x);
-        ld16f(lb + kAK + r0, ak);
-        ld16f(lb + kAG + r0, ag);
-        tc::wait_ld();
-        dstate::reg_fence(x);
-        dstate::reg_fence(ak);
-        dstate::reg_fence(ag);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float eg = ex2_ftz(gf[gfi(r0 + i, c)]), kg = kh[i] * eg, b = sbeta[r0 + i];
-            ak[i] += b * x[i] * eg;
-            ag[i] += b * x[i] * kg;
-            db[i] = x[i] * kg;
-        }
-        st16f(lb + kAK + r0, ak);
-        st16f(lb + kAG + r0, ag);
-        const float s1 = lane_sum16(db, lane);
-        if (!(lane & 1)) dbp[(0 + qd) * C + r0 + lane_sum16_col(lane)] = s1;
-        // dBv^T [v][i] (lane = value column v = c): dv = beta dBv, dbeta_i += sum_v dBv v
-        ld16f(lb + kPB + r0, x);
-        tc::wait_ld();
-        dstate::reg_fence(x);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = r0 + i;
-            const int64_t o = ((tok0 + r) * H + h) * D + c;
-            const float vv = r < L ? bfl(__ldg(a.v + o)) : 0.f;
-            db[i] = x[i] * vv;
-            if (r < L) a.dv[o] = f2b(sbeta[r] * x[i]);
-        }
-        const float s2 = lane_sum16(db, lane);
-        if (!(lane & 1)) dbp[(4 + qd) * C + r0 + lane_sum16_col(lane)] = s2;
-    }
-    tc::wait_st();
-    tc::fence_before();
-    __syncthreads();   // dT, dA_qk in place; dW, dU~^T, beta V, beta KG are read
-    tc::fence_after();
-    // ---- Xm = T^T dT (warp MMA) ----
-    {
-        const int m0 = 16 * qd, n64 = 16 * cg;
-        float acc[2][4];
-        zero_acc(acc);
-        mma_fix<2, true, true, C, C, 0, C>(acc, sbase + Sm::TB, m0, sbase + Sm::DT, n64);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint32_t *>(sm + Sm::XM + at(m0 + gq + 8 * hh, n64 + 8 * t + 2 * tq, C)) =
-                    pack_bf16(acc[t][2 * hh], acc[t][2 * hh + 1]);
-    }
-    // ---- k^ E1, q^ E1, k^ E2 and the pair scales (warp w: rows 4w .. 4w + 3, lane l: channels 4l ..) ----
-    {
-        const int c0 = 4 * lane, rr0 = 4 * warp, BR = warp >> 2;
-        uint2 qr[4], kr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = rr0 + i;
-            if (r < L) {
-                const int64_t o = ((tok0 + r) * H + h) * D + c0;
-                qr[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + o));
-                kr[i] = __ldg(reinterpret_cast<const uint2 *>(a.k + o));
-            } else {
-                qr[i] = kr[i] = make_uint2(0u, 0u);
-            }
-        }
-        const float4 gs4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * BR, c0));
-        const float4 ge4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * BR + 15, c0));
-        const float gsv[4] = {gs4.x, gs4.y, gs4.z, gs4.w}, gev[4] = {ge4.x, ge4.y, ge4.z, ge4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = rr0 + i;
-            const float4 g4 = *reinterpret_cast<const float4 *>(gf + gfi(r, c0));
-            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-            const float2 qa = bf2(qr[i].x), qb = bf2(qr[i].y), ka = bf2(kr[i].x), kb = bf2(kr[i].y);
-            const float qv[4] = {qa.x, qa.y, qb.x, qb.y}, kv[4] = {ka.x, ka.y, kb.x, kb.y};
-            const float iq = rq[r], ik = rk[r];
-            float x[4], y[4], z[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float e1 = ex2_ftz(gv[e] - gsv[e]);
-                x[e] = kv[e] * ik * e1;
-                y[e] = qv[e] * iq * e1;
-                z[e] = kv[e] * ik * ex2_ftz(gev[e] - gv[e]);
-            }
-            const uint32_t o2 = at(r, c0, C);
-            *reinterpret_cast<uint2 *>(sm + Sm::XT + o2) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
-            *reinterpret_cast<uint2 *>(sm + Sm::QT + o2) = make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
-            *reinterpret_cast<uint2 *>(sm + Sm::YT + o2) = make_uint2(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]));
-        }
-        if (warp < 10) {
-            const int PR = pair_R(warp), PI = warp - PR * (PR + 1) / 2;
-            const float4 a4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * PR, c0));
-            const float4 b4 = *reinterpret_cast<const float4 *>(gf + gfi(16 * PI + 15, c0));
-            *reinterpret_cast<float4 *>(ps + warp * D + c0) =
-                make_float4(ex2_ftz(a4.x - b4.x), ex2_ftz(a4.y - b4.y), ex2_ftz(a4.z - b4.z), ex2_ftz(a4.w - b4.w));
-        }
-    }
-    __syncthreads();   // Xm in place
-    // ---- dA_kk = strict_lower(-Xm T^T): dbeta += dA_kk . A_hat, dA_hat = beta dA_kk (both layouts) ----
-    {
-        const int m0 = 16 * qd, n64 = 16 * cg;
-        float acc[2][4];
-        zero_acc(acc);
-        mma_fix<2, false, false, C, C, 0, C>(acc, sbase + Sm::XM, m0, sbase + Sm::TB, n64);
-        float rs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int row = m0 + gq + 8 * hh, col = n64 + 8 * t + 2 * tq;
-                const float x0 = col < row ? -acc[t][2 * hh] : 0.f, x1 = col + 1 < row ? -acc[t][2 * hh + 1] : 0.f;
-                const float2 ah = col < row ? bf2(*reinterpret_cast<const uint32_t *>(sm + Sm::AH + at(row, col, C)))
-                                            : make_float2(0.f, 0.f);
-                rs[hh] += x0 * ah.x + (col + 1 < row ? x1 * ah.y : 0.f);
-                const float b = sbeta[row];
-                const uint32_t pkv = pack_bf16(b * x0, b * x1);
-                *reinterpret_cast<uint32_t *>(sm + Sm::DAH + at(row, col, C)) = pkv;
-                *reinterpret_cast<uint16_t *>(sm + Sm::DAH2 + at(col, row, C)) = (uint16_t)(pkv & 0xffffu);
-                *reinterpret_cast<uint16_t *>(sm + Sm::DAH2 + at(col + 1, row, C)) = (uint16_t)(pkv >> 16);
-            }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float x = rs[hh];
-            x += __shfl_xor_sync(0xffffffffu, x, 1);
-            x += __shfl_xor_sync(0xffffffffu, x, 2);
-            if (tq == 0) dbp[(8 + cg) * C + m0 + gq + 8 * hh] = x;
-        }
-    }
-    tc::fence_proxy_async();
-    tc::fence_before();
-    __syncthreads();   // dA_hat, dA_qk (both layouts), the pairwise operands and scales in place
-    tc::fence_after();
-    // ---- pairwise-decay sums on tcgen05, one N = 64, K = 16 product per block (channel = M) ----
-    //   row side, block I:    D_I[c][r] = sum_{i in I} Y~[i][c] dA[r][i]   (r in blocks R >= I)
-    //   column side, block R: E_R[c][i] = sum_{r in R} X~[r][c] dA[r][i]   (i in blocks I <= R)
-    constexpr uint32_t id_p = tc::idesc_bf16(128, 64, true, false, false);
-    for (int I = 0; I < 4; ++I) {
-        if (tid == 0) {
-            tc::mma(tmem + kPA, desc(dM64, Sm::YT + I * 2048), desc(dK, Sm::DAH + I * 32), id_p, 0u);
-            tc::mma(tmem + kPB, desc(dM64, Sm::YT + I * 2048), desc(dK, Sm::DAQ + I * 32), id_p, 0u);
-            tc::mma(tmem + kPC, desc(dM64, Sm::XT + I * 2048), desc(dK, Sm::DAH2 + I * 32), id_p, 0u);
-            tc::mma(tmem + kPD, desc(dM64, Sm::QT + I * 2048), desc(dK, Sm::DAQ2 + I * 32), id_p, 0u);
-            tc::commit(mb);
-        }
-        ok = wait_mb() && ok;
-        const float ge_b = gf[gfi(r0, c)], ge_e = gf[gfi(r0 + 15, c)];
-        if (cg >= I) {
-            // row side for the rows r of block R = cg: pair (R, I)
-            const float s = ps[pair_of(cg, I) * D + c];
-            float xh[16], xq[16], ak[16], aq[16], ag[16];
-            ld16f(lb + kPA + r0, xh);
-            ld16f(lb + kPB + r0, xq);
-            ld16f(lb + kAK + r0, ak);
-            ld16f(lb + kAQ + r0, aq);
-            ld16f(lb + kAG + r0, ag);
-            tc::wait_ld();
-            dstate::reg_fence(xh);
-            dstate::reg_fence(xq);
-            dstate::reg_fence(ak);
-            dstate::reg_fence(aq);
-            dstate::reg_fence(ag);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = r0 + i;
-                const uint32_t o = at(r, c, C);
-                const float e1 = ex2_ftz(gf[gfi(r, c)] - ge_b);
-                const float ph = s * xh[i], pq = s * xq[i];
-                ak[i] += e1 * ph;
-                aq[i] += e1 * pq;
-                ag[i] += bfl(*reinterpret_cast<const uint16_t *>(sm + Sm::XT + o)) * ph +
-                         bfl(*reinterpret_cast<const uint16_t *>(sm + Sm::QT + o)) * pq;
-            }
-            st16f(lb + kAK + r0, ak);
-            st16f(lb + kAQ + r0, aq);
-            st16f(lb + kAG + r0, ag);
-            tc::wait_st();
-        }
-        // column side for block R = I (the product just issued with X~ / Q~ rows of block I):
-        // columns i of block cg <= I, pair (I, cg)
-        if (cg <= I) {
-            const float s = ps[pair_of(I, cg) * D + c];
-            float xh[16], xq[16], ak[16], ag[16];
-            ld16f(lb + kPC + r0, xh);
-            ld16f(lb + kPD + r0, xq);
-            ld16f(lb + kAK + r0, ak);
-            ld16f(lb + kAG + r0, ag);
-            tc::wait_ld();
-            dstate::reg_fence(xh);
-            dstate::reg_fence(xq);
-            dstate::reg_fence(ak);
-            dstate::reg_fence(ag);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = r0 + i;
-                const float e2 = ex2_ftz(ge_e - gf[gfi(r, c)]);
-                const float p = s * (xh[i] + xq[i]);
-                ak[i] += e2 * p;
-                ag[i] -= bfl(*reinterpret_cast<const uint16_t *>(sm + Sm::YT + at(r, c, C))) * p;
-            }
-            st16f(lb + kAK + r0, ak);
-            st16f(lb + kAG + r0, ag);
-            tc::wait_st();
-        }
-        tc::fence_before();
-        __syncthreads();   // every lane read this block's results before the next products overwrite them
-        tc::fence_after();
-    }
-    // ---- dq, dk through the l2 norms; dg = reverse cumsum of dG + dG_last; dbeta ----
-    {
-        float ak[16], aq[16], ag[16];
-        ld16f(lb + kAK + r0, ak);
-        ld16f(lb + kAQ + r0, aq);
-        ld16f(lb + kAG + r0, ag);
-        tc::wait_ld();
-        dstate::reg_fence(ak);
-        dstate::reg_fence(aq);
-        dstate::reg_fence(ag);
-        float dq_[16], dk_[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            dq_[i] = qh[i] * aq[i];
-            dk_[i] = kh[i] * ak[i];
-        }
-        const float sq = lane_sum16(dq_, lane), sk = lane_sum16(dk_, lane);
-        if (!(lane & 1)) {
-            red[(r0 + lane_sum16_col(lane)) * 4 + qd] = sq;
-            red[256 + (r0 + lane_sum16_col(lane)) * 4 + qd] = sk;
-        }
-        // dG: suffix sums within this warp's block of 16 rows, block totals for the others
-#pragma unroll
-        for (int i = 14; i >= 0; --i) ag[i] += ag[i + 1];
-        tot[cg * D + c] = ag[0];
-        __syncthreads();
-        float off = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) off += dglp[i * D + c];
-        for (int g2 = cg + 1; g2 < 4; ++g2) off += tot[g2 * D + c];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = r0 + i;
-            if (r < L) {
-                const float4 s4 = *reinterpret_cast<const float4 *>(red + r * 4);
-                const float4 k4 = *reinterpret_cast<const float4 *>(red + 256 + r * 4);
-                const float dotq = s4.x + s4.y + s4.z + s4.w, dotk = k4.x + k4.y + k4.z + k4.w;
-                const int64_t o = ((tok0 + r) * H + h) * D + c;
-                a.dq[o] = f2b(rq[r] * (aq[i] - qh[i] * dotq));
-                a.dk[o] = f2b(rk[r] * (ak[i] - kh[i] * dotk));
-                a.dg[o] = ag[i] + off;
-            }
-        }
-        if (tid < L) {
-            float x = 0.f;
-#pragma unroll
-            for (int i = 0; i < 12; ++i) x += dbp[i * C + tid];
-            a.dbeta[(tok0 + tid) * H + h] = x;
-        }
-    }
-    if (!ok && tid == 0) atomicExch(a.status, kStatusTimeout);
-    tc::fence_before();
-    __syncthreads();
-    tc::fence_after();
-    if (warp == 0) tc::dealloc(tmem, kTmemCols);
-}
-}  // namespace grad2
 
 }  // namespace bwd
 
@@ -1749,16 +1149,10 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.g = g; a.beta = beta; a.cu = cu;
     a.n_docs = n_docs; a.T = T; a.H = H;
     a.ws_ck = ws_ck; a.ws_dst = ws_dst;
-    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.status = status;
-#ifdef KDA_BWD_GRAD2
-    e = cudaFuncSetAttribute(grad2::kda_bwd_grad2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad2::Sm::TOTAL);
-    if (e != cudaSuccess) return e;
-    grad2::kda_bwd_grad2_kernel<<<(unsigned)blocks, grad2::kThreads, grad2::Sm::TOTAL, stream>>>(a);
-#else
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
     e = cudaFuncSetAttribute(grad::kda_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad::Sm::TOTAL);
     if (e != cudaSuccess) return e;
     grad::kda_bwd_grad_kernel<<<(unsigned)blocks, grad::kThreads, grad::Sm::TOTAL, stream>>>(a);
-#endif
     return cudaGetLastError();
 }
 
