@@ -244,6 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     const int nchunks = (int)((doc_end - doc_start + 63) / 64);
+    // barrier waits poll in the plain forward and park the thread in the segment passes (measured)
+    constexpr bool kSuspendWaits = kMode != kDocs;
     // the checkpoint block of chunk i of this chain (kCkpt)
     auto ck_block = [&](int i) -> uint8_t * {
         return reinterpret_cast<uint8_t *>(ckpt) + ((size_t)(doc_start / 64 + doc + i) * H + h) * kCkptBytes;
@@ -362,8 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // chunk 0's inputs (one thread polls the barriers; the CTA barrier releases the rest), then its norms
     cp_async_wait_all();
     if (tid == 0) {
-        bool ok = tc::mbar_wait(mbar(kMbQK), 0u, kWaitLimit);
-        ok = tc::mbar_wait(mbar(kMbG), 0u, kWaitLimit) && ok;
+        bool ok = tc::mbar_wait<kSuspendWaits>(mbar(kMbQK), 0u, kWaitLimit);
+        ok = tc::mbar_wait<kSuspendWaits>(mbar(kMbG), 0u, kWaitLimit) && ok;
         if (!ok) *abort_flag = 1;
     }
     __syncthreads();
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // the previous step's U product is done: V, KR and its accumulator are free
-        if (tid == 0 && have_state && !tc::mbar_wait(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
+        if (tid == 0 && have_state && !tc::mbar_wait<kSuspendWaits>(mbar(kMbU), (uint32_t)((s - 1) & 1), kWaitLimit)) *abort_flag = 1;
         // the previous step's output store has read its staging buffer (Kd's buffer, rewritten below)
         if (tid == kStateTid0) tc::bulk_wait_read();
         tc::fence_before();
@@ -623,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // barrier before the W readback)
                 if (warp >= 8) {
                     if (have_next) {
-                        if (lane == 0 && !tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit)) *abort_flag = 1;
+                        if (lane == 0 && !tc::mbar_wait<kSuspendWaits>(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit)) *abort_flag = 1;
                         __syncwarp();
                         norms16((warp - 8) * 16, nL);
                     }
@@ -783,10 +785,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }   // warps 0-7
                 if (tid == 0) {
                     if constexpr (kCkpt) tc::bulk_wait_read();   // the previous chunk's B2 copy has read it
-                    bool ok = tc::mbar_wait(mbar(kMbWQ), par, kWaitLimit);
+                    bool ok = tc::mbar_wait<kSuspendWaits>(mbar(kMbWQ), par, kWaitLimit);
                     // B2 is free once the previous chunk's state product has read it
-                    if (have_state) ok = tc::mbar_wait(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
-                    if constexpr (kMode != kTransition) ok = tc::mbar_wait(mbar(kMbV), par, kWaitLimit) && ok;   // v(s) landed
+                    if (have_state) ok = tc::mbar_wait<kSuspendWaits>(mbar(kMb2), (uint32_t)((s - 1) & 1), kWaitLimit) && ok;
+                    if constexpr (kMode != kTransition) ok = tc::mbar_wait<kSuspendWaits>(mbar(kMbV), par, kWaitLimit) && ok;   // v(s) landed
                     if (!ok) *abort_flag = 1;
                     tc::fence_before();
                 }
@@ -928,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (tid == kStateTid0) tc::commit(mbar(kMb2));
                 }
                 if (tid == kStateTid0) {
-                    if (!tc::mbar_wait(mbar(kMb2), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                    if (!tc::mbar_wait<kSuspendWaits>(mbar(kMb2), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
                     tc::fence_before();
                 }
                 bar_state();
@@ -974,7 +976,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                dK + (uint64_t)((S::KDT + kk * 32) >> 4) + (uint64_t)(nbuf * (16384 >> 4)), id4, 1u);
                     tc::commit(mbar(kMb4));
                     // the output tile is staged in Kd's buffer, which the state update reads
-                    if (!tc::mbar_wait(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
+                    if (!tc::mbar_wait<kSuspendWaits>(mbar(kMb4), (uint32_t)(n & 1), kWaitLimit)) *abort_flag = 1;
                     if constexpr (kCkpt) tc::bulk_wait_read();   // and the checkpoint copy of Kd^T
                     tc::fence_before();
                 }
@@ -1046,8 +1048,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // the raw q, k and g of chunk s+1 have landed before the step ends
             if (tid == kStateTid0 && have_next) {
-                bool ok = tc::mbar_wait(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit);
-                ok = tc::mbar_wait(mbar(kMbG), (uint32_t)((s + 1) & 1), kWaitLimit) && ok;
+                bool ok = tc::mbar_wait<kSuspendWaits>(mbar(kMbQK), (uint32_t)((s + 1) & 1), kWaitLimit);
+                ok = tc::mbar_wait<kSuspendWaits>(mbar(kMbG), (uint32_t)((s + 1) & 1), kWaitLimit) && ok;
                 if (!ok) *abort_flag = 1;
             }
         }
@@ -1080,8 +1082,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) atomicExch(status, kStatusTimeout);
         // let any tensor-core work or copy still in flight land before TMEM and shared memory go away
         for (int i = 0; i < kNumMbar; ++i) {
-            tc::mbar_wait(mbar(i), 0u, kWaitLimit / 16);
-            tc::mbar_wait(mbar(i), 1u, kWaitLimit / 16);
+            tc::mbar_wait<kSuspendWaits>(mbar(i), 0u, kWaitLimit / 16);
+            tc::mbar_wait<kSuspendWaits>(mbar(i), 1u, kWaitLimit / 16);
         }
     }
     tc::fence_before();

@@ -139,23 +139,34 @@ __device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.
 __device__ __forceinline__ void mbar_init(uint32_t saddr, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr), "r"(count) : "memory");
 }
+// kSuspend: give the hardware a suspend-time hint (1 ms) so that the thread is parked until the phase
+// completes; without it the thread polls.  Which one is faster depends on the kernel: the plain
+// forward measured 1.3 % faster polling, its segment passes 2.5 % faster parked.
+template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_try(uint32_t saddr, uint32_t parity) {
     uint32_t ok;
-    // the suspend-time hint (ns) lets the hardware park the thread until the phase
-    // completes instead of spinning through the issue slots
-    asm volatile(
-        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\nselp.b32 %0, 1, 0, P;\n}\n"
-        : "=r"(ok)
-        : "r"(saddr), "r"(parity), "r"(1000000u)
-        : "memory");
+    if constexpr (kSuspend) {
+        asm volatile(
+            "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\nselp.b32 %0, 1, 0, P;\n}\n"
+            : "=r"(ok)
+            : "r"(saddr), "r"(parity), "r"(1000000u)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\nselp.b32 %0, 1, 0, P;\n}\n"
+            : "=r"(ok)
+            : "r"(saddr), "r"(parity)
+            : "memory");
+    }
     return ok != 0;
 }
 // Wait for phase `parity` to complete, giving up after ~`limit` clock cycles.  (Inlined: an out-of-line
 // copy measured 4 % slower in the forward kernel.)
+template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long long limit) {
-    if (mbar_try(saddr, parity)) return true;
+    if (mbar_try<kSuspend>(saddr, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try(saddr, parity))
+    while (!mbar_try<kSuspend>(saddr, parity))
         if (clock64() - t0 > limit) return false;
     return true;
 }
