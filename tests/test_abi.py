@@ -96,3 +96,13 @@ def test_resolve_mode():
     assert resolve_mode(RECURRENT_MAX_LEN + 1) == "chunk" and resolve_mode(65536) == "chunk"
     with pytest.raises(ValueError):
         resolve_mode(-1)
+
+
+def test_backward_workspace_size(L):
+    """The backward's workspace is one block per chunk slot and head: the forward pass's checkpoint
+    block (S^T and U~^T, B2, Kd^T, A_qk, T, A_hat, D: 123904 bytes) and the dS sweep's block (dS^T
+    and dU~^T: 49152 bytes); slots are T / 64 + n_docs per head, an upper bound that does not read
+    cu_seqlens."""
+    per = 123904 + 49152
+    for n_docs, T, H in ((1, 64, 1), (5, 1328, 4), (16, 32768, 32), (1, 65536, 32)):
+        assert L.kda_chunk_bwd_workspace_size(n_docs, T, H) == (T // 64 + n_docs) * H * per
