@@ -888,7 +888,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // two loads in flight: the next 32 columns are read while the current ones are converted;
                 // the product's first four k-steps (key channels 0-63) start once their bf16 copy is in
                 // place, while the second half is converted
-                constexpr uint32_t id2 = tc::idesc_bf16(128, 128, false, true, false);
+                // (the backward's checkpoint pass has no output: its state product needs U~ alone)
+                constexpr uint32_t id2 = tc::idesc_bf16(128, kCkpt ? 64 : 128, false, true, false);
                 auto state_mma = [&](int kk0) {   // [U~^T | (Q~ S)^T] accumulated onto [U^T | 0]
                     if (kk0 == 0 && have_intra) asm volatile("bar.sync 4, 160;" ::: "memory");
                     tc::wait_st();
@@ -963,12 +964,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (tid == kStateTid0) {
                     tc::fence_after();
                     // O^T += U~^T A_qk^T (A_qk [r][i] is the K-major B operand), then the state update
-                    constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, false, false);
+                    if constexpr (!kCkpt) {
+                        constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, false, false);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + dcol + 64, tmem + kUB + 8 * kk,
-                               dK + (uint64_t)((S::AQK + kk * 32) >> 4) + (uint64_t)(nbuf * (8192 >> 4)), id_o,
-                               1u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(tmem + dcol + 64, tmem + kUB + 8 * kk,
+                                   dK + (uint64_t)((S::AQK + kk * 32) >> 4) + (uint64_t)(nbuf * (8192 >> 4)), id_o,
+                                   1u);
+                    }
                     constexpr uint32_t id4 = tc::idesc_bf16(128, 128, false, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -984,8 +987,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_after();
                 // O^T (columns 64-127; the output scale is already applied): lane v holds o[r][v].
                 // Lane pairs swap values so that each thread writes the pair (v, v+1) of one row.  (A
-                // transition pass has no output.)
-                if constexpr (kMode != kTransition) {
+                // transition pass and the backward's checkpoint pass have no output.)
+                if constexpr (kMode != kTransition && !kCkpt) {
                     const int vcol = 32 * lq + lane;
                     const bool odd = lane & 1;
                     if (pL == 64) {
