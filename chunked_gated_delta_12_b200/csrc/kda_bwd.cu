@@ -551,6 +551,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     float *tot = reinterpret_cast<float *>(sm + Sm::TOT), *gf = reinterpret_cast<float *>(sm + Sm::GF);
     float *ps = reinterpret_cast<float *>(sm + Sm::PS);
 
+    // ---- the prep's rows of q, k, v, g first, so that their latency overlaps the tile copies below
+    //      (warp w holds rows 4w .. 4w + 3, lane l channels 4l .. 4l + 3; rows past the end are zero) ----
+    const int pc0 = 4 * lane, pr0 = 4 * warp;
+    uint2 qr[4], kr[4], vr[4];
+    float4 gr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = pr0 + i;
+        if (r < L) {
+            const int64_t o = ((tok0 + r) * H + h) * D + pc0;
+            qr[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + o));
+            kr[i] = __ldg(reinterpret_cast<const uint2 *>(a.k + o));
+            vr[i] = __ldg(reinterpret_cast<const uint2 *>(a.v + o));
+            gr[i] = __ldg(reinterpret_cast<const float4 *>(a.g + o));
+        } else {
+            qr[i] = kr[i] = vr[i] = make_uint2(0u, 0u);
+            gr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
     // ---- loads: workspace tiles as flat images, dout rows (zero past the document end) ----
     {
         // S^T, U~^T, dS^T, dU~^T: column groups -> swizzled atoms; T, A_hat: flat images
@@ -580,26 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     if (tid < C) sbeta[tid] = tid < L ? __ldg(a.beta + (tok0 + tid) * H + h) : 0.f;
     if (tid < D) dls[tid] = reinterpret_cast<const float *>(ck + Ws::DL)[tid];
 
-    // ---- prep: warp w holds rows 4w .. 4w + 3, lane l channels 4l .. 4l + 3: row norms, G (log2
-    //      units), beta k^ e^G and beta v ----
+    // ---- prep: row norms, G (log2 units), beta k^ e^G and beta v ----
     {
-        const int c0 = 4 * lane, r0 = 4 * warp;
-        uint2 qr[4], kr[4], vr[4];
-        float4 gr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = r0 + i;
-            if (r < L) {
-                const int64_t o = ((tok0 + r) * H + h) * D + c0;
-                qr[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + o));
-                kr[i] = __ldg(reinterpret_cast<const uint2 *>(a.k + o));
-                vr[i] = __ldg(reinterpret_cast<const uint2 *>(a.v + o));
-                gr[i] = __ldg(reinterpret_cast<const float4 *>(a.g + o));
-            } else {
-                qr[i] = kr[i] = vr[i] = make_uint2(0u, 0u);
-                gr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
+        const int c0 = pc0, r0 = pr0;
         float rkr[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
