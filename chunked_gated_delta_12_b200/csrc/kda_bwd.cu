@@ -572,15 +572,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
     }
     // ---- loads: workspace tiles as flat images, dout rows (zero past the document end) ----
     {
-        // S^T, U~^T, dS^T, dU~^T: column groups -> swizzled atoms; T, A_hat: flat images
+        // S^T, U~^T, dS^T, dU~^T: column groups -> swizzled atoms; T, A_hat: flat images.  Consecutive
+        // threads take consecutive 16-byte pieces of a group image (piece i of the tile is piece j of
+        // row r in group grp, i.e. grp_off(r, grp * G / 8 + j, G) = 16 i), so that every warp reads whole
+        // 128-byte lines; reading row by row across the groups instead fills shared memory at half the rate.
         const uint8_t *gsrc[4] = {ck + Ws::S, ck + Ws::UT, dsb + Ws::DS, dsb + Ws::DU};
         const int gdst[4] = {Sm::ST, Sm::UT, Sm::DST, Sm::DUT}, gcols[4] = {128, 64, 128, 64}, ggrp[4] = {16, 32, 32, 32};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-            const int per_row = gcols[t] / 8;
-            for (int i = tid; i < 128 * per_row; i += kThreads) {
-                const int r = i / per_row, m = i % per_row;
-                cp_async16(sbase + gdst[t] + at(r, 8 * m, D), gsrc[t] + grp_off(r, m, ggrp[t]), 16);
+            const int pg = ggrp[t] / 8;   // pieces per row inside a group
+            for (int i = tid; i < 16 * gcols[t]; i += kThreads) {
+                const int grp = i / (128 * pg), k = i % (128 * pg), r = k / pg, m = grp * pg + k % pg;
+                cp_async16(sbase + gdst[t] + at(r, 8 * m, D), gsrc[t] + 16 * i, 16);
             }
         }
         for (int i = tid; i < 8192 / 16; i += kThreads) {
