@@ -257,12 +257,13 @@ struct Sm {
     static constexpr int AQ = 16384;      // scale A_qk [64 t][64 s]     MN-major B (K = t, N = s)
     static constexpr int WN = 24576;      // -W^T [128 c][64 s]          K-major B (N = c, K = s)
     static constexpr int QG = 40960;      // scale QG^T [128 c][64 t]    K-major B (N = c, K = t)
-    static constexpr int DO = 57344;      // dout [64 t][128 v]          MN-major A (K = t, M = v)
-    static constexpr int DL = 73728;      // D fp32 [128]
-    static constexpr int MBAR = DL + 512; // mbarriers: inputs, dU~ product, state product
+    static constexpr int DO = 57344;      // two buffers: dout [64 t][128 v]   MN-major A (K = t, M = v)
+    static constexpr int DL = 90112;      // D fp32 [128]
+    static constexpr int MBAR = DL + 512; // mbarriers: Kd/A_qk/D copies, [-W | QG] copy, dU~ product, state product
     static constexpr int TBASE = MBAR + 32, FLAG = TBASE + 8;
     static constexpr int TOTAL = FLAG + 8;
-    static constexpr uint32_t kInBytes = 57344 + 512;   // bulk bytes per chunk (KD..WN, DL)
+    static constexpr uint32_t kBytesA = 16384 + 8192 + 512;   // Kd^T, A_qk, D
+    static constexpr uint32_t kBytesB = 32768;                // [-W^T | scale QG^T]
 };
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar) {
@@ -302,12 +303,13 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
     const int nch = (int)((d1 - d0 + C - 1) / C);
     const int64_t slot0 = d0 / C + doc;
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t mb_in = sbase + Sm::MBAR, mb_u = mb_in + 8, mb_s = mb_in + 16;
+    const uint32_t mb_a = sbase + Sm::MBAR, mb_b = mb_a + 8, mb_u = mb_a + 16, mb_s = mb_a + 24;
     volatile int *flag = reinterpret_cast<volatile int *>(sm + Sm::FLAG);
     const float *dl = reinterpret_cast<const float *>(sm + Sm::DL);
     if (warp == 0) tc::alloc(sbase + Sm::TBASE, kTmemCols);
     if (tid == 0) {
-        tc::mbar_init(mb_in, 1);
+        tc::mbar_init(mb_a, 1);
+        tc::mbar_init(mb_b, 1);
         tc::mbar_init(mb_u, 1);
         tc::mbar_init(mb_s, 1);
         *flag = 0;
@@ -327,24 +329,30 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
     constexpr uint32_t id_s1 = tc::idesc_bf16(128, 128, true, false, false);   // dO^T x QG
     constexpr uint32_t id_s2 = tc::idesc_bf16(128, 128, false, false, false);  // dU~^T_bf16 (TMEM) x (-W)
 
-    auto issue_loads = [&](int j) {
+    // Each input group of chunk j is requested as soon as its buffer is free: Kd^T, A_qk and D once
+    // chunk j+1's dU~ product and scaling have read them, [-W^T | scale QG^T] once chunk j+1's state
+    // product has, and the dout rows a whole step ahead into the second buffer.
+    auto load_a = [&](int j) {   // Kd^T, A_qk, D of chunk j (one thread)
+        const uint8_t *src = ws_ck + ((size_t)(slot0 + j) * H + h) * Ws::CK;
+        tc::mbar_expect_tx(mb_a, Sm::kBytesA);
+        bulk_load(sbase + Sm::KD, src + Ws::KD, 16384, mb_a);
+        bulk_load(sbase + Sm::AQ, src + Ws::AQ, 8192, mb_a);
+        bulk_load(sbase + Sm::DL, src + Ws::DL, 512, mb_a);
+    };
+    auto load_b = [&](int j) {   // [-W^T | scale QG^T] of chunk j (one thread)
+        const uint8_t *src = ws_ck + ((size_t)(slot0 + j) * H + h) * Ws::CK;
+        tc::mbar_expect_tx(mb_b, Sm::kBytesB);
+        bulk_load(sbase + Sm::WN, src + Ws::B2, 32768, mb_b);
+    };
+    auto load_do = [&](int j, int b) {   // dout rows of chunk j (zero past the document end) into buffer b
         const int64_t tok = d0 + (int64_t)j * C;
         const int Lj = (int)((d1 - tok) < C ? (d1 - tok) : C);
-        if (tid == 0) {
-            const uint8_t *src = ws_ck + ((size_t)(slot0 + j) * H + h) * Ws::CK;
-            tc::mbar_expect_tx(mb_in, Sm::kInBytes);
-            bulk_load(sbase + Sm::KD, src + Ws::KD, 16384, mb_in);
-            bulk_load(sbase + Sm::AQ, src + Ws::AQ, 8192, mb_in);
-            bulk_load(sbase + Sm::WN, src + Ws::B2, 32768, mb_in);   // [-W^T | scale QG^T]
-            bulk_load(sbase + Sm::DL, src + Ws::DL, 512, mb_in);
-        }
-        // dout rows (zero past the document end) into the swizzled MN-major tile
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int idx = tid + i * kThreads, t = idx >> 4, m = idx & 15;
             const bool ok = t < Lj;
             const uint16_t *src = ok ? dout + ((tok + t) * H + h) * D + 8 * m : dout;
-            cp_async16(sbase + Sm::DO + at(t, 8 * m, C), src, ok ? 16 : 0);
+            cp_async16(sbase + Sm::DO + b * 16384 + at(t, 8 * m, C), src, ok ? 16 : 0);
         }
         cp_async_commit();
     };
@@ -380,22 +388,30 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
         tc::wait_st();
     }
     store_ds(nch - 1, false);
-    issue_loads(nch - 1);
-    int last_j = nch - 1;   // the chunk whose inputs were issued last
+    load_do(nch - 1, 0);
+    if (tid == 0) {
+        load_a(nch - 1);
+        load_b(nch - 1);
+    }
+    int last_a = nch - 1, last_b = nch - 1;   // the chunks whose copies were issued last
 
     bool aborted = false;
     int n_commit_s = 0;   // completions of the state-product barrier so far (the next has parity n & 1)
     for (int j = nch - 1; j >= 0; --j) {
-        const uint32_t par = (uint32_t)((nch - 1 - j) & 1);
-        cp_async_wait_all();
+        const int b = (nch - 1 - j) & 1;   // dout buffer of chunk j
+        const uint32_t par = (uint32_t)b;
+        const uint32_t dofs = (uint32_t)(b * (16384 >> 4));
+        cp_async_wait_all();   // chunk j's dout rows (the only group in flight)
         tc::fence_proxy_async();
-        bool ok = tc::mbar_wait(mb_in, par, kWaitLimit);
+        bool ok = tc::mbar_wait(mb_a, par, kWaitLimit);
         tc::wait_st();
         tc::fence_before();
         if (__syncthreads_or(!ok)) {
             aborted = true;
             break;
         }
+        // the other dout buffer was last read by chunk j+1's products, which have completed
+        if (j > 0) load_do(j - 1, b ^ 1);
         if (tid == 0) {
             tc::fence_after();
 #pragma unroll
@@ -403,8 +419,8 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
                 mma_ts(tmem + kDU, tmem + kSB + 8 * kk, dM + (uint64_t)((Sm::KD + kk * 2048) >> 4), id_u1, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                tc::mma(tmem + kDU, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dM + (uint64_t)((Sm::AQ + kk * 2048) >> 4),
-                        id_u2, 1u);
+                tc::mma(tmem + kDU, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4) + dofs,
+                        dM + (uint64_t)((Sm::AQ + kk * 2048) >> 4), id_u2, 1u);
             tc::commit(mb_u);
         }
         // dS^T <- dS^T Diag(D) (the fp32 columns; the product above reads the bf16 copy)
@@ -439,18 +455,23 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
                         make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
             }
         }
+        ok = tc::mbar_wait(mb_b, par, kWaitLimit) && ok;   // chunk j's [-W^T | scale QG^T]
         tc::wait_st();
+        tc::fence_proxy_async();   // D was read through the generic proxy; its buffer is refilled below
         tc::fence_before();
         if (__syncthreads_or(!ok)) {
             aborted = true;
             break;
         }
+        // Kd^T and A_qk (read by the dU~ product, complete) and D (read by every thread above) are free
+        if (j > 0 && tid == 0) load_a(j - 1);
+        if (j > 0) last_a = j - 1;
         if (tid == 0) {
             tc::fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                tc::mma(tmem + kFS, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4), dK + (uint64_t)((Sm::QG + kk * 32) >> 4),
-                        id_s1, 1u);
+                tc::mma(tmem + kFS, dM + (uint64_t)((Sm::DO + kk * 2048) >> 4) + dofs,
+                        dK + (uint64_t)((Sm::QG + kk * 32) >> 4), id_s1, 1u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_ts(tmem + kFS, tmem + kUB + 8 * kk, dK + (uint64_t)((Sm::WN + kk * 32) >> 4), id_s2, 1u);
@@ -464,8 +485,8 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
             break;
         }
         if (j > 0) {
-            issue_loads(j - 1);
-            last_j = j - 1;
+            if (tid == 0) load_b(j - 1);   // [-W^T | scale QG^T] was read by the state product
+            last_b = j - 1;
             store_ds(j - 1, true);
             tc::wait_st();
         }
@@ -475,7 +496,8 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
         // operations still in flight before the CTA's shared memory and columns are released
         if (tid == 0) {
             atomicExch(status, kStatusTimeout);
-            tc::mbar_wait(mb_in, (uint32_t)((nch - 1 - last_j) & 1), kWaitLimit);
+            tc::mbar_wait(mb_a, (uint32_t)((nch - 1 - last_a) & 1), kWaitLimit);
+            tc::mbar_wait(mb_b, (uint32_t)((nch - 1 - last_b) & 1), kWaitLimit);
             tc::commit(mb_s);
             tc::mbar_wait(mb_s, (uint32_t)(n_commit_s & 1), kWaitLimit);
         }
