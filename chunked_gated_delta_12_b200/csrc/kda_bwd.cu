@@ -555,8 +555,12 @@ struct Args {
     uint16_t *dq, *dk, *dv;
     float *dg, *dbeta;
 };
+// TMA maps of dq and dk over [T, H * 128] bf16, 64 x 64 boxes with 128-byte swizzled rows
+struct OutMaps {
+    CUtensorMap dq, dk;
+};
 
-__global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a, const __grid_constant__ OutMaps om) {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
     const int H = a.H, slot = blockIdx.x / H, h = blockIdx.x % H;
@@ -1093,6 +1097,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
         }
     }
     __syncthreads();   // row dots in place; every read of G is done
+    // A whole chunk stages dq and dk as bf16 tiles in the space S^T and dW held (free since dBk),
+    // [64 rows][128] each with 128-byte swizzled rows, and writes them with four TMA stores; the
+    // per-thread pairs would otherwise leave as scattered 4-byte stores (8 rows x 16 bytes per warp
+    // instruction).  A partial chunk, whose rows past the document end belong to the next document,
+    // stores its valid rows directly.
+    const bool full = L == C;
 #pragma unroll
     for (int t = 0; t < 4; ++t)
 #pragma unroll
@@ -1105,14 +1115,29 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
                 const float sq = s4.x + s4.y + s4.z + s4.w, sk = k4.x + k4.y + k4.z + k4.w;
                 const float2 qr = bf2(qf[t][hh]), kr = bf2(kf[t][hh]);
                 const float iq = rq[row], ik = rk[row];
-                const int64_t o = ((tok0 + row) * H + h) * D + col;
-                *reinterpret_cast<uint32_t *>(a.dq + o) =
+                const uint32_t pq =
                     pack_bf16(iq * (dqn[t][2 * hh] - qr.x * iq * sq), iq * (dqn[t][2 * hh + 1] - qr.y * iq * sq));
-                *reinterpret_cast<uint32_t *>(a.dk + o) =
+                const uint32_t pk =
                     pack_bf16(ik * (dkn[t][2 * hh] - kr.x * ik * sk), ik * (dkn[t][2 * hh + 1] - kr.y * ik * sk));
+                if (full) {
+                    *reinterpret_cast<uint32_t *>(sm + Sm::ST + at(row, col, C)) = pq;
+                    *reinterpret_cast<uint32_t *>(sm + Sm::ST + 16384 + at(row, col, C)) = pk;
+                } else {
+                    const int64_t o = ((tok0 + row) * H + h) * D + col;
+                    *reinterpret_cast<uint32_t *>(a.dq + o) = pq;
+                    *reinterpret_cast<uint32_t *>(a.dk + o) = pk;
+                }
             }
         }
+    if (full) tc::fence_proxy_async();   // the staged tiles are read by the TMA engine
     __syncthreads();   // dG in place
+    if (full && tid == 0) {
+        tc::tma_store_2d(&om.dq, h * D, (int)tok0, sbase + Sm::ST);
+        tc::tma_store_2d(&om.dq, h * D + 64, (int)tok0, sbase + Sm::ST + 8192);
+        tc::tma_store_2d(&om.dk, h * D, (int)tok0, sbase + Sm::ST + 16384);
+        tc::tma_store_2d(&om.dk, h * D + 64, (int)tok0, sbase + Sm::ST + 24576);
+        tc::bulk_commit();
+    }
     // ---- dg = reverse cumsum of dG over the chunk + dG_last (which reaches every row); dbeta ----
     {
         const int c = tid & (D - 1), qd = tid >> 7;
@@ -1139,6 +1164,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a)
             a.dbeta[(tok0 + tid) * H + h] = x;
         }
     }
+    if (full && tid == 0) tc::bulk_wait();   // the TMA stores are done before shared memory goes away
 }
 }  // namespace grad
 
@@ -1159,7 +1185,7 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     const size_t blocks = ((size_t)(T / C) + (size_t)n_docs) * (size_t)H;
     uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
     uint8_t *ws_ck = ws, *ws_dst = ws + blocks * Ws::CK;
-    // 1. forward with checkpoints (its output o goes to dq, which is overwritten below)
+    // 1. forward with checkpoints (this instance forms no output; dq only gives its unused output map a base)
     cudaError_t e = launch_fwd_pipe(q, k, v, g, beta, cu, n_docs, T, H, nullptr, nullptr, dq, status, stream,
                                     reinterpret_cast<uint16_t *>(ws_ck));
     if (e != cudaSuccess) return e;
@@ -1177,9 +1203,16 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     a.n_docs = n_docs; a.T = T; a.H = H;
     a.ws_ck = ws_ck; a.ws_dst = ws_dst;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
+    grad::OutMaps om;
+    const uint64_t cols = (uint64_t)H * D;
+    if (!pipe_path::make_map(&om.dq, dq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !pipe_path::make_map(&om.dk, dk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(grad::kda_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad::Sm::TOTAL);
     if (e != cudaSuccess) return e;
-    grad::kda_bwd_grad_kernel<<<(unsigned)blocks, grad::kThreads, grad::Sm::TOTAL, stream>>>(a);
+    grad::kda_bwd_grad_kernel<<<(unsigned)blocks, grad::kThreads, grad::Sm::TOTAL, stream>>>(a, om);
     return cudaGetLastError();
 }
 

@@ -1,6 +1,7 @@
 // kda_internal.h -- launchers shared between the libkda kernel files and its C ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -40,6 +41,13 @@ cudaError_t launch_fwd_segments(bool transition, const uint16_t *q, const uint16
 cudaError_t launch_fwd_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                                  const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
                                  const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream);
+
+// 2-D TMA map over a row-major [rows, cols] tensor (cols contiguous) with box [box_rows, box_cols]
+// (kda_fwd_pipe.cu); false when the driver's encoder is unavailable or rejects the arguments.
+namespace pipe_path {
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows, uint64_t cols,
+              uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz);
+}
 
 // Recompute backward: dq, dk, dv (bf16), dg, dbeta (fp32) from the forward inputs and dout.
 // workspace holds bwd_workspace_floats(n_docs, T, H) floats (entering states of every chunk
