@@ -555,9 +555,9 @@ struct Args {
     uint16_t *dq, *dk, *dv;
     float *dg, *dbeta;
 };
-// TMA maps of dq and dk over [T, H * 128] bf16, 64 x 64 boxes with 128-byte swizzled rows
+// TMA maps of dq, dk and dv over [T, H * 128] bf16, 64 x 64 boxes with 128-byte swizzled rows
 struct OutMaps {
-    CUtensorMap dq, dk;
+    CUtensorMap dq, dk, dv;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a, const __grid_constant__ OutMaps om) {
@@ -568,6 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a,
     int64_t tok0;
     if (!slot_chunk(a.cu, a.n_docs, a.T, slot, doc, tok0, L)) return;
     const size_t blk = (size_t)slot * H + h;
+    // A whole chunk writes dq, dk and dv by TMA stores from staged tiles; a partial chunk, whose rows
+    // past the document end belong to the next document, stores its valid rows directly.
+    const bool full = L == C;
     const uint8_t *ck = a.ws_ck + blk * Ws::CK, *dsb = a.ws_dst + blk * Ws::DST;
     const uint32_t sbase = smem_u32(sm);
     float *rq = reinterpret_cast<float *>(sm + Sm::RQ), *rk = reinterpret_cast<float *>(sm + Sm::RK);
@@ -891,7 +894,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a,
                     const float2 vr = bf2(vp[t][hh]);
                     rs[hh] += x0 * vr.x + x1 * vr.y;
                     const float b = sbeta[row];
-                    *reinterpret_cast<uint32_t *>(a.dv + ((tok0 + row) * H + h) * D + col) = pack_bf16(b * x0, b * x1);
+                    const uint32_t pv = pack_bf16(b * x0, b * x1);
+                    if (full)   // dout's tile is free since dA_qk
+                        *reinterpret_cast<uint32_t *>(sm + Sm::DO + at(row, col, C)) = pv;
+                    else
+                        *reinterpret_cast<uint32_t *>(a.dv + ((tok0 + row) * H + h) * D + col) = pv;
                 }
             }
 #pragma unroll
@@ -902,7 +909,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a,
             if (tq == 0) dbp[(4 + cb) * C + m0 + gq + 8 * hh] = x;
         }
     }
+    if (full) tc::fence_proxy_async();   // the staged dv tile is read by the TMA engine
     __syncthreads();   // dT in place; dW, dU~^T, beta V, beta KG are read
+    if (full && tid == 0) {
+        tc::tma_store_2d(&om.dv, h * D, (int)tok0, sbase + Sm::DO);
+        tc::tma_store_2d(&om.dv, h * D + 64, (int)tok0, sbase + Sm::DO + 8192);
+        tc::bulk_commit();
+    }
     // ---- Xm = T^T dT ----
     {
         float acc[2][4];
@@ -1100,9 +1113,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a,
     // A whole chunk stages dq and dk as bf16 tiles in the space S^T and dW held (free since dBk),
     // [64 rows][128] each with 128-byte swizzled rows, and writes them with four TMA stores; the
     // per-thread pairs would otherwise leave as scattered 4-byte stores (8 rows x 16 bytes per warp
-    // instruction).  A partial chunk, whose rows past the document end belong to the next document,
-    // stores its valid rows directly.
-    const bool full = L == C;
+    // instruction).
 #pragma unroll
     for (int t = 0; t < 4; ++t)
 #pragma unroll
@@ -1208,6 +1219,8 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     if (!pipe_path::make_map(&om.dq, dq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B) ||
         !pipe_path::make_map(&om.dk, dk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !pipe_path::make_map(&om.dv, dv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(grad::kda_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad::Sm::TOTAL);
