@@ -555,9 +555,10 @@ struct Args {
     uint16_t *dq, *dk, *dv;
     float *dg, *dbeta;
 };
-// TMA maps of dq, dk and dv over [T, H * 128] bf16, 64 x 64 boxes with 128-byte swizzled rows
+// TMA maps of dq, dk and dv over [T, H * 128] bf16, 64 x 64 boxes with 128-byte swizzled rows, and of
+// dg over [T, H * 128] fp32, 64-row x 128-column boxes, unswizzled
 struct OutMaps {
-    CUtensorMap dq, dk, dv;
+    CUtensorMap dq, dk, dv, dg;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a, const __grid_constant__ OutMaps om) {
@@ -1163,10 +1164,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a,
 #pragma unroll
         for (int i = 0; i < 6; ++i) off += dglp[i * D + c];
         for (int q2 = qd + 1; q2 < 4; ++q2) off += tot[q2 * D + c];
+        // a whole chunk stages dg row-major in G's space (every read of G is done: barrier above) for
+        // one TMA store; a partial chunk stores its valid rows directly
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int r = 16 * qd + i;
-            if (r < L) a.dg[((tok0 + r) * H + h) * D + c] = x[i] + off;
+            if (full) gf[r * D + c] = x[i] + off;
+            else if (r < L) a.dg[((tok0 + r) * H + h) * D + c] = x[i] + off;
         }
         if (tid < L) {
             float x = 0.f;
@@ -1175,7 +1179,15 @@ __global__ void __launch_bounds__(kThreads, 1) kda_bwd_grad_kernel(const Args a,
             a.dbeta[(tok0 + tid) * H + h] = x;
         }
     }
-    if (full && tid == 0) tc::bulk_wait();   // the TMA stores are done before shared memory goes away
+    if (full) {
+        tc::fence_proxy_async();   // the staged dg tile is read by the TMA engine
+        __syncthreads();
+        if (tid == 0) {
+            tc::tma_store_2d(&om.dg, h * D, (int)tok0, sbase + Sm::GF);
+            tc::bulk_commit();
+            tc::bulk_wait_read();   // the TMA stores have read their tiles before shared memory goes away
+        }
+    }
 }
 }  // namespace grad
 
@@ -1221,7 +1233,9 @@ cudaError_t launch_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
         !pipe_path::make_map(&om.dk, dk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B) ||
         !pipe_path::make_map(&om.dv, dv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, cols, 64, 64,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !pipe_path::make_map(&om.dg, dg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)T, cols, 64, 128,
+                             CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(grad::kda_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, grad::Sm::TOTAL);
     if (e != cudaSuccess) return e;
