@@ -389,7 +389,8 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
     }
     store_ds(nch - 1, false);
     load_do(nch - 1, 0);
-    if (tid == 0) {
+    // the copies are issued by thread 32, so that thread 0 issues the products without waiting
+    if (tid == 32) {
         load_a(nch - 1);
         load_b(nch - 1);
     }
@@ -464,7 +465,7 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
             break;
         }
         // Kd^T and A_qk (read by the dU~ product, complete) and D (read by every thread above) are free
-        if (j > 0 && tid == 0) load_a(j - 1);
+        if (j > 0 && tid == 32) load_a(j - 1);
         if (j > 0) last_a = j - 1;
         if (tid == 0) {
             tc::fence_after();
@@ -485,7 +486,7 @@ kda_bwd_dstate_kernel(const uint16_t *dout, const int32_t *cu, int n_docs, int64
             break;
         }
         if (j > 0) {
-            if (tid == 0) load_b(j - 1);   // [-W^T | scale QG^T] was read by the state product
+            if (tid == 32) load_b(j - 1);   // [-W^T | scale QG^T] was read by the state product
             last_b = j - 1;
             store_ds(j - 1, true);
             tc::wait_st();
