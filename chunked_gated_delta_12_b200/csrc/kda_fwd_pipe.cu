@@ -179,9 +179,10 @@ struct Maps {
     CUtensorMap q, k, g, v, o;
 };
 
-// kCkpt: also store, per chunk and head, the state entering the chunk and the chunk's U~ into `ckpt`
-// (the backward's checkpoints: S^T[v][c] and U~^T[v][s] as bf16 in 128-byte-swizzled atoms of 128
-// rows v, 32 KB + 16 KB); a separate instance, so that the plain forward carries no trace of it.
+// kCkpt: the backward's forward pass: store, per chunk and head, the checkpoint block described at
+// kCkS..kCkptBytes into `ckpt` (the state entering the chunk, U~ and the chunk's operand tiles), and
+// form no output (neither O nor the (Q~ S)^T half of the state product); a separate instance, so that
+// the plain forward carries no trace of it.
 // kMode: what a CTA's token range is -- kDocs: document blockIdx.x / H of cu_seqlens (every plain
 // forward); kSegs: entry blockIdx.x / H of a segment table built on the device (a document cut into
 // pieces, see kda_split.cu), outputs written; kTransition: the same with v taken as zero, the

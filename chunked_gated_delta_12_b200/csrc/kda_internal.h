@@ -15,9 +15,11 @@ constexpr int kStatusTimeout = 5;
 // columns, two chunks in flight (intra-chunk work of chunk s overlapped with the
 // state update of chunk s-1).
 // h0 / ht: optional initial / final states, [n_docs * H][128][128] fp32 (NULL: zero / not written).
-// ckpt: optional, receives per chunk the state entering it, S^T[v][c], and its U~^T[v][s], both bf16 in
-// 128-byte-swizzled atoms of 128 rows (16384 + 8192 values), in slot (cu[d] / 64 + d + j) * H + h for
-// chunk j of document d (the backward's checkpoint layout).
+// ckpt: optional, receives per chunk a 123904-byte block in slot (cu[d] / 64 + d + j) * H + h for chunk j
+// of document d (the backward's checkpoint layout, kda_fwd_pipe.cu): the state entering the chunk S^T[v][c]
+// and its U~^T[v][s] (bf16, column groups of 16 and 32 values per row), the operand tiles [-W^T | Q~^T],
+// Kd^T and A_qk, T and A_hat (bf16) and e^{Gamma_last} (fp32).  With ckpt set no output is formed: out
+// only gives the unused output map a valid base.
 cudaError_t launch_fwd_pipe(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                             const float *beta, const int32_t *cu, int n_docs, int64_t T, int H,
                             const float *h0, float *ht, uint16_t *out, int *status, cudaStream_t stream,
