@@ -65,6 +65,10 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_fwd_long_segments.argtypes = [i64, i32, i32]
         L.kda_abi_version.restype = i32
         L.kda_abi_version.argtypes = []
+        L.kda_chunk_fwd_host.restype = i32
+        L.kda_chunk_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp, ctypes.c_size_t, vp]
+        L.kda_chunk_fwd_host_workspace_size.restype = ctypes.c_size_t
+        L.kda_chunk_fwd_host_workspace_size.argtypes = [i32, i64, i32]
         _lib = L
     return _lib
 
@@ -174,6 +178,39 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                                    ctypes.c_void_p(_stream_handle(stream)))
     _check(rc)
     return (out, final_state) if final_state is not None else out
+
+
+def host_workspace_bytes(n_docs: int, T: int, H: int) -> int:
+    """Device workspace bytes of ``kda_chunk_fwd_host``."""
+    return int(lib().kda_chunk_fwd_host_workspace_size(n_docs, T, H))
+
+
+def kda_chunk_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                       cu_seqlens: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                       stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """kda_chunk_fwd_host: the forward on HOST tensors (copies to the device workspace, the forward and
+    the copy of the output back are enqueued on `stream`).
+
+    q, k, v, g, beta, cu_seqlens, out: contiguous CPU tensors with kda_chunk_fwd's dtypes and shapes
+    (pinned memory for asynchronous copies); workspace: a CUDA uint8 tensor of at least
+    ``host_workspace_bytes`` bytes.  Returns out, complete once the stream is synchronised.
+    """
+    T, H, D = q.shape
+    for name, t, dt, shape in (("q", q, torch.bfloat16, (T, H, D)), ("k", k, torch.bfloat16, (T, H, D)),
+                               ("v", v, torch.bfloat16, (T, H, D)), ("g", g, torch.float32, (T, H, D)),
+                               ("beta", beta, torch.float32, (T, H)), ("out", out, torch.bfloat16, (T, H, D))):
+        if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or t.is_cuda:
+            raise KdaError(1, f"{name} must be a contiguous host {dt} tensor of shape {shape}")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise KdaError(1, "cu_seqlens must be a 1-d int32 host tensor")
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda:
+        raise KdaError(1, "workspace must be a CUDA uint8 tensor")
+    n_docs = cu_seqlens.numel() - 1
+    rc = lib().kda_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), n_docs, T, H,
+                                  _ptr(out), _ptr(workspace), workspace.numel(),
+                                  ctypes.c_void_p(_stream_handle(stream)))
+    _check(rc)
+    return out
 
 
 def kda_recurrent_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,

@@ -178,6 +178,62 @@ kda_status kda_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_
                       final_state, out, stream);
 }
 
+// Device copies of kda_chunk_fwd_host: q, k, v, out (bf16), g (fp32), beta (fp32), cu_seqlens (int32),
+// each starting on a 256-byte boundary.
+size_t kda_chunk_fwd_host_workspace_size(int n_docs, int64_t T, int H) {
+    if (n_docs < 1 || H < 1 || T < 0) return 0;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t nel = (size_t)T * (size_t)H * KDA_HEAD_DIM;
+    return 4 * up(nel * 2) + up(nel * 4) + up((size_t)T * H * 4) + up(((size_t)n_docs + 1) * 4);
+}
+
+kda_status kda_chunk_fwd_host(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                              const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                              uint16_t *out, void *workspace, size_t workspace_bytes, void *stream) {
+    g_err[0] = '\0';
+    if (n_docs < 1) return fail(KDA_ERR_INVALID_ARG, "n_docs must be >= 1 (got %d)", n_docs);
+    if (H < 1) return fail(KDA_ERR_INVALID_ARG, "H must be >= 1 (got %d)", H);
+    if (T < 0) return fail(KDA_ERR_INVALID_ARG, "T must be >= 0 (got %lld)", (long long)T);
+    if (T > (int64_t)INT32_MAX) return fail(KDA_ERR_INVALID_ARG, "T must fit int32 (cu_seqlens is int32)");
+    if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if (T == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !out) return fail(KDA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    if (!workspace || !aligned(workspace, 256))
+        return fail(KDA_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device buffer");
+    const size_t need = kda_chunk_fwd_host_workspace_size(n_docs, T, H);
+    if (workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+    int dev = -1;
+    kda_status s = check_device(&dev);
+    if (s != KDA_OK) return s;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t nel = (size_t)T * (size_t)H * KDA_HEAD_DIM;
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    uint16_t *dq = reinterpret_cast<uint16_t *>(w);
+    uint16_t *dk = reinterpret_cast<uint16_t *>(w + up(nel * 2));
+    uint16_t *dv = reinterpret_cast<uint16_t *>(w + 2 * up(nel * 2));
+    uint16_t *dout = reinterpret_cast<uint16_t *>(w + 3 * up(nel * 2));
+    float *dg = reinterpret_cast<float *>(w + 4 * up(nel * 2));
+    float *dbeta = reinterpret_cast<float *>(w + 4 * up(nel * 2) + up(nel * 4));
+    int32_t *dcu = reinterpret_cast<int32_t *>(w + 4 * up(nel * 2) + up(nel * 4) + up((size_t)T * H * 4));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    struct Copy {
+        void *dst;
+        const void *src;
+        size_t bytes;
+    } const ins[6] = {{dq, q, nel * 2}, {dk, k, nel * 2}, {dv, v, nel * 2}, {dg, g, nel * 4},
+                      {dbeta, beta, (size_t)T * H * 4}, {dcu, cu_seqlens, ((size_t)n_docs + 1) * 4}};
+    for (const Copy &c : ins) {
+        const cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "host-to-device copy: %s", cudaGetErrorString(e));
+    }
+    s = kda_chunk_fwd(dq, dk, dv, dg, dbeta, dcu, n_docs, T, H, dout, stream);
+    if (s != KDA_OK) return s;
+    const cudaError_t e = cudaMemcpyAsync(out, dout, nel * 2, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "device-to-host copy: %s", cudaGetErrorString(e));
+    return KDA_OK;
+}
+
 kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
                          uint16_t *out, void *stream) {

@@ -86,6 +86,36 @@ kda_status kda_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          int n_docs, int64_t T, int H, uint16_t *out, void *stream);
 
 /*
+ * kda_chunk_fwd_host -- kda_chunk_fwd on HOST buffers: the end-to-end call.
+ *
+ * Enqueues on `stream`, in this order: one cudaMemcpyAsync per input (q, k, v, g, beta,
+ * cu_seqlens) from host memory into the caller's device workspace, the forward of kda_chunk_fwd
+ * on those device copies, and one cudaMemcpyAsync of the output back into host `out`.  The
+ * operation and its result are kda_chunk_fwd's (bit-identical on the same inputs).
+ *
+ * Arguments: q, k, v, g, beta, cu_seqlens, out, n_docs, T, H as kda_chunk_fwd, except that the
+ * seven arrays are HOST memory (page-locked for the copies to run asynchronously at the link's
+ * rate; pageable memory works but CUDA stages it and the call may block); no alignment rule.
+ *   workspace        DEVICE memory, 256-byte aligned, at least
+ *                    kda_chunk_fwd_host_workspace_size(n_docs, T, H) bytes; it receives the
+ *                    device copies (content on entry ignored).
+ *   workspace_bytes  its size.
+ * Ownership: the caller owns every buffer.  The call is asynchronous: the host arrays must stay
+ * valid and unchanged until the stream has passed the copies, and out is complete only after the
+ * stream is synchronised.
+ * Errors: as kda_chunk_fwd, checked before anything is enqueued, plus KDA_ERR_INVALID_ARG for a
+ * missing, misaligned or small workspace and KDA_ERR_CUDA when a copy cannot be enqueued.  As in
+ * kda_chunk_fwd, cu_seqlens is validated on the device (KDA_ERR_BAD_SEQLENS via
+ * kda_device_status).
+ */
+kda_status kda_chunk_fwd_host(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                              const float *beta, const int32_t *cu_seqlens, int n_docs, int64_t T, int H,
+                              uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device workspace bytes of kda_chunk_fwd_host (0 for invalid sizes). */
+size_t kda_chunk_fwd_host_workspace_size(int n_docs, int64_t T, int H);
+
+/*
  * kda_chunk_fwd_state -- kda_chunk_fwd with an initial and a final state per chain.
  *
  * The same forward, except that the state of each (document, head) chain starts from

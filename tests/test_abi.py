@@ -106,3 +106,24 @@ def test_backward_workspace_size(L):
     per = 123904 + 49152
     for n_docs, T, H in ((1, 64, 1), (5, 1328, 4), (16, 32768, 32), (1, 65536, 32)):
         assert L.kda_chunk_bwd_workspace_size(n_docs, T, H) == (T // 64 + n_docs) * H * per
+
+
+def test_host_entry_point_checks_before_any_copy(L):
+    """kda_chunk_fwd_host (host inputs, device workspace) rejects bad sizes, pointers and workspaces
+    on the host, before anything is enqueued; its workspace holds the device copies of the inputs and
+    the output, each on a 256-byte boundary."""
+    vp = ctypes.c_void_p
+    need = L.kda_chunk_fwd_host_workspace_size(1, 64, 1)
+    up = lambda x: (x + 255) // 256 * 256
+    assert need == 4 * up(64 * 128 * 2) + up(64 * 128 * 4) + up(64 * 4) + up(2 * 4)
+    assert L.kda_chunk_fwd_host_workspace_size(0, 64, 1) == 0
+
+    def host(ws=FAKE, ws_bytes=need, n_docs=1, T=64, q=FAKE):
+        return L.kda_chunk_fwd_host(vp(q), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), n_docs, T, 1,
+                                    vp(FAKE), vp(ws), ws_bytes, None)
+    assert host(n_docs=0) == 1 and b"n_docs" in L.kda_last_error()
+    assert host(T=0) == 0
+    assert host(q=0) == 1 and b"NULL" in L.kda_last_error()
+    assert host(ws=0) == 1 and b"workspace" in L.kda_last_error()
+    assert host(ws=FAKE + 16) == 1 and b"256-byte" in L.kda_last_error()
+    assert host(ws_bytes=need - 1) == 1 and b"too small" in L.kda_last_error()

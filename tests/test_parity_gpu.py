@@ -223,3 +223,20 @@ def test_device_wait_timeout_is_reported_and_context_survives(kda):
     ref = oracle_out(d)
     rel, mx = compare(got, ref, d["cu_seqlens"], w.H)
     assert rel <= RTOL_L2 and mx <= ATOL_MAX, (rel, mx)
+
+
+def test_host_entry_point_matches_device_call(kda):
+    """kda_chunk_fwd_host (pinned host inputs and output, device workspace, copies on the stream) gives
+    the bytes kda_chunk_fwd gives on the same inputs (8 packed documents of ragged lengths, H = 8)."""
+    import torch
+    w = workload(1)
+    d = generate(w)
+    t = to_device(d)
+    want = kda.kda_chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["cu_seqlens"], split=False)
+    h = {key: x.cpu().pin_memory() for key, x in t.items()}
+    out = torch.empty(want.shape, dtype=torch.bfloat16).pin_memory()
+    ws = torch.empty(kda.host_workspace_bytes(w.n_docs, w.T, w.H), dtype=torch.uint8, device="cuda")
+    kda.kda_chunk_fwd_host(h["q"], h["k"], h["v"], h["g"], h["beta"], h["cu_seqlens"], out, ws)
+    kda.device_status()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), want.view(torch.int16).cpu())
